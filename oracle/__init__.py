@@ -1,0 +1,160 @@
+"""CPU oracle for the 1D deformable convolution forward -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports it, and it never imports the product path.
+
+The arithmetic lives in ``dcn1d_oracle.c`` (plain loops, double accumulation,
+float32 sampling positions); this module only marshals arrays.  bf16 inputs are
+widened to float32 exactly before they reach the C code.
+
+Parity status: every function is pinned by ``tests/test_oracle_pins.py``
+except the exact clamp bounds of constrained mode, which no page fixes; those
+are checked only through invariants (locality, saturation) and are
+"parity unpinned" as to the bounds themselves.
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+
+import numpy as np
+import torch
+
+from . import build as _build
+
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_p = ctypes.c_void_p
+
+
+def _f32(t):
+    """float32 contiguous numpy copy (bf16 -> f32 widening is exact)."""
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        return np.ascontiguousarray(t.detach().cpu().to(torch.float32).numpy())
+    return np.ascontiguousarray(np.asarray(t, dtype=np.float32))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Oracle:
+    """ctypes front of one build of ``dcn1d_oracle.c``."""
+
+    def __init__(self, lib_path: str):
+        lib = ctypes.CDLL(lib_path)
+        lib.oracle_out_length.restype = _i64
+        lib.oracle_out_length.argtypes = [_i64] * 5
+        lib.oracle_forward.restype = _int
+        lib.oracle_forward.argtypes = [_p] * 5 + [_i64] * 11 + [_int, _p]
+        lib.oracle_forward_points.restype = _int
+        lib.oracle_forward_points.argtypes = [_p] * 5 + [_i64] * 11 + [_int, _p, _i64, _p]
+        lib.oracle_sample_index.restype = _int
+        lib.oracle_sample_index.argtypes = [_p] + [_i64] * 8 + [_int, _p, _p]
+        lib.oracle_threads.restype = _int
+        lib.oracle_threads.argtypes = []
+        lib.oracle_set_threads.restype = None
+        lib.oracle_set_threads.argtypes = [_int]
+        self.lib = lib
+        self.path = lib_path
+
+    def out_length(self, L_in: int, K: int, stride: int, padding: int, dilation: int) -> int:
+        """Output length by the conv1d closed form; -1 when invalid."""
+        return int(self.lib.oracle_out_length(L_in, K, stride, padding, dilation))
+
+    def threads(self) -> int:
+        return int(self.lib.oracle_threads())
+
+    def set_threads(self, n: int) -> None:
+        self.lib.oracle_set_threads(int(n))
+
+    @staticmethod
+    def _dims(x, weight, offsets, stride, padding, dilation, groups, offset_groups):
+        B, C_in, L_in = x.shape
+        C_out, _, K = weight.shape
+        L_out = offsets.shape[2]
+        if offsets.shape[1] != offset_groups:
+            raise ValueError("offsets.shape[1] must equal offset_groups")
+        if weight.shape[1] * groups != C_in or offsets.shape[3] != K or offsets.shape[0] != B:
+            raise ValueError("weight/offsets shapes disagree with x and groups")
+        return (B, C_in, L_in, C_out, K, L_out, stride, padding, dilation, groups, offset_groups)
+
+    def forward(self, x, offsets, mask, weight, bias, stride, padding, dilation, groups,
+                offset_groups, unconstrained) -> np.ndarray:
+        """All outputs, float64 [B, C_out, L_out]."""
+        xs, os_, ms, ws, bs = (_f32(t) for t in (x, offsets, mask, weight, bias))
+        dims = self._dims(xs, ws, os_, stride, padding, dilation, groups, offset_groups)
+        out = np.empty((dims[0], dims[3], dims[5]), dtype=np.float64)
+        rc = self.lib.oracle_forward(_ptr(xs), _ptr(os_), _ptr(ms), _ptr(ws), _ptr(bs), *dims,
+                                     int(bool(unconstrained)), _ptr(out))
+        if rc != 0:
+            raise ValueError(f"oracle_forward rejected the shapes (code {rc})")
+        return out
+
+    def forward_points(self, x, offsets, mask, weight, bias, stride, padding, dilation, groups,
+                       offset_groups, unconstrained, points) -> np.ndarray:
+        """Selected outputs; ``points`` is an int array [n, 3] of (b, co, l)."""
+        xs, os_, ms, ws, bs = (_f32(t) for t in (x, offsets, mask, weight, bias))
+        dims = self._dims(xs, ws, os_, stride, padding, dilation, groups, offset_groups)
+        pts = np.ascontiguousarray(np.asarray(points, dtype=np.int64).reshape(-1, 3))
+        out = np.empty(pts.shape[0], dtype=np.float64)
+        rc = self.lib.oracle_forward_points(_ptr(xs), _ptr(os_), _ptr(ms), _ptr(ws), _ptr(bs),
+                                            *dims, int(bool(unconstrained)), _ptr(pts),
+                                            pts.shape[0], _ptr(out))
+        if rc != 0:
+            raise ValueError(f"oracle_forward_points rejected the arguments (code {rc})")
+        return out
+
+    def sample_index(self, offsets, L_in, K, stride, padding, dilation, unconstrained):
+        """(i0 int32, frac float32) for every tap, each shaped like ``offsets``."""
+        os_ = _f32(offsets)
+        B, G, L_out, K2 = os_.shape
+        if K2 != K:
+            raise ValueError("offsets.shape[3] must equal K")
+        i0 = np.empty(os_.shape, dtype=np.int32)
+        fr = np.empty(os_.shape, dtype=np.float32)
+        rc = self.lib.oracle_sample_index(_ptr(os_), B, G, L_in, K, L_out, stride, padding,
+                                          dilation, int(bool(unconstrained)), _ptr(i0), _ptr(fr))
+        if rc != 0:
+            raise ValueError("oracle_sample_index: offsets length disagrees with the closed form")
+        return i0, fr
+
+
+_default = None
+_lock = threading.Lock()
+
+
+def get() -> Oracle:
+    """The oracle built from this directory's source (compiled on first use)."""
+    global _default
+    with _lock:
+        if _default is None:
+            _default = Oracle(_build.build())
+    return _default
+
+
+def out_length(*a):
+    return get().out_length(*a)
+
+
+def forward(*a, **k):
+    return get().forward(*a, **k)
+
+
+def forward_points(*a, **k):
+    return get().forward_points(*a, **k)
+
+
+def sample_index(*a, **k):
+    return get().sample_index(*a, **k)
+
+
+def threads():
+    return get().threads()
+
+
+def set_threads(n):
+    return get().set_threads(n)
