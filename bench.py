@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the DeformConv1d forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|all] [--impl ours|reference]
+
+A step is one full forward pass (sampling, interpolation, mask, contraction, bias, store)
+over one batch of the named synthetic workload (default: the dc1d page's usage shape in
+fp32, B=16, C=512, K=16, dilation 3, L=128).  Inputs are resident in HBM before the timed
+region; L2 is flushed (a 256 MiB write) between steps, outside the timed events; each step
+is timed with CUDA events on the launching stream, with a barrier and a device
+synchronisation on both sides of the K timed steps, and the time is the max over ranks.
+Under torchrun each rank runs its own batch (weak scaling, no collective on the data path).
+
+``--impl reference`` times the CPU oracle instead (rank 0 only), on bounded samples of the
+same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "DeformConv1d forward TFLOP/s (HBM GB/s if depthwise) as % of B200 roofline"
+DEFAULT_WORKLOAD = "usage_f32"
+L2_FLUSH_BYTES = 256 << 20
+
+# Fallback denominators (used only when MEASURED_PEAKS.json is absent).
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+# fp32 FFMA ALU peak: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz (clocks.max.sm).
+ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# Nominal dense tensor ratios to bf16 (2.25 PFLOP/s): tf32 1.1 PFLOP/s.
+TF32_OVER_BF16 = 1.1 / 2.25
+
+
+# ------------------------------------------------------------------ peaks and roofline
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def roofline_for(kernel: str, w: W.Workload, peaks: dict):
+    """(bound, unit, peak, algorithmic amount per launch, note) of the step's main kernel."""
+    flops = w.flops() / 1e12
+    gbytes = w.algorithmic_bytes() / 1e9
+    src = peaks["source"]
+    if kernel.startswith("depthwise"):
+        return "hbm", "GB/s", peaks["hbm_gbs"], gbytes, f"HBM copy bandwidth ({src})"
+    if kernel.startswith("tcgen05_bf16"):
+        return "tensor", "TFLOP/s", peaks["bf16_tflops"], flops, f"bf16 dense GEMM burst ({src})"
+    if kernel.startswith("tcgen05_3xtf32"):
+        pk = peaks["bf16_tflops"] * TF32_OVER_BF16 / 3.0
+        return ("tensor", "TFLOP/s", pk, flops,
+                f"tf32 peak (bf16 burst {src} x 1.1/2.25 nominal) / 3 passes of 3xTF32")
+    return "alu", "TFLOP/s", ALU_F32_TFLOPS, flops, "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz"
+
+
+def load_traffic(kernel: str, w: W.Workload):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this kernel source."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    for line in lines:
+        if not line.strip() or line.startswith("#"):
+            continue
+        parts = line.split()
+        if len(parts) < 4 or parts[0] != kernel or parts[1] != w.name:
+            continue
+        src = os.path.join(ROOT, "deformable_convolution_dcn1d_b200", "csrc", parts[3])
+        want = parts[4] if len(parts) > 4 else None
+        try:
+            h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        except OSError:
+            return None
+        if want is not None and h != want:
+            return None   # the kernel changed since the counters were taken
+        return float(parts[2])
+    return None
+
+
+# ------------------------------------------------------------------ clocks during the region
+
+class ClockSampler:
+    """Polls NVML (SM clock, throttle reasons) every few ms while the timed region runs."""
+
+    REASONS = [("gpu_idle", "nvmlClocksEventReasonGpuIdle"),
+               ("applications_clocks_setting", "nvmlClocksEventReasonApplicationsClocksSetting"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("sync_boost", "nvmlClocksEventReasonSyncBoost"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown")]
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, attr in self.REASONS:
+                    if bits & getattr(nv, attr, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(value: float, ws: int, device: str = "cuda") -> float:
+    if ws == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ the CPU oracle baseline
+
+def time_oracle(w: W.Workload, inputs: dict, target_s: float, seed: int = 0):
+    """Time the oracle on a bounded random sample of the workload's outputs."""
+    import numpy as np
+    import oracle
+    per_point_flops = 2 * (w.C_in // w.groups) * w.K
+    total_points = w.B * w.C_out * w.L_out
+    rng = np.random.default_rng(seed)
+
+    def pts(n):
+        return np.stack([rng.integers(0, w.B, n), rng.integers(0, w.C_out, n),
+                         rng.integers(0, w.L_out, n)], axis=1)
+
+    args = (inputs["x"], inputs["offsets"], inputs["mask"], inputs["weight"], inputs["bias"],
+            w.stride, w.padding, w.dilation, w.groups, w.offset_groups, w.unconstrained)
+    n = 256
+    while True:
+        p = pts(n)
+        t0 = time.perf_counter()
+        oracle.forward_points(*args, p)
+        dt = time.perf_counter() - t0
+        if dt > 0.2 or n >= total_points:
+            break
+        n = min(n * 4, total_points)
+    n = int(min(total_points, max(n, n * target_s / max(dt, 1e-9))))
+    p = pts(n)
+    t0 = time.perf_counter()
+    oracle.forward_points(*args, p)
+    dt = time.perf_counter() - t0
+    return n * per_point_flops / dt / 1e12, n, dt, oracle.threads()
+
+
+def unit_value(w: W.Workload, kernel: str, seconds: float, ranks: int = 1):
+    """Whole-job throughput in the metric's unit."""
+    if kernel.startswith("depthwise"):
+        return ranks * w.algorithmic_bytes() / seconds / 1e9, "GB/s"
+    return ranks * w.flops() / seconds / 1e12, "TFLOP/s"
+
+
+# ------------------------------------------------------------------ the two arms
+
+def run_reference(args, w: W.Workload):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    inputs = W.make_inputs(w, seed=0)
+    per_point_flops = 2 * (w.C_in // w.groups) * w.K
+    # Calibrate one step to about 1 s of oracle work.
+    _, n_step, _, cores = time_oracle(w, inputs, target_s=1.0)
+    import numpy as np
+    rng = np.random.default_rng(1)
+    a = (inputs["x"], inputs["offsets"], inputs["mask"], inputs["weight"], inputs["bias"],
+         w.stride, w.padding, w.dilation, w.groups, w.offset_groups, w.unconstrained)
+
+    def step():
+        p = np.stack([rng.integers(0, w.B, n_step), rng.integers(0, w.C_out, n_step),
+                      rng.integers(0, w.L_out, n_step)], axis=1)
+        oracle.forward_points(*a, p)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    depthwise = w.groups == w.C_in == w.C_out
+    if depthwise:
+        frac = n_step * args.steps / (w.B * w.C_out * w.L_out)
+        value, unit = frac * w.algorithmic_bytes() / dt / 1e9, "GB/s"
+    else:
+        value, unit = n_step * args.steps * per_point_flops / dt / 1e12, "TFLOP/s"
+    sample = f"{n_step} random outputs per step of {w.B * w.C_out * w.L_out}"
+    return {"metric": METRIC, "value": value, "unit": unit, "impl": "reference",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, "oracle", ws, l2="n/a (CPU)"),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def workload_config(w: W.Workload, kernel: str, ws: int, l2: str):
+    return {"workload": w.name, "B": w.B, "C_in": w.C_in, "C_out": w.C_out, "K": w.K,
+            "stride": w.stride, "padding": w.padding, "dilation": w.dilation,
+            "groups": w.groups, "offset_groups": w.offset_groups, "L_in": w.L_in,
+            "L_out": w.L_out, "dtype": w.dtype, "mask": w.mask,
+            "unconstrained": w.unconstrained, "kernel": kernel, "l2": l2,
+            "parallelism": f"dp{ws} (independent batch per GPU)"}
+
+
+def run_ours(args, w: W.Workload, peaks: dict, want_cpu: bool):
+    import deformable_convolution_dcn1d_b200 as dcn
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dcn.load()
+
+    host = W.make_inputs(w, seed=rank)
+    keys = ["x", "offsets", "mask", "weight", "bias"]
+    dev_in = {k: (host[k].to(dev) if host[k] is not None else None) for k in keys}
+    out = torch.empty((w.B, w.C_out, w.L_out), dtype=w.torch_dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step(d, o):
+        dcn.dcn1d_forward(d["x"], d["offsets"], d["mask"], d["weight"], d["bias"], w.stride,
+                          w.padding, w.dilation, w.groups, w.offset_groups, w.unconstrained,
+                          out=o, stream=stream)
+
+    kernel = dcn.dcn1d_forward_kernel_name(dev_in["x"], dev_in["offsets"], dev_in["mask"],
+                                           dev_in["weight"], dev_in["bias"], w.stride,
+                                           w.padding, w.dilation, w.groups, w.offset_groups,
+                                           w.unconstrained, out)
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step(dev_in, out)
+    torch.cuda.synchronize(dev)
+    launches_per_step = dcn.dcn1d_last_launch_count()
+
+    # ---- device-resident timing
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step(dev_in, out)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(ws)
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    ms = max_over_ranks(ms, ws)
+    ms_step = ms / args.steps
+    value, unit = unit_value(w, kernel, ms_step / 1e3, ws)
+
+    # ---- end to end through the public API from pinned host buffers
+    pinned = {k: (host[k].pin_memory() if host[k] is not None else None) for k in keys}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values() if v is not None)
+    d2h = out_host.numel() * out_host.element_size()
+    scratch = {k: (torch.empty_like(v) if v is not None else None) for k, v in dev_in.items()}
+
+    def e2e_step():
+        for k in keys:
+            if pinned[k] is not None:
+                scratch[k].copy_(pinned[k], non_blocking=True)
+        step(scratch, out)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(args.warmup, 1)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        e2e_step()
+        e_ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(ws)
+    e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), ws)
+    e_value, e_unit = unit_value(w, kernel, e_ms / args.steps / 1e3, ws)
+
+    # ---- roofline of the step's kernel (one kernel per step: its time is the step time)
+    bound, r_unit, peak, per_launch, note = roofline_for(kernel, w, peaks)
+    achieved = per_launch / (ms_step / 1e3)
+    roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
+            "frac": achieved / peak, "traffic": load_traffic(kernel, w), "kernel": kernel,
+            "peak_source": note, "launches_per_step": launches_per_step}
+
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded, shapes and distributions of the named workload)",
+            "config": workload_config(w, kernel, ws,
+                                      l2="flushed between steps (256 MiB write outside the timed events)"),
+            "roofline": roof, "clocks": clk.summary(),
+            "e2e": {"value": e_value, "unit": e_unit, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h,
+                    "note": "pinned host inputs copied in, forward, output copied out, per step"},
+            "gpu_launches": launches_per_step * args.steps}
+    if want_cpu and ws == 1 and rank == 0:
+        v, n, dt, cores = time_oracle(w, host, target_s=args.cpu_seconds)
+        if kernel.startswith("depthwise"):
+            v = n / (w.B * w.C_out * w.L_out) * w.algorithmic_bytes() / dt / 1e9
+        line["cpu_baseline"] = {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
+                                "sample": f"{n} random outputs of {w.B * w.C_out * w.L_out} "
+                                          f"({dt:.1f} s)"}
+    return line if rank == 0 else None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="one of %s, or 'all'" % ", ".join(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    names = list(W.WORKLOADS) if args.workload == "all" else [args.workload]
+    ws, rank, local = dist_env()
+
+    if args.impl == "reference":
+        line = run_reference(args, W.WORKLOADS[names[0]])
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    peaks = load_peaks()
+    try:
+        for name in names:
+            line = run_ours(args, W.WORKLOADS[name], peaks,
+                            want_cpu=not args.no_cpu_baseline)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

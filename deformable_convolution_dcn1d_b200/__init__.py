@@ -1,0 +1,20 @@
+"""B200 (sm_100a) forward pass of 1D deformable convolution (DeformConv1d).
+
+The computation lives in the C-ABI CUDA library ``libdcn1d.so`` (declared in
+``include/dcn1d.h``); this package is its thin Python binding.
+"""
+from ._binding import (  # noqa: F401
+    DCN1D_BF16,
+    DCN1D_F32,
+    Dcn1dError,
+    Dcn1dTensor,
+    SIGNATURES,
+    dcn1d_forward,
+    dcn1d_forward_kernel_name,
+    dcn1d_last_launch_count,
+    dcn1d_out_length,
+    dcn1d_sample_index,
+    dcn1d_status_string,
+    lib_path,
+    load,
+)

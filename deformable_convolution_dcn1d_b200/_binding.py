@@ -1,0 +1,203 @@
+"""ctypes binding of libdcn1d.so (include/dcn1d.h).
+
+Argument marshalling only: torch tensors are described to the C ABI by their
+device pointer, dtype and shape, and the current torch CUDA stream is passed
+through.  Every step of the forward runs in the library's CUDA kernels; there
+is no Python or CPU fallback, and a missing or unbuildable library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_INT = ctypes.c_int
+_P = ctypes.c_void_p
+
+DCN1D_F32 = 0
+DCN1D_BF16 = 1
+_DTYPES = {torch.float32: DCN1D_F32, torch.bfloat16: DCN1D_BF16}
+_BAD_DTYPE = 99   # any other torch dtype: the library rejects it with DCN1D_ERR_DTYPE
+
+STATUS = {0: "DCN1D_OK", 1: "DCN1D_ERR_NULL", 2: "DCN1D_ERR_DTYPE", 3: "DCN1D_ERR_SHAPE",
+          4: "DCN1D_ERR_ARG", 5: "DCN1D_ERR_UNSUPPORTED", 6: "DCN1D_ERR_LAUNCH",
+          7: "DCN1D_ERR_TIMEOUT", 8: "DCN1D_ERR_CUDA"}
+
+
+class Dcn1dTensor(ctypes.Structure):
+    _fields_ = [("data", _P), ("dtype", _I32), ("ndim", _I32), ("shape", _I64 * 4)]
+
+
+class Dcn1dError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {dcn1d_status_string(status)} ({status})")
+
+
+_lib = None
+_lock = threading.Lock()
+
+# Exported symbols and their signatures: (name, restype, argtypes).
+_T = ctypes.POINTER(Dcn1dTensor)
+SIGNATURES = [
+    ("dcn1d_out_length", _I64, [_I64] * 5),
+    ("dcn1d_forward", _INT, [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _P]),
+    ("dcn1d_status_string", ctypes.c_char_p, [_INT]),
+    ("dcn1d_sample_index", _INT, [_T, _I64, _I64, _I64, _I64, _INT, _P, _P, _P]),
+    ("dcn1d_forward_kernel_name", ctypes.c_char_p,
+     [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T]),
+    ("dcn1d_last_launch_count", _INT, []),
+]
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def load():
+    """Load libdcn1d.so, building it from csrc/ with nvcc if it is missing or stale."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.build()
+            if not os.path.exists(path):
+                raise ImportError(f"libdcn1d.so not found at {path}")
+            lib = ctypes.CDLL(path)
+            for name, res, args in SIGNATURES:
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _desc(t):
+    """dcn1d_tensor describing a contiguous torch tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if t.ndim > 4:
+        raise ValueError("at most 4 dimensions")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    d = Dcn1dTensor()
+    d.data = t.data_ptr() if t.numel() > 0 else None
+    d.dtype = _DTYPES.get(t.dtype, _BAD_DTYPE)
+    d.ndim = t.ndim
+    for i, s in enumerate(t.shape):
+        d.shape[i] = s
+    return d
+
+
+def _ref(d):
+    return None if d is None else ctypes.byref(d)
+
+
+def _stream_ptr(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream
+
+
+def _check_device(tensors):
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("every tensor must be on a CUDA device")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("every tensor must be on the same CUDA device")
+    return dev
+
+
+def dcn1d_out_length(L_in: int, kernel_size: int, stride: int = 1, padding: int = 0,
+                     dilation: int = 1) -> int:
+    return int(load().dcn1d_out_length(L_in, kernel_size, stride, padding, dilation))
+
+
+def dcn1d_status_string(status: int) -> str:
+    return load().dcn1d_status_string(int(status)).decode()
+
+
+def dcn1d_last_launch_count() -> int:
+    return int(load().dcn1d_last_launch_count())
+
+
+def _out_for(x, weight, offsets):
+    L_out = offsets.shape[2] if offsets.ndim == 4 else 0
+    return torch.empty((x.shape[0], weight.shape[0], L_out), dtype=x.dtype, device=x.device)
+
+
+def dcn1d_forward(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=1, groups=1,
+                  offset_groups=1, unconstrained=False, out=None, stream=None):
+    """Deformable conv1d forward through the C ABI; returns ``out`` [B, C_out, L_out].
+
+    x [B, C_in, L_in]; offsets and mask [B, offset_groups, L_out, K] (mask may be None);
+    weight [C_out, C_in/groups, K]; bias [C_out] or None.  All CUDA, contiguous, one dtype
+    (float32 or bfloat16).  ``out`` is allocated with torch when not given.  Runs on
+    ``stream`` (default: the current torch stream of x's device); does not synchronise.
+    """
+    dev = _check_device((x, offsets, mask, weight, bias, out))
+    if out is None:
+        out = _out_for(x, weight, offsets)
+    descs = [_desc(t) for t in (x, offsets, mask, weight, bias, out)]
+    lib = load()
+    with torch.cuda.device(dev):
+        st = lib.dcn1d_forward(_ref(descs[0]), _ref(descs[1]), _ref(descs[2]), _ref(descs[3]),
+                               _ref(descs[4]), stride, padding, dilation, groups, offset_groups,
+                               int(bool(unconstrained)), _ref(descs[5]),
+                               _P(_stream_ptr(stream, dev)))
+    if st != 0:
+        raise Dcn1dError(st, "dcn1d_forward")
+    return out
+
+
+def dcn1d_forward_kernel_name(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=1,
+                              groups=1, offset_groups=1, unconstrained=False, out=None):
+    """Name of the kernel dcn1d_forward would launch, or None for invalid arguments."""
+    if out is None:
+        out = torch.empty((x.shape[0], weight.shape[0], offsets.shape[2]), dtype=x.dtype,
+                          device="meta")
+    descs = [_desc(t) if t is None or t.device.type != "meta" else _meta_desc(t)
+             for t in (x, offsets, mask, weight, bias, out)]
+    r = load().dcn1d_forward_kernel_name(*(_ref(d) for d in descs[:5]), stride, padding,
+                                         dilation, groups, offset_groups,
+                                         int(bool(unconstrained)), _ref(descs[5]))
+    return None if r is None else r.decode()
+
+
+def _meta_desc(t):
+    d = Dcn1dTensor()
+    d.data = 16 if t.numel() > 0 else None    # a non-NULL placeholder; never dereferenced
+    d.dtype = _DTYPES.get(t.dtype, _BAD_DTYPE)
+    d.ndim = t.ndim
+    for i, s in enumerate(t.shape):
+        d.shape[i] = s
+    return d
+
+
+def dcn1d_sample_index(offsets, L_in, stride=1, padding=0, dilation=1, unconstrained=False,
+                       stream=None):
+    """(i0 int32, frac float32) of every tap of ``offsets``, computed on the GPU."""
+    dev = _check_device((offsets,))
+    i0 = torch.empty(offsets.shape, dtype=torch.int32, device=dev)
+    fr = torch.empty(offsets.shape, dtype=torch.float32, device=dev)
+    d = _desc(offsets)
+    lib = load()
+    with torch.cuda.device(dev):
+        st = lib.dcn1d_sample_index(ctypes.byref(d), L_in, stride, padding, dilation,
+                                    int(bool(unconstrained)), _P(i0.data_ptr()),
+                                    _P(fr.data_ptr()), _P(_stream_ptr(stream, dev)))
+    if st != 0:
+        raise Dcn1dError(st, "dcn1d_sample_index")
+    return i0, fr

@@ -1,0 +1,238 @@
+// The C ABI (include/dcn1d.h): argument validation, kernel selection and
+// launch on the caller's stream.  Allocates nothing and never synchronises.
+#include <string.h>
+
+#include "common.cuh"
+
+namespace dcn1d {
+namespace {
+
+thread_local int g_last_launches = 0;
+
+constexpr int64_t kMaxElems = (int64_t)1 << 31;   // every tensor indexed with int32 rows
+constexpr int64_t kMaxPos = (int64_t)1 << 24;     // positions exact in float32
+
+int64_t numel(const dcn1d_tensor *t) {
+    int64_t n = 1;
+    for (int i = 0; i < t->ndim; ++i)
+        n *= t->shape[i];
+    return n;
+}
+
+// Descriptor present, known dtype, right rank, non-negative extents, data
+// present unless the tensor is empty.
+int check_desc(const dcn1d_tensor *t, int ndim) {
+    if (!t)
+        return DCN1D_ERR_NULL;
+    if (t->dtype != DCN1D_F32 && t->dtype != DCN1D_BF16)
+        return DCN1D_ERR_DTYPE;
+    if (t->ndim != ndim)
+        return DCN1D_ERR_SHAPE;
+    for (int i = 0; i < ndim; ++i)
+        if (t->shape[i] < 0)
+            return DCN1D_ERR_SHAPE;
+    if (!t->data && numel(t) > 0)
+        return DCN1D_ERR_NULL;
+    return DCN1D_OK;
+}
+
+bool shape_is(const dcn1d_tensor *t, int64_t a, int64_t b, int64_t c, int64_t d = -1) {
+    if (t->shape[0] != a || t->shape[1] != b || t->shape[2] != c)
+        return false;
+    return d < 0 || t->shape[3] == d;
+}
+
+enum Kernel { kDirect = 0 };
+
+const char *kernel_names[] = {"direct"};
+
+// Full validation; fills P and the chosen kernel on success.
+int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor *mask,
+             const dcn1d_tensor *w, const dcn1d_tensor *bias, int64_t stride, int64_t padding,
+             int64_t dilation, int64_t groups, int64_t offset_groups, int unconstrained,
+             const dcn1d_tensor *out, Problem *P, Kernel *kern) {
+    int st;
+    if (!x || !off || !w || !out)
+        return DCN1D_ERR_NULL;
+    if ((st = check_desc(x, 3)) || (st = check_desc(off, 4)) || (st = check_desc(w, 3)) ||
+        (st = check_desc(out, 3)))
+        return st;
+    if (mask && (st = check_desc(mask, 4)))
+        return st;
+    if (bias && (st = check_desc(bias, 1)))
+        return st;
+    const int dt = x->dtype;
+    if (off->dtype != dt || w->dtype != dt || out->dtype != dt || (mask && mask->dtype != dt) ||
+        (bias && bias->dtype != dt))
+        return DCN1D_ERR_DTYPE;
+
+    if (stride < 1 || padding < 0 || dilation < 1 || groups < 1 || offset_groups < 1)
+        return DCN1D_ERR_ARG;
+    const int64_t B = x->shape[0], C_in = x->shape[1], L_in = x->shape[2];
+    const int64_t C_out = w->shape[0], K = w->shape[2];
+    if (C_in < 1 || L_in < 1 || C_out < 1 || K < 1)
+        return DCN1D_ERR_SHAPE;
+    if (C_in % groups || C_out % groups || C_in % offset_groups)
+        return DCN1D_ERR_ARG;
+    if (w->shape[1] * groups != C_in)
+        return DCN1D_ERR_SHAPE;
+    if (stride >= kMaxPos || padding >= kMaxPos || dilation >= kMaxPos || K >= kMaxPos ||
+        L_in >= kMaxPos)
+        return DCN1D_ERR_UNSUPPORTED;
+    const int64_t L_out = dcn1d_out_length(L_in, K, stride, padding, dilation);
+    if (L_out < 1)
+        return DCN1D_ERR_ARG;
+    if (!shape_is(off, B, offset_groups, L_out, K))
+        return DCN1D_ERR_SHAPE;
+    if (mask && !shape_is(mask, B, offset_groups, L_out, K))
+        return DCN1D_ERR_SHAPE;
+    if (bias && bias->shape[0] != C_out)
+        return DCN1D_ERR_SHAPE;
+    if (!shape_is(out, B, C_out, L_out))
+        return DCN1D_ERR_SHAPE;
+    // Largest position any tap forms before its offset: (L_out-1)*s - p + d*(K-1) >= 0 and
+    // smallest -p; both must be exact in float32.
+    if ((L_out - 1) * stride + dilation * (K - 1) >= kMaxPos)
+        return DCN1D_ERR_UNSUPPORTED;
+    if (numel(x) >= kMaxElems || numel(off) >= kMaxElems || numel(w) >= kMaxElems ||
+        numel(out) >= kMaxElems)
+        return DCN1D_ERR_UNSUPPORTED;
+
+    P->B = (int)B;
+    P->C_in = (int)C_in;
+    P->L_in = (int)L_in;
+    P->C_out = (int)C_out;
+    P->K = (int)K;
+    P->L_out = (int)L_out;
+    P->stride = (int)stride;
+    P->padding = (int)padding;
+    P->dilation = (int)dilation;
+    P->groups = (int)groups;
+    P->offset_groups = (int)offset_groups;
+    P->unconstrained = unconstrained ? 1 : 0;
+    P->dtype = dt;
+    P->cin_g = (int)(C_in / groups);
+    P->cout_g = (int)(C_out / groups);
+    P->cin_per_og = (int)(C_in / offset_groups);
+    P->x = x->data;
+    P->off = off->data;
+    P->mask = mask ? mask->data : nullptr;
+    P->w = w->data;
+    P->bias = bias ? bias->data : nullptr;
+    P->out = out->data;
+    *kern = kDirect;
+    return DCN1D_OK;
+}
+
+}  // namespace
+}  // namespace dcn1d
+
+using namespace dcn1d;
+
+extern "C" {
+
+int64_t dcn1d_out_length(int64_t L_in, int64_t K, int64_t stride, int64_t padding,
+                         int64_t dilation) {
+    if (L_in < 1 || K < 1 || stride < 1 || padding < 0 || dilation < 1)
+        return -1;
+    // Arguments past 2^31 are refused so the products below cannot overflow.
+    const int64_t lim = (int64_t)1 << 31;
+    if (L_in > lim || K > lim || stride > lim || padding > lim || dilation > lim)
+        return -1;
+    const int64_t num = L_in + 2 * padding - dilation * (K - 1) - 1;
+    if (num < 0)
+        return -1;
+    return num / stride + 1;
+}
+
+const char *dcn1d_status_string(int status) {
+    switch (status) {
+    case DCN1D_OK: return "DCN1D_OK";
+    case DCN1D_ERR_NULL: return "DCN1D_ERR_NULL";
+    case DCN1D_ERR_DTYPE: return "DCN1D_ERR_DTYPE";
+    case DCN1D_ERR_SHAPE: return "DCN1D_ERR_SHAPE";
+    case DCN1D_ERR_ARG: return "DCN1D_ERR_ARG";
+    case DCN1D_ERR_UNSUPPORTED: return "DCN1D_ERR_UNSUPPORTED";
+    case DCN1D_ERR_LAUNCH: return "DCN1D_ERR_LAUNCH";
+    case DCN1D_ERR_TIMEOUT: return "DCN1D_ERR_TIMEOUT";
+    case DCN1D_ERR_CUDA: return "DCN1D_ERR_CUDA";
+    default: return "DCN1D_UNKNOWN_STATUS";
+    }
+}
+
+int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
+                  const dcn1d_tensor *weight, const dcn1d_tensor *bias, int64_t stride,
+                  int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
+                  int unconstrained, dcn1d_tensor *out, void *stream) {
+    g_last_launches = 0;
+    Problem P;
+    Kernel kern;
+    int st = validate(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
+                      offset_groups, unconstrained, out, &P, &kern);
+    if (st != DCN1D_OK)
+        return st;
+    if (P.B == 0)
+        return DCN1D_OK;   // empty batch: nothing to compute
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t err = cudaSuccess;
+    switch (kern) {
+    case kDirect:
+        err = launch_direct(P, s);
+        g_last_launches = 1;
+        break;
+    }
+    if (err != cudaSuccess) {
+        g_last_launches = 0;
+        return DCN1D_ERR_LAUNCH;
+    }
+    return DCN1D_OK;
+}
+
+const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                                      const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                                      const dcn1d_tensor *bias, int64_t stride, int64_t padding,
+                                      int64_t dilation, int64_t groups, int64_t offset_groups,
+                                      int unconstrained, const dcn1d_tensor *out) {
+    Problem P;
+    Kernel kern;
+    if (validate(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
+                 offset_groups, unconstrained, out, &P, &kern) != DCN1D_OK)
+        return nullptr;
+    return kernel_names[kern];
+}
+
+int dcn1d_last_launch_count(void) { return g_last_launches; }
+
+int dcn1d_sample_index(const dcn1d_tensor *offsets, int64_t L_in, int64_t stride,
+                       int64_t padding, int64_t dilation, int unconstrained, int32_t *i0,
+                       float *frac, void *stream) {
+    int st = check_desc(offsets, 4);
+    if (st != DCN1D_OK)
+        return st;
+    const int64_t B = offsets->shape[0], G = offsets->shape[1], L_out = offsets->shape[2],
+                  K = offsets->shape[3];
+    const int64_t n = numel(offsets);
+    if (n > 0 && (!i0 || !frac))
+        return DCN1D_ERR_NULL;
+    if (stride < 1 || padding < 0 || dilation < 1 || L_in < 1 || K < 1)
+        return DCN1D_ERR_ARG;
+    if (stride >= kMaxPos || padding >= kMaxPos || dilation >= kMaxPos || K >= kMaxPos ||
+        L_in >= kMaxPos)
+        return DCN1D_ERR_UNSUPPORTED;
+    const int64_t want = dcn1d_out_length(L_in, K, stride, padding, dilation);
+    if (want < 1)
+        return DCN1D_ERR_ARG;
+    if (L_out != want)
+        return DCN1D_ERR_SHAPE;
+    if ((L_out - 1) * stride + dilation * (K - 1) >= kMaxPos || n >= kMaxElems)
+        return DCN1D_ERR_UNSUPPORTED;
+    if (n == 0)
+        return DCN1D_OK;
+    cudaError_t err = launch_sample_index(offsets->data, offsets->dtype, (int)B, (int)G,
+                                          (int)L_out, (int)K, (int)L_in, (int)stride,
+                                          (int)padding, (int)dilation, unconstrained,
+                                          i0, frac, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? DCN1D_OK : DCN1D_ERR_LAUNCH;
+}
+
+}  // extern "C"

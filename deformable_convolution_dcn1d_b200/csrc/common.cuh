@@ -1,0 +1,42 @@
+// Internal definitions shared by the kernels and the C-ABI host code.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dcn1d.h"
+
+namespace dcn1d {
+
+// A validated forward problem.  All sizes fit in int32 (checked on the host).
+struct Problem {
+    int B, C_in, L_in, C_out, K, L_out;
+    int stride, padding, dilation, groups, offset_groups;
+    int unconstrained;
+    int dtype;                 // dcn1d_dtype
+    int cin_g, cout_g;         // channels per conv group (input, output)
+    int cin_per_og;            // input channels per offset group
+    const void *x, *off, *mask, *w, *bias;
+    void *out;
+};
+
+__device__ __forceinline__ float ld_f32(const float *p) { return __ldg(p); }
+__device__ __forceinline__ float ld_f32(const __nv_bfloat16 *p) { return __bfloat162float(__ldg(p)); }
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <class T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+
+// Kernel launchers (each returns cudaGetLastError() of its launch).
+cudaError_t launch_direct(const Problem &P, cudaStream_t stream);
+cudaError_t launch_sample_index(const void *off, int dtype, int B, int G, int L_out, int K,
+                                int L_in, int stride, int padding, int dilation,
+                                int unconstrained, int32_t *i0, float *frac,
+                                cudaStream_t stream);
+
+}  // namespace dcn1d

@@ -1,0 +1,149 @@
+/*
+ * dcn1d.h -- C ABI of the B200 (sm_100a) forward pass of 1D deformable
+ * convolution (DeformConv1d), with optional DCNv2 modulation mask.
+ *
+ * What the forward computes (sources: the "conv1d" operator page, sections
+ * "Description", "Shape" and "Axis convention"; the dc1d page "dc1d
+ * (DeformConv1d)", sections "Usage / DeformConv1d" and "Modulation (DCNv2)";
+ * the article "A Detailed Explanation of the Calculation Workflow for Dilated
+ * Convolution and Deformable Convolution", section "Deformable Convolution"
+ * and its "Step 2: Deformable Sampling"):
+ *
+ *   out[b,co,l] = bias[co] + sum_{ci in group(co)} sum_{k<K}
+ *                   weight[co, ci - c0(co), k] * m[b,g,l,k]
+ *                   * lerp(x[b,ci,:], l*stride - padding + k*dilation + offsets[b,g,l,k])
+ *
+ *   g = ci / (C_in / offset_groups) is the offset group of channel ci (all
+ *   channels of a group share offsets and mask); lerp mixes the two integer
+ *   neighbours i0 = floor(pos) and i0+1 with weights (1-f) and f, f = pos - i0,
+ *   and x reads zero outside [0, L_in-1].  Unless `unconstrained` is set, the
+ *   position is first clamped to the tap's receptive field
+ *   [l*stride - padding, l*stride - padding + dilation*(K-1)].  The position is
+ *   formed in IEEE float32 with round-to-nearest: pos = (float)base + offset;
+ *   i0 = floor(pos); f = pos - (float)i0.  Precondition: offsets are finite and
+ *   |pos| < 2^24 (a NaN or huge offset never causes an out-of-bounds access,
+ *   but its result is unspecified).  m = 1 when the mask is NULL; a mask of
+ *   all ones gives bit-for-bit the same output as a NULL mask.
+ *
+ * Memory: every tensor is a dense, contiguous, row-major array in device
+ * memory of the current CUDA device, described by a dcn1d_tensor.  The caller
+ * owns and allocates every buffer, `out` included; the library never allocates,
+ * frees or synchronises.  Work is enqueued on `stream` (a cudaStream_t; NULL is
+ * the legacy default stream) and runs asynchronously: a returned DCN1D_OK means
+ * the launch was accepted, and device-side failures surface at the caller's
+ * next synchronisation.  Thread safety: calls may be made from several host
+ * threads; outputs must not alias inputs.
+ *
+ * Errors are status codes (never an abort or a device trap).  Every argument
+ * is validated on the host before anything is launched; on a non-OK status
+ * nothing was enqueued.
+ */
+#ifndef DCN1D_H
+#define DCN1D_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dcn1d_status {
+    DCN1D_OK = 0,
+    DCN1D_ERR_NULL = 1,        /* a required pointer (descriptor or data) is NULL          */
+    DCN1D_ERR_DTYPE = 2,       /* unknown dtype, or floating tensors of mixed dtypes       */
+    DCN1D_ERR_SHAPE = 3,       /* wrong ndim, or shapes that disagree with each other      */
+    DCN1D_ERR_ARG = 4,         /* stride/padding/dilation/groups out of range, L_out < 1   */
+    DCN1D_ERR_UNSUPPORTED = 5, /* sizes past the 32-bit index or 2^24 position limits      */
+    DCN1D_ERR_LAUNCH = 6,      /* the CUDA launch itself failed (cudaGetLastError)         */
+    DCN1D_ERR_TIMEOUT = 7,     /* a kernel gave up a bounded wait (see dcn1d_device_status) */
+    DCN1D_ERR_CUDA = 8         /* another CUDA runtime call failed                         */
+} dcn1d_status;
+
+typedef enum dcn1d_dtype {
+    DCN1D_F32 = 0,             /* IEEE float32                                             */
+    DCN1D_BF16 = 1             /* bfloat16                                                 */
+} dcn1d_dtype;
+
+/* A dense, contiguous, row-major device array of `ndim` (<= 4) dimensions. */
+typedef struct dcn1d_tensor {
+    void *data;                /* device pointer; 16-byte alignment enables the fast paths */
+    int32_t dtype;             /* a dcn1d_dtype                                            */
+    int32_t ndim;
+    int64_t shape[4];          /* shape[i] for i < ndim; the rest is ignored               */
+} dcn1d_tensor;
+
+/*
+ * Output length of the convolution ("conv1d" page, "Shape"):
+ *   L_out = floor((L_in + 2*padding - dilation*(kernel_size - 1) - 1) / stride + 1).
+ * Returns -1 if L_in < 1, kernel_size < 1, stride < 1, padding < 0, dilation < 1,
+ * any argument exceeds 2^31, or the length would be < 1.  Host only; needs no
+ * device.
+ */
+int64_t dcn1d_out_length(int64_t L_in, int64_t kernel_size, int64_t stride, int64_t padding,
+                         int64_t dilation);
+
+/*
+ * The deformable convolution forward (formula at the top of this file).
+ *
+ *   x        [B, C_in, L_in]                       required
+ *   offsets  [B, offset_groups, L_out, K]          required; L_out must equal
+ *                                                  dcn1d_out_length(L_in, K, ...)
+ *   mask     [B, offset_groups, L_out, K] or NULL  applied as given (no sigmoid)
+ *   weight   [C_out, C_in / groups, K]             required
+ *   bias     [C_out] or NULL
+ *   out      [B, C_out, L_out]                     required, written entirely
+ *
+ * All floating tensors share one dtype (F32 or BF16); the arithmetic is fp32
+ * (bf16 operands of the tensor-core contraction, fp32 accumulation), and `out`
+ * is written in that same dtype ("conv1d" page: the computation stays in the
+ * input dtype).  groups must divide C_in and C_out; offset_groups must divide
+ * C_in; stride >= 1, padding >= 0, dilation >= 1 ("conv1d" page, "Arguments").
+ * `unconstrained` != 0 lets taps sample anywhere (dc1d page, "Usage").
+ *
+ * Returns DCN1D_OK, or DCN1D_ERR_NULL / _DTYPE / _SHAPE / _ARG / _UNSUPPORTED on
+ * invalid arguments (nothing launched), DCN1D_ERR_LAUNCH if a launch failed.
+ */
+int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
+                  const dcn1d_tensor *weight, const dcn1d_tensor *bias, int64_t stride,
+                  int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
+                  int unconstrained, dcn1d_tensor *out, void *stream);
+
+/* A static, human-readable name of a status code ("DCN1D_OK", ...). Never NULL. */
+const char *dcn1d_status_string(int status);
+
+/*
+ * The sampling step alone, for testing the integer decisions bit for bit: for
+ * every tap of `offsets` ([B, G, L_out, K], F32 or BF16, device memory) write
+ * the integer neighbour i0 = floor(pos) to `i0` and the fraction f = pos - i0
+ * to `frac` (each a device array of B*G*L_out*K elements, same order as
+ * offsets), using the same device function as the forward kernels.  L_out
+ * must equal dcn1d_out_length(L_in, K, stride, padding, dilation).
+ * Errors as for dcn1d_forward.
+ */
+int dcn1d_sample_index(const dcn1d_tensor *offsets, int64_t L_in, int64_t stride,
+                       int64_t padding, int64_t dilation, int unconstrained, int32_t *i0,
+                       float *frac, void *stream);
+
+/*
+ * Which kernel dcn1d_forward would launch for these arguments, as a static
+ * string ("direct", "depthwise", "tcgen05_bf16", ...), or NULL if the arguments
+ * are invalid.  Host only; launches nothing.  For tests and benchmarks.
+ */
+const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                                      const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                                      const dcn1d_tensor *bias, int64_t stride, int64_t padding,
+                                      int64_t dilation, int64_t groups, int64_t offset_groups,
+                                      int unconstrained, const dcn1d_tensor *out);
+
+/*
+ * Number of kernels the last accepted dcn1d_forward call on this host thread
+ * enqueued (0 if none).  For counting launches in benchmarks.
+ */
+int dcn1d_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCN1D_H */
