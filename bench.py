@@ -395,14 +395,20 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (small cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     names = list(W.WORKLOADS) if args.workload == "all" else [args.workload]
     ws, rank, local = dist_env()
 
+    def pick(name):
+        w = W.WORKLOADS[name]
+        return w.with_batch(args.batch) if args.batch else w
+
     if args.impl == "reference":
-        line = run_reference(args, W.WORKLOADS[names[0]])
+        line = run_reference(args, pick(names[0]))
         if line is not None:
             print(json.dumps(line), flush=True)
         return
@@ -416,8 +422,7 @@ def main():
     peaks = load_peaks()
     try:
         for name in names:
-            line = run_ours(args, W.WORKLOADS[name], peaks,
-                            want_cpu=not args.no_cpu_baseline)
+            line = run_ours(args, pick(name), peaks, want_cpu=not args.no_cpu_baseline)
             if line is not None:
                 print(json.dumps(line), flush=True)
     finally:

@@ -42,9 +42,15 @@ bool shape_is(const dcn1d_tensor *t, int64_t a, int64_t b, int64_t c, int64_t d 
     return d < 0 || t->shape[3] == d;
 }
 
-enum Kernel { kDirect = 0 };
+enum Kernel { kDirect = 0, kDepthwise = 1 };
 
-const char *kernel_names[] = {"direct"};
+const char *kernel_names[] = {"direct", "depthwise"};
+
+Kernel select_kernel(const Problem &P) {
+    if (depthwise_supported(P))
+        return kDepthwise;
+    return kDirect;
+}
 
 // Full validation; fills P and the chosen kernel on success.
 int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor *mask,
@@ -120,7 +126,7 @@ int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor 
     P->w = w->data;
     P->bias = bias ? bias->data : nullptr;
     P->out = out->data;
-    *kern = kDirect;
+    *kern = select_kernel(*P);
     return DCN1D_OK;
 }
 
@@ -178,6 +184,10 @@ int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1
     switch (kern) {
     case kDirect:
         err = launch_direct(P, s);
+        g_last_launches = 1;
+        break;
+    case kDepthwise:
+        err = launch_depthwise(P, s);
         g_last_launches = 1;
         break;
     }

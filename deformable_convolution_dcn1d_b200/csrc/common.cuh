@@ -34,6 +34,8 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 // Kernel launchers (each returns cudaGetLastError() of its launch).
 cudaError_t launch_direct(const Problem &P, cudaStream_t stream);
+bool depthwise_supported(const Problem &P);
+cudaError_t launch_depthwise(const Problem &P, cudaStream_t stream);
 cudaError_t launch_sample_index(const void *off, int dtype, int B, int G, int L_out, int K,
                                 int L_in, int stride, int padding, int dilation,
                                 int unconstrained, int32_t *i0, float *frac,

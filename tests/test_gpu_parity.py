@@ -145,10 +145,15 @@ def test_zero_offsets_match_cudnn_conv1d(w):
     td = to_dev(t)
     td["offsets"] = torch.zeros_like(td["offsets"])
     y = gpu_forward(w, td, mask=None)
-    ref = F.conv1d(td["x"].float(), td["weight"].float(),
-                   td["bias"].float() if td["bias"] is not None else None, stride=w.stride,
-                   padding=w.padding, dilation=w.dilation, groups=w.groups)
-    torch.cuda.synchronize()
+    prev = torch.backends.cudnn.allow_tf32
+    torch.backends.cudnn.allow_tf32 = False   # the reference itself must be true fp32
+    try:
+        ref = F.conv1d(td["x"].float(), td["weight"].float(),
+                       td["bias"].float() if td["bias"] is not None else None, stride=w.stride,
+                       padding=w.padding, dilation=w.dilation, groups=w.groups)
+        torch.cuda.synchronize()
+    finally:
+        torch.backends.cudnn.allow_tf32 = prev
     err = (y.float() - ref).abs().max().item() / ref.abs().max().item()
     assert err <= TOL[w.dtype], (w.name, err)
 
