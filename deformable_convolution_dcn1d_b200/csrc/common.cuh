@@ -32,6 +32,11 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(v);
 }
 
+// The kernels that use the conversion-free floor (sampler.cuh) need every
+// signal position below 2^22: then any tap whose floor lands inside the signal
+// had |pos| < 2^22, where that floor is exact.
+inline bool fast_floor_ok(const Problem &P) { return P.L_in < (1 << 22); }
+
 // Kernel launchers (each returns cudaGetLastError() of its launch).
 cudaError_t launch_direct(const Problem &P, cudaStream_t stream);
 bool depthwise_supported(const Problem &P);

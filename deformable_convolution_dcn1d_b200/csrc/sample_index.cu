@@ -1,5 +1,5 @@
 // The sampling step alone: (i0, f) of every tap of an offsets tensor, from
-// the same device function the forward kernels use.  Used to test the integer
+// the same device functions the forward kernels use.  Used to test the integer
 // decisions bit for bit.
 #include "common.cuh"
 #include "sampler.cuh"
@@ -17,8 +17,11 @@ __global__ void __launch_bounds__(256) sample_index_kernel(const T *off, int64_t
         return;
     const int k = (int)(t % K);
     const int l = (int)((t / K) % L_out);
-    Tap tp = sample_tap(l * stride - padding, k, dilation, dilation * (K - 1), ld_f32(off + t),
-                        unconstrained != 0);
+    // The fast floor the forward kernels use wherever it is exact; the conversion
+    // floor elsewhere, so every tap matches the definition bit for bit.
+    const float pos = tap_position(l * stride - padding, k, dilation, dilation * (K - 1),
+                                   ld_f32(off + t), unconstrained != 0);
+    Tap tp = (fabsf(pos) < (float)kFastPosLimit) ? tap_floor_fast(pos) : tap_floor_exact(pos);
     i0[t] = tp.i0;
     frac[t] = tp.f;
 }
