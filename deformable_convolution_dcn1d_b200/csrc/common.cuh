@@ -32,10 +32,14 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(v);
 }
 
-// The kernels that use the conversion-free floor (sampler.cuh) need every
-// signal position below 2^22: then any tap whose floor lands inside the signal
-// had |pos| < 2^22, where that floor is exact.
-inline bool fast_floor_ok(const Problem &P) { return P.L_in < (1 << 22); }
+// The kernels that use the conversion-free floor (sampler.cuh) need the signal
+// and its staged windows well inside (-2^22, 2^22): then any tap whose floor
+// lands inside a window or the signal had |pos| < 2^22, where that floor is
+// exact, and the bit patterns it yields for larger |pos| cannot alias a
+// window index.
+inline bool fast_floor_ok(const Problem &P) {
+    return P.L_in < (1 << 21) && P.padding < (1 << 21);
+}
 
 // Kernel launchers (each returns cudaGetLastError() of its launch).
 cudaError_t launch_direct(const Problem &P, cudaStream_t stream);

@@ -1,22 +1,23 @@
 // Depthwise kernel (groups == C_in == C_out): out[b,c,l] = bias[c] +
 // sum_k w[c,0,k] * m * lerp(x[b,c,:], pos(l,k)).  There is no contraction
 // across channels, so the op is bound by HBM: x, offsets, mask and out should
-// each cross the bus once, and the per-output instruction count must stay
-// below what the HBM rate leaves (~55 thread-instructions per output on B200
-// at full bandwidth for K=3 bf16).
+// each cross the bus once, and the per-output instruction count has to stay
+// below what the HBM rate leaves (about 55 thread-instructions per output on
+// B200 at full bandwidth for K=3 bf16).
 //
 // One CTA owns one (b, c) row and a tile of TL consecutive outputs.
 //  1. The x window its taps can reach (receptive fields plus a margin for
-//     deformed taps) is staged in shared memory as neighbour PAIRS
-//     (x[i], x[i+1]) in fp32, read from DRAM with 16-byte loads and zero
-//     outside the signal, so one 8-byte shared load gives both neighbours.
-//  2. Lane j of each warp owns output l0 + j (+ 32*warp, + 256*iteration):
-//     lanes touch consecutive offsets (coalesced) and gather pairs at nearly
-//     consecutive positions (few bank conflicts).  Taps whose pair lies outside
-//     the window (an offset beyond the margin) read global memory instead, so
-//     any offset value is handled.
-// The floor is the conversion-free fast floor (exact for |pos| < 2^22, the
-// range this kernel is selected for).
+//     deformed taps) is staged in shared memory as neighbour PAIRS: word r
+//     holds (x[wlo+r], x[wlo+r+1]) -- two bf16 in one 32-bit word (fp32: a
+//     float2) -- read from DRAM with 16-byte loads, zero outside the signal.
+//     One shared load then gives both neighbours of a tap.
+//  2. A thread owns groups of 8 consecutive outputs: their 8*K offsets (and
+//     mask) arrive as 16-byte vectors and the 8 results leave as one 16-byte
+//     store.  The arithmetic runs on output pairs with packed f32x2
+//     instructions.  Taps whose pair lies outside the window (an offset beyond
+//     the margin) read global memory instead, so any offset value is handled.
+// The floor is the conversion-free fast floor (exact for |pos| < 2^22; the
+// kernel is selected only for L_in < 2^22).
 #include "common.cuh"
 #include "sampler.cuh"
 
@@ -24,48 +25,121 @@ namespace dcn1d {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;   // outputs per thread per iteration (their loads go out together)
+constexpr int kGroup = 8;   // consecutive outputs per thread-iteration
 
 template <class T>
-struct Vec;   // 16 bytes of T
+struct Traits;
 template <>
-struct Vec<float> {
-    static constexpr int n = 4;
+struct Traits<__nv_bfloat16> {
+    static constexpr int VN = 8;   // elements per 16-byte vector
+    using Word = uint32_t;         // one neighbour pair in the window
 };
 template <>
-struct Vec<__nv_bfloat16> {
-    static constexpr int n = 8;
+struct Traits<float> {
+    static constexpr int VN = 4;
+    using Word = float2;
 };
 
 struct DwArgs {
     Problem P;
-    int TL;          // outputs per tile
+    int TL;          // outputs per tile (multiple of kGroup, or the whole row)
     int tiles;       // tiles per row
     int margin;      // extra positions staged on each side for deformed taps
-    int win_elems;   // shared-memory window length (pairs)
+    int win_elems;   // window length in pairs
 };
 
-__device__ __forceinline__ void unpack16(const uint4 &v, float (&o)[8], const __nv_bfloat16 *) {
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+// 16 bytes of T -> floats.
+__device__ __forceinline__ void unpack16(const uint4 &v, float *o, const __nv_bfloat16 *) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        float2 f = __bfloat1622float2(h[i]);
-        o[2 * i] = f.x;
-        o[2 * i + 1] = f.y;
+        o[2 * i] = __uint_as_float(w[i] << 16);
+        o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
 }
-__device__ __forceinline__ void unpack16(const uint4 &v, float (&o)[8], const float *) {
+__device__ __forceinline__ void unpack16(const uint4 &v, float *o, const float *) {
     o[0] = __uint_as_float(v.x);
     o[1] = __uint_as_float(v.y);
     o[2] = __uint_as_float(v.z);
     o[3] = __uint_as_float(v.w);
 }
 
+__device__ __forceinline__ float2 pair_floats(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ float2 pair_floats(float2 w) { return w; }
+
+// Stage VN window pairs starting at position p0 (window index r0).
+__device__ __forceinline__ void stage_pairs(uint32_t *xp, int r0, const __nv_bfloat16 *row, int p0,
+                                            int L, bool vec_ok) {
+    uint32_t w[5];
+    if (vec_ok && p0 >= 0 && p0 + 8 <= L) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(row + p0));
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int p = p0 + 2 * i;
+            const uint32_t lo = (p >= 0 && p < L) ? (uint32_t)__bfloat16_as_ushort(row[p]) : 0u;
+            const uint32_t hi = (p + 1 >= 0 && p + 1 < L) ? (uint32_t)__bfloat16_as_ushort(row[p + 1]) : 0u;
+            w[i] = lo | (hi << 16);
+        }
+    }
+    const int pn = p0 + 8;
+    w[4] = (pn >= 0 && pn < L) ? (uint32_t)__bfloat16_as_ushort(row[pn]) : 0u;
+    uint4 a, b;   // pair(i) = (x[i], x[i+1]): even i is a whole word, odd i straddles two
+    a.x = w[0];
+    a.y = __byte_perm(w[0], w[1], 0x5432);
+    a.z = w[1];
+    a.w = __byte_perm(w[1], w[2], 0x5432);
+    b.x = w[2];
+    b.y = __byte_perm(w[2], w[3], 0x5432);
+    b.z = w[3];
+    b.w = __byte_perm(w[3], w[4], 0x5432);
+    reinterpret_cast<uint4 *>(xp + r0)[0] = a;
+    reinterpret_cast<uint4 *>(xp + r0)[1] = b;
+}
+__device__ __forceinline__ void stage_pairs(float2 *xp, int r0, const float *row, int p0, int L,
+                                            bool vec_ok) {
+    float x[5];
+    if (vec_ok && p0 >= 0 && p0 + 4 <= L) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(row + p0));
+        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            x[i] = (p0 + i >= 0 && p0 + i < L) ? row[p0 + i] : 0.0f;
+    }
+    x[4] = (p0 + 4 >= 0 && p0 + 4 < L) ? row[p0 + 4] : 0.0f;
+    float4 *dst = reinterpret_cast<float4 *>(xp + r0);
+    dst[0] = make_float4(x[0], x[1], x[1], x[2]);
+    dst[1] = make_float4(x[2], x[3], x[3], x[4]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16 *dst, const float *r) {
+    uint4 o;
+    o.x = pack_bf16x2(r[0], r[1]);
+    o.y = pack_bf16x2(r[2], r[3]);
+    o.z = pack_bf16x2(r[4], r[5]);
+    o.w = pack_bf16x2(r[6], r[7]);
+    *reinterpret_cast<uint4 *>(dst) = o;
+}
+__device__ __forceinline__ void store8(float *dst, const float *r) {
+    reinterpret_cast<float4 *>(dst)[0] = make_float4(r[0], r[1], r[2], r[3]);
+    reinterpret_cast<float4 *>(dst)[1] = make_float4(r[4], r[5], r[6], r[7]);
+}
+
 template <class T, int K, bool UNC, bool MASK>
 __global__ void __launch_bounds__(kThreads) depthwise_kernel(DwArgs A) {
-    extern __shared__ __align__(16) float2 xp[];   // xp[r] = (X(wlo + r), X(wlo + r + 1))
+    using Word = typename Traits<T>::Word;
+    constexpr int VN = Traits<T>::VN;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    Word *xp = reinterpret_cast<Word *>(smem_raw);   // xp[r] = (X(wlo + r), X(wlo + r + 1))
     const Problem &P = A.P;
-    constexpr int VN = Vec<T>::n;
 
     const int tile = blockIdx.x % A.tiles;
     const int bc = blockIdx.x / A.tiles;   // b * C + c
@@ -76,37 +150,16 @@ __global__ void __launch_bounds__(kThreads) depthwise_kernel(DwArgs A) {
     const int span = P.dilation * (K - 1);
 
     const T *xrow = static_cast<const T *>(P.x) + (int64_t)bc * P.L_in;
-    // Window [wlo, wlo + wn): wlo rounded down to a multiple of VN for aligned vectors.
+    // Window [wlo, wlo + wn): wlo rounded down to a multiple of 8 for aligned vectors.
     int wlo = l0 * P.stride - P.padding - A.margin;
-    wlo = (wlo >= 0) ? (wlo / VN) * VN : -(((-wlo) + VN - 1) / VN) * VN;
+    wlo = (wlo >= 0) ? (wlo / 8) * 8 : -(((-wlo) + 7) / 8) * 8;
     const int whi_needed = (l1 - 1) * P.stride - P.padding + span + 2 + A.margin;
-    const int wn = min(A.win_elems, ((whi_needed - wlo) + VN - 1) / VN * VN);
+    const int wn = min(A.win_elems, ((whi_needed - wlo) + 7) / 8 * 8);
 
     // ---- 1. stage the window as neighbour pairs
     const bool xvec = ((reinterpret_cast<uintptr_t>(xrow) & 15) == 0);
-    for (int v = threadIdx.x; v < wn / VN; v += kThreads) {
-        const int p0 = wlo + v * VN;
-        float raw[VN + 1];
-        if (xvec && p0 >= 0 && p0 + VN <= P.L_in) {
-            float tmp[8];
-            unpack16(__ldg(reinterpret_cast<const uint4 *>(xrow + p0)), tmp,
-                     static_cast<const T *>(nullptr));
-#pragma unroll
-            for (int j = 0; j < VN; ++j)
-                raw[j] = tmp[j];
-        } else {
-#pragma unroll
-            for (int j = 0; j < VN; ++j) {
-                const int p = p0 + j;
-                raw[j] = (p >= 0 && p < P.L_in) ? ld_f32(xrow + p) : 0.0f;
-            }
-        }
-        const int pn = p0 + VN;
-        raw[VN] = (pn >= 0 && pn < P.L_in) ? ld_f32(xrow + pn) : 0.0f;
-#pragma unroll
-        for (int j = 0; j < VN; ++j)
-            xp[v * VN + j] = make_float2(raw[j], raw[j + 1]);
-    }
+    for (int v = threadIdx.x; v < wn / VN; v += kThreads)
+        stage_pairs(xp, v * VN, xrow, wlo + v * VN, P.L_in, xvec);
 
     // ---- per-row constants
     const int og = c / P.cin_per_og;
@@ -120,77 +173,121 @@ __global__ void __launch_bounds__(kThreads) depthwise_kernel(DwArgs A) {
         kd[k] = (float)(k * P.dilation);
     }
     const float bias = P.bias ? ld_f32(static_cast<const T *>(P.bias) + c) : 0.0f;
+    const float sf = (float)P.stride;
     const float spanf = (float)span;
     T *orow_out = static_cast<T *>(P.out) + (int64_t)bc * P.L_out;
+    const bool vec = ((reinterpret_cast<uintptr_t>(offp) & 15) == 0) &&
+                     (!MASK || (reinterpret_cast<uintptr_t>(maskp) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(orow_out) & 15) == 0) && ((l0 % kGroup) == 0);
+    // bits(t) - kWinBits = floor(pos) - wlo for t = RD(pos + 1.5*2^23).
+    const unsigned kWinBits = kFloorMagicBits + (unsigned)wlo;
     __syncthreads();
 
-    // ---- 2. outputs: lane-consecutive, kUnroll per thread per iteration
-    const float step_f = (float)(kThreads * P.stride);   // start advance between a thread's outputs
-    for (int lb = l0 + threadIdx.x; lb < l1; lb += kThreads * kUnroll) {
-        float of[kUnroll][K], mk[kUnroll][K];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int l = lb + u * kThreads;
-#pragma unroll
-            for (int k = 0; k < K; ++k) {
-                of[u][k] = (l < l1) ? ld_f32(offp + (int64_t)l * K + k) : 0.0f;
-                if (MASK)
-                    mk[u][k] = (l < l1) ? ld_f32(maskp + (int64_t)l * K + k) : 0.0f;
-            }
+    // Both neighbours of a tap whose floor is t (see tap_floor_fast).
+    auto gather = [&](float t, float pos, float &x0, float &x1) {
+        const unsigned r = __float_as_uint(t) - kWinBits;
+        if (r < (unsigned)(wn - 1)) {
+            const float2 p = pair_floats(xp[r]);
+            x0 = p.x;
+            x1 = p.y;
+        } else {   // beyond the staged window: exact floor, global loads
+            const Tap e = tap_floor_exact(pos);
+            x0 = (e.i0 >= 0 && e.i0 < P.L_in) ? ld_f32(xrow + e.i0) : 0.0f;
+            x1 = (e.i0 >= -1 && e.i0 < P.L_in - 1) ? ld_f32(xrow + e.i0 + 1) : 0.0f;
         }
-        float startf = (float)(lb * P.stride - P.padding);
+    };
+
+    // ---- 2. groups of 8 consecutive outputs, arithmetic on output pairs
+    const int ngroups = vec ? (l1 - l0) / kGroup : 0;
+    for (int gi = threadIdx.x; gi < ngroups; gi += kThreads) {
+        const int lg = l0 + gi * kGroup;
+        float of[kGroup * K], mk[MASK ? kGroup * K : 1];
+        const uint4 *ov = reinterpret_cast<const uint4 *>(offp + (int64_t)lg * K);
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int l = lb + u * kThreads;
-            float acc = bias;
+        for (int j = 0; j < kGroup * K / VN; ++j)
+            unpack16(__ldg(ov + j), of + j * VN, static_cast<const T *>(nullptr));
+        if constexpr (MASK) {
+            const uint4 *mv = reinterpret_cast<const uint4 *>(maskp + (int64_t)lg * K);
+#pragma unroll
+            for (int j = 0; j < kGroup * K / VN; ++j)
+                unpack16(__ldg(mv + j), mk + j * VN, static_cast<const T *>(nullptr));
+        }
+        const float s0 = (float)(lg * P.stride - P.padding);
+        float res[kGroup];
+#pragma unroll
+        for (int i = 0; i < kGroup; i += 2) {
+            // receptive-field starts of outputs i and i+1
+            const float2 st = make_float2(__fadd_rn(s0, (float)i * sf), __fadd_rn(s0, (float)(i + 1) * sf));
+            float2 acc = make_float2(bias, bias);
 #pragma unroll
             for (int k = 0; k < K; ++k) {
-                float pos = __fadd_rn(__fadd_rn(startf, kd[k]), of[u][k]);
-                if (!UNC)
-                    pos = fminf(fmaxf(pos, startf), __fadd_rn(startf, spanf));
-                const Tap t = tap_floor_fast(pos);
-                const unsigned r = (unsigned)t.i0 - (unsigned)wlo;   // wraps when outside
-                float2 x01;
-                if (r < (unsigned)(wn - 1)) {
-                    x01 = xp[r];
-                } else {
-                    x01.x = (t.i0 >= 0 && t.i0 < P.L_in) ? ld_f32(xrow + t.i0) : 0.0f;
-                    x01.y = (t.i0 >= -1 && t.i0 < P.L_in - 1) ? ld_f32(xrow + t.i0 + 1) : 0.0f;
+                float2 pos = __fadd2_rn(__fadd2_rn(st, make_float2(kd[k], kd[k])),
+                                        make_float2(of[i * K + k], of[(i + 1) * K + k]));
+                if (!UNC) {
+                    pos.x = fminf(fmaxf(pos.x, st.x), __fadd_rn(st.x, spanf));
+                    pos.y = fminf(fmaxf(pos.y, st.y), __fadd_rn(st.y, spanf));
                 }
-                float v = __fmaf_rn(t.f, __fsub_rn(x01.y, x01.x), x01.x);
-                if (MASK)
-                    v = __fmul_rn(v, mk[u][k]);
-                acc = __fmaf_rn(wk[k], v, acc);
+                const float2 t = __fadd2_rd(pos, make_float2(kFloorMagic, kFloorMagic));
+                const float2 fl = __fadd2_rn(t, make_float2(-kFloorMagic, -kFloorMagic));
+                const float2 f = __fadd2_rn(pos, make_float2(-fl.x, -fl.y));
+                float2 x0, x1;
+                gather(t.x, pos.x, x0.x, x1.x);
+                gather(t.y, pos.y, x0.y, x1.y);
+                float2 v = __ffma2_rn(f, __fadd2_rn(x1, make_float2(-x0.x, -x0.y)), x0);
+                if constexpr (MASK)
+                    v = __fmul2_rn(v, make_float2(mk[i * K + k], mk[(i + 1) * K + k]));
+                acc = __ffma2_rn(make_float2(wk[k], wk[k]), v, acc);
             }
-            if (l < l1)
-                orow_out[l] = from_f32<T>(acc);
-            startf = __fadd_rn(startf, step_f);
+            res[i] = acc.x;
+            res[i + 1] = acc.y;
         }
+        store8(orow_out + lg, res);
+    }
+
+    // ---- scalar path: everything when vectors are not allowed, else the ragged end
+    const int lstart = l0 + ngroups * kGroup;
+    for (int l = lstart + threadIdx.x; l < l1; l += kThreads) {
+        const float st = (float)(l * P.stride - P.padding);
+        float acc = bias;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            float pos = __fadd_rn(__fadd_rn(st, kd[k]), ld_f32(offp + (int64_t)l * K + k));
+            if (!UNC)
+                pos = fminf(fmaxf(pos, st), __fadd_rn(st, spanf));
+            const float t = __fadd_rd(pos, kFloorMagic);
+            const float f = __fsub_rn(pos, __fsub_rn(t, kFloorMagic));
+            float x0, x1;
+            gather(t, pos, x0, x1);
+            float v = __fmaf_rn(f, __fsub_rn(x1, x0), x0);
+            if constexpr (MASK)
+                v = __fmul_rn(v, ld_f32(maskp + (int64_t)l * K + k));
+            acc = __fmaf_rn(wk[k], v, acc);
+        }
+        orow_out[l] = from_f32<T>(acc);
     }
 }
 
 template <class T, int K, bool UNC, bool MASK>
 cudaError_t launch_kum(const Problem &P, cudaStream_t stream) {
-    constexpr int VN = Vec<T>::n;
+    using Word = typename Traits<T>::Word;
     DwArgs A;
     A.P = P;
     A.margin = UNC ? 32 : 0;
     const int span = P.dilation * (K - 1);
     // Window of a tile of TL outputs: the reach of its taps plus the margin on both sides,
-    // plus slack for rounding its start down to a vector boundary.
+    // plus slack for rounding its start down to a multiple of 8.
     auto win_elems = [&](int TL) -> int64_t {
-        return ((int64_t)(TL - 1) * P.stride + span + 2 + 2 * A.margin + VN + VN - 1) / VN * VN +
-               VN;
+        return ((int64_t)(TL - 1) * P.stride + span + 2 + 2 * A.margin + 7 + 7) / 8 * 8 + 8;
     };
     int TL = 4096;
-    while (TL > 32 && win_elems(TL) * (int64_t)sizeof(float2) > 48 * 1024)
+    while (TL > 32 && win_elems(TL) * (int64_t)sizeof(Word) > 48 * 1024)
         TL /= 2;
     if (TL >= P.L_out)
         TL = P.L_out;
     A.TL = TL;
     A.tiles = (P.L_out + TL - 1) / TL;
     A.win_elems = (int)win_elems(TL);
-    const size_t smem = (size_t)A.win_elems * sizeof(float2);
+    const size_t smem = (size_t)A.win_elems * sizeof(Word);
     if (smem > 48 * 1024)
         return cudaErrorInvalidValue;   // the host selection rule keeps this from happening
     const int64_t blocks = (int64_t)A.tiles * P.B * P.C_in;
@@ -231,7 +328,7 @@ bool depthwise_supported(const Problem &P) {
         return false;
     // The window of the smallest tile (32 outputs) must fit in 48 KB of shared memory.
     const int64_t win = 31LL * P.stride + (int64_t)P.dilation * (P.K - 1) + 2 + 64 + 32;
-    return win * (int64_t)sizeof(float2) <= 48 * 1024;
+    return win * 8 <= 48 * 1024;
 }
 
 cudaError_t launch_depthwise(const Problem &P, cudaStream_t stream) {
