@@ -9,6 +9,7 @@ from ._binding import (  # noqa: F401
     Dcn1dError,
     Dcn1dTensor,
     SIGNATURES,
+    dcn1d_device_status,
     dcn1d_forward,
     dcn1d_forward_kernel_name,
     dcn1d_last_launch_count,

@@ -53,6 +53,7 @@ SIGNATURES = [
     ("dcn1d_forward_kernel_name", ctypes.c_char_p,
      [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T]),
     ("dcn1d_last_launch_count", _INT, []),
+    ("dcn1d_device_status", _INT, [_P]),
 ]
 
 
@@ -131,6 +132,15 @@ def dcn1d_status_string(status: int) -> str:
 
 def dcn1d_last_launch_count() -> int:
     return int(load().dcn1d_last_launch_count())
+
+
+def dcn1d_device_status(stream=None, device=None) -> int:
+    """Synchronise ``stream`` and return (and clear) the kernels' bounded-wait status:
+    0 (DCN1D_OK) or 7 (DCN1D_ERR_TIMEOUT)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    lib = load()
+    with torch.cuda.device(dev):
+        return int(lib.dcn1d_device_status(_P(_stream_ptr(stream, dev))))
 
 
 def _out_for(x, weight, offsets):

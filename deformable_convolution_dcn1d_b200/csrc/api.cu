@@ -42,13 +42,15 @@ bool shape_is(const dcn1d_tensor *t, int64_t a, int64_t b, int64_t c, int64_t d 
     return d < 0 || t->shape[3] == d;
 }
 
-enum Kernel { kDirect = 0, kDepthwise = 1 };
+enum Kernel { kDirect = 0, kDepthwise = 1, kTcBf16 = 2 };
 
-const char *kernel_names[] = {"direct", "depthwise"};
+const char *kernel_names[] = {"direct", "depthwise", "tcgen05_bf16"};
 
 Kernel select_kernel(const Problem &P) {
     if (depthwise_supported(P))
         return kDepthwise;
+    if (tc_bf16_supported(P))
+        return kTcBf16;
     return kDirect;
 }
 
@@ -131,6 +133,32 @@ int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor 
 }
 
 }  // namespace
+
+// One status word per device (a __device__ variable exists once per device).
+__device__ unsigned int g_device_status = 0;
+
+unsigned int *device_status_ptr() {
+    static unsigned int *ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess)
+            return nullptr;
+        ptrs[dev] = static_cast<unsigned int *>(p);
+    }
+    return ptrs[dev];
+}
+
+cudaError_t read_and_clear_device_status(unsigned int *word) {
+    cudaError_t e = cudaMemcpyFromSymbol(word, g_device_status, sizeof(unsigned int));
+    if (e != cudaSuccess)
+        return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_device_status, &zero, sizeof(unsigned int));
+}
+
 }  // namespace dcn1d
 
 using namespace dcn1d;
@@ -190,6 +218,10 @@ int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1
         err = launch_depthwise(P, s);
         g_last_launches = 1;
         break;
+    case kTcBf16:
+        err = launch_tc_bf16(P, s);
+        g_last_launches = 1;
+        break;
     }
     if (err != cudaSuccess) {
         g_last_launches = 0;
@@ -212,6 +244,15 @@ const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor 
 }
 
 int dcn1d_last_launch_count(void) { return g_last_launches; }
+
+int dcn1d_device_status(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return DCN1D_ERR_CUDA;
+    unsigned int word = 0;
+    if (read_and_clear_device_status(&word) != cudaSuccess)
+        return DCN1D_ERR_CUDA;
+    return word ? DCN1D_ERR_TIMEOUT : DCN1D_OK;
+}
 
 int dcn1d_sample_index(const dcn1d_tensor *offsets, int64_t L_in, int64_t stride,
                        int64_t padding, int64_t dilation, int unconstrained, int32_t *i0,

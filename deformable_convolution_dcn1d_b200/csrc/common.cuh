@@ -38,13 +38,19 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // exact, and the bit patterns it yields for larger |pos| cannot alias a
 // window index.
 inline bool fast_floor_ok(const Problem &P) {
-    return P.L_in < (1 << 21) && P.padding < (1 << 21);
+    return (int64_t)P.L_in + 2 * (int64_t)P.padding < (1 << 21);
 }
 
 // Kernel launchers (each returns cudaGetLastError() of its launch).
 cudaError_t launch_direct(const Problem &P, cudaStream_t stream);
 bool depthwise_supported(const Problem &P);
 cudaError_t launch_depthwise(const Problem &P, cudaStream_t stream);
+// The device status word (bounded-wait failures) of the current device, as a
+// device address to hand to kernels (NULL on failure), and its read-and-reset.
+unsigned int *device_status_ptr();
+cudaError_t read_and_clear_device_status(unsigned int *word);
+bool tc_bf16_supported(const Problem &P);
+cudaError_t launch_tc_bf16(const Problem &P, cudaStream_t stream);
 cudaError_t launch_sample_index(const void *off, int dtype, int B, int G, int L_out, int K,
                                 int L_in, int stride, int padding, int dilation,
                                 int unconstrained, int32_t *i0, float *frac,

@@ -11,9 +11,8 @@
 
 namespace dcn1d {
 
-// Device-wide error word: kernels OR bits into it when a bounded wait gives up.
-// Read and cleared by dcn1d_device_status().
-extern __device__ unsigned int g_device_status;
+// Kernels OR this bit into the device status word (its address is a kernel
+// argument, see device_status_ptr) when a bounded wait gives up.
 constexpr unsigned kStatusTimeout = 1u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -65,6 +64,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 struct BoundedWait {
     volatile int *abort;   // shared-memory flag of this CTA
     uint64_t limit_ns;
+    unsigned int *status;  // device status word
 
     __device__ __forceinline__ bool operator()(uint32_t bar, uint32_t parity) const {
         if (mbar_try_wait(bar, parity))
@@ -76,7 +76,7 @@ struct BoundedWait {
             if (*abort)
                 return false;
             if ((i & 15) == 15 && globaltimer_ns() - t0 > limit_ns) {
-                atomicOr(&g_device_status, kStatusTimeout);
+                atomicOr(status, kStatusTimeout);
                 *abort = 1;
                 return false;
             }

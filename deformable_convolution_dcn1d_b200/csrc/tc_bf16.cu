@@ -1,0 +1,561 @@
+// Fused deformable-im2col + tcgen05 tensor-core contraction, bf16 inputs and
+// fp32 accumulation (conv groups with C_out/groups <= 256).
+//
+// Per conv group g the forward is a GEMM over the reduction index kk = (ci, k)
+// of the group (k fastest, the weight's own order):
+//   D[n, co] = sum_kk cols[n, kk] * W[g*Cg_out + co, kk],   n = output position l
+// where cols[n, kk] = m * lerp(x[b, ci, :], pos(l, k)) is the deformable im2col
+// ("conv1d" page, "Description", with the sampling of the deformable-
+// convolution article, "Step 2").  The cols never exist in global memory:
+//
+//  * a TILE is 128 consecutive output positions of one (g, b) and all
+//    Cg_out output channels; the CTA is persistent over tiles;
+//  * TMA warp: per 64-wide k-block, one TMA load of the weight tile
+//    W[co 0..N-1][kk block] (128-byte swizzle, K-major: the MMA's B operand)
+//    and one or two TMA loads of the x window [channels of the block][up to
+//    503 positions] (zero-filled outside the signal) into a stage;
+//  * producer warps (8 = two per TMEM lane quarter): thread = output row; it
+//    turns its row's taps into (window address, fraction, mask) once per
+//    offset group, then for each k-block computes 32 col values from the
+//    staged window and writes them, packed bf16x2, straight into TENSOR
+//    MEMORY with tcgen05.st (the MMA's A operand) -- no shared-memory round
+//    trip for the cols;
+//  * MMA warp: one thread issues 4 tcgen05.mma (M=128, N=Cg_out, K=16) per
+//    k-block, A from tensor memory, B from shared memory, D (fp32) in tensor
+//    memory, and commits completion to the stage's "empty" barrier;
+//  * epilogue warps (4): tcgen05.ld the accumulator, add the bias, round to
+//    bf16 and store; lanes are consecutive l, so each store is 64 contiguous
+//    bytes of out[b, co, :].
+// Stages are chained by mbarriers; every wait is bounded (sm100.cuh).
+#include <string.h>
+
+#include "common.cuh"
+#include "sampler.cuh"
+#include "sm100.cuh"
+
+namespace dcn1d {
+
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kRows = 128;         // output positions per tile = TMEM lanes
+constexpr int kBK = 64;            // reduction elements per k-block
+constexpr int kSeg = 32;           // reduction elements per producer warp and k-block
+constexpr int kBox = 256;          // x window box width (positions)
+constexpr int kBoxStep = 248;      // second box starts here (8 positions of overlap)
+constexpr int kWinMax = 503;       // window positions usable by a tap (pair inside one box)
+constexpr int kRowBytes = kBox * 2;
+constexpr int kThreads = 14 * 32;
+constexpr int kEpiWarp0 = 0;       // warps 0-3
+constexpr int kProdWarp0 = 4;      // warps 4-11
+constexpr int kTmaWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColD = 0;      // D: columns [0, N)
+constexpr uint32_t kColA = 256;    // A stages: columns [256 + 32 s, +32)
+constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s
+
+struct TcArgs {
+    Problem P;
+    int N;             // MMA N = Cg_out (multiple of 32, <= 256)
+    int num_kb;        // k-blocks per tile
+    int tiles_l;       // tiles per (g, b)
+    int num_tiles;
+    int nch;           // x rows per stage
+    int nbox;          // x boxes per stage (1 or 2)
+    int margin;        // staged positions beyond the receptive fields (unconstrained)
+    uint32_t w_stage_bytes, x_stage_bytes, x_box_bytes;
+    uint32_t off_w, off_x, off_bias, off_bar;   // shared-memory layout
+    unsigned int *status;                       // device status word
+};
+
+struct Tile {
+    int g, b, lbase, wx0;
+};
+
+__device__ __forceinline__ Tile decode_tile(const TcArgs &A, int t) {
+    Tile r;
+    const int lt = t % A.tiles_l;
+    const int gb = t / A.tiles_l;
+    r.b = gb % A.P.B;
+    r.g = gb / A.P.B;
+    r.lbase = lt * kRows;
+    int w = r.lbase * A.P.stride - A.P.padding - A.margin;
+    r.wx0 = (w >= 0) ? (w / 8) * 8 : -(((-w) + 7) / 8) * 8;
+    return r;
+}
+
+__device__ __forceinline__ float lds_bf16(uint32_t addr) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return __uint_as_float((uint32_t)v << 16);
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Per-row tap state of one offset group.
+template <int K>
+struct Taps {
+    uint32_t addr[K];   // byte offset of the pair in a stage (box and position; row added later)
+    float f[K];
+    float m[K];
+    float pos[K];       // for taps outside the window (slow path)
+    uint32_t slow;      // bit k: tap k outside the staged window
+};
+
+// 32 col values of one row for the reduction elements kk0 .. kk0+31 of a k-block
+// whose first channel is c_lo; phase K0 = kk0 % K is a compile-time constant.
+template <int K, int K0, bool MASK, bool SLOW>
+__device__ __forceinline__ void produce_segment(uint32_t (&out)[16], const Taps<K> &tp,
+                                                uint32_t xrow_addr, const __nv_bfloat16 *xg,
+                                                int64_t xg_row_stride, int L_in) {
+    float v[kSeg];
+#pragma unroll
+    for (int jj = 0; jj < kSeg; ++jj) {
+        const int kidx = (K0 + jj) % K;
+        const int crel = (K0 + jj) / K;
+        float x0, x1;
+        if (SLOW && ((tp.slow >> kidx) & 1u)) {
+            const Tap e = tap_floor_exact(tp.pos[kidx]);
+            const __nv_bfloat16 *row = xg + crel * xg_row_stride;
+            x0 = (e.i0 >= 0 && e.i0 < L_in) ? ld_f32(row + e.i0) : 0.0f;
+            x1 = (e.i0 >= -1 && e.i0 < L_in - 1) ? ld_f32(row + e.i0 + 1) : 0.0f;
+            float r = __fmaf_rn(e.f, __fsub_rn(x1, x0), x0);
+            v[jj] = MASK ? __fmul_rn(r, tp.m[kidx]) : r;
+        } else {
+            const uint32_t a = xrow_addr + tp.addr[kidx] + crel * kRowBytes;
+            x0 = lds_bf16(a);
+            x1 = lds_bf16(a + 2);
+            float r = __fmaf_rn(tp.f[kidx], __fsub_rn(x1, x0), x0);
+            v[jj] = MASK ? __fmul_rn(r, tp.m[kidx]) : r;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        out[i] = pack2(v[2 * i], v[2 * i + 1]);
+}
+
+template <int K, bool MASK, bool SLOW, int K0 = 0>
+__device__ __forceinline__ void produce_dispatch(int k0, uint32_t (&out)[16], const Taps<K> &tp,
+                                                 uint32_t xrow_addr, const __nv_bfloat16 *xg,
+                                                 int64_t xg_row_stride, int L_in) {
+    if constexpr (K0 < K) {
+        if (k0 == K0)
+            produce_segment<K, K0, MASK, SLOW>(out, tp, xrow_addr, xg, xg_row_stride, L_in);
+        else
+            produce_dispatch<K, MASK, SLOW, K0 + 1>(k0, out, tp, xrow_addr, xg, xg_row_stride,
+                                                    L_in);
+    }
+}
+
+template <int K, bool MASK>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_bf16_kernel(const __grid_constant__ TcArgs A, const __grid_constant__ CUtensorMap wmap,
+                   const __grid_constant__ CUtensorMap xmap) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const Problem &P = A.P;
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+
+    // The 128-byte swizzle needs 1024-byte aligned stages: align the base by hand
+    // (the launch reserves 1 KB of slack for this).
+    const uint32_t sraw = smem_u32(smem_raw);
+    const uint32_t sbase = (sraw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - sraw);
+    const uint32_t w_st0 = sbase + A.off_w;
+    const uint32_t x_st0 = sbase + A.off_x;
+    const uint32_t bar0 = sbase + A.off_bar;
+    auto bar_full = [&](int s) { return bar0 + 8u * s; };
+    auto bar_empty = [&](int s) { return bar0 + 8u * (kStages + s); };
+    auto bar_afull = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+    const uint32_t bar_dfull = bar0 + 8u * (3 * kStages);
+    const uint32_t bar_dempty = bar0 + 8u * (3 * kStages + 1);
+    const uint32_t bar_drain = bar0 + 8u * (3 * kStages + 2);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + A.off_bar + 8 * (3 * kStages + 3));
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_empty(s), 1);
+            mbar_init(bar_afull(s), 8);
+        }
+        mbar_init(bar_dfull, 1);
+        mbar_init(bar_dempty, 4);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+        tc_fence_before();
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        tma_prefetch_desc(&wmap);
+        tma_prefetch_desc(&xmap);
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const BoundedWait wait{abort_flag, kWaitNs, A.status};
+
+    if (warp == kTmaWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
+                const Tile T = decode_tile(A, t);
+                const int xrow0 = T.b * P.C_in + T.g * P.cin_g;
+                for (int kb = 0; kb < A.num_kb; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!wait(bar_empty(s), ph ^ 1u))
+                        goto tma_done;
+                    mbar_arrive_expect_tx(bar_full(s), A.w_stage_bytes + A.x_stage_bytes);
+                    tma_load_2d(w_st0 + s * A.w_stage_bytes, &wmap, kb * kBK, T.g * P.cout_g,
+                                bar_full(s));
+                    const int c_lo = (kb * kBK) / K;
+                    const uint32_t xdst = x_st0 + s * A.x_stage_bytes;
+                    tma_load_2d(xdst, &xmap, T.wx0, xrow0 + c_lo, bar_full(s));
+                    if (A.nbox == 2)
+                        tma_load_2d(xdst + A.x_box_bytes, &xmap, T.wx0 + kBoxStep, xrow0 + c_lo,
+                                    bar_full(s));
+                }
+            }
+        tma_done:
+            // Let every load this thread issued land before the CTA can exit
+            // (bounded; on the normal path they have all been consumed already).
+            volatile int never = 0;
+            const BoundedWait drain{&never, kWaitNs, A.status};
+            for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
+                drain(bar_full(j % kStages), (j / kStages) & 1u);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, A.N);
+            uint32_t it = 0, tc = 0;
+            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
+                if (!wait(bar_dempty, (tc & 1u) ^ 1u))
+                    goto mma_done;
+                tc_fence_after();
+                for (int kb = 0; kb < A.num_kb; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!wait(bar_full(s), ph) || !wait(bar_afull(s), ph))
+                        goto mma_done;
+                    tc_fence_after();
+                    const uint32_t wst = w_st0 + s * A.w_stage_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        mma_bf16_ts(tmem + kColD, tmem + kColA + 32u * s + 8u * kk,
+                                    sw128_kmajor_desc(wst + 32u * kk), idesc,
+                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar_empty(s));
+                }
+                mma_commit(bar_dfull);
+            }
+        mma_done:
+            // Every MMA issued has completed once this commit arrives.
+            mma_commit(bar_drain);
+            volatile int never = 0;
+            const BoundedWait drain{&never, kWaitNs, A.status};
+            drain(bar_drain, 0);
+        }
+    } else if (warp >= kProdWarp0 && warp < kProdWarp0 + 8) {
+        // ------------------------------------------------------------ col producers
+        const int q = warp % 4;                // TMEM lane quarter
+        const int h = (warp - kProdWarp0) / 4; // which 32 of the 64 elements of a k-block
+        const int row = 32 * q + lane;
+        const float M = kFloorMagic;
+        uint32_t it = 0;
+        for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
+            const Tile T = decode_tile(A, t);
+            const int l = T.lbase + row;
+            const bool valid = l < P.L_out;
+            const float start = (float)(l * P.stride - P.padding);
+            const float spanf = (float)(P.dilation * (K - 1));
+            const uint32_t win_bits = kFloorMagicBits + (uint32_t)T.wx0;
+            const __nv_bfloat16 *xb =
+                static_cast<const __nv_bfloat16 *>(P.x) + (int64_t)T.b * P.C_in * P.L_in;
+            Taps<K> tp;
+            int og_cur = -1;
+            for (int kb = 0; kb < A.num_kb; ++kb, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1u;
+                const int kk0 = kb * kBK + kSeg * h;
+                const int c_first = kk0 / K;             // group-relative channel
+                const int k0 = kk0 - c_first * K;
+                const int c_lo = (kb * kBK) / K;
+                const int og = (T.g * P.cin_g + c_first) / P.cin_per_og;
+                if (og != og_cur) {
+                    og_cur = og;
+                    const int64_t obase =
+                        (((int64_t)T.b * P.offset_groups + og) * P.L_out + (valid ? l : 0)) * K;
+                    const __nv_bfloat16 *op = static_cast<const __nv_bfloat16 *>(P.off) + obase;
+                    const __nv_bfloat16 *mp =
+                        MASK ? static_cast<const __nv_bfloat16 *>(P.mask) + obase : nullptr;
+                    tp.slow = 0;
+#pragma unroll
+                    for (int k = 0; k < K; ++k) {
+                        float pos = __fadd_rn(__fadd_rn(start, (float)(k * P.dilation)),
+                                              ld_f32(op + k));
+                        if (!P.unconstrained)
+                            pos = fminf(fmaxf(pos, start), __fadd_rn(start, spanf));
+                        const float tt = __fadd_rd(pos, M);
+                        const uint32_t rel = __float_as_uint(tt) - win_bits;   // i0 - wx0
+                        tp.f[k] = __fsub_rn(pos, __fsub_rn(tt, M));
+                        tp.pos[k] = pos;
+                        tp.m[k] = MASK ? ld_f32(mp + k) : 1.0f;
+                        if (rel < (uint32_t)(kBox - 1)) {
+                            tp.addr[k] = rel * 2u;
+                        } else if (A.nbox == 2 && rel < (uint32_t)kWinMax) {
+                            tp.addr[k] = A.x_box_bytes + (rel - kBoxStep) * 2u;
+                        } else {
+                            tp.addr[k] = 0;
+                            tp.slow |= 1u << k;
+                        }
+                        if (!valid) {   // rows past L_out: finite zeros, never stored
+                            tp.f[k] = 0.0f;
+                            tp.m[k] = 0.0f;
+                            tp.addr[k] = 0;
+                            tp.slow &= ~(1u << k);
+                        }
+                    }
+                }
+                if (!__all_sync(0xffffffffu, wait(bar_full(s), ph)))
+                    goto prod_done;
+                {
+                    const uint32_t xrow_addr =
+                        x_st0 + s * A.x_stage_bytes + (uint32_t)(c_first - c_lo) * kRowBytes;
+                    const __nv_bfloat16 *xg =
+                        xb + (int64_t)(T.g * P.cin_g + c_first) * P.L_in;
+                    uint32_t packed[16];
+                    if (__any_sync(0xffffffffu, tp.slow != 0))
+                        produce_dispatch<K, MASK, true>(k0, packed, tp, xrow_addr, xg, P.L_in,
+                                                        P.L_in);
+                    else
+                        produce_dispatch<K, MASK, false>(k0, packed, tp, xrow_addr, xg, P.L_in,
+                                                         P.L_in);
+                    tmem_st16(tmem + ((uint32_t)(32 * q) << 16) + kColA + 32u * s + 16u * h,
+                              packed);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar_afull(s));
+                }
+            }
+        }
+    prod_done:;
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp;
+        const int row = 32 * q + lane;
+        uint32_t tc = 0;
+        for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
+            const Tile T = decode_tile(A, t);
+            const int l = T.lbase + row;
+            const bool valid = l < P.L_out;
+            const __nv_bfloat16 *biasp =
+                P.bias ? static_cast<const __nv_bfloat16 *>(P.bias) + T.g * P.cout_g : nullptr;
+            if (!__all_sync(0xffffffffu, wait(bar_dfull, tc & 1u)))
+                goto epi_done;
+            tc_fence_after();
+            __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(P.out) +
+                                  ((int64_t)T.b * P.C_out + (int64_t)T.g * P.cout_g) * P.L_out + l;
+            for (int cc = 0; cc < A.N / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + kColD + 32u * cc, v);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int co = 32 * cc + i;
+                        const float bv = biasp ? ld_f32(biasp + co) : 0.0f;   // broadcast load
+                        outp[(int64_t)co * P.L_out] = __float2bfloat16_rn(__uint_as_float(v[i]) + bv);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_dempty);
+        }
+    epi_done:;
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+struct Plan {
+    TcArgs A;
+    size_t smem;
+};
+
+bool make_plan(const Problem &P, Plan *out) {
+    TcArgs A;
+    memset(&A, 0, sizeof(A));
+    A.P = P;
+    A.status = nullptr;
+    const int Kg = P.cin_g * P.K;
+    A.N = P.cout_g;
+    A.num_kb = Kg / kBK;
+    A.tiles_l = (P.L_out + kRows - 1) / kRows;
+    A.num_tiles = P.groups * P.B * A.tiles_l;
+    A.nch = (kBK - 1) / P.K + 2;
+    A.margin = P.unconstrained ? 32 : 0;
+    const int64_t need = (int64_t)(kRows - 1) * P.stride + (int64_t)P.dilation * (P.K - 1) + 2 +
+                         2 * A.margin + 7;
+    if (need > kWinMax)
+        return false;
+    A.nbox = need > kBox - 1 ? 2 : 1;
+    A.w_stage_bytes = (uint32_t)A.N * 128u;
+    A.x_box_bytes = (uint32_t)A.nch * kRowBytes;
+    A.x_stage_bytes = A.x_box_bytes * A.nbox;
+    A.off_w = 0;
+    A.off_x = A.off_w + kStages * A.w_stage_bytes;
+    A.off_bias = A.off_x + kStages * A.x_stage_bytes;
+    A.off_bar = A.off_bias;
+    size_t smem = A.off_bar + 8 * (3 * kStages + 3) + 16 + 1024;   // + alignment slack
+    if (smem > 227 * 1024)
+        return false;
+    // At least half the SM's shared memory, so two CTAs (each allocating all 512
+    // tensor-memory columns) never share an SM.
+    if (smem < 116 * 1024)
+        smem = 116 * 1024;
+    out->A = A;
+    out->smem = smem;
+    return true;
+}
+
+template <int K, bool MASK>
+cudaError_t launch_km(const Plan &pl, cudaStream_t stream) {
+    const Problem &P = pl.A.P;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return cudaErrorNotSupported;
+    alignas(64) CUtensorMap wmap, xmap;
+    const int Kg = P.cin_g * P.K;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)Kg, (cuuint64_t)P.C_out};
+        cuuint64_t strides[1] = {(cuuint64_t)Kg * 2};
+        cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)pl.A.N};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(P.w), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)P.L_in, (cuuint64_t)P.B * P.C_in};
+        cuuint64_t strides[1] = {(cuuint64_t)P.L_in * 2};
+        cuuint32_t box[2] = {(cuuint32_t)kBox, (cuuint32_t)pl.A.nch};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(P.x), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    auto kern = tc_bf16_kernel<K, MASK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)pl.smem);
+    if (e != cudaSuccess)
+        return e;
+    const int sms = sm_count();
+    if (sms <= 0)
+        return cudaErrorNoDevice;
+    const int grid = pl.A.num_tiles < sms ? pl.A.num_tiles : sms;
+    kern<<<grid, kThreads, pl.smem, stream>>>(pl.A, wmap, xmap);
+    return cudaGetLastError();
+}
+
+template <int K>
+cudaError_t launch_k(const Plan &pl, cudaStream_t stream) {
+    return pl.A.P.mask ? launch_km<K, true>(pl, stream) : launch_km<K, false>(pl, stream);
+}
+
+}  // namespace
+
+
+bool tc_bf16_supported(const Problem &P) {
+    if (P.dtype != DCN1D_BF16 || !fast_floor_ok(P))
+        return false;
+    if (!(P.K == 3 || P.K == 4 || P.K == 5 || P.K == 7 || P.K == 9))
+        return false;
+    if (P.cout_g % 32 != 0 || P.cout_g > 256)
+        return false;
+    if ((P.cin_g * P.K) % kBK != 0)
+        return false;
+    if (P.L_in % 8 != 0)   // TMA row stride must be a multiple of 16 bytes
+        return false;
+    // Offsets are uniform across each 32-element segment of the reduction.
+    const bool og_whole_group = (P.cin_per_og % P.cin_g) == 0;
+    if (!og_whole_group && (P.cin_per_og * P.K) % kSeg != 0)
+        return false;
+    if ((reinterpret_cast<uintptr_t>(P.x) & 15) || (reinterpret_cast<uintptr_t>(P.w) & 15))
+        return false;
+    Plan pl;
+    return make_plan(P, &pl);
+}
+
+cudaError_t launch_tc_bf16(const Problem &P, cudaStream_t stream) {
+    Plan pl;
+    if (!make_plan(P, &pl))
+        return cudaErrorInvalidValue;
+    pl.A.status = device_status_ptr();
+    if (!pl.A.status)
+        return cudaErrorInvalidDevice;
+    switch (P.K) {
+    case 3: return launch_k<3>(pl, stream);
+    case 4: return launch_k<4>(pl, stream);
+    case 5: return launch_k<5>(pl, stream);
+    case 7: return launch_k<7>(pl, stream);
+    case 9: return launch_k<9>(pl, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace dcn1d

@@ -137,6 +137,17 @@ const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor 
                                       int unconstrained, const dcn1d_tensor *out);
 
 /*
+ * Device-side status of the kernels enqueued so far on the current device.
+ * Kernels that wait on on-chip barriers bound every wait (about 2 s); a kernel
+ * that gives up records it in a device status word and exits, leaving its
+ * output incomplete.  This call synchronises `stream`, reads and clears that
+ * word, and returns DCN1D_ERR_TIMEOUT if any kernel gave up since the last
+ * call, DCN1D_ERR_CUDA if the synchronisation or the read failed, else
+ * DCN1D_OK.  It is the only entry point that synchronises.
+ */
+int dcn1d_device_status(void *stream);
+
+/*
  * Number of kernels the last accepted dcn1d_forward call on this host thread
  * enqueued (0 if none).  For counting launches in benchmarks.
  */

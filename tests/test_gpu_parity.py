@@ -21,8 +21,8 @@ REDUCED = [
     reduced(W.TINY_F32),
     reduced(W.USAGE_F32, B=2),
     reduced(W.DEPTHWISE_BF16, B=2, C_in=64, C_out=64, groups=64, offset_groups=64, L_in=3001),
-    reduced(W.MODULATED_BF16, B=2, L_in=333),
-    reduced(W.LARGE_BF16, B=2, L_in=700),
+    reduced(W.MODULATED_BF16, B=2, L_in=336),   # L_out 336 = 2 tiles of 128 + 80
+    reduced(W.LARGE_BF16, B=2, L_in=696),       # L_out 344 = 2 tiles of 128 + 88
 ]
 
 

@@ -1,0 +1,56 @@
+"""GPU parity of the fused tensor-core (tcgen05) bf16 path: shapes chosen so that the
+library selects it, asserted, then compared with the oracle; plus the device status word
+(no bounded wait may have given up)."""
+import pytest
+import torch
+
+import deformable_convolution_dcn1d_b200 as dcn
+import oracle
+import workloads as W
+from gpu_util import TOL, gpu_forward, kernel_name, norm_err, oracle_full, to_dev
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # name, B, C_in, C_out, K, L_in, s, p, d, groups, og, mask, unc, off_scale
+    ("g1_k5_mask_constrained", 2, 128, 128, 5, 256, 1, 2, 1, 1, 4, True, False, 3.0),
+    ("g2_k9_strided_unc", 2, 256, 128, 9, 264, 2, 4, 2, 2, 2, False, True, 2.0),
+    ("g4_k4_cout32", 1, 128, 128, 4, 512, 1, 1, 1, 4, 4, False, True, 4.0),
+    ("g1_k4_cout96_ragged", 3, 64, 96, 4, 200, 1, 3, 3, 1, 1, True, True, 2.0),
+    ("g1_k7_og_per_32", 1, 64, 64, 7, 136, 1, 3, 1, 1, 2, False, False, 2.5),
+    ("far_offsets_slow_taps", 2, 64, 64, 5, 256, 1, 2, 1, 1, 1, False, True, 80.0),
+    ("l_out_below_one_tile", 2, 128, 256, 5, 64, 1, 2, 1, 1, 4, True, False, 3.0),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_tc_bf16_parity(case):
+    name, B, Ci, Co, K, L, s, p, d, G, og, mask, unc, sc = case
+    L_out = oracle.out_length(L, K, s, p, d)
+    w, t = W.small_case(21, B=B, C_in=Ci, C_out=Co, K=K, stride=s, padding=p, dilation=d,
+                        groups=G, offset_groups=og, L_in=L, L_out=L_out, dtype="bf16",
+                        mask=mask, unconstrained=unc, off_scale=sc)
+    td = to_dev(t)
+    assert kernel_name(w, td) == "tcgen05_bf16", kernel_name(w, td)
+    y = gpu_forward(w, td)
+    assert dcn.dcn1d_device_status() == 0
+    r = oracle_full(w, t)
+    err = norm_err(y.double().cpu().numpy(), r)
+    assert err <= TOL["bf16"], (name, err)
+
+
+@pytest.mark.parametrize("w", [W.MODULATED_BF16, W.LARGE_BF16], ids=lambda w: w.name)
+def test_named_dense_workloads_take_the_tensor_core_path(w):
+    t = W.make_inputs(w.with_batch(1), seed=0)
+    td = to_dev(t)
+    assert kernel_name(w.with_batch(1), td) == "tcgen05_bf16"
+
+
+def test_device_status_clean_after_many_launches():
+    w, t = W.small_case(5, B=2, C_in=128, C_out=128, K=5, stride=1, padding=2, dilation=1,
+                        groups=1, offset_groups=4, L_in=512, L_out=512, dtype="bf16")
+    td = to_dev(t)
+    ys = [gpu_forward(w, td) for _ in range(20)]
+    assert dcn.dcn1d_device_status() == 0
+    for y in ys[1:]:
+        assert torch.equal(ys[0].view(torch.int16), y.view(torch.int16))
