@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kThreads) depthwise_kernel(DwArgs A) {
     const unsigned kWinBits = kFloorMagicBits + (unsigned)wlo;
     __syncthreads();
 
-    // Both neighbours of a tap whose floor is t (see tap_floor_fast).
+    // Both neighbours of a tap whose floor is t (see tap_floor_fast); checked.
     auto gather = [&](float t, float pos, float &x0, float &x1) {
         const unsigned r = __float_as_uint(t) - kWinBits;
         if (r < (unsigned)(wn - 1)) {
@@ -196,50 +196,112 @@ __global__ void __launch_bounds__(kThreads) depthwise_kernel(DwArgs A) {
             x1 = (e.i0 >= -1 && e.i0 < P.L_in - 1) ? ld_f32(xrow + e.i0 + 1) : 0.0f;
         }
     };
+    // Unchecked: the caller knows the pair is inside the window.
+    auto gather_fast = [&](float t) -> Word {
+        return xp[__float_as_uint(t) - kWinBits];
+    };
+    // Largest |offset| that keeps every tap of an output inside the window (margin),
+    // as a bf16/fp32 bit threshold on |offset| bits.
+    const float off_limit = (float)(A.margin - 1);
 
     // ---- 2. groups of 8 consecutive outputs, arithmetic on output pairs
     const int ngroups = vec ? (l1 - l0) / kGroup : 0;
     for (int gi = threadIdx.x; gi < ngroups; gi += kThreads) {
         const int lg = l0 + gi * kGroup;
-        float of[kGroup * K], mk[MASK ? kGroup * K : 1];
+        constexpr int NW = kGroup * K * (int)sizeof(T) / 4;   // 32-bit words of offsets per group
+        uint32_t ow[NW], mw[MASK ? NW : 1];
         const uint4 *ov = reinterpret_cast<const uint4 *>(offp + (int64_t)lg * K);
 #pragma unroll
-        for (int j = 0; j < kGroup * K / VN; ++j)
-            unpack16(__ldg(ov + j), of + j * VN, static_cast<const T *>(nullptr));
+        for (int j = 0; j < NW / 4; ++j) {
+            const uint4 v = __ldg(ov + j);
+            ow[4 * j] = v.x; ow[4 * j + 1] = v.y; ow[4 * j + 2] = v.z; ow[4 * j + 3] = v.w;
+        }
         if constexpr (MASK) {
             const uint4 *mv = reinterpret_cast<const uint4 *>(maskp + (int64_t)lg * K);
 #pragma unroll
-            for (int j = 0; j < kGroup * K / VN; ++j)
-                unpack16(__ldg(mv + j), mk + j * VN, static_cast<const T *>(nullptr));
+            for (int j = 0; j < NW / 4; ++j) {
+                const uint4 v = __ldg(mv + j);
+                mw[4 * j] = v.x; mw[4 * j + 1] = v.y; mw[4 * j + 2] = v.z; mw[4 * j + 3] = v.w;
+            }
+        }
+        // element e (= i*K + k) of the group's offsets / mask as a float
+        auto elem = [&](const uint32_t *w, int e) -> float {
+            if constexpr (sizeof(T) == 2)
+                return (e & 1) ? __uint_as_float(w[e >> 1] & 0xFFFF0000u)
+                               : __uint_as_float(w[e >> 1] << 16);
+            else
+                return __uint_as_float(w[e]);
+        };
+        // In unconstrained mode the window covers every tap with |offset| <= margin-1;
+        // constrained taps are clamped into the receptive field, always inside.
+        bool inside = true;
+        if constexpr (UNC) {
+            if constexpr (sizeof(T) == 2) {
+                uint32_t amax = 0;
+#pragma unroll
+                for (int j = 0; j < NW; ++j)
+                    amax = __vmaxu2(amax, ow[j] & 0x7FFF7FFFu);
+                const uint32_t lim = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rz(off_limit));
+                inside = ((amax & 0xFFFFu) <= lim) && ((amax >> 16) <= lim);
+            } else {
+                float amax = 0.0f;
+#pragma unroll
+                for (int j = 0; j < NW; ++j)
+                    amax = fmaxf(amax, fabsf(__uint_as_float(ow[j])));
+                inside = amax <= off_limit;   // false for NaN
+            }
         }
         const float s0 = (float)(lg * P.stride - P.padding);
         float res[kGroup];
+        if (__all_sync(0xffffffffu, inside)) {
 #pragma unroll
-        for (int i = 0; i < kGroup; i += 2) {
-            // receptive-field starts of outputs i and i+1
-            const float2 st = make_float2(__fadd_rn(s0, (float)i * sf), __fadd_rn(s0, (float)(i + 1) * sf));
-            float2 acc = make_float2(bias, bias);
+            for (int i = 0; i < kGroup; i += 2) {
+                const float2 st = make_float2(__fadd_rn(s0, (float)i * sf),
+                                              __fadd_rn(s0, (float)(i + 1) * sf));
+                float2 acc = make_float2(bias, bias);
 #pragma unroll
-            for (int k = 0; k < K; ++k) {
-                float2 pos = __fadd2_rn(__fadd2_rn(st, make_float2(kd[k], kd[k])),
-                                        make_float2(of[i * K + k], of[(i + 1) * K + k]));
-                if (!UNC) {
-                    pos.x = fminf(fmaxf(pos.x, st.x), __fadd_rn(st.x, spanf));
-                    pos.y = fminf(fmaxf(pos.y, st.y), __fadd_rn(st.y, spanf));
+                for (int k = 0; k < K; ++k) {
+                    float2 pos = __fadd2_rn(__fadd2_rn(st, make_float2(kd[k], kd[k])),
+                                            make_float2(elem(ow, i * K + k), elem(ow, (i + 1) * K + k)));
+                    if (!UNC) {
+                        pos.x = fminf(fmaxf(pos.x, st.x), __fadd_rn(st.x, spanf));
+                        pos.y = fminf(fmaxf(pos.y, st.y), __fadd_rn(st.y, spanf));
+                    }
+                    const float2 t = __fadd2_rd(pos, make_float2(kFloorMagic, kFloorMagic));
+                    const float2 f = __ffma2_rn(__fadd2_rn(t, make_float2(-kFloorMagic, -kFloorMagic)),
+                                                make_float2(-1.0f, -1.0f), pos);
+                    const float2 pa = pair_floats(gather_fast(t.x));
+                    const float2 pb = pair_floats(gather_fast(t.y));
+                    const float2 x0 = make_float2(pa.x, pb.x), x1 = make_float2(pa.y, pb.y);
+                    float2 v = __ffma2_rn(f, __ffma2_rn(x0, make_float2(-1.0f, -1.0f), x1), x0);
+                    if constexpr (MASK)
+                        v = __fmul2_rn(v, make_float2(elem(mw, i * K + k), elem(mw, (i + 1) * K + k)));
+                    acc = __ffma2_rn(make_float2(wk[k], wk[k]), v, acc);
                 }
-                const float2 t = __fadd2_rd(pos, make_float2(kFloorMagic, kFloorMagic));
-                const float2 fl = __fadd2_rn(t, make_float2(-kFloorMagic, -kFloorMagic));
-                const float2 f = __fadd2_rn(pos, make_float2(-fl.x, -fl.y));
-                float2 x0, x1;
-                gather(t.x, pos.x, x0.x, x1.x);
-                gather(t.y, pos.y, x0.y, x1.y);
-                float2 v = __ffma2_rn(f, __fadd2_rn(x1, make_float2(-x0.x, -x0.y)), x0);
-                if constexpr (MASK)
-                    v = __fmul2_rn(v, make_float2(mk[i * K + k], mk[(i + 1) * K + k]));
-                acc = __ffma2_rn(make_float2(wk[k], wk[k]), v, acc);
+                res[i] = acc.x;
+                res[i + 1] = acc.y;
             }
-            res[i] = acc.x;
-            res[i + 1] = acc.y;
+        } else {
+#pragma unroll
+            for (int i = 0; i < kGroup; ++i) {
+                const float st = __fadd_rn(s0, (float)i * sf);
+                float acc = bias;
+#pragma unroll
+                for (int k = 0; k < K; ++k) {
+                    float pos = __fadd_rn(__fadd_rn(st, kd[k]), elem(ow, i * K + k));
+                    if (!UNC)
+                        pos = fminf(fmaxf(pos, st), __fadd_rn(st, spanf));
+                    const float t = __fadd_rd(pos, kFloorMagic);
+                    const float f = __fsub_rn(pos, __fsub_rn(t, kFloorMagic));
+                    float x0, x1;
+                    gather(t, pos, x0, x1);
+                    float v = __fmaf_rn(f, __fsub_rn(x1, x0), x0);
+                    if constexpr (MASK)
+                        v = __fmul_rn(v, elem(mw, i * K + k));
+                    acc = __fmaf_rn(wk[k], v, acc);
+                }
+                res[i] = acc;
+            }
         }
         store8(orow_out + lg, res);
     }

@@ -85,10 +85,17 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs &A, int t) {
     return r;
 }
 
-__device__ __forceinline__ float lds_bf16(uint32_t addr) {
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
     unsigned short v;
     asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-    return __uint_as_float((uint32_t)v << 16);
+    return (uint32_t)v;
+}
+
+__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t u) {
+    return *reinterpret_cast<__nv_bfloat162 *>(&u);
+}
+__device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 h) {
+    return *reinterpret_cast<uint32_t *>(&h);
 }
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -96,46 +103,65 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Per-row tap state of one offset group.
+// Per-row tap state of one offset group.  Elements come in pairs (kk, kk+1),
+// i.e. taps (k, (k+1) % K), so fractions and mask values are kept pre-packed
+// as bf16x2 pairs indexed by the first tap of the pair.
 template <int K>
 struct Taps {
-    uint32_t addr[K];   // byte offset of the pair in a stage (box and position; row added later)
-    float f[K];
-    float m[K];
-    float pos[K];       // for taps outside the window (slow path)
-    uint32_t slow;      // bit k: tap k outside the staged window
+    uint32_t addr[K];    // byte offset of the tap's neighbour pair in a stage row
+    uint32_t fpair[K];   // bf16x2 (f_k, f_{(k+1)%K})
+    uint32_t mpair[K];   // bf16x2 (m_k, m_{(k+1)%K})
+    float pos[K];        // position, for taps outside the window (slow path)
+    uint32_t slow;       // bit k: tap k outside the staged window
 };
 
-// 32 col values of one row for the reduction elements kk0 .. kk0+31 of a k-block
-// whose first channel is c_lo; phase K0 = kk0 % K is a compile-time constant.
+// The col value of one element by the slow path: exact floor, global loads.
+template <int K, bool MASK>
+__device__ __forceinline__ float slow_element(const Taps<K> &tp, int kidx, int hi,
+                                              const __nv_bfloat16 *row, int L_in) {
+    const Tap e = tap_floor_exact(tp.pos[kidx]);
+    const float x0 = (e.i0 >= 0 && e.i0 < L_in) ? ld_f32(row + e.i0) : 0.0f;
+    const float x1 = (e.i0 >= -1 && e.i0 < L_in - 1) ? ld_f32(row + e.i0 + 1) : 0.0f;
+    const float r = __fmaf_rn(e.f, __fsub_rn(x1, x0), x0);
+    if (!MASK)
+        return r;
+    const uint32_t mp = tp.mpair[(kidx + K - hi) % K];
+    return __fmul_rn(r, __uint_as_float(hi ? (mp & 0xFFFF0000u) : (mp << 16)));
+}
+
+// 32 col values of one row for the reduction elements kk0 .. kk0+31 of a k-block,
+// packed bf16x2 (element 2i in the low half of out[i]).  Phase K0 = kk0 % K is a
+// compile-time constant, so every tap index below is static.  The lerp
+// x0 + f (x1 - x0) runs in bf16x2 arithmetic on element pairs.
 template <int K, int K0, bool MASK, bool SLOW>
 __device__ __forceinline__ void produce_segment(uint32_t (&out)[16], const Taps<K> &tp,
                                                 uint32_t xrow_addr, const __nv_bfloat16 *xg,
                                                 int64_t xg_row_stride, int L_in) {
-    float v[kSeg];
+    uint32_t base[K];
 #pragma unroll
-    for (int jj = 0; jj < kSeg; ++jj) {
-        const int kidx = (K0 + jj) % K;
-        const int crel = (K0 + jj) / K;
-        float x0, x1;
-        if (SLOW && ((tp.slow >> kidx) & 1u)) {
-            const Tap e = tap_floor_exact(tp.pos[kidx]);
-            const __nv_bfloat16 *row = xg + crel * xg_row_stride;
-            x0 = (e.i0 >= 0 && e.i0 < L_in) ? ld_f32(row + e.i0) : 0.0f;
-            x1 = (e.i0 >= -1 && e.i0 < L_in - 1) ? ld_f32(row + e.i0 + 1) : 0.0f;
-            float r = __fmaf_rn(e.f, __fsub_rn(x1, x0), x0);
-            v[jj] = MASK ? __fmul_rn(r, tp.m[kidx]) : r;
-        } else {
-            const uint32_t a = xrow_addr + tp.addr[kidx] + crel * kRowBytes;
-            x0 = lds_bf16(a);
-            x1 = lds_bf16(a + 2);
-            float r = __fmaf_rn(tp.f[kidx], __fsub_rn(x1, x0), x0);
-            v[jj] = MASK ? __fmul_rn(r, tp.m[kidx]) : r;
+    for (int k = 0; k < K; ++k)
+        base[k] = xrow_addr + tp.addr[k];
+#pragma unroll
+    for (int i = 0; i < kSeg / 2; ++i) {
+        const int k0 = (K0 + 2 * i) % K, c0 = (K0 + 2 * i) / K;
+        const int k1 = (K0 + 2 * i + 1) % K, c1 = (K0 + 2 * i + 1) / K;
+        const uint32_t a0 = base[k0] + c0 * kRowBytes;
+        const uint32_t a1 = base[k1] + c1 * kRowBytes;
+        const uint32_t x0 = __byte_perm(lds_u16(a0), lds_u16(a1), 0x5410);
+        const uint32_t x1 = __byte_perm(lds_u16(a0 + 2), lds_u16(a1 + 2), 0x5410);
+        __nv_bfloat162 v = __hfma2(as_bf2(tp.fpair[k0]), __hsub2(as_bf2(x1), as_bf2(x0)), as_bf2(x0));
+        if (MASK)
+            v = __hmul2(v, as_bf2(tp.mpair[k0]));
+        out[i] = as_u32(v);
+        if (SLOW && (((tp.slow >> k0) | (tp.slow >> k1)) & 1u)) {
+            float lo = __low2float(v), hi = __high2float(v);
+            if ((tp.slow >> k0) & 1u)
+                lo = slow_element<K, MASK>(tp, k0, 0, xg + c0 * xg_row_stride, L_in);
+            if ((tp.slow >> k1) & 1u)
+                hi = slow_element<K, MASK>(tp, k1, 1, xg + c1 * xg_row_stride, L_in);
+            out[i] = pack2(lo, hi);
         }
     }
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-        out[i] = pack2(v[2 * i], v[2 * i + 1]);
 }
 
 template <int K, bool MASK, bool SLOW, int K0 = 0>
@@ -168,6 +194,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t w_st0 = sbase + A.off_w;
     const uint32_t x_st0 = sbase + A.off_x;
     const uint32_t bar0 = sbase + A.off_bar;
+    float *bias_s = reinterpret_cast<float *>(smem + A.off_bias);
+    for (int i = threadIdx.x; i < P.C_out; i += kThreads)
+        bias_s[i] = P.bias ? ld_f32(static_cast<const __nv_bfloat16 *>(P.bias) + i) : 0.0f;
     auto bar_full = [&](int s) { return bar0 + 8u * s; };
     auto bar_empty = [&](int s) { return bar0 + 8u * (kStages + s); };
     auto bar_afull = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
@@ -272,14 +301,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = (warp - kProdWarp0) / 4; // which 32 of the 64 elements of a k-block
         const int row = 32 * q + lane;
         const float M = kFloorMagic;
+        const float spanf = (float)(P.dilation * (K - 1));
+        // Offsets (and mask) of the next (tile, offset group) this thread needs, loaded
+        // one group ahead so the global-load latency hides behind the current group.
+        float raw_off[K], raw_m[K];
+        int pf_t = -1, pf_og = -1;
+        auto prefetch = [&](int t, int og) {
+            pf_t = t;
+            pf_og = og;
+            if (t >= A.num_tiles)
+                return;
+            const Tile T = decode_tile(A, t);
+            const int l = T.lbase + row;
+            const int64_t obase =
+                (((int64_t)T.b * P.offset_groups + og) * P.L_out + (l < P.L_out ? l : 0)) * K;
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                raw_off[k] = ld_f32(static_cast<const __nv_bfloat16 *>(P.off) + obase + k);
+                raw_m[k] = MASK ? ld_f32(static_cast<const __nv_bfloat16 *>(P.mask) + obase + k) : 1.0f;
+            }
+        };
+        auto first_og = [&](int t) {
+            return (decode_tile(A, t).g * P.cin_g) / P.cin_per_og;
+        };
+        if ((int)blockIdx.x < A.num_tiles)
+            prefetch(blockIdx.x, first_og(blockIdx.x));
         uint32_t it = 0;
         for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
             const Tile T = decode_tile(A, t);
             const int l = T.lbase + row;
             const bool valid = l < P.L_out;
             const float start = (float)(l * P.stride - P.padding);
-            const float spanf = (float)(P.dilation * (K - 1));
             const uint32_t win_bits = kFloorMagicBits + (uint32_t)T.wx0;
+            const int og_last = (T.g * P.cin_g + P.cin_g - 1) / P.cin_per_og;
             const __nv_bfloat16 *xb =
                 static_cast<const __nv_bfloat16 *>(P.x) + (int64_t)T.b * P.C_in * P.L_in;
             Taps<K> tp;
@@ -294,23 +348,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int og = (T.g * P.cin_g + c_first) / P.cin_per_og;
                 if (og != og_cur) {
                     og_cur = og;
-                    const int64_t obase =
-                        (((int64_t)T.b * P.offset_groups + og) * P.L_out + (valid ? l : 0)) * K;
-                    const __nv_bfloat16 *op = static_cast<const __nv_bfloat16 *>(P.off) + obase;
-                    const __nv_bfloat16 *mp =
-                        MASK ? static_cast<const __nv_bfloat16 *>(P.mask) + obase : nullptr;
+                    if (pf_t != t || pf_og != og)
+                        prefetch(t, og);   // not predicted: load now
+                    float f[K], m[K];
                     tp.slow = 0;
 #pragma unroll
                     for (int k = 0; k < K; ++k) {
-                        float pos = __fadd_rn(__fadd_rn(start, (float)(k * P.dilation)),
-                                              ld_f32(op + k));
+                        float pos = __fadd_rn(__fadd_rn(start, (float)(k * P.dilation)), raw_off[k]);
                         if (!P.unconstrained)
                             pos = fminf(fmaxf(pos, start), __fadd_rn(start, spanf));
                         const float tt = __fadd_rd(pos, M);
                         const uint32_t rel = __float_as_uint(tt) - win_bits;   // i0 - wx0
-                        tp.f[k] = __fsub_rn(pos, __fsub_rn(tt, M));
+                        f[k] = __fsub_rn(pos, __fsub_rn(tt, M));
+                        m[k] = raw_m[k];
                         tp.pos[k] = pos;
-                        tp.m[k] = MASK ? ld_f32(mp + k) : 1.0f;
                         if (rel < (uint32_t)(kBox - 1)) {
                             tp.addr[k] = rel * 2u;
                         } else if (A.nbox == 2 && rel < (uint32_t)kWinMax) {
@@ -320,12 +371,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tp.slow |= 1u << k;
                         }
                         if (!valid) {   // rows past L_out: finite zeros, never stored
-                            tp.f[k] = 0.0f;
-                            tp.m[k] = 0.0f;
+                            f[k] = 0.0f;
+                            m[k] = 0.0f;
                             tp.addr[k] = 0;
                             tp.slow &= ~(1u << k);
                         }
                     }
+#pragma unroll
+                    for (int k = 0; k < K; ++k) {
+                        tp.fpair[k] = pack2(f[k], f[(k + 1) % K]);
+                        tp.mpair[k] = pack2(m[k], m[(k + 1) % K]);
+                    }
+                    // next group: the following offset group of this tile, else the
+                    // first one of the next tile
+                    if (og < og_last)
+                        prefetch(t, og + 1);
+                    else if (t + (int)gridDim.x < A.num_tiles)
+                        prefetch(t + gridDim.x, first_og(t + gridDim.x));
                 }
                 if (!__all_sync(0xffffffffu, wait(bar_full(s), ph)))
                     goto prod_done;
@@ -361,8 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Tile T = decode_tile(A, t);
             const int l = T.lbase + row;
             const bool valid = l < P.L_out;
-            const __nv_bfloat16 *biasp =
-                P.bias ? static_cast<const __nv_bfloat16 *>(P.bias) + T.g * P.cout_g : nullptr;
+            const float *biasg = bias_s + T.g * P.cout_g;
             if (!__all_sync(0xffffffffu, wait(bar_dfull, tc & 1u)))
                 goto epi_done;
             tc_fence_after();
@@ -376,8 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int co = 32 * cc + i;
-                        const float bv = biasp ? ld_f32(biasp + co) : 0.0f;   // broadcast load
-                        outp[(int64_t)co * P.L_out] = __float2bfloat16_rn(__uint_as_float(v[i]) + bv);
+                        outp[(int64_t)co * P.L_out] =
+                            __float2bfloat16_rn(__uint_as_float(v[i]) + biasg[co]);
                     }
                 }
             }
@@ -458,7 +519,7 @@ bool make_plan(const Problem &P, Plan *out) {
     A.off_w = 0;
     A.off_x = A.off_w + kStages * A.w_stage_bytes;
     A.off_bias = A.off_x + kStages * A.x_stage_bytes;
-    A.off_bar = A.off_bias;
+    A.off_bar = A.off_bias + (uint32_t)((P.C_out * 4 + 15) / 16 * 16);
     size_t smem = A.off_bar + 8 * (3 * kStages + 3) + 16 + 1024;   // + alignment slack
     if (smem > 227 * 1024)
         return false;
@@ -536,6 +597,8 @@ bool tc_bf16_supported(const Problem &P) {
     if (!og_whole_group && (P.cin_per_og * P.K) % kSeg != 0)
         return false;
     if ((reinterpret_cast<uintptr_t>(P.x) & 15) || (reinterpret_cast<uintptr_t>(P.w) & 15))
+        return false;
+    if (P.C_out > 8192)   // the bias is staged in shared memory
         return false;
     Plan pl;
     return make_plan(P, &pl);
