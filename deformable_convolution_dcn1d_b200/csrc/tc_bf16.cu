@@ -14,18 +14,21 @@
 //    W[co 0..N-1][kk block] (128-byte swizzle, K-major: the MMA's B operand)
 //    and one or two TMA loads of the x window [channels of the block][up to
 //    503 positions] (zero-filled outside the signal) into a stage;
-//  * producer warps (8 = two per TMEM lane quarter): thread = output row; it
-//    turns its row's taps into (window address, fraction, mask) once per
-//    offset group, then for each k-block computes 32 col values from the
-//    staged window and writes them, packed bf16x2, straight into TENSOR
-//    MEMORY with tcgen05.st (the MMA's A operand) -- no shared-memory round
-//    trip for the cols;
+//  * producer warps (16 = four per TMEM lane quarter): thread = output row;
+//    it turns its row's taps into (window address, fraction pair, mask pair)
+//    once per offset group, then for each k-block computes 16 col values from
+//    the staged window in bf16x2 arithmetic and writes them straight into
+//    TENSOR MEMORY with tcgen05.st (the MMA's A operand) -- no shared-memory
+//    round trip for the cols;
 //  * MMA warp: one thread issues 4 tcgen05.mma (M=128, N=Cg_out, K=16) per
 //    k-block, A from tensor memory, B from shared memory, D (fp32) in tensor
 //    memory, and commits completion to the stage's "empty" barrier;
-//  * epilogue warps (4): tcgen05.ld the accumulator, add the bias, round to
+//  * epilogue, by the same 16 warps (each drains a quarter of its lane
+//    quarter's columns): tcgen05.ld the accumulator, add the bias, round to
 //    bf16 and store; lanes are consecutive l, so each store is 64 contiguous
-//    bytes of out[b, co, :].
+//    bytes of out[b, co, :].  A tile's epilogue runs after the producers have
+//    staged the first kStages k-blocks of their next tile, so the MMA resumes
+//    on ready stages as soon as the accumulator is free.
 // Stages are chained by mbarriers; every wait is bounded (sm100.cuh).
 #include <string.h>
 
@@ -40,16 +43,15 @@ namespace {
 constexpr int kStages = 4;
 constexpr int kRows = 128;         // output positions per tile = TMEM lanes
 constexpr int kBK = 64;            // reduction elements per k-block
-constexpr int kSeg = 32;           // reduction elements per producer warp and k-block
+constexpr int kSeg = 16;           // reduction elements per producer warp and k-block
 constexpr int kBox = 256;          // x window box width (positions)
 constexpr int kBoxStep = 248;      // second box starts here (8 positions of overlap)
 constexpr int kWinMax = 503;       // window positions usable by a tap (pair inside one box)
 constexpr int kRowBytes = kBox * 2;
-constexpr int kThreads = 14 * 32;
-constexpr int kEpiWarp0 = 0;       // warps 0-3
-constexpr int kProdWarp0 = 4;      // warps 4-11
-constexpr int kTmaWarp = 12;
-constexpr int kMmaWarp = 13;
+constexpr int kProdWarps = 16;     // producer + epilogue warps 0-15: 4 per TMEM lane quarter
+constexpr int kTmaWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 18 * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColD = 0;      // D: columns [0, N)
 constexpr uint32_t kColA = 256;    // A stages: columns [256 + 32 s, +32)
@@ -129,12 +131,12 @@ __device__ __forceinline__ float slow_element(const Taps<K> &tp, int kidx, int h
     return __fmul_rn(r, __uint_as_float(hi ? (mp & 0xFFFF0000u) : (mp << 16)));
 }
 
-// 32 col values of one row for the reduction elements kk0 .. kk0+31 of a k-block,
+// kSeg col values of one row for the reduction elements kk0 .. kk0+kSeg-1 of a k-block,
 // packed bf16x2 (element 2i in the low half of out[i]).  Phase K0 = kk0 % K is a
 // compile-time constant, so every tap index below is static.  The lerp
 // x0 + f (x1 - x0) runs in bf16x2 arithmetic on element pairs.
 template <int K, int K0, bool MASK, bool SLOW>
-__device__ __forceinline__ void produce_segment(uint32_t (&out)[16], const Taps<K> &tp,
+__device__ __forceinline__ void produce_segment(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
                                                 uint32_t xrow_addr, const __nv_bfloat16 *xg,
                                                 int64_t xg_row_stride, int L_in) {
     uint32_t base[K];
@@ -165,7 +167,7 @@ __device__ __forceinline__ void produce_segment(uint32_t (&out)[16], const Taps<
 }
 
 template <int K, bool MASK, bool SLOW, int K0 = 0>
-__device__ __forceinline__ void produce_dispatch(int k0, uint32_t (&out)[16], const Taps<K> &tp,
+__device__ __forceinline__ void produce_dispatch(int k0, uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
                                                  uint32_t xrow_addr, const __nv_bfloat16 *xg,
                                                  int64_t xg_row_stride, int L_in) {
     if constexpr (K0 < K) {
@@ -178,7 +180,7 @@ __device__ __forceinline__ void produce_dispatch(int k0, uint32_t (&out)[16], co
 }
 
 template <int K, bool MASK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(112)
     tc_bf16_kernel(const __grid_constant__ TcArgs A, const __grid_constant__ CUtensorMap wmap,
                    const __grid_constant__ CUtensorMap xmap) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -210,10 +212,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar_full(s), 1);
             mbar_init(bar_empty(s), 1);
-            mbar_init(bar_afull(s), 8);
+            mbar_init(bar_afull(s), kProdWarps);
         }
         mbar_init(bar_dfull, 1);
-        mbar_init(bar_dempty, 4);
+        mbar_init(bar_dempty, kProdWarps);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -295,11 +297,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             const BoundedWait drain{&never, kWaitNs, A.status};
             drain(bar_drain, 0);
         }
-    } else if (warp >= kProdWarp0 && warp < kProdWarp0 + 8) {
-        // ------------------------------------------------------------ col producers
+    } else if (warp < kProdWarps) {
+        // ------------------------------------------------------------ col producers + epilogue
         const int q = warp % 4;                // TMEM lane quarter
-        const int h = (warp - kProdWarp0) / 4; // which 32 of the 64 elements of a k-block
+        const int h = warp / 4;                // which 16 of the 64 elements of a k-block
         const int row = 32 * q + lane;
+        // Epilogue of tile t (tile count tcnt): this warp's share of the accumulator columns.
+        auto epilogue = [&](int t, uint32_t tcnt) -> bool {
+            const Tile T = decode_tile(A, t);
+            const int l = T.lbase + row;
+            const bool valid = l < P.L_out;
+            const float *biasg = bias_s + T.g * P.cout_g;
+            if (!__all_sync(0xffffffffu, wait(bar_dfull, tcnt & 1u)))
+                return false;
+            tc_fence_after();
+            __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(P.out) +
+                                  ((int64_t)T.b * P.C_out + (int64_t)T.g * P.cout_g) * P.L_out + l;
+            for (int cc = h; cc < A.N / 32; cc += 4) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + kColD + 32u * cc, v);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int co = 32 * cc + i;
+                        outp[(int64_t)co * P.L_out] =
+                            __float2bfloat16_rn(__uint_as_float(v[i]) + biasg[co]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_dempty);
+            return true;
+        };
+        int pend_t = -1;        // tile whose epilogue is still to do
+        uint32_t pend_cnt = 0, tcount = 0;
         const float M = kFloorMagic;
         const float spanf = (float)(P.dilation * (K - 1));
         // Offsets (and mask) of the next (tile, offset group) this thread needs, loaded
@@ -396,58 +430,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                         x_st0 + s * A.x_stage_bytes + (uint32_t)(c_first - c_lo) * kRowBytes;
                     const __nv_bfloat16 *xg =
                         xb + (int64_t)(T.g * P.cin_g + c_first) * P.L_in;
-                    uint32_t packed[16];
+                    uint32_t packed[kSeg / 2];
                     if (__any_sync(0xffffffffu, tp.slow != 0))
                         produce_dispatch<K, MASK, true>(k0, packed, tp, xrow_addr, xg, P.L_in,
                                                         P.L_in);
                     else
                         produce_dispatch<K, MASK, false>(k0, packed, tp, xrow_addr, xg, P.L_in,
                                                          P.L_in);
-                    tmem_st16(tmem + ((uint32_t)(32 * q) << 16) + kColA + 32u * s + 16u * h,
-                              packed);
+                    tmem_st8(tmem + ((uint32_t)(32 * q) << 16) + kColA + 32u * s + 8u * h,
+                             packed);
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
                         mbar_arrive(bar_afull(s));
                 }
-            }
-        }
-    prod_done:;
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ epilogue
-        const int q = warp;
-        const int row = 32 * q + lane;
-        uint32_t tc = 0;
-        for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
-            const Tile T = decode_tile(A, t);
-            const int l = T.lbase + row;
-            const bool valid = l < P.L_out;
-            const float *biasg = bias_s + T.g * P.cout_g;
-            if (!__all_sync(0xffffffffu, wait(bar_dfull, tc & 1u)))
-                goto epi_done;
-            tc_fence_after();
-            __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(P.out) +
-                                  ((int64_t)T.b * P.C_out + (int64_t)T.g * P.cout_g) * P.L_out + l;
-            for (int cc = 0; cc < A.N / 32; ++cc) {
-                uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + kColD + 32u * cc, v);
-                tmem_wait_ld();
-                if (valid) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int co = 32 * cc + i;
-                        outp[(int64_t)co * P.L_out] =
-                            __float2bfloat16_rn(__uint_as_float(v[i]) + biasg[co]);
-                    }
+                if (pend_t >= 0 && kb == (A.num_kb < kStages ? A.num_kb : kStages) - 1) {
+                    if (!epilogue(pend_t, pend_cnt))
+                        goto prod_done;
+                    pend_t = -1;
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(bar_dempty);
+            pend_t = t;
+            pend_cnt = tcount++;
         }
-    epi_done:;
+        if (pend_t >= 0)
+            epilogue(pend_t, pend_cnt);
+    prod_done:;
     }
 
     // ---------------------------------------------------------------- teardown
