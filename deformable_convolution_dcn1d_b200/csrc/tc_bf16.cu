@@ -180,7 +180,9 @@ __device__ __forceinline__ void produce_dispatch(int k0, uint32_t (&out)[kSeg / 
 }
 
 template <int K, bool MASK>
-__global__ void __maxnreg__(112)
+// 18 warps: 5 land on some SM sub-partitions, each of which holds 16K registers,
+// so a thread may use at most 16384 / (5 * 32) -> 96 registers.
+__global__ void __maxnreg__(96)
     tc_bf16_kernel(const __grid_constant__ TcArgs A, const __grid_constant__ CUtensorMap wmap,
                    const __grid_constant__ CUtensorMap xmap) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -313,14 +315,14 @@ __global__ void __maxnreg__(112)
             tc_fence_after();
             __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(P.out) +
                                   ((int64_t)T.b * P.C_out + (int64_t)T.g * P.cout_g) * P.L_out + l;
-            for (int cc = h; cc < A.N / 32; cc += 4) {
-                uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + kColD + 32u * cc, v);
+            for (int cc = h; cc < A.N / 16; cc += 4) {
+                uint32_t v[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + kColD + 16u * cc, v);
                 tmem_wait_ld();
                 if (valid) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int co = 32 * cc + i;
+                    for (int i = 0; i < 16; ++i) {
+                        const int co = 16 * cc + i;
                         outp[(int64_t)co * P.L_out] =
                             __float2bfloat16_rn(__uint_as_float(v[i]) + biasg[co]);
                     }
