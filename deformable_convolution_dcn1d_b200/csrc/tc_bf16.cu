@@ -16,10 +16,11 @@
 //    503 positions] (zero-filled outside the signal) into a stage;
 //  * producer warps (16 = four per TMEM lane quarter): thread = output row;
 //    it turns its row's taps into (window address, fraction pair, mask pair)
-//    once per offset group, then for each k-block computes 16 col values from
-//    the staged window in bf16x2 arithmetic and writes them straight into
-//    TENSOR MEMORY with tcgen05.st (the MMA's A operand) -- no shared-memory
-//    round trip for the cols;
+//    once per offset group; the four warps of a quarter split the work as
+//    (k-block parity) x (half of the k-block), so two k-blocks are produced at
+//    once and each warp computes 32 col values per k-block from the staged
+//    window in bf16x2 arithmetic, written straight into TENSOR MEMORY with
+//    tcgen05.st (the MMA's A operand) -- no shared-memory round trip;
 //  * MMA warp: one thread issues 4 tcgen05.mma (M=128, N=Cg_out, K=16) per
 //    k-block, A from tensor memory, B from shared memory, D (fp32) in tensor
 //    memory, and commits completion to the stage's "empty" barrier;
@@ -43,7 +44,7 @@ namespace {
 constexpr int kStages = 4;
 constexpr int kRows = 128;         // output positions per tile = TMEM lanes
 constexpr int kBK = 64;            // reduction elements per k-block
-constexpr int kSeg = 16;           // reduction elements per producer warp and k-block
+constexpr int kSeg = 32;           // reduction elements per producer warp and k-block
 constexpr int kBox = 256;          // x window box width (positions)
 constexpr int kBoxStep = 248;      // second box starts here (8 positions of overlap)
 constexpr int kWinMax = 503;       // window positions usable by a tap (pair inside one box)
@@ -214,7 +215,7 @@ __global__ void __maxnreg__(96)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar_full(s), 1);
             mbar_init(bar_empty(s), 1);
-            mbar_init(bar_afull(s), kProdWarps);
+            mbar_init(bar_afull(s), kProdWarps / 2);
         }
         mbar_init(bar_dfull, 1);
         mbar_init(bar_dempty, kProdWarps);
@@ -302,7 +303,9 @@ __global__ void __maxnreg__(96)
     } else if (warp < kProdWarps) {
         // ------------------------------------------------------------ col producers + epilogue
         const int q = warp % 4;                // TMEM lane quarter
-        const int h = warp / 4;                // which 16 of the 64 elements of a k-block
+        const int h = warp / 4;                // epilogue share (0..3)
+        const int par = h >> 1;                // k-blocks of this parity
+        const int half = h & 1;                // which 32 of the 64 elements of a k-block
         const int row = 32 * q + lane;
         // Epilogue of tile t (tile count tcnt): this warp's share of the accumulator columns.
         auto epilogue = [&](int t, uint32_t tcnt) -> bool {
@@ -362,7 +365,6 @@ __global__ void __maxnreg__(96)
         };
         if ((int)blockIdx.x < A.num_tiles)
             prefetch(blockIdx.x, first_og(blockIdx.x));
-        uint32_t it = 0;
         for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
             const Tile T = decode_tile(A, t);
             const int l = T.lbase + row;
@@ -373,15 +375,24 @@ __global__ void __maxnreg__(96)
             const __nv_bfloat16 *xb =
                 static_cast<const __nv_bfloat16 *>(P.x) + (int64_t)T.b * P.C_in * P.L_in;
             Taps<K> tp;
+            // Offset group of the first channel of this warp's first segment; it only
+            // grows with the channel, so it is tracked against the next boundary.
             int og_cur = -1;
-            for (int kb = 0; kb < A.num_kb; ++kb, ++it) {
+            int og = (T.g * P.cin_g) / P.cin_per_og;
+            int og_next_c = (og + 1) * P.cin_per_og - T.g * P.cin_g;   // group-relative
+            const int kb_first = par, kb_first_stage = (A.num_kb < kStages ? A.num_kb : kStages);
+            for (int kb = kb_first; kb < A.num_kb; kb += 2) {
+                const uint32_t it = tcount * (uint32_t)A.num_kb + (uint32_t)kb;
                 const int s = it % kStages;
                 const uint32_t ph = (it / kStages) & 1u;
-                const int kk0 = kb * kBK + kSeg * h;
+                const int kk0 = kb * kBK + kSeg * half;
                 const int c_first = kk0 / K;             // group-relative channel
                 const int k0 = kk0 - c_first * K;
                 const int c_lo = (kb * kBK) / K;
-                const int og = (T.g * P.cin_g + c_first) / P.cin_per_og;
+                while (c_first >= og_next_c) {
+                    ++og;
+                    og_next_c += P.cin_per_og;
+                }
                 if (og != og_cur) {
                     og_cur = og;
                     if (pf_t != t || pf_og != og)
@@ -439,19 +450,24 @@ __global__ void __maxnreg__(96)
                     else
                         produce_dispatch<K, MASK, false>(k0, packed, tp, xrow_addr, xg, P.L_in,
                                                          P.L_in);
-                    tmem_st8(tmem + ((uint32_t)(32 * q) << 16) + kColA + 32u * s + 8u * h,
-                             packed);
+                    tmem_st16(tmem + ((uint32_t)(32 * q) << 16) + kColA + 32u * s + 16u * half,
+                              packed);
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
                         mbar_arrive(bar_afull(s));
                 }
-                if (pend_t >= 0 && kb == (A.num_kb < kStages ? A.num_kb : kStages) - 1) {
+                if (pend_t >= 0 && kb + 2 >= kb_first_stage) {
                     if (!epilogue(pend_t, pend_cnt))
                         goto prod_done;
                     pend_t = -1;
                 }
+            }
+            if (pend_t >= 0) {   // this warp had no k-block late enough in the tile
+                if (!epilogue(pend_t, pend_cnt))
+                    goto prod_done;
+                pend_t = -1;
             }
             pend_t = t;
             pend_cnt = tcount++;
