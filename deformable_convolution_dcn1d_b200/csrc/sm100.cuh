@@ -57,10 +57,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps (without issuing) until
+// the phase completes or about `hint_ns` pass.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // A wait on an mbarrier phase that gives up after `limit_ns` of wall time or as
 // soon as another role of the CTA has given up (shared abort flag).  On giving
 // up it records kStatusTimeout in the device status word and raises the abort
-// flag, so every role leaves its loop and the CTA can drain and exit.
+// flag, so every role leaves its loop and the CTA can drain and exit.  While
+// waiting the thread is suspended in hardware, so waiting roles do not take
+// issue slots from working warps.
 struct BoundedWait {
     volatile int *abort;   // shared-memory flag of this CTA
     uint64_t limit_ns;
@@ -70,12 +87,12 @@ struct BoundedWait {
         if (mbar_try_wait(bar, parity))
             return true;
         const uint64_t t0 = globaltimer_ns();
-        for (uint32_t i = 0;; ++i) {
-            if (mbar_try_wait(bar, parity))
+        for (;;) {
+            if (mbar_try_wait_sleep(bar, parity, 20000u))
                 return true;
             if (*abort)
                 return false;
-            if ((i & 15) == 15 && globaltimer_ns() - t0 > limit_ns) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 atomicOr(status, kStatusTimeout);
                 *abort = 1;
                 return false;

@@ -345,12 +345,11 @@ __global__ void __maxnreg__(96)
         // one group ahead so the global-load latency hides behind the current group.
         float raw_off[K], raw_m[K];
         int pf_t = -1, pf_og = -1;
-        auto prefetch = [&](int t, int og) {
+        auto prefetch = [&](int t, const Tile &T, int og) {
             pf_t = t;
             pf_og = og;
             if (t >= A.num_tiles)
                 return;
-            const Tile T = decode_tile(A, t);
             const int l = T.lbase + row;
             const int64_t obase =
                 (((int64_t)T.b * P.offset_groups + og) * P.L_out + (l < P.L_out ? l : 0)) * K;
@@ -360,13 +359,13 @@ __global__ void __maxnreg__(96)
                 raw_m[k] = MASK ? ld_f32(static_cast<const __nv_bfloat16 *>(P.mask) + obase + k) : 1.0f;
             }
         };
-        auto first_og = [&](int t) {
-            return (decode_tile(A, t).g * P.cin_g) / P.cin_per_og;
-        };
-        if ((int)blockIdx.x < A.num_tiles)
-            prefetch(blockIdx.x, first_og(blockIdx.x));
+        if ((int)blockIdx.x < A.num_tiles) {
+            const Tile T0 = decode_tile(A, blockIdx.x);
+            prefetch(blockIdx.x, T0, (T0.g * P.cin_g) / P.cin_per_og);
+        }
         for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
             const Tile T = decode_tile(A, t);
+            const int t_next = t + (int)gridDim.x;
             const int l = T.lbase + row;
             const bool valid = l < P.L_out;
             const float start = (float)(l * P.stride - P.padding);
@@ -396,7 +395,7 @@ __global__ void __maxnreg__(96)
                 if (og != og_cur) {
                     og_cur = og;
                     if (pf_t != t || pf_og != og)
-                        prefetch(t, og);   // not predicted: load now
+                        prefetch(t, T, og);   // not predicted: load now
                     float f[K], m[K];
                     tp.slow = 0;
 #pragma unroll
@@ -432,9 +431,11 @@ __global__ void __maxnreg__(96)
                     // next group: the following offset group of this tile, else the
                     // first one of the next tile
                     if (og < og_last)
-                        prefetch(t, og + 1);
-                    else if (t + (int)gridDim.x < A.num_tiles)
-                        prefetch(t + gridDim.x, first_og(t + gridDim.x));
+                        prefetch(t, T, og + 1);
+                    else if (t_next < A.num_tiles) {
+                        const Tile Tn = decode_tile(A, t_next);   // once per tile
+                        prefetch(t_next, Tn, (Tn.g * P.cin_g) / P.cin_per_og);
+                    }
                 }
                 if (!__all_sync(0xffffffffu, wait(bar_full(s), ph)))
                     goto prod_done;
