@@ -88,10 +88,11 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs &A, int t) {
     return r;
 }
 
+// 16-bit shared load, zero-extended into a 32-bit register by the load itself.
 __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
-    unsigned short v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-    return (uint32_t)v;
+    uint32_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
 }
 
 __device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t u) {
@@ -167,17 +168,23 @@ __device__ __forceinline__ void produce_segment(uint32_t (&out)[kSeg / 2], const
     }
 }
 
-template <int K, bool MASK, bool SLOW, int K0 = 0>
+// Jump to the segment code of phase k0 (a switch, so one indirect branch).
+template <int K, bool MASK, bool SLOW>
 __device__ __forceinline__ void produce_dispatch(int k0, uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
                                                  uint32_t xrow_addr, const __nv_bfloat16 *xg,
                                                  int64_t xg_row_stride, int L_in) {
-    if constexpr (K0 < K) {
-        if (k0 == K0)
-            produce_segment<K, K0, MASK, SLOW>(out, tp, xrow_addr, xg, xg_row_stride, L_in);
-        else
-            produce_dispatch<K, MASK, SLOW, K0 + 1>(k0, out, tp, xrow_addr, xg, xg_row_stride,
-                                                    L_in);
+#define DCN1D_PHASE(P_)                                                                          \
+    case P_:                                                                                    \
+        if constexpr (P_ < K)                                                                   \
+            produce_segment<K, (P_ < K ? P_ : 0), MASK, SLOW>(out, tp, xrow_addr, xg,             \
+                                                              xg_row_stride, L_in);             \
+        break;
+    switch (k0) {
+        DCN1D_PHASE(0) DCN1D_PHASE(1) DCN1D_PHASE(2) DCN1D_PHASE(3) DCN1D_PHASE(4)
+        DCN1D_PHASE(5) DCN1D_PHASE(6) DCN1D_PHASE(7) DCN1D_PHASE(8)
+        default: break;
     }
+#undef DCN1D_PHASE
 }
 
 template <int K, bool MASK>
