@@ -54,6 +54,10 @@ SIGNATURES = [
      [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T]),
     ("dcn1d_last_launch_count", _INT, []),
     ("dcn1d_device_status", _INT, [_P]),
+    ("dcn1d_forward_workspace_size", _I64,
+     [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T]),
+    ("dcn1d_forward_ws", _INT,
+     [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _P, ctypes.c_size_t, _P]),
 ]
 
 
@@ -149,27 +153,58 @@ def _out_for(x, weight, offsets):
 
 
 def dcn1d_forward(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=1, groups=1,
-                  offset_groups=1, unconstrained=False, out=None, stream=None):
+                  offset_groups=1, unconstrained=False, out=None, stream=None, workspace=None):
     """Deformable conv1d forward through the C ABI; returns ``out`` [B, C_out, L_out].
 
     x [B, C_in, L_in]; offsets and mask [B, offset_groups, L_out, K] (mask may be None);
     weight [C_out, C_in/groups, K]; bias [C_out] or None.  All CUDA, contiguous, one dtype
-    (float32 or bfloat16).  ``out`` is allocated with torch when not given.  Runs on
-    ``stream`` (default: the current torch stream of x's device); does not synchronise.
+    (float32 or bfloat16).  ``out`` is allocated with torch when not given.  The scratch the
+    fastest path needs (``dcn1d_forward_workspace_size``) is allocated with torch unless a
+    uint8 CUDA tensor ``workspace`` is given; ``workspace=False`` asks for the path without
+    scratch.  Runs on ``stream`` (default: the current torch stream of x's device); does not
+    synchronise.
     """
     dev = _check_device((x, offsets, mask, weight, bias, out))
     if out is None:
         out = _out_for(x, weight, offsets)
     descs = [_desc(t) for t in (x, offsets, mask, weight, bias, out)]
     lib = load()
+    refs = [_ref(d) for d in descs]
     with torch.cuda.device(dev):
-        st = lib.dcn1d_forward(_ref(descs[0]), _ref(descs[1]), _ref(descs[2]), _ref(descs[3]),
-                               _ref(descs[4]), stride, padding, dilation, groups, offset_groups,
-                               int(bool(unconstrained)), _ref(descs[5]),
-                               _P(_stream_ptr(stream, dev)))
+        ws_ptr, ws_bytes = None, 0
+        if workspace is not False:
+            need = int(lib.dcn1d_forward_workspace_size(*refs[:5], stride, padding, dilation,
+                                                        groups, offset_groups,
+                                                        int(bool(unconstrained)), refs[5]))
+            if need < 0:
+                raise Dcn1dError(-need, "dcn1d_forward_workspace_size")
+            if need > 0:
+                if workspace is None:
+                    workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+                if workspace.numel() < need or workspace.dtype != torch.uint8:
+                    raise ValueError(f"workspace must be a uint8 tensor of >= {need} bytes")
+                ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+        st = lib.dcn1d_forward_ws(*refs[:5], stride, padding, dilation, groups, offset_groups,
+                                  int(bool(unconstrained)), refs[5], _P(ws_ptr), ws_bytes,
+                                  _P(_stream_ptr(stream, dev)))
     if st != 0:
         raise Dcn1dError(st, "dcn1d_forward")
     return out
+
+
+def dcn1d_forward_workspace_size(x, offsets, mask, weight, bias, stride=1, padding=0,
+                                 dilation=1, groups=1, offset_groups=1, unconstrained=False,
+                                 out=None) -> int:
+    """Bytes of scratch the fastest path needs for these arguments (0 if none)."""
+    if out is None:
+        out = _out_for(x, weight, offsets)
+    descs = [_desc(t) for t in (x, offsets, mask, weight, bias, out)]
+    need = int(load().dcn1d_forward_workspace_size(*(_ref(d) for d in descs[:5]), stride,
+                                                   padding, dilation, groups, offset_groups,
+                                                   int(bool(unconstrained)), _ref(descs[5])))
+    if need < 0:
+        raise Dcn1dError(-need, "dcn1d_forward_workspace_size")
+    return need
 
 
 def dcn1d_forward_kernel_name(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=1,

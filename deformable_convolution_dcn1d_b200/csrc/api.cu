@@ -1,5 +1,6 @@
 // The C ABI (include/dcn1d.h): argument validation, kernel selection and
 // launch on the caller's stream.  Allocates nothing and never synchronises.
+#include <stdint.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -42,23 +43,34 @@ bool shape_is(const dcn1d_tensor *t, int64_t a, int64_t b, int64_t c, int64_t d 
     return d < 0 || t->shape[3] == d;
 }
 
-enum Kernel { kDirect = 0, kDepthwise = 1, kTcBf16 = 2 };
+enum Kernel { kDirect = 0, kDepthwise = 1, kTcBf16 = 2, kTcTf32 = 3 };
 
-const char *kernel_names[] = {"direct", "depthwise", "tcgen05_bf16"};
+const char *kernel_names[] = {"direct", "depthwise", "tcgen05_bf16", "tcgen05_3xtf32"};
 
-Kernel select_kernel(const Problem &P) {
+// The fastest kernel for P, given `ws_bytes` of caller workspace (SIZE_MAX: any amount).
+Kernel select_kernel(const Problem &P, size_t ws_bytes) {
     if (depthwise_supported(P))
         return kDepthwise;
     if (tc_bf16_supported(P))
         return kTcBf16;
+    if (tc_tf32_supported(P) && ws_bytes >= tc_tf32_workspace(P))
+        return kTcTf32;
     return kDirect;
+}
+
+size_t workspace_bytes(const Problem &P) {
+    if (depthwise_supported(P) || tc_bf16_supported(P))
+        return 0;
+    if (tc_tf32_supported(P))
+        return tc_tf32_workspace(P);
+    return 0;
 }
 
 // Full validation; fills P and the chosen kernel on success.
 int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor *mask,
              const dcn1d_tensor *w, const dcn1d_tensor *bias, int64_t stride, int64_t padding,
              int64_t dilation, int64_t groups, int64_t offset_groups, int unconstrained,
-             const dcn1d_tensor *out, Problem *P, Kernel *kern) {
+             const dcn1d_tensor *out, Problem *P) {
     int st;
     if (!x || !off || !w || !out)
         return DCN1D_ERR_NULL;
@@ -128,7 +140,6 @@ int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor 
     P->w = w->data;
     P->bias = bias ? bias->data : nullptr;
     P->out = out->data;
-    *kern = select_kernel(*P);
     return DCN1D_OK;
 }
 
@@ -194,40 +205,65 @@ const char *dcn1d_status_string(int status) {
     }
 }
 
+int dcn1d_forward_ws(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                     const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                     const dcn1d_tensor *bias, int64_t stride, int64_t padding, int64_t dilation,
+                     int64_t groups, int64_t offset_groups, int unconstrained, dcn1d_tensor *out,
+                     void *workspace, size_t workspace_bytes, void *stream) {
+    g_last_launches = 0;
+    Problem P;
+    int st = validate(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
+                      offset_groups, unconstrained, out, &P);
+    if (st != DCN1D_OK)
+        return st;
+    if (workspace_bytes > 0 && !workspace)
+        return DCN1D_ERR_NULL;
+    if (P.B == 0)
+        return DCN1D_OK;   // empty batch: nothing to compute
+    const Kernel kern = select_kernel(P, workspace ? workspace_bytes : 0);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t err = cudaSuccess;
+    int launches = 1;
+    switch (kern) {
+    case kDirect:
+        err = launch_direct(P, s);
+        break;
+    case kDepthwise:
+        err = launch_depthwise(P, s);
+        break;
+    case kTcBf16:
+        err = launch_tc_bf16(P, s);
+        break;
+    case kTcTf32:
+        err = launch_tc_tf32(P, workspace, s);
+        launches = tc_tf32_launches(P);
+        break;
+    }
+    if (err != cudaSuccess)
+        return DCN1D_ERR_LAUNCH;
+    g_last_launches = launches;
+    return DCN1D_OK;
+}
+
 int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
                   const dcn1d_tensor *weight, const dcn1d_tensor *bias, int64_t stride,
                   int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
                   int unconstrained, dcn1d_tensor *out, void *stream) {
-    g_last_launches = 0;
+    return dcn1d_forward_ws(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
+                            offset_groups, unconstrained, out, nullptr, 0, stream);
+}
+
+int64_t dcn1d_forward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                                     const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                                     const dcn1d_tensor *bias, int64_t stride, int64_t padding,
+                                     int64_t dilation, int64_t groups, int64_t offset_groups,
+                                     int unconstrained, const dcn1d_tensor *out) {
     Problem P;
-    Kernel kern;
-    int st = validate(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
-                      offset_groups, unconstrained, out, &P, &kern);
+    const int st = validate(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
+                            offset_groups, unconstrained, out, &P);
     if (st != DCN1D_OK)
-        return st;
-    if (P.B == 0)
-        return DCN1D_OK;   // empty batch: nothing to compute
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t err = cudaSuccess;
-    switch (kern) {
-    case kDirect:
-        err = launch_direct(P, s);
-        g_last_launches = 1;
-        break;
-    case kDepthwise:
-        err = launch_depthwise(P, s);
-        g_last_launches = 1;
-        break;
-    case kTcBf16:
-        err = launch_tc_bf16(P, s);
-        g_last_launches = 1;
-        break;
-    }
-    if (err != cudaSuccess) {
-        g_last_launches = 0;
-        return DCN1D_ERR_LAUNCH;
-    }
-    return DCN1D_OK;
+        return -st;
+    return (int64_t)workspace_bytes(P);
 }
 
 const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
@@ -236,11 +272,10 @@ const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor 
                                       int64_t dilation, int64_t groups, int64_t offset_groups,
                                       int unconstrained, const dcn1d_tensor *out) {
     Problem P;
-    Kernel kern;
     if (validate(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
-                 offset_groups, unconstrained, out, &P, &kern) != DCN1D_OK)
+                 offset_groups, unconstrained, out, &P) != DCN1D_OK)
         return nullptr;
-    return kernel_names[kern];
+    return kernel_names[select_kernel(P, SIZE_MAX)];
 }
 
 int dcn1d_last_launch_count(void) { return g_last_launches; }

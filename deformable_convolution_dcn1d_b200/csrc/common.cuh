@@ -49,6 +49,10 @@ cudaError_t launch_depthwise(const Problem &P, cudaStream_t stream);
 // device address to hand to kernels (NULL on failure), and its read-and-reset.
 unsigned int *device_status_ptr();
 cudaError_t read_and_clear_device_status(unsigned int *word);
+bool tc_tf32_supported(const Problem &P);
+size_t tc_tf32_workspace(const Problem &P);
+int tc_tf32_launches(const Problem &P);
+cudaError_t launch_tc_tf32(const Problem &P, void *workspace, cudaStream_t stream);
 bool tc_bf16_supported(const Problem &P);
 cudaError_t launch_tc_bf16(const Problem &P, cudaStream_t stream);
 cudaError_t launch_sample_index(const void *off, int dtype, int B, int G, int L_out, int K,

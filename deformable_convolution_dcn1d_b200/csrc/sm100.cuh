@@ -237,4 +237,20 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
 
+// ---------------------------------------------------------------- host helpers (host_util.cu)
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (NULL if unavailable).
+EncodeTiledFn encode_fn();
+// Number of SMs of the current device (0 on failure).
+int sm_count();
+// A 2D tiled tensor map over a row-major [rows][cols] array (elements of `elem_bytes`).
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t cols,
+               uint64_t rows, uint32_t elem_bytes, uint32_t box_cols, uint32_t box_rows,
+               CUtensorMapSwizzle swizzle);
+
 }  // namespace dcn1d

@@ -497,35 +497,6 @@ __global__ void __maxnreg__(96)
 
 // ------------------------------------------------------------------ host side
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-int sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess)
-        return 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return 0;
-    return n;
-}
-
 struct Plan {
     TcArgs A;
     size_t smem;
@@ -570,31 +541,14 @@ bool make_plan(const Problem &P, Plan *out) {
 template <int K, bool MASK>
 cudaError_t launch_km(const Plan &pl, cudaStream_t stream) {
     const Problem &P = pl.A.P;
-    EncodeTiledFn enc = encode_fn();
-    if (!enc)
-        return cudaErrorNotSupported;
     alignas(64) CUtensorMap wmap, xmap;
     const int Kg = P.cin_g * P.K;
-    {
-        cuuint64_t dims[2] = {(cuuint64_t)Kg, (cuuint64_t)P.C_out};
-        cuuint64_t strides[1] = {(cuuint64_t)Kg * 2};
-        cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)pl.A.N};
-        cuuint32_t estr[2] = {1, 1};
-        if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(P.w), dims, strides,
-                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    {
-        cuuint64_t dims[2] = {(cuuint64_t)P.L_in, (cuuint64_t)P.B * P.C_in};
-        cuuint64_t strides[1] = {(cuuint64_t)P.L_in * 2};
-        cuuint32_t box[2] = {(cuuint32_t)kBox, (cuuint32_t)pl.A.nch};
-        cuuint32_t estr[2] = {1, 1};
-        if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(P.x), dims, strides,
-                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
+    if (!encode_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P.w, (uint64_t)Kg, (uint64_t)P.C_out,
+                   2, kBK, (uint32_t)pl.A.N, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!encode_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P.x, (uint64_t)P.L_in,
+                   (uint64_t)P.B * P.C_in, 2, kBox, (uint32_t)pl.A.nch, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
     auto kern = tc_bf16_kernel<K, MASK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)pl.smem);

@@ -1,0 +1,711 @@
+// Fused deformable-im2col + tcgen05 tensor-core contraction for fp32 inputs,
+// accurate to fp32 through three TF32 products ("3xTF32").
+//
+// Same GEMM as the bf16 kernel (see tc_bf16.cu): per conv group and block of N
+// output channels, D[n, co] = sum_kk cols[n, kk] * W[co, kk] over kk = (ci, k).
+// TF32 keeps 10 mantissa bits, so every fp32 operand v is split exactly into
+// hi = v with its low 13 mantissa bits cleared (a tf32 value) and lo = v - hi,
+// and the MMA accumulates hi*hi + hi*lo + lo*hi in fp32; the dropped lo*lo
+// term is about 2^-22 of the product.
+//
+//  * A one-pass kernel splits the weight into W_hi and W_lo in the workspace.
+//  * The main kernel has the bf16 kernel's roles: a TMA warp loads the W_hi and
+//    W_lo tiles (128-byte swizzle) and the fp32 x window of each 32-wide
+//    k-block; 16 producer warps interpolate 16 columns each in fp32 and write
+//    their hi and lo parts straight into tensor memory (A operand); one thread
+//    issues 3 tcgen05.mma kind::tf32 per 8-wide k step; the producers drain D.
+//  * Small-N, large-K problems are split along the reduction (split-K) across
+//    CTAs; each split writes fp32 partial sums to the workspace and a third
+//    kernel adds them in a fixed order, plus the bias -- deterministic.
+#include <string.h>
+
+#include "common.cuh"
+#include "sampler.cuh"
+#include "sm100.cuh"
+
+namespace dcn1d {
+
+namespace {
+
+constexpr int kStages = 3;
+constexpr int kRows = 128;         // output positions per tile = TMEM lanes
+constexpr int kBK = 32;            // reduction elements per k-block (one 128-byte fp32 row)
+constexpr int kSeg = 16;           // reduction elements per producer warp and k-block
+constexpr int kBox = 256;          // x window box width (positions)
+constexpr int kBoxStep = 248;      // second box starts here (8 positions of overlap)
+constexpr int kWinMax = 503;
+constexpr int kRowBytes = kBox * 4;
+constexpr int kProdWarps = 16;
+constexpr int kTmaWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 18 * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColD = 0;      // D: columns [0, N)
+constexpr uint32_t kColA = 256;    // A stage s: hi [256 + 64 s, +32), lo [256 + 64 s + 32, +32)
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint32_t kTf32Mask = 0xFFFFE000u;
+
+struct TfArgs {
+    Problem P;
+    int N;              // MMA N = output channels per block (multiple of 32, <= 256)
+    int n_cob;          // channel blocks per conv group
+    int num_kb;         // k-blocks of the whole reduction
+    int kb_per_split;   // k-blocks per split
+    int splits;
+    int tiles_l;        // l-tiles per batch row
+    int num_units;      // splits * groups * n_cob * B * tiles_l
+    int nch, nbox, margin;
+    uint32_t w_stage_bytes, x_stage_bytes, x_box_bytes;
+    uint32_t off_w, off_wlo, off_x, off_bias, off_bar;
+    unsigned int *status;
+    float *partial;     // [splits][B][C_out][L_out] when splits > 1
+};
+
+struct Unit {
+    int split, g, cob, b, lbase, wx0, kb0, kb1;
+};
+
+__device__ __forceinline__ Unit decode_unit(const TfArgs &A, int u) {
+    Unit r;
+    const int lt = u % A.tiles_l;
+    int t = u / A.tiles_l;
+    r.b = t % A.P.B;
+    t /= A.P.B;
+    r.cob = t % A.n_cob;
+    t /= A.n_cob;
+    r.g = t % A.P.groups;
+    r.split = t / A.P.groups;
+    r.lbase = lt * kRows;
+    int w = r.lbase * A.P.stride - A.P.padding - A.margin;
+    r.wx0 = (w >= 0) ? (w / 8) * 8 : -(((-w) + 7) / 8) * 8;
+    r.kb0 = r.split * A.kb_per_split;
+    r.kb1 = min(A.num_kb, r.kb0 + A.kb_per_split);
+    return r;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::tf32.
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
+    return (1u << 4)                       // D format: f32
+           | (2u << 7)                     // A format: tf32
+           | (2u << 10)                    // B format: tf32
+           | ((uint32_t)(N >> 3) << 17)
+           | ((uint32_t)(M >> 4) << 24);
+}
+
+template <int K>
+struct TapsF {
+    uint32_t addr[K];   // byte offset of the tap's neighbour pair in a stage row
+    float f[K];
+    float m[K];
+    uint32_t slow;      // bit k: tap k outside the staged window
+};
+
+// One col value by the slow path: the position is recomputed from the offset
+// in global memory, exact floor, neighbours from global memory.
+template <bool MASK>
+__device__ __forceinline__ float slow_value(const Problem &P, float start, int k, float off,
+                                            float m, const float *row) {
+    float pos = __fadd_rn(__fadd_rn(start, (float)(k * P.dilation)), off);
+    if (!P.unconstrained)
+        pos = fminf(fmaxf(pos, start), __fadd_rn(start, (float)(P.dilation * (P.K - 1))));
+    const Tap e = tap_floor_exact(pos);
+    const float x0 = (e.i0 >= 0 && e.i0 < P.L_in) ? row[e.i0] : 0.0f;
+    const float x1 = (e.i0 >= -1 && e.i0 < P.L_in - 1) ? row[e.i0 + 1] : 0.0f;
+    const float v = __fmaf_rn(e.f, __fsub_rn(x1, x0), x0);
+    return MASK ? __fmul_rn(v, m) : v;
+}
+
+// 8 col values (elements j0 .. j0+7 of a segment whose phase is K0), split in
+// tf32 hi and lo parts.
+template <int K, int K0, int J0, bool MASK, bool SLOW>
+__device__ __forceinline__ void produce8(uint32_t (&hi)[8], uint32_t (&lo)[8], const TapsF<K> &tp,
+                                         uint32_t xrow_addr, const Problem &P, float start,
+                                         const float *xg, const float *offrow,
+                                         const float *maskrow) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int kidx = (K0 + J0 + i) % K;
+        const int crel = (K0 + J0 + i) / K;
+        float v;
+        if (SLOW && ((tp.slow >> kidx) & 1u)) {
+            v = slow_value<MASK>(P, start, kidx, offrow[kidx], MASK ? maskrow[kidx] : 1.0f,
+                                 xg + (int64_t)crel * P.L_in);
+        } else {
+            const uint32_t a = xrow_addr + tp.addr[kidx] + crel * kRowBytes;
+            const float x0 = lds_f32(a), x1 = lds_f32(a + 4);
+            v = __fmaf_rn(tp.f[kidx], __fsub_rn(x1, x0), x0);
+            if (MASK)
+                v = __fmul_rn(v, tp.m[kidx]);
+        }
+        const uint32_t h = __float_as_uint(v) & kTf32Mask;
+        hi[i] = h;
+        lo[i] = __float_as_uint(__fsub_rn(v, __uint_as_float(h)));
+    }
+}
+
+template <int K, int K0, bool MASK, bool SLOW>
+__device__ __forceinline__ void produce_segment(uint32_t tmem_hi, uint32_t tmem_lo,
+                                                const TapsF<K> &tp, uint32_t xrow_addr,
+                                                const Problem &P, float start, const float *xg,
+                                                const float *offrow, const float *maskrow) {
+    uint32_t hi[8], lo[8];
+    produce8<K, K0, 0, MASK, SLOW>(hi, lo, tp, xrow_addr, P, start, xg, offrow, maskrow);
+    tmem_st8(tmem_hi, hi);
+    tmem_st8(tmem_lo, lo);
+    produce8<K, K0, 8, MASK, SLOW>(hi, lo, tp, xrow_addr, P, start, xg, offrow, maskrow);
+    tmem_st8(tmem_hi + 8, hi);
+    tmem_st8(tmem_lo + 8, lo);
+}
+
+template <int K, bool MASK, bool SLOW>
+__device__ __forceinline__ void produce_dispatch(int k0, uint32_t tmem_hi, uint32_t tmem_lo,
+                                                 const TapsF<K> &tp, uint32_t xrow_addr,
+                                                 const Problem &P, float start, const float *xg,
+                                                 const float *offrow, const float *maskrow) {
+#define DCN1D_PHASE(P_)                                                                        \
+    case P_:                                                                                  \
+        if constexpr (P_ < K)                                                                 \
+            produce_segment<K, (P_ < K ? P_ : 0), MASK, SLOW>(tmem_hi, tmem_lo, tp, xrow_addr, \
+                                                              P, start, xg, offrow, maskrow); \
+        break;
+    switch (k0) {
+        DCN1D_PHASE(0) DCN1D_PHASE(1) DCN1D_PHASE(2) DCN1D_PHASE(3) DCN1D_PHASE(4)
+        DCN1D_PHASE(5) DCN1D_PHASE(6) DCN1D_PHASE(7) DCN1D_PHASE(8) DCN1D_PHASE(9)
+        DCN1D_PHASE(10) DCN1D_PHASE(11) DCN1D_PHASE(12) DCN1D_PHASE(13) DCN1D_PHASE(14)
+        DCN1D_PHASE(15)
+        default: break;
+    }
+#undef DCN1D_PHASE
+}
+
+// 18 warps: at most 96 registers per thread (5 warps share a 16K-register sub-partition).
+template <int K, bool MASK>
+__global__ void __maxnreg__(96)
+    tc_tf32_kernel(const __grid_constant__ TfArgs A, const __grid_constant__ CUtensorMap whimap,
+                   const __grid_constant__ CUtensorMap wlomap,
+                   const __grid_constant__ CUtensorMap xmap) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const Problem &P = A.P;
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+
+    const uint32_t sraw = smem_u32(smem_raw);
+    const uint32_t sbase = (sraw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - sraw);
+    const uint32_t w_st0 = sbase + A.off_w;
+    const uint32_t wlo_st0 = sbase + A.off_wlo;
+    const uint32_t x_st0 = sbase + A.off_x;
+    const uint32_t bar0 = sbase + A.off_bar;
+    float *bias_s = reinterpret_cast<float *>(smem + A.off_bias);
+    for (int i = threadIdx.x; i < P.C_out; i += kThreads)
+        bias_s[i] = P.bias ? static_cast<const float *>(P.bias)[i] : 0.0f;
+    auto bar_full = [&](int s) { return bar0 + 8u * s; };
+    auto bar_empty = [&](int s) { return bar0 + 8u * (kStages + s); };
+    auto bar_afull = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+    const uint32_t bar_dfull = bar0 + 8u * (3 * kStages);
+    const uint32_t bar_dempty = bar0 + 8u * (3 * kStages + 1);
+    const uint32_t bar_drain = bar0 + 8u * (3 * kStages + 2);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + A.off_bar + 8 * (3 * kStages + 3));
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_empty(s), 1);
+            mbar_init(bar_afull(s), kProdWarps / 2);
+        }
+        mbar_init(bar_dfull, 1);
+        mbar_init(bar_dempty, kProdWarps);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+        tc_fence_before();
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        tma_prefetch_desc(&whimap);
+        tma_prefetch_desc(&wlomap);
+        tma_prefetch_desc(&xmap);
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const BoundedWait wait{abort_flag, kWaitNs, A.status};
+
+    if (warp == kTmaWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int u = blockIdx.x; u < A.num_units; u += gridDim.x) {
+                const Unit U = decode_unit(A, u);
+                const int xrow0 = U.b * P.C_in + U.g * P.cin_g;
+                const int corow = U.g * P.cout_g + U.cob * A.N;
+                for (int kb = U.kb0; kb < U.kb1; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!wait(bar_empty(s), ph ^ 1u))
+                        goto tma_done;
+                    mbar_arrive_expect_tx(bar_full(s), 2 * A.w_stage_bytes + A.x_stage_bytes);
+                    tma_load_2d(w_st0 + s * A.w_stage_bytes, &whimap, kb * kBK, corow, bar_full(s));
+                    tma_load_2d(wlo_st0 + s * A.w_stage_bytes, &wlomap, kb * kBK, corow, bar_full(s));
+                    const int c_lo = (kb * kBK) / K;
+                    const uint32_t xdst = x_st0 + s * A.x_stage_bytes;
+                    tma_load_2d(xdst, &xmap, U.wx0, xrow0 + c_lo, bar_full(s));
+                    if (A.nbox == 2)
+                        tma_load_2d(xdst + A.x_box_bytes, &xmap, U.wx0 + kBoxStep, xrow0 + c_lo,
+                                    bar_full(s));
+                }
+            }
+        tma_done:
+            volatile int never = 0;
+            const BoundedWait drain{&never, kWaitNs, A.status};
+            for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
+                drain(bar_full(j % kStages), (j / kStages) & 1u);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_tf32_f32(128, A.N);
+            uint32_t it = 0, tc = 0;
+            for (int u = blockIdx.x; u < A.num_units; u += gridDim.x, ++tc) {
+                const Unit U = decode_unit(A, u);
+                if (!wait(bar_dempty, (tc & 1u) ^ 1u))
+                    goto mma_done;
+                tc_fence_after();
+                for (int kb = U.kb0; kb < U.kb1; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!wait(bar_full(s), ph) || !wait(bar_afull(s), ph))
+                        goto mma_done;
+                    tc_fence_after();
+                    const uint32_t whi = w_st0 + s * A.w_stage_bytes;
+                    const uint32_t wlo = wlo_st0 + s * A.w_stage_bytes;
+                    const uint32_t ahi = tmem + kColA + 64u * s;
+                    const uint32_t alo = ahi + 32u;
+#pragma unroll
+                    for (int j = 0; j < kBK / 8; ++j) {
+                        const uint32_t acc = (kb > U.kb0 || j > 0) ? 1u : 0u;
+                        mma_tf32_ts(tmem + kColD, ahi + 8u * j, sw128_kmajor_desc(whi + 32u * j),
+                                    idesc, acc);
+                        mma_tf32_ts(tmem + kColD, ahi + 8u * j, sw128_kmajor_desc(wlo + 32u * j),
+                                    idesc, 1u);
+                        mma_tf32_ts(tmem + kColD, alo + 8u * j, sw128_kmajor_desc(whi + 32u * j),
+                                    idesc, 1u);
+                    }
+                    mma_commit(bar_empty(s));
+                }
+                mma_commit(bar_dfull);
+            }
+        mma_done:
+            mma_commit(bar_drain);
+            volatile int never = 0;
+            const BoundedWait drain{&never, kWaitNs, A.status};
+            drain(bar_drain, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ producers + epilogue
+        const int q = warp % 4;          // TMEM lane quarter
+        const int h = warp / 4;          // epilogue share (0..3)
+        const int par = h >> 1;          // k-blocks of this parity (relative to the unit start)
+        const int half = h & 1;          // which 16 of the 32 elements of a k-block
+        const int row = 32 * q + lane;
+        const float M = kFloorMagic;
+        const float spanf = (float)(P.dilation * (K - 1));
+
+        auto epilogue = [&](int u, uint32_t tcnt) -> bool {
+            const Unit U = decode_unit(A, u);
+            const int l = U.lbase + row;
+            const bool valid = l < P.L_out;
+            const int co0 = U.g * P.cout_g + U.cob * A.N;
+            if (!__all_sync(0xffffffffu, wait(bar_dfull, tcnt & 1u)))
+                return false;
+            tc_fence_after();
+            float *dst;
+            bool add_bias;
+            if (A.splits > 1) {
+                dst = A.partial + ((((int64_t)U.split * P.B + U.b) * P.C_out + co0) * P.L_out + l);
+                add_bias = false;
+            } else {
+                dst = static_cast<float *>(P.out) + (((int64_t)U.b * P.C_out + co0) * P.L_out + l);
+                add_bias = true;
+            }
+            for (int cc = h; cc < A.N / 16; cc += 4) {
+                uint32_t v[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + kColD + 16u * cc, v);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int co = 16 * cc + i;
+                        const float b = add_bias ? bias_s[co0 + co] : 0.0f;
+                        dst[(int64_t)co * P.L_out] = __fadd_rn(__uint_as_float(v[i]), b);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_dempty);
+            return true;
+        };
+
+        // Offsets (and mask) of the next (unit, offset group), loaded one group ahead.
+        float raw_off[K], raw_m[K];
+        int pf_u = -1, pf_og = -1;
+        auto prefetch = [&](int u, const Unit &U, int og) {
+            pf_u = u;
+            pf_og = og;
+            if (u >= A.num_units)
+                return;
+            const int l = U.lbase + row;
+            const int64_t obase =
+                (((int64_t)U.b * P.offset_groups + og) * P.L_out + (l < P.L_out ? l : 0)) * K;
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                raw_off[k] = static_cast<const float *>(P.off)[obase + k];
+                raw_m[k] = MASK ? static_cast<const float *>(P.mask)[obase + k] : 1.0f;
+            }
+        };
+        auto og_of = [&](const Unit &U, int kb) {
+            return (U.g * P.cin_g + (kb * kBK) / K) / P.cin_per_og;
+        };
+        if ((int)blockIdx.x < A.num_units) {
+            const Unit U0 = decode_unit(A, blockIdx.x);
+            prefetch(blockIdx.x, U0, og_of(U0, U0.kb0));
+        }
+        int pend_u = -1;
+        uint32_t pend_cnt = 0, ucount = 0, it_base = 0;
+        for (int u = blockIdx.x; u < A.num_units; u += gridDim.x) {
+            const Unit U = decode_unit(A, u);
+            const int u_next = u + (int)gridDim.x;
+            const int l = U.lbase + row;
+            const bool valid = l < P.L_out;
+            const float start = (float)(l * P.stride - P.padding);
+            const uint32_t win_bits = kFloorMagicBits + (uint32_t)U.wx0;
+            const int og_last = (U.g * P.cin_g + ((U.kb1 * kBK - 1) / K)) / P.cin_per_og;
+            const float *xb = static_cast<const float *>(P.x) + (int64_t)U.b * P.C_in * P.L_in;
+            TapsF<K> tp;
+            int og_cur = -1;
+            int og = og_of(U, U.kb0);
+            int og_next_c = (og + 1) * P.cin_per_og - U.g * P.cin_g;   // group-relative
+            const int nkb = U.kb1 - U.kb0;
+            const int kb_first_stage = (nkb < kStages ? nkb : kStages);
+            for (int r = par; r < nkb; r += 2) {
+                const int kb = U.kb0 + r;
+                const uint32_t it = it_base + (uint32_t)r;
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1u;
+                const int kk0 = kb * kBK + kSeg * half;
+                const int c_first = kk0 / K;
+                const int k0 = kk0 - c_first * K;
+                const int c_lo = (kb * kBK) / K;
+                while (c_first >= og_next_c) {
+                    ++og;
+                    og_next_c += P.cin_per_og;
+                }
+                if (og != og_cur) {
+                    og_cur = og;
+                    if (pf_u != u || pf_og != og)
+                        prefetch(u, U, og);
+                    tp.slow = 0;
+#pragma unroll
+                    for (int k = 0; k < K; ++k) {
+                        float pos = __fadd_rn(__fadd_rn(start, (float)(k * P.dilation)), raw_off[k]);
+                        if (!P.unconstrained)
+                            pos = fminf(fmaxf(pos, start), __fadd_rn(start, spanf));
+                        const float tt = __fadd_rd(pos, M);
+                        const uint32_t rel = __float_as_uint(tt) - win_bits;   // i0 - wx0
+                        tp.f[k] = __fsub_rn(pos, __fsub_rn(tt, M));
+                        tp.m[k] = raw_m[k];
+                        if (rel < (uint32_t)(kBox - 1)) {
+                            tp.addr[k] = rel * 4u;
+                        } else if (A.nbox == 2 && rel < (uint32_t)kWinMax) {
+                            tp.addr[k] = A.x_box_bytes + (rel - kBoxStep) * 4u;
+                        } else {
+                            tp.addr[k] = 0;
+                            tp.slow |= 1u << k;
+                        }
+                        if (!valid) {
+                            tp.f[k] = 0.0f;
+                            tp.m[k] = 0.0f;
+                            tp.addr[k] = 0;
+                            tp.slow &= ~(1u << k);
+                        }
+                    }
+                    if (og < og_last) {
+                        prefetch(u, U, og + 1);
+                    } else if (u_next < A.num_units) {
+                        const Unit Un = decode_unit(A, u_next);
+                        prefetch(u_next, Un, og_of(Un, Un.kb0));
+                    }
+                }
+                if (!__all_sync(0xffffffffu, wait(bar_full(s), ph)))
+                    goto prod_done;
+                {
+                    const uint32_t xrow_addr =
+                        x_st0 + s * A.x_stage_bytes + (uint32_t)(c_first - c_lo) * kRowBytes;
+                    const float *xg = xb + (int64_t)(U.g * P.cin_g + c_first) * P.L_in;
+                    const int64_t obase = (((int64_t)U.b * P.offset_groups + og) * P.L_out +
+                                           (valid ? l : 0)) * K;
+                    const float *offrow = static_cast<const float *>(P.off) + obase;
+                    const float *maskrow = MASK ? static_cast<const float *>(P.mask) + obase : nullptr;
+                    const uint32_t lanebase = tmem + ((uint32_t)(32 * q) << 16);
+                    const uint32_t thi = lanebase + kColA + 64u * s + 16u * half;
+                    if (__any_sync(0xffffffffu, tp.slow != 0))
+                        produce_dispatch<K, MASK, true>(k0, thi, thi + 32u, tp, xrow_addr, P, start,
+                                                        xg, offrow, maskrow);
+                    else
+                        produce_dispatch<K, MASK, false>(k0, thi, thi + 32u, tp, xrow_addr, P,
+                                                         start, xg, offrow, maskrow);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar_afull(s));
+                }
+                if (pend_u >= 0 && r + 2 >= kb_first_stage) {
+                    if (!epilogue(pend_u, pend_cnt))
+                        goto prod_done;
+                    pend_u = -1;
+                }
+            }
+            if (pend_u >= 0) {
+                if (!epilogue(pend_u, pend_cnt))
+                    goto prod_done;
+                pend_u = -1;
+            }
+            pend_u = u;
+            pend_cnt = ucount++;
+            it_base += (uint32_t)nkb;
+        }
+        if (pend_u >= 0)
+            epilogue(pend_u, pend_cnt);
+    prod_done:;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// W_hi = W with the low 13 mantissa bits cleared (exactly a tf32 value), W_lo = W - W_hi.
+__global__ void __launch_bounds__(256) split_tf32_kernel(const float *w, float *hi, float *lo,
+                                                         int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = w[i];
+        const float h = __uint_as_float(__float_as_uint(v) & kTf32Mask);
+        hi[i] = h;
+        lo[i] = __fsub_rn(v, h);
+    }
+}
+
+// out[b, co, l] = bias[co] + sum over splits of the partial sums, in split order.
+__global__ void __launch_bounds__(256) reduce_splits_kernel(const float *partial, const float *bias,
+                                                            float *out, int splits, int C_out,
+                                                            int L_out, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float acc = 0.0f;
+        for (int s = 0; s < splits; ++s)
+            acc = __fadd_rn(acc, partial[(int64_t)s * n + i]);
+        if (bias)
+            acc = __fadd_rn(acc, bias[(i / L_out) % C_out]);
+        out[i] = acc;
+    }
+}
+
+struct TfPlan {
+    TfArgs A;
+    size_t smem;
+    size_t ws_whi, ws_wlo, ws_partial, ws_total;   // workspace layout (bytes)
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Grid of a grid-stride elementwise kernel of 256-thread blocks over n elements.
+unsigned grid_for(int64_t n, int sms) {
+    const int64_t want = (n + 255) / 256, cap = 8LL * sms;
+    return (unsigned)(want < cap ? want : cap);
+}
+
+bool make_tf_plan(const Problem &P, TfPlan *out) {
+    TfArgs A;
+    memset(&A, 0, sizeof(A));
+    A.P = P;
+    const int Kg = P.cin_g * P.K;
+    A.N = P.cout_g < 256 ? P.cout_g : 256;
+    if (P.cout_g % A.N != 0)
+        return false;
+    A.n_cob = P.cout_g / A.N;
+    A.num_kb = Kg / kBK;
+    A.tiles_l = (P.L_out + kRows - 1) / kRows;
+    const int base_units = P.groups * A.n_cob * P.B * A.tiles_l;
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    int splits = sms / (base_units > 0 ? base_units : 1);
+    const int max_splits = A.num_kb / 8 > 0 ? A.num_kb / 8 : 1;   // at least 8 k-blocks a split
+    if (splits > max_splits)
+        splits = max_splits;
+    if (splits < 1)
+        splits = 1;
+    A.kb_per_split = (A.num_kb + splits - 1) / splits;
+    A.splits = (A.num_kb + A.kb_per_split - 1) / A.kb_per_split;
+    A.num_units = A.splits * base_units;
+    A.nch = (kBK - 1) / P.K + 2;
+    A.margin = P.unconstrained ? 32 : 0;
+    const int64_t need = (int64_t)(kRows - 1) * P.stride + (int64_t)P.dilation * (P.K - 1) + 2 +
+                         2 * A.margin + 7;
+    if (need > kWinMax)
+        return false;
+    A.nbox = need > kBox - 1 ? 2 : 1;
+    A.w_stage_bytes = (uint32_t)A.N * 128u;
+    A.x_box_bytes = (uint32_t)A.nch * kRowBytes;
+    A.x_stage_bytes = A.x_box_bytes * A.nbox;
+    A.off_w = 0;
+    A.off_wlo = A.off_w + kStages * A.w_stage_bytes;
+    A.off_x = A.off_wlo + kStages * A.w_stage_bytes;
+    A.off_bias = A.off_x + kStages * A.x_stage_bytes;
+    A.off_bar = A.off_bias + (uint32_t)((P.C_out * 4 + 15) / 16 * 16);
+    size_t smem = A.off_bar + 8 * (3 * kStages + 3) + 16 + 1024;
+    if (smem > 227 * 1024)
+        return false;
+    if (smem < 116 * 1024)
+        smem = 116 * 1024;
+    TfPlan pl;
+    pl.A = A;
+    pl.smem = smem;
+    const size_t wbytes = (size_t)P.C_out * Kg * 4;
+    pl.ws_whi = 0;
+    pl.ws_wlo = align256(wbytes);
+    pl.ws_partial = pl.ws_wlo + align256(wbytes);
+    pl.ws_total = pl.ws_partial +
+                  (A.splits > 1 ? align256((size_t)A.splits * P.B * P.C_out * P.L_out * 4) : 0);
+    *out = pl;
+    return true;
+}
+
+template <int K, bool MASK>
+cudaError_t launch_tf_km(const TfPlan &pl, void *ws, cudaStream_t stream) {
+    const Problem &P = pl.A.P;
+    TfArgs A = pl.A;
+    A.status = device_status_ptr();
+    if (!A.status)
+        return cudaErrorInvalidDevice;
+    unsigned char *wsb = static_cast<unsigned char *>(ws);
+    float *whi = reinterpret_cast<float *>(wsb + pl.ws_whi);
+    float *wlo = reinterpret_cast<float *>(wsb + pl.ws_wlo);
+    A.partial = A.splits > 1 ? reinterpret_cast<float *>(wsb + pl.ws_partial) : nullptr;
+    const int Kg = P.cin_g * P.K;
+    alignas(64) CUtensorMap mhi, mlo, mx;
+    if (!encode_2d(&mhi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, whi, (uint64_t)Kg, (uint64_t)P.C_out, 4,
+                   kBK, (uint32_t)A.N, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&mlo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, wlo, (uint64_t)Kg, (uint64_t)P.C_out, 4,
+                   kBK, (uint32_t)A.N, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, P.x, (uint64_t)P.L_in,
+                   (uint64_t)P.B * P.C_in, 4, kBox, (uint32_t)A.nch, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    const int sms = sm_count();
+    if (sms <= 0)
+        return cudaErrorNoDevice;
+    const int64_t nw = (int64_t)P.C_out * Kg;
+    split_tf32_kernel<<<(unsigned)grid_for(nw, sms), 256, 0, stream>>>(
+        static_cast<const float *>(P.w), whi, wlo, nw);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    auto kern = tc_tf32_kernel<K, MASK>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+    if (e != cudaSuccess)
+        return e;
+    const int grid = A.num_units < sms ? A.num_units : sms;
+    kern<<<grid, kThreads, pl.smem, stream>>>(A, mhi, mlo, mx);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || A.splits == 1)
+        return e;
+    const int64_t n = (int64_t)P.B * P.C_out * P.L_out;
+    reduce_splits_kernel<<<(unsigned)grid_for(n, sms), 256, 0, stream>>>(
+        A.partial, static_cast<const float *>(P.bias), static_cast<float *>(P.out), A.splits,
+        P.C_out, P.L_out, n);
+    return cudaGetLastError();
+}
+
+template <int K>
+cudaError_t launch_tf_k(const TfPlan &pl, void *ws, cudaStream_t stream) {
+    return pl.A.P.mask ? launch_tf_km<K, true>(pl, ws, stream)
+                       : launch_tf_km<K, false>(pl, ws, stream);
+}
+
+}  // namespace
+
+bool tc_tf32_supported(const Problem &P) {
+    if (P.dtype != DCN1D_F32 || !fast_floor_ok(P))
+        return false;
+    if (P.K < 1 || P.K > 16)
+        return false;
+    if (P.cout_g % 32 != 0)
+        return false;
+    if ((P.cin_g * P.K) % kBK != 0)
+        return false;
+    if (P.L_in % 4 != 0)   // TMA row stride must be a multiple of 16 bytes
+        return false;
+    const bool og_whole_group = (P.cin_per_og % P.cin_g) == 0;
+    if (!og_whole_group && (P.cin_per_og * P.K) % kSeg != 0)
+        return false;
+    if ((reinterpret_cast<uintptr_t>(P.x) & 15) || (reinterpret_cast<uintptr_t>(P.w) & 15))
+        return false;
+    if (P.C_out > 8192)
+        return false;
+    TfPlan pl;
+    return make_tf_plan(P, &pl);
+}
+
+size_t tc_tf32_workspace(const Problem &P) {
+    TfPlan pl;
+    return make_tf_plan(P, &pl) ? pl.ws_total : 0;
+}
+
+int tc_tf32_launches(const Problem &P) {
+    TfPlan pl;
+    return make_tf_plan(P, &pl) ? (pl.A.splits > 1 ? 3 : 2) : 0;
+}
+
+cudaError_t launch_tc_tf32(const Problem &P, void *workspace, cudaStream_t stream) {
+    TfPlan pl;
+    if (!make_tf_plan(P, &pl) || !workspace)
+        return cudaErrorInvalidValue;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255)
+        return cudaErrorInvalidValue;
+    switch (P.K) {
+#define DCN1D_K(K_) \
+    case K_: return launch_tf_k<K_>(pl, workspace, stream);
+        DCN1D_K(1) DCN1D_K(2) DCN1D_K(3) DCN1D_K(4) DCN1D_K(5) DCN1D_K(6) DCN1D_K(7) DCN1D_K(8)
+        DCN1D_K(9) DCN1D_K(10) DCN1D_K(11) DCN1D_K(12) DCN1D_K(13) DCN1D_K(14) DCN1D_K(15)
+        DCN1D_K(16)
+#undef DCN1D_K
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace dcn1d

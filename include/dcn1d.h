@@ -101,6 +101,9 @@ int64_t dcn1d_out_length(int64_t L_in, int64_t kernel_size, int64_t stride, int6
  * C_in; stride >= 1, padding >= 0, dilation >= 1 ("conv1d" page, "Arguments").
  * `unconstrained` != 0 lets taps sample anywhere (dc1d page, "Usage").
  *
+ * Needs no scratch memory: where the fastest path would (see
+ * dcn1d_forward_workspace_size), a path without scratch runs instead.
+ *
  * Returns DCN1D_OK, or DCN1D_ERR_NULL / _DTYPE / _SHAPE / _ARG / _UNSUPPORTED on
  * invalid arguments (nothing launched), DCN1D_ERR_LAUNCH if a launch failed.
  */
@@ -108,6 +111,36 @@ int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1
                   const dcn1d_tensor *weight, const dcn1d_tensor *bias, int64_t stride,
                   int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
                   int unconstrained, dcn1d_tensor *out, void *stream);
+
+/*
+ * Scratch memory (bytes) the fastest path for these arguments needs, or 0 when
+ * it needs none; a negative value is minus the status code of invalid
+ * arguments.  Host only.  The fp32 tensor-core path needs scratch: the weight
+ * split into tf32 high and low parts (2 * C_out * (C_in/groups) * K floats)
+ * and, when the reduction is split across CTAs, the fp32 partial sums
+ * (splits * B * C_out * L_out floats).
+ */
+int64_t dcn1d_forward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                                     const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                                     const dcn1d_tensor *bias, int64_t stride, int64_t padding,
+                                     int64_t dilation, int64_t groups, int64_t offset_groups,
+                                     int unconstrained, const dcn1d_tensor *out);
+
+/*
+ * dcn1d_forward with caller-provided scratch: `workspace` is a device buffer
+ * of `workspace_bytes` bytes, 256-byte aligned, owned by the caller and used
+ * only during the work enqueued on `stream` (calls that overlap on the GPU
+ * must use different workspaces).  With at least
+ * dcn1d_forward_workspace_size() bytes the fastest path runs; with less (or
+ * NULL and 0) the call behaves exactly like dcn1d_forward.  A non-zero size
+ * with a NULL pointer is DCN1D_ERR_NULL.  Other arguments and errors as for
+ * dcn1d_forward.
+ */
+int dcn1d_forward_ws(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
+                     const dcn1d_tensor *weight, const dcn1d_tensor *bias, int64_t stride,
+                     int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
+                     int unconstrained, dcn1d_tensor *out, void *workspace,
+                     size_t workspace_bytes, void *stream);
 
 /* A static, human-readable name of a status code ("DCN1D_OK", ...). Never NULL. */
 const char *dcn1d_status_string(int status);
@@ -126,9 +159,11 @@ int dcn1d_sample_index(const dcn1d_tensor *offsets, int64_t L_in, int64_t stride
                        float *frac, void *stream);
 
 /*
- * Which kernel dcn1d_forward would launch for these arguments, as a static
- * string ("direct", "depthwise", "tcgen05_bf16", ...), or NULL if the arguments
- * are invalid.  Host only; launches nothing.  For tests and benchmarks.
+ * Which kernel dcn1d_forward_ws launches for these arguments when given at
+ * least dcn1d_forward_workspace_size() bytes of scratch, as a static string
+ * ("direct", "depthwise", "tcgen05_bf16", "tcgen05_3xtf32"), or NULL if the
+ * arguments are invalid.  Host only; launches nothing.  For tests and
+ * benchmarks.
  */
 const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
                                       const dcn1d_tensor *mask, const dcn1d_tensor *weight,
@@ -148,8 +183,8 @@ const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor 
 int dcn1d_device_status(void *stream);
 
 /*
- * Number of kernels the last accepted dcn1d_forward call on this host thread
- * enqueued (0 if none).  For counting launches in benchmarks.
+ * Number of kernels the last accepted dcn1d_forward / dcn1d_forward_ws call on
+ * this host thread enqueued (0 if none).  For counting launches in benchmarks.
  */
 int dcn1d_last_launch_count(void);
 

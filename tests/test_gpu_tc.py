@@ -54,3 +54,56 @@ def test_device_status_clean_after_many_launches():
     assert dcn.dcn1d_device_status() == 0
     for y in ys[1:]:
         assert torch.equal(ys[0].view(torch.int16), y.view(torch.int16))
+
+
+# ---------------------------------------------------------------- fp32: 3xTF32 tensor-core path
+
+TF32_CASES = [
+    # name, B, C_in, C_out, K, L_in, s, p, d, groups, og, mask, unc, off_scale
+    ("usage_shape_b2_split", 2, 512, 512, 16, 128, 1, 0, 3, 1, 1, False, False, 1.5),
+    ("no_split_small_k", 2, 32, 64, 8, 200, 1, 4, 1, 1, 1, False, True, 2.0),
+    ("groups2_mask_og4", 2, 64, 128, 4, 160, 2, 2, 2, 2, 4, True, False, 3.0),
+    ("far_offsets_slow_taps", 1, 64, 64, 8, 256, 1, 3, 1, 1, 2, False, True, 90.0),
+    ("cout_512_two_blocks", 1, 64, 512, 4, 300, 1, 1, 1, 1, 1, True, True, 2.0),
+]
+
+
+@pytest.mark.parametrize("case", TF32_CASES, ids=[c[0] for c in TF32_CASES])
+def test_tc_tf32_parity(case):
+    name, B, Ci, Co, K, L, s, p, d, G, og, mask, unc, sc = case
+    L_out = oracle.out_length(L, K, s, p, d)
+    w, t = W.small_case(31, B=B, C_in=Ci, C_out=Co, K=K, stride=s, padding=p, dilation=d,
+                        groups=G, offset_groups=og, L_in=L, L_out=L_out, dtype="f32",
+                        mask=mask, unconstrained=unc, off_scale=sc)
+    td = to_dev(t)
+    assert kernel_name(w, td) == "tcgen05_3xtf32", kernel_name(w, td)
+    y = gpu_forward(w, td)
+    assert dcn.dcn1d_device_status() == 0
+    r = oracle_full(w, t)
+    err = norm_err(y.double().cpu().numpy(), r)
+    assert err <= TOL["f32"], (name, err)
+
+
+def test_tf32_without_workspace_takes_the_direct_path():
+    """dcn1d_forward without scratch runs a path that needs none, with the same result."""
+    w = W.USAGE_F32.with_batch(2)
+    td = to_dev(W.make_inputs(w, seed=2))
+    a = gpu_forward(w, td)
+    b = dcn.dcn1d_forward(td["x"], td["offsets"], td["mask"], td["weight"], td["bias"],
+                          w.stride, w.padding, w.dilation, w.groups, w.offset_groups,
+                          w.unconstrained, workspace=False)
+    torch.cuda.synchronize()
+    assert dcn.dcn1d_last_launch_count() == 1
+    err = (a.double() - b.double()).abs().max().item() / b.double().abs().max().item()
+    assert err <= 2e-5
+
+
+def test_tf32_deterministic_across_calls():
+    w = W.USAGE_F32.with_batch(3)
+    td = to_dev(W.make_inputs(w, seed=5))
+    a = gpu_forward(w, td)
+    launches = dcn.dcn1d_last_launch_count()
+    b = gpu_forward(w, td)
+    torch.cuda.synchronize()
+    assert launches >= 2
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
