@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     SIGNATURES,
     dcn1d_device_status,
     dcn1d_forward,
+    dcn1d_forward_noalloc,
     dcn1d_forward_workspace_size,
     dcn1d_forward_kernel_name,
     dcn1d_last_launch_count,

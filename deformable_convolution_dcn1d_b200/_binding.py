@@ -58,6 +58,8 @@ SIGNATURES = [
      [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T]),
     ("dcn1d_forward_ws", _INT,
      [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _P, ctypes.c_size_t, _P]),
+    ("dcn1d_forward_noalloc", _INT,
+     [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _P]),
 ]
 
 
@@ -189,6 +191,26 @@ def dcn1d_forward(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=
                                   _P(_stream_ptr(stream, dev)))
     if st != 0:
         raise Dcn1dError(st, "dcn1d_forward")
+    return out
+
+
+def dcn1d_forward_noalloc(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=1,
+                          groups=1, offset_groups=1, unconstrained=False, out=None, stream=None):
+    """The forward for callers that cannot allocate device memory: the library's own
+    48 MiB static scratch instead of a workspace.  ``out`` must be given (this call
+    allocates nothing).  Calls whose GPU work overlaps share the scratch and race."""
+    if out is None:
+        raise ValueError("dcn1d_forward_noalloc allocates nothing: pass out")
+    dev = _check_device((x, offsets, mask, weight, bias, out))
+    descs = [_desc(t) for t in (x, offsets, mask, weight, bias, out)]
+    lib = load()
+    with torch.cuda.device(dev):
+        st = lib.dcn1d_forward_noalloc(*(_ref(d) for d in descs[:5]), stride, padding,
+                                       dilation, groups, offset_groups,
+                                       int(bool(unconstrained)), _ref(descs[5]),
+                                       _P(_stream_ptr(stream, dev)))
+    if st != 0:
+        raise Dcn1dError(st, "dcn1d_forward_noalloc")
     return out
 
 

@@ -142,6 +142,41 @@ int dcn1d_forward_ws(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const d
                      int unconstrained, dcn1d_tensor *out, void *workspace,
                      size_t workspace_bytes, void *stream);
 
+/*
+ * dcn1d_forward for callers that cannot allocate device memory: code running
+ * where cudaMalloc is not allowed or not wanted (a real-time loop, a runtime
+ * that owns every allocation, a host that reserved all device memory up
+ * front).  The pages describe no counterpart of this entry point; it exists
+ * only for such callers.
+ *
+ * Same arguments, kernels and results as dcn1d_forward_ws given enough
+ * scratch, but the scratch is a fixed array of 48 MiB inside the library
+ * (static device memory: every GPU that loads the library may hold it until
+ * the process exits).  The caller still passes all inputs and `out`; this call
+ * itself allocates and frees nothing.
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * (with that device current) and caches it; make that first call before any
+ * stream capture.
+ *
+ * Scratch limit: arguments whose fastest path needs more than 48 MiB
+ * (dcn1d_forward_workspace_size) are rejected with DCN1D_ERR_UNSUPPORTED and
+ * nothing is launched.  Arguments that need no scratch run as dcn1d_forward.
+ *
+ * Sharing: every call on a device uses the same array and it keeps the last
+ * call's contents; each call writes every scratch byte it reads, so nothing
+ * needs clearing, but calls whose work overlaps on the GPU (different streams,
+ * or host threads) race on the array and must be serialised by the caller.
+ *
+ * Returns the codes of dcn1d_forward, DCN1D_ERR_UNSUPPORTED past the scratch
+ * limit, or DCN1D_ERR_CUDA if the address lookup failed.
+ */
+int dcn1d_forward_noalloc(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                          const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                          const dcn1d_tensor *bias, int64_t stride, int64_t padding,
+                          int64_t dilation, int64_t groups, int64_t offset_groups,
+                          int unconstrained, dcn1d_tensor *out, void *stream);
+
 /* A static, human-readable name of a status code ("DCN1D_OK", ...). Never NULL. */
 const char *dcn1d_status_string(int status);
 
