@@ -311,12 +311,18 @@ def run_ours(args, w: W.Workload, peaks: dict, want_cpu: bool):
     # ---- device-resident timing
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # The library records these around its main kernel (helper kernels stay outside).
+    k_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for e in k_starts + k_ends:
+        e.record(stream)   # creates the CUDA event (torch creates events lazily)
     barrier(ws)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)
+            dcn.dcn1d_set_timing_events(k_starts[i], k_ends[i])
             step(dev_in, out)
             ends[i].record(stream)
         torch.cuda.synchronize(dev)
@@ -324,6 +330,8 @@ def run_ours(args, w: W.Workload, peaks: dict, want_cpu: bool):
     ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     ms = max_over_ranks(ms, ws)
     ms_step = ms / args.steps
+    ms_kernel = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(k_starts, k_ends)),
+                               ws) / args.steps
     value, unit = unit_value(w, kernel, ms_step / 1e3, ws)
 
     # ---- end to end through the public API from pinned host buffers
@@ -359,10 +367,12 @@ def run_ours(args, w: W.Workload, peaks: dict, want_cpu: bool):
 
     # ---- roofline of the step's kernel (one kernel per step: its time is the step time)
     bound, r_unit, peak, per_launch, note = roofline_for(kernel, w, peaks)
-    achieved = per_launch / (ms_step / 1e3)
+    achieved = per_launch / (ms_kernel / 1e3)
     roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
             "frac": achieved / peak, "traffic": load_traffic(kernel, w), "kernel": kernel,
-            "peak_source": note, "launches_per_step": launches_per_step}
+            "peak_source": note, "launches_per_step": launches_per_step,
+            "kernel_ms": ms_kernel,
+            "timing": "CUDA events the library records around its main kernel, per step"}
 
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,

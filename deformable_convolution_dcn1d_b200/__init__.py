@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     dcn1d_last_launch_count,
     dcn1d_out_length,
     dcn1d_sample_index,
+    dcn1d_set_timing_events,
     dcn1d_status_string,
     lib_path,
     load,

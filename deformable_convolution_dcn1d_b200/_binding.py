@@ -58,6 +58,7 @@ SIGNATURES = [
      [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T]),
     ("dcn1d_forward_ws", _INT,
      [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _P, ctypes.c_size_t, _P]),
+    ("dcn1d_set_timing_events", None, [_P, _P]),
     ("dcn1d_forward_noalloc", _INT,
      [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _P]),
 ]
@@ -138,6 +139,12 @@ def dcn1d_status_string(status: int) -> str:
 
 def dcn1d_last_launch_count() -> int:
     return int(load().dcn1d_last_launch_count())
+
+
+def dcn1d_set_timing_events(begin, end) -> None:
+    """The next forward on this thread records these torch.cuda.Events around its main kernel."""
+    load().dcn1d_set_timing_events(_P(begin.cuda_event if begin is not None else None),
+                                   _P(end.cuda_event if end is not None else None))
 
 
 def dcn1d_device_status(stream=None, device=None) -> int:

@@ -9,6 +9,7 @@ namespace dcn1d {
 namespace {
 
 thread_local int g_last_launches = 0;
+thread_local cudaEvent_t g_time_begin = nullptr, g_time_end = nullptr;
 
 constexpr int64_t kMaxElems = (int64_t)1 << 31;   // every tensor indexed with int32 rows
 constexpr int64_t kMaxPos = (int64_t)1 << 24;     // positions exact in float32
@@ -145,6 +146,17 @@ int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor 
 
 }  // namespace
 
+void timing_begin(cudaStream_t stream) {
+    if (g_time_begin)
+        cudaEventRecord(g_time_begin, stream);
+}
+
+void timing_end(cudaStream_t stream) {
+    if (g_time_end)
+        cudaEventRecord(g_time_end, stream);
+    g_time_begin = g_time_end = nullptr;   // one forward only
+}
+
 // One status word per device (a __device__ variable exists once per device).
 __device__ unsigned int g_device_status = 0;
 
@@ -226,10 +238,14 @@ int dcn1d_forward_ws(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
     int launches = 1;
     switch (kern) {
     case kDirect:
+        timing_begin(s);
         err = launch_direct(P, s);
+        timing_end(s);
         break;
     case kDepthwise:
+        timing_begin(s);
         err = launch_depthwise(P, s);
+        timing_end(s);
         break;
     case kTcBf16:
         err = launch_tc_bf16(P, s);
@@ -279,6 +295,11 @@ const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor 
 }
 
 int dcn1d_last_launch_count(void) { return g_last_launches; }
+
+void dcn1d_set_timing_events(void *begin, void *end) {
+    g_time_begin = static_cast<cudaEvent_t>(begin);
+    g_time_end = static_cast<cudaEvent_t>(end);
+}
 
 int dcn1d_device_status(void *stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)

@@ -41,6 +41,12 @@ inline bool fast_floor_ok(const Problem &P) {
     return (int64_t)P.L_in + 2 * (int64_t)P.padding < (1 << 21);
 }
 
+// Benchmark timing hook (dcn1d_set_timing_events): launchers call these right
+// before and right after the launch of their main kernel; they record the
+// events set for this host thread, if any, on `stream`.
+void timing_begin(cudaStream_t stream);
+void timing_end(cudaStream_t stream);
+
 // Kernel launchers (each returns cudaGetLastError() of its launch).
 cudaError_t launch_direct(const Problem &P, cudaStream_t stream);
 bool depthwise_supported(const Problem &P);

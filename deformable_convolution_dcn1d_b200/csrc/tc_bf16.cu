@@ -558,7 +558,9 @@ cudaError_t launch_km(const Plan &pl, cudaStream_t stream) {
     if (sms <= 0)
         return cudaErrorNoDevice;
     const int grid = pl.A.num_tiles < sms ? pl.A.num_tiles : sms;
+    timing_begin(stream);
     kern<<<grid, kThreads, pl.smem, stream>>>(pl.A, wmap, xmap);
+    timing_end(stream);
     return cudaGetLastError();
 }
 

@@ -640,7 +640,9 @@ cudaError_t launch_tf_km(const TfPlan &pl, void *ws, cudaStream_t stream) {
     if (e != cudaSuccess)
         return e;
     const int grid = A.num_units < sms ? A.num_units : sms;
+    timing_begin(stream);
     kern<<<grid, kThreads, pl.smem, stream>>>(A, mhi, mlo, mx);
+    timing_end(stream);
     e = cudaGetLastError();
     if (e != cudaSuccess || A.splits == 1)
         return e;

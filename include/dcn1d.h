@@ -207,6 +207,15 @@ const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor 
                                       int unconstrained, const dcn1d_tensor *out);
 
 /*
+ * For benchmarks: the next dcn1d_forward / dcn1d_forward_ws call on this host
+ * thread records `begin` (a cudaEvent_t) on its stream right before launching
+ * its main kernel and `end` right after it, then forgets both.  A forward that
+ * launches helper kernels (weight split, split-K reduction) keeps them outside
+ * the pair.  NULL events record nothing.
+ */
+void dcn1d_set_timing_events(void *begin, void *end);
+
+/*
  * Device-side status of the kernels enqueued so far on the current device.
  * Kernels that wait on on-chip barriers bound every wait (about 2 s); a kernel
  * that gives up records it in a device status word and exits, leaving its
