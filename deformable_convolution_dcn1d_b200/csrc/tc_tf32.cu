@@ -52,35 +52,58 @@ struct TfArgs {
     int num_kb;         // k-blocks of the whole reduction
     int kb_per_split;   // k-blocks per split
     int splits;
-    int tiles_l;        // l-tiles per batch row
-    int num_units;      // splits * groups * n_cob * B * tiles_l
+    int flat;           // 1: tiles run over the flattened positions n = b * L_out + l
+                        // 0: tiles stay inside one batch row (tiles_l per row)
+    int tiles_l;
+    int n_tiles;
+    int num_units;      // splits * groups * n_cob * n_tiles
     int nch, nbox, margin;
-    uint32_t w_stage_bytes, x_stage_bytes, x_box_bytes;
+    int nslots;         // batch rows a tile can touch (x window staged per row)
+    uint32_t w_stage_bytes, x_stage_bytes, x_box_bytes, x_slot_bytes;
     uint32_t off_w, off_wlo, off_x, off_bias, off_bar;
     unsigned int *status;
     float *partial;     // [splits][B][C_out][L_out] when splits > 1
 };
 
+// A unit of work: one split of the reduction for one tile of up to 128
+// consecutive flattened output positions n = b * L_out + l in [nbase, n_end)
+// and one block of N output channels of conv group g.  A flat tile may span
+// several batch rows b_first ..; "slot" j is batch row b_first + j.
 struct Unit {
-    int split, g, cob, b, lbase, wx0, kb0, kb1;
+    int split, g, cob, nbase, n_end, b_first, nslots, kb0, kb1;
 };
+
+__device__ __forceinline__ int floor8(int w) { return (w >= 0) ? (w / 8) * 8 : -(((-w) + 7) / 8) * 8; }
 
 __device__ __forceinline__ Unit decode_unit(const TfArgs &A, int u) {
     Unit r;
-    const int lt = u % A.tiles_l;
-    int t = u / A.tiles_l;
-    r.b = t % A.P.B;
-    t /= A.P.B;
+    const int nt = u % A.n_tiles;
+    int t = u / A.n_tiles;
     r.cob = t % A.n_cob;
     t /= A.n_cob;
     r.g = t % A.P.groups;
     r.split = t / A.P.groups;
-    r.lbase = lt * kRows;
-    int w = r.lbase * A.P.stride - A.P.padding - A.margin;
-    r.wx0 = (w >= 0) ? (w / 8) * 8 : -(((-w) + 7) / 8) * 8;
+    if (A.flat) {
+        r.nbase = nt * kRows;
+        r.n_end = min(r.nbase + kRows, A.P.B * A.P.L_out);
+    } else {
+        const int b = nt / A.tiles_l;
+        const int lb = (nt - b * A.tiles_l) * kRows;
+        r.nbase = b * A.P.L_out + lb;
+        r.n_end = b * A.P.L_out + min(lb + kRows, A.P.L_out);
+    }
+    r.b_first = r.nbase / A.P.L_out;
+    r.nslots = (r.n_end - 1) / A.P.L_out - r.b_first + 1;
     r.kb0 = r.split * A.kb_per_split;
     r.kb1 = min(A.num_kb, r.kb0 + A.kb_per_split);
     return r;
+}
+
+// First staged position of slot j's window: its first output's receptive field
+// minus the margin, rounded down to 8 (TMA coordinates are 16-byte aligned).
+__device__ __forceinline__ int slot_wx0(const TfArgs &A, const Unit &U, int j) {
+    const int lmin = (j == 0) ? U.nbase - U.b_first * A.P.L_out : 0;
+    return floor8(lmin * A.P.stride - A.P.padding - A.margin);
 }
 
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
@@ -256,22 +279,26 @@ __global__ void __maxnreg__(96)
             uint32_t it = 0;
             for (int u = blockIdx.x; u < A.num_units; u += gridDim.x) {
                 const Unit U = decode_unit(A, u);
-                const int xrow0 = U.b * P.C_in + U.g * P.cin_g;
                 const int corow = U.g * P.cout_g + U.cob * A.N;
+                const uint32_t tx = 2 * A.w_stage_bytes + (uint32_t)U.nslots * A.x_slot_bytes;
                 for (int kb = U.kb0; kb < U.kb1; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
                     if (!wait(bar_empty(s), ph ^ 1u))
                         goto tma_done;
-                    mbar_arrive_expect_tx(bar_full(s), 2 * A.w_stage_bytes + A.x_stage_bytes);
+                    mbar_arrive_expect_tx(bar_full(s), tx);
                     tma_load_2d(w_st0 + s * A.w_stage_bytes, &whimap, kb * kBK, corow, bar_full(s));
                     tma_load_2d(wlo_st0 + s * A.w_stage_bytes, &wlomap, kb * kBK, corow, bar_full(s));
                     const int c_lo = (kb * kBK) / K;
-                    const uint32_t xdst = x_st0 + s * A.x_stage_bytes;
-                    tma_load_2d(xdst, &xmap, U.wx0, xrow0 + c_lo, bar_full(s));
-                    if (A.nbox == 2)
-                        tma_load_2d(xdst + A.x_box_bytes, &xmap, U.wx0 + kBoxStep, xrow0 + c_lo,
-                                    bar_full(s));
+                    for (int j = 0; j < U.nslots; ++j) {   // one window per batch row of the tile
+                        const int xrow = (U.b_first + j) * P.C_in + U.g * P.cin_g + c_lo;
+                        const int wx0 = slot_wx0(A, U, j);
+                        const uint32_t xdst = x_st0 + s * A.x_stage_bytes + j * A.x_slot_bytes;
+                        tma_load_2d(xdst, &xmap, wx0, xrow, bar_full(s));
+                        if (A.nbox == 2)
+                            tma_load_2d(xdst + A.x_box_bytes, &xmap, wx0 + kBoxStep, xrow,
+                                        bar_full(s));
+                    }
                 }
             }
         tma_done:
@@ -332,8 +359,10 @@ __global__ void __maxnreg__(96)
 
         auto epilogue = [&](int u, uint32_t tcnt) -> bool {
             const Unit U = decode_unit(A, u);
-            const int l = U.lbase + row;
-            const bool valid = l < P.L_out;
+            const int n = U.nbase + row;
+            const bool valid = n < U.n_end;
+            const int b = valid ? n / P.L_out : 0;
+            const int l = valid ? n - b * P.L_out : 0;
             const int co0 = U.g * P.cout_g + U.cob * A.N;
             if (!__all_sync(0xffffffffu, wait(bar_dfull, tcnt & 1u)))
                 return false;
@@ -341,10 +370,10 @@ __global__ void __maxnreg__(96)
             float *dst;
             bool add_bias;
             if (A.splits > 1) {
-                dst = A.partial + ((((int64_t)U.split * P.B + U.b) * P.C_out + co0) * P.L_out + l);
+                dst = A.partial + ((((int64_t)U.split * P.B + b) * P.C_out + co0) * P.L_out + l);
                 add_bias = false;
             } else {
-                dst = static_cast<float *>(P.out) + (((int64_t)U.b * P.C_out + co0) * P.L_out + l);
+                dst = static_cast<float *>(P.out) + (((int64_t)b * P.C_out + co0) * P.L_out + l);
                 add_bias = true;
             }
             for (int cc = h; cc < A.N / 16; cc += 4) {
@@ -355,8 +384,8 @@ __global__ void __maxnreg__(96)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int co = 16 * cc + i;
-                        const float b = add_bias ? bias_s[co0 + co] : 0.0f;
-                        dst[(int64_t)co * P.L_out] = __fadd_rn(__uint_as_float(v[i]), b);
+                        const float bv = add_bias ? bias_s[co0 + co] : 0.0f;
+                        dst[(int64_t)co * P.L_out] = __fadd_rn(__uint_as_float(v[i]), bv);
                     }
                 }
             }
@@ -375,9 +404,10 @@ __global__ void __maxnreg__(96)
             pf_og = og;
             if (u >= A.num_units)
                 return;
-            const int l = U.lbase + row;
-            const int64_t obase =
-                (((int64_t)U.b * P.offset_groups + og) * P.L_out + (l < P.L_out ? l : 0)) * K;
+            const int n = U.nbase + row;
+            const int b = n < U.n_end ? n / P.L_out : 0;
+            const int l = n < U.n_end ? n - b * P.L_out : 0;
+            const int64_t obase = (((int64_t)b * P.offset_groups + og) * P.L_out + l) * K;
 #pragma unroll
             for (int k = 0; k < K; ++k) {
                 raw_off[k] = static_cast<const float *>(P.off)[obase + k];
@@ -396,12 +426,16 @@ __global__ void __maxnreg__(96)
         for (int u = blockIdx.x; u < A.num_units; u += gridDim.x) {
             const Unit U = decode_unit(A, u);
             const int u_next = u + (int)gridDim.x;
-            const int l = U.lbase + row;
-            const bool valid = l < P.L_out;
+            const int n = U.nbase + row;
+            const bool valid = n < U.n_end;
+            const int b = valid ? n / P.L_out : U.b_first;
+            const int l = valid ? n - b * P.L_out : 0;
+            const int slot = b - U.b_first;                 // this row's window in the stage
+            const uint32_t slot_off = (uint32_t)slot * A.x_slot_bytes;
             const float start = (float)(l * P.stride - P.padding);
-            const uint32_t win_bits = kFloorMagicBits + (uint32_t)U.wx0;
+            const uint32_t win_bits = kFloorMagicBits + (uint32_t)slot_wx0(A, U, slot);
             const int og_last = (U.g * P.cin_g + ((U.kb1 * kBK - 1) / K)) / P.cin_per_og;
-            const float *xb = static_cast<const float *>(P.x) + (int64_t)U.b * P.C_in * P.L_in;
+            const float *xb = static_cast<const float *>(P.x) + (int64_t)b * P.C_in * P.L_in;
             TapsF<K> tp;
             int og_cur = -1;
             int og = og_of(U, U.kb0);
@@ -436,14 +470,14 @@ __global__ void __maxnreg__(96)
                         tp.f[k] = __fsub_rn(pos, __fsub_rn(tt, M));
                         tp.m[k] = raw_m[k];
                         if (rel < (uint32_t)(kBox - 1)) {
-                            tp.addr[k] = rel * 4u;
+                            tp.addr[k] = slot_off + rel * 4u;
                         } else if (A.nbox == 2 && rel < (uint32_t)kWinMax) {
-                            tp.addr[k] = A.x_box_bytes + (rel - kBoxStep) * 4u;
+                            tp.addr[k] = slot_off + A.x_box_bytes + (rel - kBoxStep) * 4u;
                         } else {
                             tp.addr[k] = 0;
                             tp.slow |= 1u << k;
                         }
-                        if (!valid) {
+                        if (!valid) {   // rows past the last output: finite zeros, never stored
                             tp.f[k] = 0.0f;
                             tp.m[k] = 0.0f;
                             tp.addr[k] = 0;
@@ -463,8 +497,7 @@ __global__ void __maxnreg__(96)
                     const uint32_t xrow_addr =
                         x_st0 + s * A.x_stage_bytes + (uint32_t)(c_first - c_lo) * kRowBytes;
                     const float *xg = xb + (int64_t)(U.g * P.cin_g + c_first) * P.L_in;
-                    const int64_t obase = (((int64_t)U.b * P.offset_groups + og) * P.L_out +
-                                           (valid ? l : 0)) * K;
+                    const int64_t obase = (((int64_t)b * P.offset_groups + og) * P.L_out + l) * K;
                     const float *offrow = static_cast<const float *>(P.off) + obase;
                     const float *maskrow = MASK ? static_cast<const float *>(P.mask) + obase : nullptr;
                     const uint32_t lanebase = tmem + ((uint32_t)(32 * q) << 16);
@@ -551,18 +584,64 @@ unsigned grid_for(int64_t n, int sms) {
     return (unsigned)(want < cap ? want : cap);
 }
 
+// Shared-memory layout of A for the given tile mode; false if it does not fit.
+bool layout_tf(const Problem &P, TfArgs &A, size_t *smem_out) {
+    const int64_t rows = P.L_out < kRows ? P.L_out : kRows;   // outputs of one batch row in a tile
+    const int64_t need = (rows - 1) * P.stride + (int64_t)P.dilation * (P.K - 1) + 2 +
+                         2 * A.margin + 7;
+    if (need > kWinMax)
+        return false;
+    A.nbox = need > kBox - 1 ? 2 : 1;
+    if (A.flat) {
+        const int slots = (kRows - 1 + P.L_out - 1) / P.L_out + 1;
+        A.nslots = slots < P.B ? slots : P.B;
+    } else {
+        A.nslots = 1;
+    }
+    A.w_stage_bytes = (uint32_t)A.N * 128u;
+    A.x_box_bytes = (uint32_t)A.nch * kRowBytes;
+    A.x_slot_bytes = A.x_box_bytes * A.nbox;
+    A.x_stage_bytes = A.x_slot_bytes * A.nslots;
+    A.off_w = 0;
+    A.off_wlo = A.off_w + kStages * A.w_stage_bytes;
+    A.off_x = A.off_wlo + kStages * A.w_stage_bytes;
+    A.off_bias = A.off_x + kStages * A.x_stage_bytes;
+    A.off_bar = A.off_bias + (uint32_t)((P.C_out * 4 + 15) / 16 * 16);
+    size_t smem = A.off_bar + 8 * (3 * kStages + 3) + 16 + 1024;
+    if (smem > 227 * 1024)
+        return false;
+    *smem_out = smem < 116 * 1024 ? 116 * 1024 : smem;   // one CTA per SM
+    return true;
+}
+
 bool make_tf_plan(const Problem &P, TfPlan *out) {
     TfArgs A;
     memset(&A, 0, sizeof(A));
     A.P = P;
     const int Kg = P.cin_g * P.K;
+    if ((int64_t)P.B * P.L_out + kRows > INT32_MAX || (int64_t)P.B * P.C_in > INT32_MAX)
+        return false;   // flattened position and TMA row indices are 32-bit
     A.N = P.cout_g < 256 ? P.cout_g : 256;
     if (P.cout_g % A.N != 0)
         return false;
     A.n_cob = P.cout_g / A.N;
     A.num_kb = Kg / kBK;
+    A.nch = (kBK - 1) / P.K + 2;
+    A.margin = P.unconstrained ? 32 : 0;
+    size_t smem = 0;
+    // Flat tiles fill all 128 MMA rows when L_out is not a multiple of 128;
+    // row tiles need only one x window per stage.
+    A.flat = (P.L_out % kRows != 0) ? 1 : 0;
+    if (!layout_tf(P, A, &smem)) {
+        if (!A.flat)
+            return false;
+        A.flat = 0;
+        if (!layout_tf(P, A, &smem))
+            return false;
+    }
     A.tiles_l = (P.L_out + kRows - 1) / kRows;
-    const int base_units = P.groups * A.n_cob * P.B * A.tiles_l;
+    A.n_tiles = A.flat ? (int)(((int64_t)P.B * P.L_out + kRows - 1) / kRows) : P.B * A.tiles_l;
+    const int base_units = P.groups * A.n_cob * A.n_tiles;
     const int sms = sm_count() > 0 ? sm_count() : 148;
     int splits = sms / (base_units > 0 ? base_units : 1);
     const int max_splits = A.num_kb / 8 > 0 ? A.num_kb / 8 : 1;   // at least 8 k-blocks a split
@@ -573,26 +652,6 @@ bool make_tf_plan(const Problem &P, TfPlan *out) {
     A.kb_per_split = (A.num_kb + splits - 1) / splits;
     A.splits = (A.num_kb + A.kb_per_split - 1) / A.kb_per_split;
     A.num_units = A.splits * base_units;
-    A.nch = (kBK - 1) / P.K + 2;
-    A.margin = P.unconstrained ? 32 : 0;
-    const int64_t need = (int64_t)(kRows - 1) * P.stride + (int64_t)P.dilation * (P.K - 1) + 2 +
-                         2 * A.margin + 7;
-    if (need > kWinMax)
-        return false;
-    A.nbox = need > kBox - 1 ? 2 : 1;
-    A.w_stage_bytes = (uint32_t)A.N * 128u;
-    A.x_box_bytes = (uint32_t)A.nch * kRowBytes;
-    A.x_stage_bytes = A.x_box_bytes * A.nbox;
-    A.off_w = 0;
-    A.off_wlo = A.off_w + kStages * A.w_stage_bytes;
-    A.off_x = A.off_wlo + kStages * A.w_stage_bytes;
-    A.off_bias = A.off_x + kStages * A.x_stage_bytes;
-    A.off_bar = A.off_bias + (uint32_t)((P.C_out * 4 + 15) / 16 * 16);
-    size_t smem = A.off_bar + 8 * (3 * kStages + 3) + 16 + 1024;
-    if (smem > 227 * 1024)
-        return false;
-    if (smem < 116 * 1024)
-        smem = 116 * 1024;
     TfPlan pl;
     pl.A = A;
     pl.smem = smem;

@@ -65,6 +65,12 @@ TF32_CASES = [
     ("groups2_mask_og4", 2, 64, 128, 4, 160, 2, 2, 2, 2, 4, True, False, 3.0),
     ("far_offsets_slow_taps", 1, 64, 64, 8, 256, 1, 3, 1, 1, 2, False, True, 90.0),
     ("cout_512_two_blocks", 1, 64, 512, 4, 300, 1, 1, 1, 1, 1, True, True, 2.0),
+    # L_out = 256: tiles stay inside one batch row
+    ("row_tiles_lout_256", 2, 32, 64, 9, 264, 1, 0, 1, 1, 1, False, False, 2.0),
+    # L_out = 21: one 128-row tile spans 8 batch rows, the last tile is ragged
+    ("short_rows_span_8_batches", 9, 64, 64, 8, 28, 1, 0, 1, 1, 1, True, False, 2.0),
+    # two x windows per batch row do not fit beside N = 256 twice: row tiles instead
+    ("flat_falls_back_to_rows", 2, 32, 256, 16, 300, 2, 0, 1, 1, 1, False, False, 2.0),
 ]
 
 
