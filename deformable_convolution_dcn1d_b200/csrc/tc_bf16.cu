@@ -33,6 +33,8 @@
 // Stages are chained by mbarriers; every wait is bounded (sm100.cuh).
 #include <string.h>
 
+#include <utility>
+
 #include "common.cuh"
 #include "sampler.cuh"
 #include "sm100.cuh"
@@ -68,6 +70,7 @@ struct TcArgs {
     int nbox;          // x boxes per stage (1 or 2)
     int margin;        // staged positions beyond the receptive fields (unconstrained)
     uint32_t w_stage_bytes, x_stage_bytes, x_box_bytes;
+    int pair_store;    // 1: L_out even and out 4-byte aligned (32-bit epilogue stores)
     uint32_t off_w, off_x, off_bias, off_bar;   // shared-memory layout
     unsigned int *status;                       // device status word
 };
@@ -88,10 +91,12 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs &A, int t) {
     return r;
 }
 
-// 16-bit shared load, zero-extended into a 32-bit register by the load itself.
+// 16-bit shared load at addr + OFF, zero-extended into a 32-bit register by the
+// load itself (the offset rides in the instruction, not in an extra add).
+template <uint32_t OFF>
 __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
     uint32_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(addr));
+    asm volatile("ld.shared.u16 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
     return v;
 }
 
@@ -133,10 +138,45 @@ __device__ __forceinline__ float slow_element(const Taps<K> &tp, int kidx, int h
     return __fmul_rn(r, __uint_as_float(hi ? (mp & 0xFFFF0000u) : (mp << 16)));
 }
 
+// Col values 2I and 2I+1 of a segment whose first element has phase K0 = kk0 % K:
+// taps (k0, k1) of channel rows (c0, c1) relative to the segment's first channel.
+// The lerp x0 + f (x1 - x0) runs on the two elements in bf16x2 arithmetic.
+template <int K, int K0, bool MASK, bool SLOW, int I>
+__device__ __forceinline__ void produce_pair(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
+                                             const uint32_t (&base)[K], const __nv_bfloat16 *xg,
+                                             int64_t xg_row_stride, int L_in) {
+    constexpr int k0 = (K0 + 2 * I) % K, c0 = (K0 + 2 * I) / K;
+    constexpr int k1 = (K0 + 2 * I + 1) % K, c1 = (K0 + 2 * I + 1) / K;
+    constexpr uint32_t o0 = c0 * kRowBytes, o1 = c1 * kRowBytes;
+    const uint32_t x0 =
+        __byte_perm(lds_u16<o0>(base[k0]), lds_u16<o1>(base[k1]), 0x5410);
+    const uint32_t x1 =
+        __byte_perm(lds_u16<o0 + 2>(base[k0]), lds_u16<o1 + 2>(base[k1]), 0x5410);
+    __nv_bfloat162 v = __hfma2(as_bf2(tp.fpair[k0]), __hsub2(as_bf2(x1), as_bf2(x0)), as_bf2(x0));
+    if (MASK)
+        v = __hmul2(v, as_bf2(tp.mpair[k0]));
+    out[I] = as_u32(v);
+    if (SLOW && (((tp.slow >> k0) | (tp.slow >> k1)) & 1u)) {
+        float lo = __low2float(v), hi = __high2float(v);
+        if ((tp.slow >> k0) & 1u)
+            lo = slow_element<K, MASK>(tp, k0, 0, xg + c0 * xg_row_stride, L_in);
+        if ((tp.slow >> k1) & 1u)
+            hi = slow_element<K, MASK>(tp, k1, 1, xg + c1 * xg_row_stride, L_in);
+        out[I] = pack2(lo, hi);
+    }
+}
+
+template <int K, int K0, bool MASK, bool SLOW, int... Is>
+__device__ __forceinline__ void produce_pairs(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
+                                              const uint32_t (&base)[K], const __nv_bfloat16 *xg,
+                                              int64_t xg_row_stride, int L_in,
+                                              std::integer_sequence<int, Is...>) {
+    (produce_pair<K, K0, MASK, SLOW, Is>(out, tp, base, xg, xg_row_stride, L_in), ...);
+}
+
 // kSeg col values of one row for the reduction elements kk0 .. kk0+kSeg-1 of a k-block,
 // packed bf16x2 (element 2i in the low half of out[i]).  Phase K0 = kk0 % K is a
-// compile-time constant, so every tap index below is static.  The lerp
-// x0 + f (x1 - x0) runs in bf16x2 arithmetic on element pairs.
+// compile-time constant, so every tap index and row offset below is static.
 template <int K, int K0, bool MASK, bool SLOW>
 __device__ __forceinline__ void produce_segment(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
                                                 uint32_t xrow_addr, const __nv_bfloat16 *xg,
@@ -145,27 +185,8 @@ __device__ __forceinline__ void produce_segment(uint32_t (&out)[kSeg / 2], const
 #pragma unroll
     for (int k = 0; k < K; ++k)
         base[k] = xrow_addr + tp.addr[k];
-#pragma unroll
-    for (int i = 0; i < kSeg / 2; ++i) {
-        const int k0 = (K0 + 2 * i) % K, c0 = (K0 + 2 * i) / K;
-        const int k1 = (K0 + 2 * i + 1) % K, c1 = (K0 + 2 * i + 1) / K;
-        const uint32_t a0 = base[k0] + c0 * kRowBytes;
-        const uint32_t a1 = base[k1] + c1 * kRowBytes;
-        const uint32_t x0 = __byte_perm(lds_u16(a0), lds_u16(a1), 0x5410);
-        const uint32_t x1 = __byte_perm(lds_u16(a0 + 2), lds_u16(a1 + 2), 0x5410);
-        __nv_bfloat162 v = __hfma2(as_bf2(tp.fpair[k0]), __hsub2(as_bf2(x1), as_bf2(x0)), as_bf2(x0));
-        if (MASK)
-            v = __hmul2(v, as_bf2(tp.mpair[k0]));
-        out[i] = as_u32(v);
-        if (SLOW && (((tp.slow >> k0) | (tp.slow >> k1)) & 1u)) {
-            float lo = __low2float(v), hi = __high2float(v);
-            if ((tp.slow >> k0) & 1u)
-                lo = slow_element<K, MASK>(tp, k0, 0, xg + c0 * xg_row_stride, L_in);
-            if ((tp.slow >> k1) & 1u)
-                hi = slow_element<K, MASK>(tp, k1, 1, xg + c1 * xg_row_stride, L_in);
-            out[i] = pack2(lo, hi);
-        }
-    }
+    produce_pairs<K, K0, MASK, SLOW>(out, tp, base, xg, xg_row_stride, L_in,
+                                     std::make_integer_sequence<int, kSeg / 2>{});
 }
 
 // Jump to the segment code of phase k0 (a switch, so one indirect branch).
