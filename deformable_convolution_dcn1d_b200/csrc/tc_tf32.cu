@@ -8,8 +8,9 @@
 // and the MMA accumulates hi*hi + hi*lo + lo*hi in fp32; the dropped lo*lo
 // term is about 2^-22 of the product.
 //
-//  * A one-pass kernel splits the weight into W_hi and W_lo in the workspace.
-//  * The main kernel has the bf16 kernel's roles: a TMA warp loads the W_hi and
+//  * A one-pass kernel writes W_lo to the workspace; W itself serves as W_hi,
+//    since the tf32 MMA ignores the low 13 mantissa bits of an fp32 operand.
+//  * The main kernel has the bf16 kernel's roles: a TMA warp loads the W and
 //    W_lo tiles (128-byte swizzle) and the fp32 x window of each 32-wide
 //    k-block; 16 producer warps interpolate 16 columns each in fp32 and write
 //    their hi and lo parts straight into tensor memory (A operand); one thread
@@ -543,15 +544,15 @@ __global__ void __maxnreg__(96)
     }
 }
 
-// W_hi = W with the low 13 mantissa bits cleared (exactly a tf32 value), W_lo = W - W_hi.
-__global__ void __launch_bounds__(256) split_tf32_kernel(const float *w, float *hi, float *lo,
-                                                         int64_t n) {
+// W_lo = W - W_hi, W_hi = W with the low 13 mantissa bits cleared (a tf32 value).
+// W_hi itself is never stored: tcgen05.mma kind::tf32 ignores the low 13 mantissa
+// bits of an fp32 operand (its results on W are bit-identical to those on W_hi), so
+// the main kernel reads W as the high part.
+__global__ void __launch_bounds__(256) split_tf32_kernel(const float *w, float *lo, int64_t n) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
         const float v = w[i];
-        const float h = __uint_as_float(__float_as_uint(v) & kTf32Mask);
-        hi[i] = h;
-        lo[i] = __fsub_rn(v, h);
+        lo[i] = __fsub_rn(v, __uint_as_float(__float_as_uint(v) & kTf32Mask));
     }
 }
 
@@ -573,7 +574,7 @@ __global__ void __launch_bounds__(256) reduce_splits_kernel(const float *partial
 struct TfPlan {
     TfArgs A;
     size_t smem;
-    size_t ws_whi, ws_wlo, ws_partial, ws_total;   // workspace layout (bytes)
+    size_t ws_wlo, ws_partial, ws_total;   // workspace layout (bytes)
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -656,9 +657,8 @@ bool make_tf_plan(const Problem &P, TfPlan *out) {
     pl.A = A;
     pl.smem = smem;
     const size_t wbytes = (size_t)P.C_out * Kg * 4;
-    pl.ws_whi = 0;
-    pl.ws_wlo = align256(wbytes);
-    pl.ws_partial = pl.ws_wlo + align256(wbytes);
+    pl.ws_wlo = 0;
+    pl.ws_partial = align256(wbytes);
     pl.ws_total = pl.ws_partial +
                   (A.splits > 1 ? align256((size_t)A.splits * P.B * P.C_out * P.L_out * 4) : 0);
     *out = pl;
@@ -673,12 +673,11 @@ cudaError_t launch_tf_km(const TfPlan &pl, void *ws, cudaStream_t stream) {
     if (!A.status)
         return cudaErrorInvalidDevice;
     unsigned char *wsb = static_cast<unsigned char *>(ws);
-    float *whi = reinterpret_cast<float *>(wsb + pl.ws_whi);
     float *wlo = reinterpret_cast<float *>(wsb + pl.ws_wlo);
     A.partial = A.splits > 1 ? reinterpret_cast<float *>(wsb + pl.ws_partial) : nullptr;
     const int Kg = P.cin_g * P.K;
     alignas(64) CUtensorMap mhi, mlo, mx;
-    if (!encode_2d(&mhi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, whi, (uint64_t)Kg, (uint64_t)P.C_out, 4,
+    if (!encode_2d(&mhi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, P.w, (uint64_t)Kg, (uint64_t)P.C_out, 4,
                    kBK, (uint32_t)A.N, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&mlo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, wlo, (uint64_t)Kg, (uint64_t)P.C_out, 4,
                    kBK, (uint32_t)A.N, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -690,7 +689,7 @@ cudaError_t launch_tf_km(const TfPlan &pl, void *ws, cudaStream_t stream) {
         return cudaErrorNoDevice;
     const int64_t nw = (int64_t)P.C_out * Kg;
     split_tf32_kernel<<<(unsigned)grid_for(nw, sms), 256, 0, stream>>>(
-        static_cast<const float *>(P.w), whi, wlo, nw);
+        static_cast<const float *>(P.w), wlo, nw);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;

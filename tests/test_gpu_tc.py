@@ -113,3 +113,23 @@ def test_tf32_deterministic_across_calls():
     torch.cuda.synchronize()
     assert launches >= 2
     assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+# The three-product split reaches about fp32 accuracy; one TF32 product per term (or a
+# tensor core that rounded, instead of truncating, the fp32 weight it reads as the high
+# part) gives about 1e-4 on this shape.  The bound pins the split, not just the tolerance.
+TF32_SPLIT_BOUND = 1e-5
+
+
+@pytest.mark.parametrize("scale_low_bits", [False, True], ids=["plain", "low_bits_set"])
+def test_tf32_three_products_reach_fp32_accuracy(scale_low_bits):
+    w = W.USAGE_F32.with_batch(2)
+    t = W.make_inputs(w, seed=11)
+    if scale_low_bits:   # weights whose low mantissa bits are all populated
+        t["weight"] = (t["weight"].double() * (1.0 + 2.0 ** -12)).float()
+    td = to_dev(t)
+    assert kernel_name(w, td) == "tcgen05_3xtf32"
+    y = gpu_forward(w, td)
+    assert dcn.dcn1d_device_status() == 0
+    err = norm_err(y.double().cpu().numpy(), oracle_full(w, t))
+    assert err <= TF32_SPLIT_BOUND, err
