@@ -548,11 +548,24 @@ __global__ void __maxnreg__(96)
 // W_hi itself is never stored: tcgen05.mma kind::tf32 ignores the low 13 mantissa
 // bits of an fp32 operand (its results on W are bit-identical to those on W_hi), so
 // the main kernel reads W as the high part.
-__global__ void __launch_bounds__(256) split_tf32_kernel(const float *w, float *lo, int64_t n) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const float v = w[i];
-        lo[i] = __fsub_rn(v, __uint_as_float(__float_as_uint(v) & kTf32Mask));
+// 16-byte accesses, four in flight per thread (n4 = element count / 4).
+__device__ __forceinline__ float lo_part(float v) {
+    return __fsub_rn(v, __uint_as_float(__float_as_uint(v) & kTf32Mask));
+}
+
+__global__ void __launch_bounds__(256) split_tf32_kernel(const float4 *w, float4 *lo, int64_t n4) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += 4 * stride) {
+        float4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (i + j * stride < n4)
+                v[j] = w[i + j * stride];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (i + j * stride < n4)
+                lo[i + j * stride] =
+                    make_float4(lo_part(v[j].x), lo_part(v[j].y), lo_part(v[j].z), lo_part(v[j].w));
     }
 }
 
@@ -567,6 +580,38 @@ __global__ void __launch_bounds__(256) reduce_splits_kernel(const float *partial
             acc = __fadd_rn(acc, partial[(int64_t)s * n + i]);
         if (bias)
             acc = __fadd_rn(acc, bias[(i / L_out) % C_out]);
+        out[i] = acc;
+    }
+}
+
+// The same sums four outputs at a time with 16-byte accesses (n % 4 == 0, out 16-byte
+// aligned, L_out >= 4 so that four consecutive outputs span at most two channels).
+__global__ void __launch_bounds__(256) reduce_splits_kernel4(const float4 *partial,
+                                                             const float *bias, float4 *out,
+                                                             int splits, int C_out, int L_out,
+                                                             int64_t n4) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 4
+        for (int s = 0; s < splits; ++s) {
+            const float4 p = partial[(int64_t)s * n4 + i];
+            acc.x = __fadd_rn(acc.x, p.x);
+            acc.y = __fadd_rn(acc.y, p.y);
+            acc.z = __fadd_rn(acc.z, p.z);
+            acc.w = __fadd_rn(acc.w, p.w);
+        }
+        if (bias) {
+            const int64_t row = (4 * i) / L_out;        // (b, co) row of the first output
+            const int l = (int)(4 * i - row * L_out);
+            const int co = (int)(row % C_out);
+            const int co_next = co + 1 == C_out ? 0 : co + 1;
+            const float b0 = bias[co], b1 = bias[co_next];
+            acc.x = __fadd_rn(acc.x, b0);
+            acc.y = __fadd_rn(acc.y, l + 1 < L_out ? b0 : b1);
+            acc.z = __fadd_rn(acc.z, l + 2 < L_out ? b0 : b1);
+            acc.w = __fadd_rn(acc.w, l + 3 < L_out ? b0 : b1);
+        }
         out[i] = acc;
     }
 }
@@ -687,9 +732,9 @@ cudaError_t launch_tf_km(const TfPlan &pl, void *ws, cudaStream_t stream) {
     const int sms = sm_count();
     if (sms <= 0)
         return cudaErrorNoDevice;
-    const int64_t nw = (int64_t)P.C_out * Kg;
-    split_tf32_kernel<<<(unsigned)grid_for(nw, sms), 256, 0, stream>>>(
-        static_cast<const float *>(P.w), wlo, nw);
+    const int64_t nw4 = (int64_t)P.C_out * Kg / 4;   // Kg is a multiple of 32
+    split_tf32_kernel<<<(unsigned)grid_for((nw4 + 3) / 4, sms), 256, 0, stream>>>(
+        static_cast<const float4 *>(P.w), reinterpret_cast<float4 *>(wlo), nw4);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
@@ -705,9 +750,14 @@ cudaError_t launch_tf_km(const TfPlan &pl, void *ws, cudaStream_t stream) {
     if (e != cudaSuccess || A.splits == 1)
         return e;
     const int64_t n = (int64_t)P.B * P.C_out * P.L_out;
-    reduce_splits_kernel<<<(unsigned)grid_for(n, sms), 256, 0, stream>>>(
-        A.partial, static_cast<const float *>(P.bias), static_cast<float *>(P.out), A.splits,
-        P.C_out, P.L_out, n);
+    if (n % 4 == 0 && P.L_out >= 4 && (reinterpret_cast<uintptr_t>(P.out) & 15) == 0)
+        reduce_splits_kernel4<<<(unsigned)grid_for(n / 4, sms), 256, 0, stream>>>(
+            reinterpret_cast<const float4 *>(A.partial), static_cast<const float *>(P.bias),
+            static_cast<float4 *>(P.out), A.splits, P.C_out, P.L_out, n / 4);
+    else
+        reduce_splits_kernel<<<(unsigned)grid_for(n, sms), 256, 0, stream>>>(
+            A.partial, static_cast<const float *>(P.bias), static_cast<float *>(P.out), A.splits,
+            P.C_out, P.L_out, n);
     return cudaGetLastError();
 }
 

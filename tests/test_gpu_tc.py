@@ -71,6 +71,8 @@ TF32_CASES = [
     ("short_rows_span_8_batches", 9, 64, 64, 8, 28, 1, 0, 1, 1, 1, True, False, 2.0),
     # two x windows per batch row do not fit beside N = 256 twice: row tiles instead
     ("flat_falls_back_to_rows", 2, 32, 256, 16, 300, 2, 0, 1, 1, 1, False, False, 2.0),
+    # L_out = 1, 16 reduction splits: the split sums take the one-output-at-a-time path
+    ("lout_1_scalar_reduce", 2, 256, 64, 16, 16, 1, 0, 1, 1, 1, False, False, 2.0),
 ]
 
 
@@ -133,3 +135,20 @@ def test_tf32_three_products_reach_fp32_accuracy(scale_low_bits):
     assert dcn.dcn1d_device_status() == 0
     err = norm_err(y.double().cpu().numpy(), oracle_full(w, t))
     assert err <= TF32_SPLIT_BOUND, err
+
+
+def test_tf32_split_sums_into_a_misaligned_output():
+    """An output view that is only 4-byte aligned takes the one-at-a-time reduction; the
+    result is the same bits as with an aligned output."""
+    w = W.USAGE_F32.with_batch(2)
+    td = to_dev(W.make_inputs(w, seed=13))
+    ref = gpu_forward(w, td)
+    buf = torch.full((ref.numel() + 1,), float("nan"), device="cuda")
+    out = buf[1:].view(ref.shape)
+    assert out.data_ptr() % 16 != 0
+    y = dcn.dcn1d_forward(td["x"], td["offsets"], td["mask"], td["weight"], td["bias"], w.stride,
+                          w.padding, w.dilation, w.groups, w.offset_groups, w.unconstrained,
+                          out=out)
+    torch.cuda.synchronize()
+    assert dcn.dcn1d_device_status() == 0
+    assert torch.equal(y.view(torch.int32), ref.view(torch.int32))
