@@ -1,4 +1,4 @@
-"""CPU oracle for the 1D deformable convolution forward -- TEST INFRASTRUCTURE.
+"""CPU oracle for the 1D deformable convolution forward and backward -- TEST INFRASTRUCTURE.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The product path (the CUDA library and
@@ -8,10 +8,11 @@ The arithmetic lives in ``dcn1d_oracle.c`` (plain loops, double accumulation,
 float32 sampling positions); this module only marshals arrays.  bf16 inputs are
 widened to float32 exactly before they reach the C code.
 
-Parity status: every function is pinned by ``tests/test_oracle_pins.py``
-except the exact clamp bounds of constrained mode, which no page fixes; those
-are checked only through invariants (locality, saturation) and are
-"parity unpinned" as to the bounds themselves.
+Parity status: every function is pinned by ``tests/test_oracle_pins.py`` (forward)
+and ``tests/test_oracle_backward_pins.py`` (backward: finite differences of the
+forward, conv1d autograd for zero offsets) except the exact clamp bounds of
+constrained mode, which no page fixes; those are checked only through invariants
+(locality, saturation) and are "parity unpinned" as to the bounds themselves.
 """
 from __future__ import annotations
 
@@ -54,6 +55,8 @@ class Oracle:
         lib.oracle_forward_points.argtypes = [_p] * 5 + [_i64] * 11 + [_int, _p, _i64, _p]
         lib.oracle_sample_index.restype = _int
         lib.oracle_sample_index.argtypes = [_p] + [_i64] * 8 + [_int, _p, _p]
+        lib.oracle_backward.restype = _int
+        lib.oracle_backward.argtypes = [_p] * 5 + [_i64] * 11 + [_int] + [_p] * 5
         lib.oracle_threads.restype = _int
         lib.oracle_threads.argtypes = []
         lib.oracle_set_threads.restype = None
@@ -108,6 +111,27 @@ class Oracle:
             raise ValueError(f"oracle_forward_points rejected the arguments (code {rc})")
         return out
 
+    def backward(self, x, offsets, mask, weight, grad_out, stride, padding, dilation, groups,
+                 offset_groups, unconstrained) -> dict:
+        """Gradients of sum(grad_out * forward) as float64 arrays: grad_x, grad_offsets,
+        grad_mask (None without a mask), grad_weight, grad_bias."""
+        xs, os_, ms, ws, gs = (_f32(t) for t in (x, offsets, mask, weight, grad_out))
+        dims = self._dims(xs, ws, os_, stride, padding, dilation, groups, offset_groups)
+        if gs.shape != (dims[0], dims[3], dims[5]):
+            raise ValueError("grad_out must be [B, C_out, L_out]")
+        g = {"grad_x": np.empty(xs.shape, dtype=np.float64),
+             "grad_offsets": np.empty(os_.shape, dtype=np.float64),
+             "grad_mask": np.empty(os_.shape, dtype=np.float64) if ms is not None else None,
+             "grad_weight": np.empty(ws.shape, dtype=np.float64),
+             "grad_bias": np.empty(ws.shape[0], dtype=np.float64)}
+        rc = self.lib.oracle_backward(_ptr(xs), _ptr(os_), _ptr(ms), _ptr(ws), _ptr(gs), *dims,
+                                      int(bool(unconstrained)), _ptr(g["grad_x"]),
+                                      _ptr(g["grad_offsets"]), _ptr(g["grad_mask"]),
+                                      _ptr(g["grad_weight"]), _ptr(g["grad_bias"]))
+        if rc != 0:
+            raise ValueError(f"oracle_backward rejected the shapes (code {rc})")
+        return g
+
     def sample_index(self, offsets, L_in, K, stride, padding, dilation, unconstrained):
         """(i0 int32, frac float32) for every tap, each shaped like ``offsets``."""
         os_ = _f32(offsets)
@@ -150,6 +174,10 @@ def forward_points(*a, **k):
 
 def sample_index(*a, **k):
     return get().sample_index(*a, **k)
+
+
+def backward(*a, **k):
+    return get().backward(*a, **k)
 
 
 def threads():

@@ -73,16 +73,22 @@ int64_t oracle_out_length(int64_t L_in, int64_t K, int64_t s, int64_t p, int64_t
 
 /* One tap's sampling position: the undeformed tap l*s - p + k*d plus the
  * learned offset (deformable-convolution formula, 1D), clamped in constrained
- * mode, split into its integer neighbour i0 and fraction f. */
+ * mode, split into its integer neighbour i0 and fraction f.  If gate is not
+ * NULL it receives the clamp's derivative (backward): 0 when the clamp moved
+ * the position, 1 otherwise (bounds included). */
 static void sample_position(int64_t l, int64_t k, float off, const oracle_shape *S,
-                            int64_t *i0, float *f)
+                            int64_t *i0, float *f, double *gate)
 {
     int64_t start = l * S->stride - S->padding;
     int64_t base = start + k * S->dilation;
     float pos = (float)base + off;
+    if (gate)
+        *gate = 1.0;
     if (!S->unconstrained) {
         float lo = (float)start;
         float hi = (float)(start + S->dilation * (S->K - 1));
+        if (gate && (pos < lo || pos > hi))
+            *gate = 0.0;
         if (pos < lo) pos = lo;
         if (pos > hi) pos = hi;
     }
@@ -116,7 +122,7 @@ static double output_point(const float *x, const float *off, const float *mask,
             int64_t oidx = ((b * S->offset_groups + og) * S->L_out + l) * S->K + k;
             int64_t i0;
             float f;
-            sample_position(l, k, off[oidx], S, &i0, &f);
+            sample_position(l, k, off[oidx], S, &i0, &f, NULL);
             double v = (1.0 - (double)f) * x_at(x, S, b, ci, i0) + (double)f * x_at(x, S, b, ci, i0 + 1);
             if (mask)
                 v *= (double)mask[oidx];
@@ -196,7 +202,7 @@ int oracle_sample_index(const float *off, int64_t B, int64_t G, int64_t L_in, in
         int64_t l = (t / K) % L_out;
         int64_t i0;
         float f;
-        sample_position(l, k, off[t], &S, &i0, &f);
+        sample_position(l, k, off[t], &S, &i0, &f, NULL);
         i0_out[t] = (int32_t)i0;
         f_out[t] = f;
     }
@@ -221,4 +227,118 @@ void oracle_set_threads(int n)
 #else
     (void)n;
 #endif
+}
+
+/* ------------------------------------------------------------------ backward
+ *
+ * Gradients of the forward above with respect to every input, for an upstream
+ * gradient gout[B, C_out, L_out] (the loss is sum(gout * out)).
+ *
+ * Source: "dc1d (DeformConv1d)" page, opening paragraph: the layer is plain
+ * tensor code and is trained through torch.autograd, so its gradient is the
+ * derivative of the forward as written; the "Demo notebook" note checks the
+ * offset gradient against a finite difference.  Writing v = (1-f) X(i0) + f X(i0+1)
+ * and dv(b,ci,l,k) = sum_{co in the conv group of ci} gout[b,co,l] W[co,ci-c0,k]:
+ *
+ *   grad_bias[co]        = sum_{b,l} gout[b,co,l]
+ *   grad_weight[co,c,k]  = sum_{b,l} gout[b,co,l] * m * v
+ *   grad_x[b,ci,i0]     += m (1-f) dv,   grad_x[b,ci,i0+1] += m f dv   (inside [0, L_in) only)
+ *   grad_mask[b,g,l,k]   = sum_{ci in offset group g} v dv
+ *   grad_offsets[b,g,l,k]= sum_{ci in offset group g} m (X(i0+1) - X(i0)) dv * gate
+ *
+ * Readings (listed in the design notes): floor() contributes nothing (the
+ * slope inside a unit cell is X(i0+1) - X(i0), the right-hand one at an
+ * integer position); in constrained mode the clamp passes the offset gradient
+ * when lo <= pos <= hi (bounds included, as torch.clamp does) and stops it
+ * outside (gate = 0 there); the position's float32 rounding counts as exact.
+ * Every output array may be NULL (skipped); all are float64.
+ */
+int oracle_backward(const float *x, const float *off, const float *mask, const float *w,
+                    const float *gout, int64_t B, int64_t C_in, int64_t L_in, int64_t C_out,
+                    int64_t K, int64_t L_out, int64_t stride, int64_t padding, int64_t dilation,
+                    int64_t groups, int64_t offset_groups, int unconstrained, double *gx,
+                    double *goff, double *gmask, double *gw, double *gbias)
+{
+    oracle_shape S = {B, C_in, L_in, C_out, K, L_out, stride, padding,
+                      dilation, groups, offset_groups, unconstrained};
+    if (check_shape(&S))
+        return 1;
+    const int64_t cin_g = C_in / groups, cout_g = C_out / groups;
+    const int64_t cin_per_og = C_in / offset_groups;
+
+    /* grad_x, grad_offsets, grad_mask: one (b, offset group) per iteration owns
+     * the x rows of its channels and its offset/mask entries. */
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t og = 0; og < offset_groups; ++og) {
+            for (int64_t ci = og * cin_per_og; ci < (og + 1) * cin_per_og; ++ci)
+                if (gx)
+                    for (int64_t i = 0; i < L_in; ++i)
+                        gx[(b * C_in + ci) * L_in + i] = 0.0;
+            for (int64_t l = 0; l < L_out; ++l)
+                for (int64_t k = 0; k < K; ++k) {
+                    int64_t oidx = ((b * offset_groups + og) * L_out + l) * K + k;
+                    int64_t i0;
+                    float f;
+                    double gate;
+                    sample_position(l, k, off[oidx], &S, &i0, &f, &gate);
+                    double m = mask ? (double)mask[oidx] : 1.0;
+                    double sum_off = 0.0, sum_mask = 0.0;
+                    for (int64_t ci = og * cin_per_og; ci < (og + 1) * cin_per_og; ++ci) {
+                        int64_t g = ci / cin_g, c = ci - g * cin_g;
+                        double dv = 0.0;
+                        for (int64_t co = g * cout_g; co < (g + 1) * cout_g; ++co)
+                            dv += (double)gout[(b * C_out + co) * L_out + l] *
+                                  (double)w[(co * cin_g + c) * K + k];
+                        double x0 = x_at(x, &S, b, ci, i0), x1 = x_at(x, &S, b, ci, i0 + 1);
+                        if (gx) {
+                            if (i0 >= 0 && i0 < L_in)
+                                gx[(b * C_in + ci) * L_in + i0] += m * (1.0 - (double)f) * dv;
+                            if (i0 + 1 >= 0 && i0 + 1 < L_in)
+                                gx[(b * C_in + ci) * L_in + i0 + 1] += m * (double)f * dv;
+                        }
+                        sum_off += m * (x1 - x0) * dv;
+                        sum_mask += ((1.0 - (double)f) * x0 + (double)f * x1) * dv;
+                    }
+                    if (goff)
+                        goff[oidx] = sum_off * gate;
+                    if (gmask)
+                        gmask[oidx] = sum_mask;
+                }
+        }
+
+    /* grad_weight: one (co, c) per iteration. */
+    if (gw) {
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+        for (int64_t co = 0; co < C_out; ++co)
+            for (int64_t c = 0; c < cin_g; ++c) {
+                int64_t g = co / cout_g, ci = g * cin_g + c, og = ci / cin_per_og;
+                for (int64_t k = 0; k < K; ++k) {
+                    double acc = 0.0;
+                    for (int64_t b = 0; b < B; ++b)
+                        for (int64_t l = 0; l < L_out; ++l) {
+                            int64_t oidx = ((b * offset_groups + og) * L_out + l) * K + k;
+                            int64_t i0;
+                            float f;
+                            sample_position(l, k, off[oidx], &S, &i0, &f, NULL);
+                            double v = (1.0 - (double)f) * x_at(x, &S, b, ci, i0) +
+                                       (double)f * x_at(x, &S, b, ci, i0 + 1);
+                            if (mask)
+                                v = v * (double)mask[oidx];
+                            acc += (double)gout[(b * C_out + co) * L_out + l] * v;
+                        }
+                    gw[(co * cin_g + c) * K + k] = acc;
+                }
+            }
+    }
+
+    if (gbias)
+        for (int64_t co = 0; co < C_out; ++co) {
+            double acc = 0.0;
+            for (int64_t b = 0; b < B; ++b)
+                for (int64_t l = 0; l < L_out; ++l)
+                    acc += (double)gout[(b * C_out + co) * L_out + l];
+            gbias[co] = acc;
+        }
+    return 0;
 }
