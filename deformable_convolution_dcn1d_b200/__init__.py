@@ -1,4 +1,4 @@
-"""B200 (sm_100a) forward pass of 1D deformable convolution (DeformConv1d).
+"""B200 (sm_100a) forward and backward passes of 1D deformable convolution (DeformConv1d).
 
 The computation lives in the C-ABI CUDA library ``libdcn1d.so`` (declared in
 ``include/dcn1d.h``); this package is its thin Python binding.
@@ -8,7 +8,9 @@ from ._binding import (  # noqa: F401
     DCN1D_F32,
     Dcn1dError,
     Dcn1dTensor,
+    GRADS,
     SIGNATURES,
+    dcn1d_backward,
     dcn1d_device_status,
     dcn1d_forward,
     dcn1d_forward_noalloc,

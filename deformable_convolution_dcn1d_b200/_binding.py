@@ -61,6 +61,11 @@ SIGNATURES = [
     ("dcn1d_set_timing_events", None, [_P, _P]),
     ("dcn1d_forward_noalloc", _INT,
      [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _P]),
+    ("dcn1d_backward_workspace_size", _I64,
+     [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _T, _T, _T, _T]),
+    ("dcn1d_backward", _INT,
+     [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _T, _T, _T, _T, _P,
+      ctypes.c_size_t, _P]),
 ]
 
 
@@ -199,6 +204,55 @@ def dcn1d_forward(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=
     if st != 0:
         raise Dcn1dError(st, "dcn1d_forward")
     return out
+
+
+GRADS = ("x", "offsets", "mask", "weight", "bias")
+
+
+def dcn1d_backward(x, offsets, mask, weight, grad_out, stride=1, padding=0, dilation=1,
+                   groups=1, offset_groups=1, unconstrained=False, wanted=GRADS, grads=None,
+                   workspace=None, stream=None):
+    """Gradients of sum(grad_out * forward) through the C ABI.
+
+    Returns a dict {name: tensor} for the names in ``wanted`` (a subset of "x", "offsets",
+    "mask", "weight", "bias"; "mask" only when a mask is given), each shaped like its
+    input (bias: [C_out]) in the inputs' dtype.  ``grads`` may supply some of those
+    tensors (they are overwritten); the rest, and the scratch the call needs, are
+    allocated with torch unless a uint8 CUDA tensor ``workspace`` is given.  Runs on
+    ``stream``; does not synchronise.
+    """
+    wanted = tuple(n for n in wanted if n != "mask" or mask is not None)
+    unknown = set(wanted) - set(GRADS)
+    if unknown:
+        raise ValueError(f"unknown gradients {sorted(unknown)}")
+    dev = _check_device((x, offsets, mask, weight, grad_out))
+    like = {"x": x, "offsets": offsets, "mask": mask, "weight": weight}
+    out = dict(grads or {})
+    for n in wanted:
+        if n not in out:
+            shape = (weight.shape[0],) if n == "bias" else like[n].shape
+            out[n] = torch.empty(shape, dtype=x.dtype, device=dev)
+    ins = [_desc(t) for t in (x, offsets, mask, weight, grad_out)]
+    gd = [_desc(out.get(n)) for n in GRADS]
+    lib = load()
+    refs = [_ref(d) for d in ins] + [_ref(d) for d in gd]
+    args = (stride, padding, dilation, groups, offset_groups, int(bool(unconstrained)))
+    with torch.cuda.device(dev):
+        need = int(lib.dcn1d_backward_workspace_size(*refs[:5], *args, *refs[5:]))
+        if need < 0:
+            raise Dcn1dError(-need, "dcn1d_backward_workspace_size")
+        ws_ptr, ws_bytes = None, 0
+        if need > 0:
+            if workspace is None:
+                workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+            if workspace.numel() < need or workspace.dtype != torch.uint8:
+                raise ValueError(f"workspace must be a uint8 tensor of >= {need} bytes")
+            ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+        st = lib.dcn1d_backward(*refs[:5], *args, *refs[5:], _P(ws_ptr), ws_bytes,
+                                _P(_stream_ptr(stream, dev)))
+    if st != 0:
+        raise Dcn1dError(st, "dcn1d_backward")
+    return {n: out[n] for n in wanted}
 
 
 def dcn1d_forward_noalloc(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=1,

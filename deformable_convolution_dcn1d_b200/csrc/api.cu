@@ -144,6 +144,55 @@ int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor 
     return DCN1D_OK;
 }
 
+// Validation of a backward call: the forward's checks with grad_out in the place
+// of out, then every wanted gradient against its input's dtype and shape.
+int validate_backward(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor *mask,
+                      const dcn1d_tensor *w, const dcn1d_tensor *gout, int64_t stride,
+                      int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
+                      int unconstrained, const dcn1d_tensor *gx, const dcn1d_tensor *goff,
+                      const dcn1d_tensor *gmask, const dcn1d_tensor *gw, const dcn1d_tensor *gbias,
+                      Problem *P, BackwardGrads *G) {
+    int st = validate(x, off, mask, w, nullptr, stride, padding, dilation, groups, offset_groups,
+                      unconstrained, gout, P);
+    if (st != DCN1D_OK)
+        return st;
+    auto like = [&](const dcn1d_tensor *g, const dcn1d_tensor *in, int nd) -> int {
+        if (!g)
+            return DCN1D_OK;
+        if (!in)
+            return DCN1D_ERR_ARG;   // a mask gradient without a mask
+        const int s2 = check_desc(g, nd);
+        if (s2 != DCN1D_OK)
+            return s2;
+        if (g->dtype != x->dtype)
+            return DCN1D_ERR_DTYPE;
+        for (int i = 0; i < nd; ++i)
+            if (g->shape[i] != in->shape[i])
+                return DCN1D_ERR_SHAPE;
+        return DCN1D_OK;
+    };
+    if ((st = like(gx, x, 3)) || (st = like(goff, off, 4)) || (st = like(gmask, mask, 4)) ||
+        (st = like(gw, w, 3)))
+        return st;
+    if (gbias) {
+        if ((st = check_desc(gbias, 1)) != DCN1D_OK)
+            return st;
+        if (gbias->dtype != x->dtype)
+            return DCN1D_ERR_DTYPE;
+        if (gbias->shape[0] != P->C_out)
+            return DCN1D_ERR_SHAPE;
+    }
+    if ((int64_t)P->B * P->groups > 65535)   // one GEMM grid slice per (batch, group)
+        return DCN1D_ERR_UNSUPPORTED;
+    G->gout = gout->data;
+    G->x = gx ? gx->data : nullptr;
+    G->off = goff ? goff->data : nullptr;
+    G->mask = gmask ? gmask->data : nullptr;
+    G->w = gw ? gw->data : nullptr;
+    G->bias = gbias ? gbias->data : nullptr;
+    return DCN1D_OK;
+}
+
 }  // namespace
 
 void timing_begin(cudaStream_t stream) {
@@ -280,6 +329,52 @@ int64_t dcn1d_forward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *
     if (st != DCN1D_OK)
         return -st;
     return (int64_t)workspace_bytes(P);
+}
+
+int64_t dcn1d_backward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                                      const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                                      const dcn1d_tensor *grad_out, int64_t stride,
+                                      int64_t padding, int64_t dilation, int64_t groups,
+                                      int64_t offset_groups, int unconstrained,
+                                      const dcn1d_tensor *grad_x, const dcn1d_tensor *grad_offsets,
+                                      const dcn1d_tensor *grad_mask,
+                                      const dcn1d_tensor *grad_weight,
+                                      const dcn1d_tensor *grad_bias) {
+    Problem P;
+    BackwardGrads G;
+    const int st = validate_backward(x, offsets, mask, weight, grad_out, stride, padding,
+                                     dilation, groups, offset_groups, unconstrained, grad_x,
+                                     grad_offsets, grad_mask, grad_weight, grad_bias, &P, &G);
+    if (st != DCN1D_OK)
+        return -(int64_t)st;
+    return (int64_t)backward_workspace(P, G);
+}
+
+int dcn1d_backward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
+                   const dcn1d_tensor *weight, const dcn1d_tensor *grad_out, int64_t stride,
+                   int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
+                   int unconstrained, dcn1d_tensor *grad_x, dcn1d_tensor *grad_offsets,
+                   dcn1d_tensor *grad_mask, dcn1d_tensor *grad_weight, dcn1d_tensor *grad_bias,
+                   void *workspace, size_t workspace_bytes, void *stream) {
+    g_last_launches = 0;
+    Problem P;
+    BackwardGrads G;
+    const int st = validate_backward(x, offsets, mask, weight, grad_out, stride, padding,
+                                     dilation, groups, offset_groups, unconstrained, grad_x,
+                                     grad_offsets, grad_mask, grad_weight, grad_bias, &P, &G);
+    if (st != DCN1D_OK)
+        return st;
+    const size_t need = backward_workspace(P, G);
+    if (need > 0 && !workspace)
+        return DCN1D_ERR_NULL;
+    if (need > workspace_bytes || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return DCN1D_ERR_ARG;
+    int launches = 0;
+    if (launch_backward(P, G, workspace, static_cast<cudaStream_t>(stream), &launches) !=
+        cudaSuccess)
+        return DCN1D_ERR_LAUNCH;
+    g_last_launches = launches;
+    return DCN1D_OK;
 }
 
 const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor *offsets,

@@ -1,0 +1,386 @@
+// Backward pass of the 1D deformable convolution: gradients of sum(grad_out * y)
+// with respect to x, the offsets, the mask, the weight and the bias.
+//
+// The layer is trained through autograd on the forward as written ("dc1d
+// (DeformConv1d)" page, opening paragraph; its demo notebook checks the offset
+// gradient against a finite difference), so the backward is that derivative.
+// With v = (1-f) x[i0] + f x[i0+1] the sampled value of tap (l, k) in channel
+// ci and dv = sum_co W[co, ci, k] grad_out[b, co, l] over the conv group:
+//   grad_weight[co, c, k] = sum_{b,l} grad_out[b, co, l] * m * v
+//   grad_x[b, ci, i0]    += m (1-f) dv,    grad_x[b, ci, i0+1] += m f dv
+//   grad_mask[b, g, l, k] = sum_{ci in offset group g} v dv
+//   grad_offsets         = sum_{ci in g} m (x[i0+1] - x[i0]) dv   (0 where the
+//                          constrained clamp moved the position)
+//   grad_bias[co]         = sum_{b,l} grad_out[b, co, l]
+//
+// Kernels, all fp32 arithmetic whatever the input type:
+//  1. dcols[b, (c,k), l] = sum_co W[co, (c,k)] grad_out[b, co, l]: a batched GEMM
+//     per (batch, conv group) on CUDA cores;
+//  2. the sampling gradient: one thread per (batch, 16-channel chunk, offset
+//     group, tap, position) recomputes the tap's position once, then for its
+//     channels scatters grad_x, sums the offset and mask gradients (atomics
+//     into fp32 scratch: the order of those sums is not fixed) and writes the
+//     sampled columns m*v that the weight gradient needs;
+//  3. grad_weight = sum_b grad_out[b] cols[b]^T: the same GEMM kernel, summing
+//     over the batch inside the tile loop (a fixed order);
+//  4. grad_bias: one block per channel, a fixed-order tree reduction;
+//  5. the fp32 scratch of grad_x / grad_offsets / grad_mask is written out in
+//     the input type.
+#include <string.h>
+
+#include "common.cuh"
+#include "sampler.cuh"
+
+namespace dcn1d {
+
+namespace {
+
+constexpr int kBM = 64, kBN = 64, kBKd = 16;   // GEMM tile
+constexpr int kChunk = 16;                     // channels per sampling-gradient thread
+
+// C[zb, zg][m][n] = sum_{r < R} sum_{kk < Kd} A[zb, zg, r][m][kk] * B[zb, zg, r][kk][n]
+// with blockIdx.z = zb * ng + zg; every stride in elements.
+struct GemmArgs {
+    int M, N, Kd, R, ng;
+    int64_t a_sm, a_sk, a_sb, a_sg, a_sr;
+    int64_t b_sk, b_sn, b_sb, b_sg, b_sr;
+    int64_t c_sm, c_sn, c_sb, c_sg;
+};
+
+// 64x64 output tile per 256 threads, 4x4 per thread; A_MC: A is contiguous along m
+// (else along kk), B_NC: B is contiguous along n (else along kk) -- the tile loads
+// run along the contiguous direction.
+template <class TA, class TB, class TC, bool A_MC, bool B_NC>
+__global__ void __launch_bounds__(256) gemm_kernel(const TA *__restrict__ A,
+                                                   const TB *__restrict__ B, TC *__restrict__ C,
+                                                   const GemmArgs g) {
+    __shared__ __align__(16) float As[kBKd][kBM + 4];
+    __shared__ __align__(16) float Bs[kBKd][kBN + 4];
+    const int tid = threadIdx.x;
+    const int m0 = blockIdx.y * kBM, n0 = blockIdx.x * kBN;
+    const int zb = blockIdx.z / g.ng, zg = blockIdx.z - zb * g.ng;
+    const TA *Az = A + zb * g.a_sb + zg * g.a_sg;
+    const TB *Bz = B + zb * g.b_sb + zg * g.b_sg;
+    const int tm = (tid / 16) * 4, tn = (tid % 16) * 4;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            acc[i][j] = 0.0f;
+    for (int r = 0; r < g.R; ++r) {
+        const TA *Ar = Az + r * g.a_sr;
+        const TB *Br = Bz + r * g.b_sr;
+        for (int k0 = 0; k0 < g.Kd; k0 += kBKd) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int e = tid + i * 256;
+                const int m = A_MC ? e % kBM : e / kBKd;
+                const int kk = A_MC ? e / kBM : e % kBKd;
+                const bool in = m0 + m < g.M && k0 + kk < g.Kd;
+                As[kk][m] = in ? to_f32(Ar[(int64_t)(m0 + m) * g.a_sm + (int64_t)(k0 + kk) * g.a_sk])
+                               : 0.0f;
+                const int n = B_NC ? e % kBN : e / kBKd;
+                const int kb = B_NC ? e / kBN : e % kBKd;
+                const bool inb = n0 + n < g.N && k0 + kb < g.Kd;
+                Bs[kb][n] = inb ? to_f32(Br[(int64_t)(k0 + kb) * g.b_sk + (int64_t)(n0 + n) * g.b_sn])
+                                : 0.0f;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int kk = 0; kk < kBKd; ++kk) {
+                const float4 a = *reinterpret_cast<const float4 *>(&As[kk][tm]);
+                const float4 b = *reinterpret_cast<const float4 *>(&Bs[kk][tn]);
+                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        acc[i][j] = __fmaf_rn(av[i], bv[j], acc[i][j]);
+            }
+            __syncthreads();
+        }
+    }
+    TC *Cz = C + zb * g.c_sb + zg * g.c_sg;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (m0 + tm + i < g.M && n0 + tn + j < g.N)
+                Cz[(int64_t)(m0 + tm + i) * g.c_sm + (int64_t)(n0 + tn + j) * g.c_sn] =
+                    from_f32<TC>(acc[i][j]);
+}
+
+template <class TA, class TB, class TC, bool A_MC, bool B_NC>
+cudaError_t run_gemm(const TA *A, const TB *B, TC *C, const GemmArgs &g, int nz,
+                     cudaStream_t stream) {
+    const dim3 grid((g.N + kBN - 1) / kBN, (g.M + kBM - 1) / kBM, nz);
+    gemm_kernel<TA, TB, TC, A_MC, B_NC><<<grid, 256, 0, stream>>>(A, B, C, g);
+    return cudaGetLastError();
+}
+
+struct SampArgs {
+    Problem P;
+    int nchunk;                  // channel chunks per offset group
+    const float *dcols;          // [B][C_in*K][L_out] or NULL
+    float *cols;                 // [B][C_in*K][L_out] or NULL
+    float *gx, *goff, *gmask;    // fp32 scratch, each may be NULL
+};
+
+// Thread = (b, chunk, offset group, k, l), l fastest.
+template <class T, bool MASK>
+__global__ void __launch_bounds__(256) sample_grad_kernel(const SampArgs a) {
+    const Problem &P = a.P;
+    const int64_t n = (int64_t)P.B * a.nchunk * P.offset_groups * P.K * P.L_out;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n)
+        return;
+    const int l = (int)(t % P.L_out);
+    int64_t r = t / P.L_out;
+    const int k = (int)(r % P.K);
+    r /= P.K;
+    const int og = (int)(r % P.offset_groups);
+    r /= P.offset_groups;
+    const int chunk = (int)(r % a.nchunk);
+    const int b = (int)(r / a.nchunk);
+
+    const int start = l * P.stride - P.padding;
+    const int64_t oidx = (((int64_t)b * P.offset_groups + og) * P.L_out + l) * P.K + k;
+    const float off = ld_f32(static_cast<const T *>(P.off) + oidx);
+    const float m = MASK ? ld_f32(static_cast<const T *>(P.mask) + oidx) : 1.0f;
+    const int span = P.dilation * (P.K - 1);
+    const float raw = __fadd_rn(__int2float_rn(start + k * P.dilation), off);
+    // The clamp passes the gradient inside its closed range (NaN: no gradient).
+    const bool gate = P.unconstrained ||
+                      (raw >= __int2float_rn(start) && raw <= __int2float_rn(start + span));
+    const Tap tp = sample_tap(start, k, P.dilation, span, off, P.unconstrained);
+    const float mf = __fmul_rn(m, tp.f), m1f = __fmul_rn(m, __fsub_rn(1.0f, tp.f));
+    const bool in0 = tp.i0 >= 0 && tp.i0 < P.L_in;
+    const bool in1 = tp.i0 >= -1 && tp.i0 < P.L_in - 1;
+
+    const int c_begin = og * P.cin_per_og + chunk * kChunk;
+    const int c_end = min(c_begin + kChunk, (og + 1) * P.cin_per_og);
+    float s_off = 0.0f, s_mask = 0.0f;
+    for (int ci = c_begin; ci < c_end; ++ci) {
+        const T *row = static_cast<const T *>(P.x) + ((int64_t)b * P.C_in + ci) * P.L_in;
+        const float x0 = in0 ? ld_f32(row + tp.i0) : 0.0f;
+        const float x1 = in1 ? ld_f32(row + tp.i0 + 1) : 0.0f;
+        const float v = __fadd_rn(__fmul_rn(__fsub_rn(1.0f, tp.f), x0), __fmul_rn(tp.f, x1));
+        const int64_t cidx = (((int64_t)b * P.C_in + ci) * P.K + k) * P.L_out + l;
+        if (a.cols)
+            a.cols[cidx] = __fmul_rn(m, v);
+        if (a.dcols) {
+            const float dv = a.dcols[cidx];
+            if (a.gx) {
+                float *gxr = a.gx + ((int64_t)b * P.C_in + ci) * P.L_in;
+                if (in0)
+                    atomicAdd(gxr + tp.i0, __fmul_rn(m1f, dv));
+                if (in1)
+                    atomicAdd(gxr + tp.i0 + 1, __fmul_rn(mf, dv));
+            }
+            s_off = __fmaf_rn(__fmul_rn(m, __fsub_rn(x1, x0)), dv, s_off);
+            s_mask = __fmaf_rn(v, dv, s_mask);
+        }
+    }
+    if (a.goff && gate)
+        atomicAdd(a.goff + oidx, s_off);
+    if (a.gmask)
+        atomicAdd(a.gmask + oidx, s_mask);
+}
+
+// grad_bias[co] = sum over (b, l) of grad_out[b, co, l]: one block per channel,
+// a fixed-order reduction.
+template <class T>
+__global__ void __launch_bounds__(256) bias_grad_kernel(const T *gout, T *gbias, int B,
+                                                        int C_out, int L_out) {
+    __shared__ float part[256];
+    const int co = blockIdx.x;
+    float s = 0.0f;
+    for (int64_t i = threadIdx.x; i < (int64_t)B * L_out; i += blockDim.x) {
+        const int b = (int)(i / L_out), l = (int)(i - (int64_t)b * L_out);
+        s = __fadd_rn(s, ld_f32(gout + ((int64_t)b * C_out + co) * L_out + l));
+    }
+    part[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if ((int)threadIdx.x < w)
+            part[threadIdx.x] = __fadd_rn(part[threadIdx.x], part[threadIdx.x + w]);
+        __syncthreads();
+    }
+    if (threadIdx.x == 0)
+        gbias[co] = from_f32<T>(part[0]);
+}
+
+template <class T>
+__global__ void __launch_bounds__(256) write_out_kernel(const float *src, T *dst, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = from_f32<T>(src[i]);
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct WsLayout {
+    size_t dcols, cols, gx, goff, gmask, total;   // byte offsets (SIZE_MAX: not used)
+};
+
+WsLayout ws_layout(const Problem &P, const BackwardGrads &G) {
+    WsLayout w;
+    const size_t ncol = (size_t)P.B * P.C_in * P.K * P.L_out * 4;
+    const size_t noff = (size_t)P.B * P.offset_groups * P.L_out * P.K * 4;
+    const bool need_dcols = G.x || G.off || G.mask;
+    size_t at = 0;
+    w.dcols = need_dcols ? at : SIZE_MAX;
+    at += need_dcols ? align256(ncol) : 0;
+    w.cols = G.w ? at : SIZE_MAX;
+    at += G.w ? align256(ncol) : 0;
+    w.gx = G.x ? at : SIZE_MAX;
+    at += G.x ? align256((size_t)P.B * P.C_in * P.L_in * 4) : 0;
+    w.goff = G.off ? at : SIZE_MAX;
+    at += G.off ? align256(noff) : 0;
+    w.gmask = G.mask ? at : SIZE_MAX;
+    at += G.mask ? align256(noff) : 0;
+    w.total = at;
+    return w;
+}
+
+unsigned grid_1d(int64_t n) {
+    const int64_t want = (n + 255) / 256;
+    return (unsigned)(want < 65535LL * 16 ? want : 65535LL * 16);
+}
+
+template <class T>
+cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cudaStream_t s,
+                         int *launches) {
+    const WsLayout L = ws_layout(P, G);
+    unsigned char *wsb = static_cast<unsigned char *>(ws);
+    float *dcols = L.dcols != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.dcols) : nullptr;
+    float *cols = L.cols != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.cols) : nullptr;
+    float *gx = L.gx != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.gx) : nullptr;
+    float *goff = L.goff != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.goff) : nullptr;
+    float *gmask = L.gmask != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.gmask) : nullptr;
+    const T *w = static_cast<const T *>(P.w);
+    const T *gout = static_cast<const T *>(G.gout);
+    const int Kg = P.cin_g * P.K;
+    const bool want_dcols = G.x || G.off || G.mask;   // (scratch pointers are NULL when
+    const bool want_cols = G.w != nullptr;           //  their size is zero)
+    cudaError_t e;
+    int n = 0;
+    const int64_t nx = (int64_t)P.B * P.C_in * P.L_in;
+    const int64_t noff = (int64_t)P.B * P.offset_groups * P.L_out * P.K;
+    if (gx && (e = cudaMemsetAsync(gx, 0, nx * 4, s)) != cudaSuccess)
+        return e;
+    if (goff && (e = cudaMemsetAsync(goff, 0, noff * 4, s)) != cudaSuccess)
+        return e;
+    if (gmask && (e = cudaMemsetAsync(gmask, 0, noff * 4, s)) != cudaSuccess)
+        return e;
+
+    if (want_dcols && P.B > 0) {   // 1. dcols[b][g*Kg + m][l] = sum_co W[g*cout_g + co][m] * gout[b][g*cout_g + co][l]
+        GemmArgs g;
+        memset(&g, 0, sizeof(g));
+        g.M = Kg;
+        g.N = P.L_out;
+        g.Kd = P.cout_g;
+        g.R = 1;
+        g.ng = P.groups;
+        g.a_sm = 1;
+        g.a_sk = Kg;
+        g.a_sg = (int64_t)P.cout_g * Kg;
+        g.b_sk = P.L_out;
+        g.b_sn = 1;
+        g.b_sb = (int64_t)P.C_out * P.L_out;
+        g.b_sg = (int64_t)P.cout_g * P.L_out;
+        g.c_sm = P.L_out;
+        g.c_sn = 1;
+        g.c_sb = (int64_t)P.C_in * P.K * P.L_out;
+        g.c_sg = (int64_t)Kg * P.L_out;
+        if ((e = run_gemm<T, T, float, true, true>(w, gout, dcols, g, P.B * P.groups, s)) !=
+            cudaSuccess)
+            return e;
+        ++n;
+    }
+    if (want_dcols || want_cols) {   // 2. sampling gradient and sampled columns
+        SampArgs a;
+        memset(&a, 0, sizeof(a));
+        a.P = P;
+        a.nchunk = (P.cin_per_og + kChunk - 1) / kChunk;
+        a.dcols = dcols;
+        a.cols = cols;
+        a.gx = gx;
+        a.goff = goff;
+        a.gmask = gmask;
+        const int64_t nt = (int64_t)P.B * a.nchunk * P.offset_groups * P.K * P.L_out;
+        const unsigned blocks = (unsigned)((nt + 255) / 256);
+        if (nt == 0) {
+            // empty batch: no columns, no sampling gradient
+        } else if (P.mask)
+            sample_grad_kernel<T, true><<<blocks, 256, 0, s>>>(a);
+        else
+            sample_grad_kernel<T, false><<<blocks, 256, 0, s>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+        n += nt > 0;
+    }
+    if (want_cols) {   // 3. gW (zeros for an empty batch: no term is summed)[g*cout_g + co][m] = sum_b sum_l gout[b][g*cout_g + co][l] * cols[b][g*Kg + m][l]
+        GemmArgs g;
+        memset(&g, 0, sizeof(g));
+        g.M = P.cout_g;
+        g.N = Kg;
+        g.Kd = P.L_out;
+        g.R = P.B;
+        g.ng = P.groups;
+        g.a_sm = P.L_out;
+        g.a_sk = 1;
+        g.a_sg = (int64_t)P.cout_g * P.L_out;
+        g.a_sr = (int64_t)P.C_out * P.L_out;
+        g.b_sk = 1;
+        g.b_sn = P.L_out;
+        g.b_sg = (int64_t)Kg * P.L_out;
+        g.b_sr = (int64_t)P.C_in * P.K * P.L_out;
+        g.c_sm = Kg;
+        g.c_sn = 1;
+        g.c_sg = (int64_t)P.cout_g * Kg;
+        if ((e = run_gemm<T, float, T, false, false>(gout, cols, static_cast<T *>(G.w), g,
+                                                       P.groups, s)) != cudaSuccess)
+            return e;
+        ++n;
+    }
+    if (G.bias) {   // 4.
+        bias_grad_kernel<T><<<P.C_out, 256, 0, s>>>(gout, static_cast<T *>(G.bias), P.B, P.C_out,
+                                                    P.L_out);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+        ++n;
+    }
+    // 5. scratch -> outputs in the input type
+    if (gx && nx > 0) {
+        write_out_kernel<T><<<grid_1d(nx), 256, 0, s>>>(gx, static_cast<T *>(G.x), nx);
+        ++n;
+    }
+    if (goff && noff > 0) {
+        write_out_kernel<T><<<grid_1d(noff), 256, 0, s>>>(goff, static_cast<T *>(G.off), noff);
+        ++n;
+    }
+    if (gmask && noff > 0) {
+        write_out_kernel<T><<<grid_1d(noff), 256, 0, s>>>(gmask, static_cast<T *>(G.mask), noff);
+        ++n;
+    }
+    *launches = n;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t backward_workspace(const Problem &P, const BackwardGrads &G) {
+    return ws_layout(P, G).total;
+}
+
+cudaError_t launch_backward(const Problem &P, const BackwardGrads &G, void *workspace,
+                            cudaStream_t stream, int *launches) {
+    *launches = 0;
+    return P.dtype == DCN1D_BF16
+               ? run_backward<__nv_bfloat16>(P, G, workspace, stream, launches)
+               : run_backward<float>(P, G, workspace, stream, launches);
+}
+
+}  // namespace dcn1d

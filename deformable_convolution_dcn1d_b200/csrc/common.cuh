@@ -61,6 +61,15 @@ int tc_tf32_launches(const Problem &P);
 cudaError_t launch_tc_tf32(const Problem &P, void *workspace, cudaStream_t stream);
 bool tc_bf16_supported(const Problem &P);
 cudaError_t launch_tc_bf16(const Problem &P, cudaStream_t stream);
+// Backward (backward.cu): the upstream gradient and the wanted gradients (each
+// output NULL when not wanted), all in the problem's dtype and its inputs' shapes.
+struct BackwardGrads {
+    const void *gout;                    // [B, C_out, L_out]
+    void *x, *off, *mask, *w, *bias;     // outputs
+};
+size_t backward_workspace(const Problem &P, const BackwardGrads &G);
+cudaError_t launch_backward(const Problem &P, const BackwardGrads &G, void *workspace,
+                            cudaStream_t stream, int *launches);
 cudaError_t launch_sample_index(const void *off, int dtype, int B, int G, int L_out, int K,
                                 int L_in, int stride, int padding, int dilation,
                                 int unconstrained, int32_t *i0, float *frac,

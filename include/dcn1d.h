@@ -115,10 +115,10 @@ int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1
 /*
  * Scratch memory (bytes) the fastest path for these arguments needs, or 0 when
  * it needs none; a negative value is minus the status code of invalid
- * arguments.  Host only.  The fp32 tensor-core path needs scratch: the weight
- * split into tf32 high and low parts (2 * C_out * (C_in/groups) * K floats)
- * and, when the reduction is split across CTAs, the fp32 partial sums
- * (splits * B * C_out * L_out floats).
+ * arguments.  Host only.  The fp32 tensor-core path needs scratch: the low
+ * tf32 part of the weight (C_out * (C_in/groups) * K floats; the weight itself
+ * serves as the high part) and, when the reduction is split across CTAs, the
+ * fp32 partial sums (splits * B * C_out * L_out floats).
  */
 int64_t dcn1d_forward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
                                      const dcn1d_tensor *mask, const dcn1d_tensor *weight,
@@ -176,6 +176,57 @@ int dcn1d_forward_noalloc(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
                           const dcn1d_tensor *bias, int64_t stride, int64_t padding,
                           int64_t dilation, int64_t groups, int64_t offset_groups,
                           int unconstrained, dcn1d_tensor *out, void *stream);
+
+/*
+ * Backward pass: the gradients of sum(grad_out * forward(...)) with respect to
+ * x, offsets, mask, weight and bias.  The pages train the layer through
+ * autograd on the forward as written (the dc1d page, opening paragraph; its
+ * demo notebook checks the offset gradient against a finite difference), so
+ * these are that derivative: with v = (1-f) x[i0] + f x[i0+1] and
+ * dv = sum_co weight[co, c, k] * grad_out[b, co, l] over the conv group,
+ *   grad_weight[co,c,k] = sum_{b,l} grad_out[b,co,l] * m * v
+ *   grad_x[b,ci,i0] += m (1-f) dv,  grad_x[b,ci,i0+1] += m f dv  (in range only)
+ *   grad_mask[b,g,l,k]  = sum_{ci in offset group g} v * dv
+ *   grad_offsets[b,g,l,k] = sum_{ci in g} m (x[i0+1] - x[i0]) dv, and 0 where
+ *                           the constrained clamp moved the position (a
+ *                           position exactly on a bound passes the gradient)
+ *   grad_bias[co]       = sum_{b,l} grad_out[b,co,l]
+ * floor() contributes nothing (inside a unit cell the slope is x[i0+1]-x[i0]).
+ *
+ * Arguments: the forward's inputs (bias is not needed), grad_out [B, C_out,
+ * L_out] in their dtype, and the gradients wanted, each NULL when not wanted
+ * and otherwise shaped like its input in the same dtype (grad_mask needs a
+ * mask: DCN1D_ERR_ARG otherwise).  Every wanted gradient is overwritten.
+ * Arithmetic is fp32 for both dtypes; grad_x, grad_offsets and grad_mask are
+ * sums of atomic fp32 additions, so their low bits may differ between calls;
+ * grad_weight and grad_bias are summed in a fixed order.
+ *
+ * Scratch: `workspace` (256-byte aligned, owned by the caller, used only by the
+ * work enqueued on `stream`) of at least dcn1d_backward_workspace_size() bytes:
+ * fp32 column buffers of B * C_in * K * L_out floats (one for the gradient
+ * sampled columns when any of grad_x / grad_offsets / grad_mask is wanted, one
+ * for the sampled columns when grad_weight is wanted) plus fp32 accumulators of
+ * grad_x, grad_offsets and grad_mask.  Too small or misaligned:
+ * DCN1D_ERR_ARG; NULL with a non-zero need: DCN1D_ERR_NULL.
+ * Other errors as for dcn1d_forward; B * groups above 65535 is
+ * DCN1D_ERR_UNSUPPORTED.
+ */
+int64_t dcn1d_backward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                                      const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                                      const dcn1d_tensor *grad_out, int64_t stride,
+                                      int64_t padding, int64_t dilation, int64_t groups,
+                                      int64_t offset_groups, int unconstrained,
+                                      const dcn1d_tensor *grad_x, const dcn1d_tensor *grad_offsets,
+                                      const dcn1d_tensor *grad_mask,
+                                      const dcn1d_tensor *grad_weight,
+                                      const dcn1d_tensor *grad_bias);
+
+int dcn1d_backward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
+                   const dcn1d_tensor *weight, const dcn1d_tensor *grad_out, int64_t stride,
+                   int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
+                   int unconstrained, dcn1d_tensor *grad_x, dcn1d_tensor *grad_offsets,
+                   dcn1d_tensor *grad_mask, dcn1d_tensor *grad_weight, dcn1d_tensor *grad_bias,
+                   void *workspace, size_t workspace_bytes, void *stream);
 
 /* A static, human-readable name of a status code ("DCN1D_OK", ...). Never NULL. */
 const char *dcn1d_status_string(int status);
