@@ -12,7 +12,8 @@ synchronisation on both sides of the K timed steps, and the time is the max over
 Under torchrun each rank runs its own batch (weak scaling, no collective on the data path).
 
 ``--impl reference`` times the CPU oracle instead (rank 0 only), on bounded samples of the
-same workload.
+same workload.  ``--pass backward`` prints one line for the backward pass instead (all
+gradients of one batch per step; the work counted is its two contractions).
 """
 from __future__ import annotations
 
@@ -32,6 +33,7 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "DeformConv1d forward TFLOP/s (HBM GB/s if depthwise) as % of B200 roofline"
+METRIC_BACKWARD = "DeformConv1d backward TFLOP/s as % of B200 roofline"
 DEFAULT_WORKLOAD = "usage_f32"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -395,6 +397,89 @@ def run_ours(args, w: W.Workload, peaks: dict, want_cpu: bool):
     return line if rank == 0 else None
 
 
+# ------------------------------------------------------------------ the backward pass
+
+def time_oracle_backward(w: W.Workload, host: dict, gout: torch.Tensor):
+    """The oracle's backward on a batch-1 slice of the workload: TFLOP/s, seconds, threads."""
+    import oracle
+    w1 = w.with_batch(1)
+    sl = {k: (v[:1] if (v is not None and k in ("x", "offsets", "mask")) else v)
+          for k, v in host.items()}
+    t0 = time.perf_counter()
+    oracle.backward(sl["x"], sl["offsets"], sl["mask"], sl["weight"], gout[:1], w.stride,
+                    w.padding, w.dilation, w.groups, w.offset_groups, w.unconstrained)
+    dt = time.perf_counter() - t0
+    return 2 * w1.flops() / dt / 1e12, dt, oracle.threads()
+
+
+def run_backward_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
+    """One backward step = all five gradients of one batch; the work counted is the two
+    contractions (2x the forward's flops); the rest (sampling gradient) is overhead."""
+    import deformable_convolution_dcn1d_b200 as dcn
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dcn.load()
+    host = W.make_inputs(w, seed=rank)
+    gout_h = torch.randn(w.B, w.C_out, w.L_out,
+                         generator=torch.Generator().manual_seed(100 + rank)).to(host["x"].dtype)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in host.items()}
+    gout = gout_h.to(dev)
+    wanted = tuple(n for n in dcn.GRADS if n != "mask" or d["mask"] is not None)
+    like = {"x": d["x"], "offsets": d["offsets"], "mask": d["mask"], "weight": d["weight"]}
+    grads = {n: torch.empty((w.C_out,) if n == "bias" else like[n].shape, dtype=d["x"].dtype,
+                            device=dev) for n in wanted}
+    args_c = (w.stride, w.padding, w.dilation, w.groups, w.offset_groups, w.unconstrained)
+    need = dcn.dcn1d_backward_workspace_size(d["x"], d["offsets"], d["mask"], d["weight"], gout,
+                                             *args_c, wanted=wanted)
+    scratch = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        dcn.dcn1d_backward(d["x"], d["offsets"], d["mask"], d["weight"], gout, *args_c,
+                           wanted=wanted, grads=grads, workspace=scratch, stream=stream)
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    launches = dcn.dcn1d_last_launch_count()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(ws)
+    ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), ws) / args.steps
+    per_gpu = 2 * w.flops() / (ms / 1e3) / 1e12
+    line = {"metric": METRIC_BACKWARD, "value": per_gpu * ws, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded, shapes and distributions of the named workload)",
+            "config": workload_config(w, "backward", ws,
+                                      l2="flushed between steps (256 MiB write outside the timed events)"),
+            "roofline": {"bound": "alu", "achieved": per_gpu, "peak": ALU_F32_TFLOPS,
+                         "unit": "TFLOP/s", "frac": per_gpu / ALU_F32_TFLOPS, "traffic": None,
+                         "kernel": "backward: two CUDA-core fp32 GEMMs + sampling gradient",
+                         "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz",
+                         "launches_per_step": launches,
+                         "timing": "CUDA events around the whole backward call, per step"},
+            "clocks": clk.summary(), "gpu_launches": launches * args.steps,
+            "workspace_bytes": need}
+    if want_cpu and ws == 1 and rank == 0:
+        v, dt, cores = time_oracle_backward(w, host, gout_h)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": f"all gradients of batch element 0 ({dt:.1f} s)"}
+    return line if rank == 0 else None
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -405,6 +490,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+                    help="time the forward (the default line) or the backward pass")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (small cases for profiling)")
     args = ap.parse_args()
@@ -432,7 +519,8 @@ def main():
     peaks = load_peaks()
     try:
         for name in names:
-            line = run_ours(args, pick(name), peaks, want_cpu=not args.no_cpu_baseline)
+            run = run_backward_pass if args.which == "backward" else run_ours
+            line = run(args, pick(name), peaks, want_cpu=not args.no_cpu_baseline)
             if line is not None:
                 print(json.dumps(line), flush=True)
     finally:

@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     GRADS,
     SIGNATURES,
     dcn1d_backward,
+    dcn1d_backward_workspace_size,
     dcn1d_device_status,
     dcn1d_forward,
     dcn1d_forward_noalloc,

@@ -255,6 +255,37 @@ def dcn1d_backward(x, offsets, mask, weight, grad_out, stride=1, padding=0, dila
     return {n: out[n] for n in wanted}
 
 
+def dcn1d_backward_workspace_size(x, offsets, mask, weight, grad_out, stride=1, padding=0,
+                                  dilation=1, groups=1, offset_groups=1, unconstrained=False,
+                                  wanted=GRADS) -> int:
+    """Bytes of scratch dcn1d_backward needs for these arguments and wanted gradients."""
+    wanted = tuple(n for n in wanted if n != "mask" or mask is not None)
+    like = {"x": x, "offsets": offsets, "mask": mask, "weight": weight}
+    probe = {n: torch.empty((weight.shape[0],) if n == "bias" else like[n].shape,
+                            dtype=x.dtype, device="meta") for n in wanted}
+    gd = [_desc_meta(probe.get(n)) for n in GRADS]
+    ins = [_desc(t) for t in (x, offsets, mask, weight, grad_out)]
+    need = int(load().dcn1d_backward_workspace_size(
+        *(_ref(d) for d in ins), stride, padding, dilation, groups, offset_groups,
+        int(bool(unconstrained)), *(_ref(d) for d in gd)))
+    if need < 0:
+        raise Dcn1dError(-need, "dcn1d_backward_workspace_size")
+    return need
+
+
+def _desc_meta(t):
+    """Descriptor of a shape-only tensor (a non-NULL placeholder pointer: sizing only)."""
+    if t is None:
+        return None
+    d = Dcn1dTensor()
+    d.data = ctypes.c_void_p(256)
+    d.dtype = _DTYPES.get(t.dtype, _BAD_DTYPE)
+    d.ndim = t.ndim
+    for i, n in enumerate(t.shape):
+        d.shape[i] = n
+    return d
+
+
 def dcn1d_forward_noalloc(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=1,
                           groups=1, offset_groups=1, unconstrained=False, out=None, stream=None):
     """The forward for callers that cannot allocate device memory: the library's own
