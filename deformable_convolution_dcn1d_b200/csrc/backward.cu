@@ -15,14 +15,15 @@
 //
 // Kernels, all fp32 arithmetic whatever the input type:
 //  1. dcols[b, (c,k), l] = sum_co W[co, (c,k)] grad_out[b, co, l]: a batched GEMM
-//     per (batch, conv group) on CUDA cores;
+//     per (batch, conv group) on CUDA cores (64x64 tiles, 4x4 per thread);
 //  2. the sampling gradient: one thread per (batch, 16-channel chunk, offset
 //     group, tap, position) recomputes the tap's position once, then for its
 //     channels scatters grad_x, sums the offset and mask gradients (atomics
 //     into fp32 scratch: the order of those sums is not fixed) and writes the
 //     sampled columns m*v that the weight gradient needs;
 //  3. grad_weight = sum_b grad_out[b] cols[b]^T: the same GEMM kernel, summing
-//     over the batch inside the tile loop (a fixed order);
+//     over the batch inside the tile loop; when that grid is small the batch sum
+//     is split across CTAs into fp32 slices added in split order (a fixed order);
 //  4. grad_bias: one block per channel, a fixed-order tree reduction;
 //  5. the fp32 scratch of grad_x / grad_offsets / grad_mask is written out in
 //     the input type.
@@ -30,6 +31,7 @@
 
 #include "common.cuh"
 #include "sampler.cuh"
+#include "sm100.cuh"
 
 namespace dcn1d {
 
@@ -117,6 +119,19 @@ cudaError_t run_gemm(const TA *A, const TB *B, TC *C, const GemmArgs &g, int nz,
     const dim3 grid((g.N + kBN - 1) / kBN, (g.M + kBM - 1) / kBM, nz);
     gemm_kernel<TA, TB, TC, A_MC, B_NC><<<grid, 256, 0, stream>>>(A, B, C, g);
     return cudaGetLastError();
+}
+
+// out[i] = sum over s < S of part[s][i] in split order, written in the output type.
+template <class T>
+__global__ void __launch_bounds__(256) sum_splits_kernel(const float *part, T *out, int S,
+                                                         int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float acc = 0.0f;
+        for (int s = 0; s < S; ++s)
+            acc = __fadd_rn(acc, part[(int64_t)s * n + i]);
+        out[i] = from_f32<T>(acc);
+    }
 }
 
 struct SampArgs {
@@ -220,8 +235,25 @@ __global__ void __launch_bounds__(256) write_out_kernel(const float *src, T *dst
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Splits of the weight gradient's batch sum: the largest divisor of B that brings the
+// grid to about two waves of the SMs (1: no split, the GEMM writes grad_weight itself).
+int wgrad_splits(const Problem &P) {
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    const int64_t tiles = (int64_t)((P.cin_g * P.K + kBN - 1) / kBN) *
+                          ((P.cout_g + kBM - 1) / kBM) * P.groups;
+    int want = (int)((2 * sms + tiles - 1) / tiles);
+    if (want > P.B)
+        want = P.B;
+    int S = 1;
+    for (int d = 1; d <= want; ++d)
+        if (P.B % d == 0)
+            S = d;
+    return S;
+}
+
 struct WsLayout {
-    size_t dcols, cols, gx, goff, gmask, total;   // byte offsets (SIZE_MAX: not used)
+    size_t dcols, cols, gx, goff, gmask, wpart, total;   // byte offsets (SIZE_MAX: not used)
+    int wsplits;
 };
 
 WsLayout ws_layout(const Problem &P, const BackwardGrads &G) {
@@ -240,6 +272,9 @@ WsLayout ws_layout(const Problem &P, const BackwardGrads &G) {
     at += G.off ? align256(noff) : 0;
     w.gmask = G.mask ? at : SIZE_MAX;
     at += G.mask ? align256(noff) : 0;
+    w.wsplits = G.w ? wgrad_splits(P) : 1;
+    w.wpart = w.wsplits > 1 ? at : SIZE_MAX;
+    at += w.wsplits > 1 ? align256((size_t)w.wsplits * P.C_out * P.cin_g * P.K * 4) : 0;
     w.total = at;
     return w;
 }
@@ -259,6 +294,7 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
     float *gx = L.gx != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.gx) : nullptr;
     float *goff = L.goff != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.goff) : nullptr;
     float *gmask = L.gmask != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.gmask) : nullptr;
+    float *wpart = L.wpart != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.wpart) : nullptr;
     const T *w = static_cast<const T *>(P.w);
     const T *gout = static_cast<const T *>(G.gout);
     const int Kg = P.cin_g * P.K;
@@ -275,7 +311,8 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
     if (gmask && (e = cudaMemsetAsync(gmask, 0, noff * 4, s)) != cudaSuccess)
         return e;
 
-    if (want_dcols && P.B > 0) {   // 1. dcols[b][g*Kg + m][l] = sum_co W[g*cout_g + co][m] * gout[b][g*cout_g + co][l]
+    if (want_dcols && P.B > 0) {
+        // 1. dcols[b][g*Kg + m][l] = sum_co W[g*cout_g + co][m] * gout[b][g*cout_g + co][l]
         GemmArgs g;
         memset(&g, 0, sizeof(g));
         g.M = Kg;
@@ -321,29 +358,48 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
             return e;
         n += nt > 0;
     }
-    if (want_cols) {   // 3. gW (zeros for an empty batch: no term is summed)[g*cout_g + co][m] = sum_b sum_l gout[b][g*cout_g + co][l] * cols[b][g*Kg + m][l]
+    if (want_cols) {
+        // 3. gW[g*cout_g + co][m] = sum_b sum_l gout[b][g*cout_g + co][l] * cols[b][g*Kg + m][l]
+        // (zeros for an empty batch).  Split s of the batch sum covers batches
+        // [s * rps, (s + 1) * rps) (blockIdx.z = s * groups + group) and writes its own
+        // fp32 slice; the slices are then added in split order.
+        const int S = L.wsplits, rps = S > 1 ? P.B / S : P.B;
         GemmArgs g;
         memset(&g, 0, sizeof(g));
         g.M = P.cout_g;
         g.N = Kg;
         g.Kd = P.L_out;
-        g.R = P.B;
+        g.R = rps;
         g.ng = P.groups;
         g.a_sm = P.L_out;
         g.a_sk = 1;
         g.a_sg = (int64_t)P.cout_g * P.L_out;
         g.a_sr = (int64_t)P.C_out * P.L_out;
+        g.a_sb = g.a_sr * rps;
         g.b_sk = 1;
         g.b_sn = P.L_out;
         g.b_sg = (int64_t)Kg * P.L_out;
         g.b_sr = (int64_t)P.C_in * P.K * P.L_out;
+        g.b_sb = g.b_sr * rps;
         g.c_sm = Kg;
         g.c_sn = 1;
         g.c_sg = (int64_t)P.cout_g * Kg;
-        if ((e = run_gemm<T, float, T, false, false>(gout, cols, static_cast<T *>(G.w), g,
-                                                       P.groups, s)) != cudaSuccess)
-            return e;
-        ++n;
+        g.c_sb = (int64_t)P.C_out * Kg;
+        if (S > 1) {
+            if ((e = run_gemm<T, float, float, false, false>(gout, cols, wpart, g, S * P.groups,
+                                                             s)) != cudaSuccess)
+                return e;
+            const int64_t nw = (int64_t)P.C_out * Kg;
+            sum_splits_kernel<T><<<grid_1d(nw), 256, 0, s>>>(wpart, static_cast<T *>(G.w), S, nw);
+            if ((e = cudaGetLastError()) != cudaSuccess)
+                return e;
+            n += 2;
+        } else {
+            if ((e = run_gemm<T, float, T, false, false>(gout, cols, static_cast<T *>(G.w), g,
+                                                           P.groups, s)) != cudaSuccess)
+                return e;
+            ++n;
+        }
     }
     if (G.bias) {   // 4.
         bias_grad_kernel<T><<<P.C_out, 256, 0, s>>>(gout, static_cast<T *>(G.bias), P.B, P.C_out,

@@ -48,22 +48,6 @@ struct DwArgs {
     int win_elems;   // window length in pairs
 };
 
-// 16 bytes of T -> floats.
-__device__ __forceinline__ void unpack16(const uint4 &v, float *o, const __nv_bfloat16 *) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        o[2 * i] = __uint_as_float(w[i] << 16);
-        o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-__device__ __forceinline__ void unpack16(const uint4 &v, float *o, const float *) {
-    o[0] = __uint_as_float(v.x);
-    o[1] = __uint_as_float(v.y);
-    o[2] = __uint_as_float(v.z);
-    o[3] = __uint_as_float(v.w);
-}
-
 __device__ __forceinline__ float2 pair_floats(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
