@@ -42,6 +42,13 @@ def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
+def _pads(padding):
+    """(left, right) zeros around the signal from an int or a (left, right) pair."""
+    if isinstance(padding, (tuple, list)):
+        return int(padding[0]), int(padding[1])
+    return int(padding), int(padding)
+
+
 class Oracle:
     """ctypes front of one build of ``dcn1d_oracle.c``."""
 
@@ -50,13 +57,15 @@ class Oracle:
         lib.oracle_out_length.restype = _i64
         lib.oracle_out_length.argtypes = [_i64] * 5
         lib.oracle_forward.restype = _int
-        lib.oracle_forward.argtypes = [_p] * 5 + [_i64] * 11 + [_int, _p]
+        lib.oracle_out_length_lr.restype = _i64
+        lib.oracle_out_length_lr.argtypes = [_i64] * 6
+        lib.oracle_forward.argtypes = [_p] * 5 + [_i64] * 12 + [_int, _p]
         lib.oracle_forward_points.restype = _int
-        lib.oracle_forward_points.argtypes = [_p] * 5 + [_i64] * 11 + [_int, _p, _i64, _p]
+        lib.oracle_forward_points.argtypes = [_p] * 5 + [_i64] * 12 + [_int, _p, _i64, _p]
         lib.oracle_sample_index.restype = _int
         lib.oracle_sample_index.argtypes = [_p] + [_i64] * 8 + [_int, _p, _p]
         lib.oracle_backward.restype = _int
-        lib.oracle_backward.argtypes = [_p] * 5 + [_i64] * 11 + [_int] + [_p] * 5
+        lib.oracle_backward.argtypes = [_p] * 5 + [_i64] * 12 + [_int] + [_p] * 5
         lib.oracle_threads.restype = _int
         lib.oracle_threads.argtypes = []
         lib.oracle_set_threads.restype = None
@@ -64,9 +73,11 @@ class Oracle:
         self.lib = lib
         self.path = lib_path
 
-    def out_length(self, L_in: int, K: int, stride: int, padding: int, dilation: int) -> int:
-        """Output length by the conv1d closed form; -1 when invalid."""
-        return int(self.lib.oracle_out_length(L_in, K, stride, padding, dilation))
+    def out_length(self, L_in: int, K: int, stride: int, padding, dilation: int) -> int:
+        """Output length by the conv1d closed form; -1 when invalid.  ``padding`` is an int
+        (both sides) or a (left, right) pair."""
+        pl, pr = _pads(padding)
+        return int(self.lib.oracle_out_length_lr(L_in, K, stride, pl, pr, dilation))
 
     def threads(self) -> int:
         return int(self.lib.oracle_threads())
@@ -83,7 +94,8 @@ class Oracle:
             raise ValueError("offsets.shape[1] must equal offset_groups")
         if weight.shape[1] * groups != C_in or offsets.shape[3] != K or offsets.shape[0] != B:
             raise ValueError("weight/offsets shapes disagree with x and groups")
-        return (B, C_in, L_in, C_out, K, L_out, stride, padding, dilation, groups, offset_groups)
+        pl, pr = _pads(padding)
+        return (B, C_in, L_in, C_out, K, L_out, stride, pl, pr, dilation, groups, offset_groups)
 
     def forward(self, x, offsets, mask, weight, bias, stride, padding, dilation, groups,
                 offset_groups, unconstrained) -> np.ndarray:

@@ -37,6 +37,10 @@
  *  - Receptive field of output l: [l*s - p, l*s - p + d*(K-1)]; in constrained
  *    mode the sampling position is clamped to it BEFORE the floor.
  *  - Offset group of channel ci: ci / (C_in / offset_groups) (contiguous blocks).
+ *  - Padding "valid" is 0 and "same" (stride 1) is d(K-1)/2 zeros on the left and the
+ *    rest on the right, as nn.Conv1d does (the dc1d page uses both strings and says its
+ *    output length is nn.Conv1d's closed form); `padding` is the left side, and
+ *    `padding_right` enters only the output length.
  *  - Sampling position: pos = (float)base + off in IEEE float32 with round to
  *    nearest; i0 = floor(pos); f = pos - (float)i0 in float32.  The
  *    interpolation and the sums are then done in double.
@@ -57,18 +61,33 @@ typedef struct {
     int64_t B, C_in, L_in, C_out, K, L_out;
     int64_t stride, padding, dilation, groups, offset_groups;
     int unconstrained;
+    int64_t padding_right;   /* zeros after the signal; `padding` is the left side */
 } oracle_shape;
 
-/* "conv1d", "Shape" and "Description": L_out = floor((L_in + 2p - d(K-1) - 1)/s + 1).
+/* "conv1d", "Shape" and "Description": L_out = floor((L_in + 2p - d(K-1) - 1)/s + 1),
+ * here with the padding of each side separate: 2p -> pl + pr ("same" padding of the dc1d
+ * page pads d(K-1)/2 on the left and the rest on the right, as nn.Conv1d does).
  * Returns -1 for out-of-range arguments or when the length would be < 1. */
-int64_t oracle_out_length(int64_t L_in, int64_t K, int64_t s, int64_t p, int64_t d)
+static int64_t out_length_lr(int64_t L_in, int64_t K, int64_t s, int64_t pl, int64_t pr,
+                             int64_t d)
 {
-    if (L_in < 1 || K < 1 || s < 1 || p < 0 || d < 1)
+    if (L_in < 1 || K < 1 || s < 1 || pl < 0 || pr < 0 || d < 1)
         return -1;
-    int64_t num = L_in + 2 * p - d * (K - 1) - 1;
+    int64_t num = L_in + pl + pr - d * (K - 1) - 1;
     if (num < 0)          /* then floor(num/s + 1) <= 0 */
         return -1;
     return num / s + 1;   /* num >= 0: integer division is the floor */
+}
+
+int64_t oracle_out_length(int64_t L_in, int64_t K, int64_t s, int64_t p, int64_t d)
+{
+    return out_length_lr(L_in, K, s, p, p, d);
+}
+
+int64_t oracle_out_length_lr(int64_t L_in, int64_t K, int64_t s, int64_t pl, int64_t pr,
+                             int64_t d)
+{
+    return out_length_lr(L_in, K, s, pl, pr, d);
 }
 
 /* One tap's sampling position: the undeformed tap l*s - p + k*d plus the
@@ -140,7 +159,8 @@ static int check_shape(const oracle_shape *S)
         return 1;
     if (S->offset_groups < 1 || S->C_in % S->offset_groups)
         return 1;
-    if (oracle_out_length(S->L_in, S->K, S->stride, S->padding, S->dilation) != S->L_out)
+    if (out_length_lr(S->L_in, S->K, S->stride, S->padding, S->padding_right, S->dilation) !=
+        S->L_out)
         return 1;
     return 0;
 }
@@ -148,11 +168,12 @@ static int check_shape(const oracle_shape *S)
 /* Every output: out[B, C_out, L_out] in double.  Returns 0, or 1 on bad shape. */
 int oracle_forward(const float *x, const float *off, const float *mask, const float *w,
                    const float *bias, int64_t B, int64_t C_in, int64_t L_in, int64_t C_out,
-                   int64_t K, int64_t L_out, int64_t stride, int64_t padding, int64_t dilation,
-                   int64_t groups, int64_t offset_groups, int unconstrained, double *out)
+                   int64_t K, int64_t L_out, int64_t stride, int64_t padding,
+                   int64_t padding_right, int64_t dilation, int64_t groups,
+                   int64_t offset_groups, int unconstrained, double *out)
 {
     oracle_shape S = {B, C_in, L_in, C_out, K, L_out, stride, padding,
-                      dilation, groups, offset_groups, unconstrained};
+                      dilation, groups, offset_groups, unconstrained, padding_right};
     if (check_shape(&S))
         return 1;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
@@ -167,12 +188,12 @@ int oracle_forward(const float *x, const float *off, const float *mask, const fl
 int oracle_forward_points(const float *x, const float *off, const float *mask, const float *w,
                           const float *bias, int64_t B, int64_t C_in, int64_t L_in,
                           int64_t C_out, int64_t K, int64_t L_out, int64_t stride,
-                          int64_t padding, int64_t dilation, int64_t groups,
-                          int64_t offset_groups, int unconstrained, const int64_t *points,
-                          int64_t n, double *out)
+                          int64_t padding, int64_t padding_right, int64_t dilation,
+                          int64_t groups, int64_t offset_groups, int unconstrained,
+                          const int64_t *points, int64_t n, double *out)
 {
     oracle_shape S = {B, C_in, L_in, C_out, K, L_out, stride, padding,
-                      dilation, groups, offset_groups, unconstrained};
+                      dilation, groups, offset_groups, unconstrained, padding_right};
     if (check_shape(&S))
         return 1;
     for (int64_t i = 0; i < n; ++i) {
@@ -192,7 +213,8 @@ int oracle_sample_index(const float *off, int64_t B, int64_t G, int64_t L_in, in
                         int64_t L_out, int64_t stride, int64_t padding, int64_t dilation,
                         int unconstrained, int32_t *i0_out, float *f_out)
 {
-    oracle_shape S = {B, G, L_in, G, K, L_out, stride, padding, dilation, 1, G, unconstrained};
+    oracle_shape S = {B, G, L_in, G, K, L_out, stride, padding, dilation, 1, G, unconstrained,
+                      padding};
     if (oracle_out_length(L_in, K, stride, padding, dilation) != L_out)
         return 1;
     int64_t n = B * G * L_out * K;
@@ -255,12 +277,13 @@ void oracle_set_threads(int n)
  */
 int oracle_backward(const float *x, const float *off, const float *mask, const float *w,
                     const float *gout, int64_t B, int64_t C_in, int64_t L_in, int64_t C_out,
-                    int64_t K, int64_t L_out, int64_t stride, int64_t padding, int64_t dilation,
-                    int64_t groups, int64_t offset_groups, int unconstrained, double *gx,
-                    double *goff, double *gmask, double *gw, double *gbias)
+                    int64_t K, int64_t L_out, int64_t stride, int64_t padding,
+                    int64_t padding_right, int64_t dilation, int64_t groups,
+                    int64_t offset_groups, int unconstrained, double *gx, double *goff,
+                    double *gmask, double *gw, double *gbias)
 {
     oracle_shape S = {B, C_in, L_in, C_out, K, L_out, stride, padding,
-                      dilation, groups, offset_groups, unconstrained};
+                      dilation, groups, offset_groups, unconstrained, padding_right};
     if (check_shape(&S))
         return 1;
     const int64_t cin_g = C_in / groups, cout_g = C_out / groups;

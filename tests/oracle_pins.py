@@ -24,6 +24,7 @@ from __future__ import annotations
 
 import fractions
 import math
+import warnings
 
 import numpy as np
 import torch
@@ -388,6 +389,43 @@ def pin_offset_group_reading(o):
         assert np.array_equal(a, c)
 
 
+def pin_asymmetric_padding(o):
+    """Padding given per side: zero offsets equal torch's conv1d on the explicitly padded
+    signal (F.pad, library routine) with padding 0; the dc1d page's "same" (stride 1,
+    d(K-1) odd: d(K-1)//2 on the left, the rest on the right) equals torch's own
+    padding="same" and keeps L_out = L_in."""
+    cases = [  # B, C_in, C_out, K, L_in, s, (pl, pr), d, groups, og
+        (2, 4, 6, 4, 15, 1, (1, 2), 1, 2, 2),
+        (1, 6, 3, 3, 20, 2, (0, 3), 2, 3, 1),
+        (2, 4, 4, 2, 11, 1, (2, 0), 3, 4, 4),
+    ]
+    for i, (B, Ci, Co, K, L, s, pads, d, G, og) in enumerate(cases):
+        g = torch.Generator().manual_seed(700 + i)
+        x = torch.randn(B, Ci, L, generator=g)
+        w = torch.randn(Co, Ci // G, K, generator=g)
+        b = torch.randn(Co, generator=g)
+        L_out = o.out_length(L, K, s, pads, d)
+        ref = F.conv1d(F.pad(x.double(), pads), w.double(), b.double(), stride=s, dilation=d,
+                       groups=G)
+        assert L_out == ref.shape[2], (i, L_out, ref.shape)
+        offs = torch.zeros(B, og, L_out, K)
+        for unc in (False, True):
+            y = o.forward(x, offs, None, w, b, s, pads, d, G, og, unc)
+            assert rel_err(y, ref) < 1e-12, (i, unc)
+    for K, d in ((4, 1), (2, 3), (6, 1)):   # d(K-1) odd: one more zero on the right
+        g = torch.Generator().manual_seed(800 + K)
+        x = torch.randn(2, 3, 16, generator=g)
+        w = torch.randn(5, 3, K, generator=g)
+        tot = d * (K - 1)
+        pads = (tot // 2, tot - tot // 2)
+        assert o.out_length(16, K, 1, pads, d) == 16
+        with warnings.catch_warnings():   # torch notes that it pads a copy for this case
+            warnings.simplefilter("ignore", UserWarning)
+            ref = F.conv1d(x.double(), w.double(), None, padding="same", dilation=d)
+        y = o.forward(x, torch.zeros(2, 1, 16, K), None, w, None, 1, pads, d, 1, 1, False)
+        assert rel_err(y, ref) < 1e-12, (K, d)
+
+
 ALL_PINS = [
     pin_out_length_page_examples,
     pin_out_length_closed_form,
@@ -403,4 +441,5 @@ ALL_PINS = [
     pin_constrained_locality,
     pin_sample_index,
     pin_offset_group_reading,
+    pin_asymmetric_padding,
 ]

@@ -34,8 +34,10 @@ CASES = [
     (1, 4, 4, 3, 12, 2, 2, 2, 1, 1, False, True),
     (2, 2, 4, 4, 9, 1, 0, 1, 2, 1, True, True),
     (1, 6, 3, 2, 7, 1, 1, 3, 3, 3, True, False),
+    (2, 4, 4, 4, 11, 1, (1, 2), 1, 2, 2, True, False),   # "same" with d(K-1) odd
 ]
-IDS = ["g2_og2_mask_constrained", "strided_dilated_unc", "k4_mask_unc", "depthwise_like_dil3"]
+IDS = ["g2_og2_mask_constrained", "strided_dilated_unc", "k4_mask_unc", "depthwise_like_dil3",
+       "same_padding_asymmetric"]
 
 
 def _bf16_grid(a):
@@ -110,7 +112,9 @@ def pin_conv1d_autograd(o, case):
     x = torch.tensor(t["x"], dtype=torch.float64, requires_grad=True)
     w = torch.tensor(t["weight"], dtype=torch.float64, requires_grad=True)
     b = torch.tensor(t["bias"], dtype=torch.float64, requires_grad=True)
-    y = torch.nn.functional.conv1d(x, w, b, stride=s, padding=p, dilation=d, groups=G)
+    pads = tuple(p) if isinstance(p, tuple) else (p, p)
+    y = torch.nn.functional.conv1d(torch.nn.functional.pad(x, pads), w, b, stride=s,
+                                   dilation=d, groups=G)
     (y * torch.tensor(t["gout"], dtype=torch.float64)).sum().backward()
     for got, ref in ((g["grad_x"], x.grad), (g["grad_weight"], w.grad), (g["grad_bias"], b.grad)):
         assert np.allclose(got, ref.numpy(), rtol=1e-12, atol=1e-12)
