@@ -24,4 +24,5 @@ from ._binding import (  # noqa: F401
     dcn1d_status_string,
     lib_path,
     load,
+    resolve_padding,
 )

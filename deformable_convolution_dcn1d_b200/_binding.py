@@ -66,7 +66,37 @@ SIGNATURES = [
     ("dcn1d_backward", _INT,
      [_T, _T, _T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _T, _T, _T, _T, _P,
       ctypes.c_size_t, _P]),
+    ("dcn1d_out_length_lr", _I64, [_I64] * 6),
+    ("dcn1d_forward_lr_kernel_name", ctypes.c_char_p, [_T, _T, _T, _T, _T] + [_I64] * 6 + [_INT, _T]),
+    ("dcn1d_forward_lr", _INT,
+     [_T, _T, _T, _T, _T] + [_I64] * 6 + [_INT, _T, _P, ctypes.c_size_t, _P]),
+    ("dcn1d_forward_lr_workspace_size", _I64, [_T, _T, _T, _T, _T] + [_I64] * 6 + [_INT, _T]),
+    ("dcn1d_backward_lr_workspace_size", _I64,
+     [_T, _T, _T, _T, _T] + [_I64] * 6 + [_INT] + [_T] * 5),
+    ("dcn1d_backward_lr", _INT,
+     [_T, _T, _T, _T, _T] + [_I64] * 6 + [_INT] + [_T] * 5 + [_P, ctypes.c_size_t, _P]),
 ]
+
+
+def resolve_padding(padding, kernel_size, stride=1, dilation=1):
+    """(left, right) zeros around the signal from an int (both sides), a (left, right)
+    pair, "valid" (none) or "same" (stride 1: dilation*(kernel_size-1) // 2 on the left,
+    the rest on the right, so that L_out = L_in -- nn.Conv1d's reading, which the dc1d
+    page's output-length rule follows)."""
+    if isinstance(padding, str):
+        if padding == "valid":
+            return 0, 0
+        if padding == "same":
+            if stride != 1:
+                raise ValueError('padding="same" needs stride 1')
+            tot = dilation * (kernel_size - 1)
+            return tot // 2, tot - tot // 2
+        raise ValueError(f"unknown padding {padding!r}")
+    if isinstance(padding, (tuple, list)):
+        if len(padding) != 2:
+            raise ValueError("padding pair must be (left, right)")
+        return int(padding[0]), int(padding[1])
+    return int(padding), int(padding)
 
 
 def lib_path() -> str:
@@ -133,9 +163,11 @@ def _check_device(tensors):
     return dev
 
 
-def dcn1d_out_length(L_in: int, kernel_size: int, stride: int = 1, padding: int = 0,
+def dcn1d_out_length(L_in: int, kernel_size: int, stride: int = 1, padding=0,
                      dilation: int = 1) -> int:
-    return int(load().dcn1d_out_length(L_in, kernel_size, stride, padding, dilation))
+    """Output length (-1 when invalid); ``padding`` as in resolve_padding."""
+    pl, pr = resolve_padding(padding, kernel_size, stride, dilation)
+    return int(load().dcn1d_out_length_lr(L_in, kernel_size, stride, pl, pr, dilation))
 
 
 def dcn1d_status_string(status: int) -> str:
@@ -172,12 +204,14 @@ def dcn1d_forward(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=
 
     x [B, C_in, L_in]; offsets and mask [B, offset_groups, L_out, K] (mask may be None);
     weight [C_out, C_in/groups, K]; bias [C_out] or None.  All CUDA, contiguous, one dtype
-    (float32 or bfloat16).  ``out`` is allocated with torch when not given.  The scratch the
+    (float32 or bfloat16).  ``padding``: an int, a (left, right) pair, "valid" or "same"
+    (see resolve_padding).  ``out`` is allocated with torch when not given.  The scratch the
     fastest path needs (``dcn1d_forward_workspace_size``) is allocated with torch unless a
     uint8 CUDA tensor ``workspace`` is given; ``workspace=False`` asks for the path without
     scratch.  Runs on ``stream`` (default: the current torch stream of x's device); does not
     synchronise.
     """
+    pl, pr = resolve_padding(padding, weight.shape[2], stride, dilation)
     dev = _check_device((x, offsets, mask, weight, bias, out))
     if out is None:
         out = _out_for(x, weight, offsets)
@@ -187,9 +221,9 @@ def dcn1d_forward(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=
     with torch.cuda.device(dev):
         ws_ptr, ws_bytes = None, 0
         if workspace is not False:
-            need = int(lib.dcn1d_forward_workspace_size(*refs[:5], stride, padding, dilation,
-                                                        groups, offset_groups,
-                                                        int(bool(unconstrained)), refs[5]))
+            need = int(lib.dcn1d_forward_lr_workspace_size(*refs[:5], stride, pl, pr, dilation,
+                                                           groups, offset_groups,
+                                                           int(bool(unconstrained)), refs[5]))
             if need < 0:
                 raise Dcn1dError(-need, "dcn1d_forward_workspace_size")
             if need > 0:
@@ -198,7 +232,7 @@ def dcn1d_forward(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=
                 if workspace.numel() < need or workspace.dtype != torch.uint8:
                     raise ValueError(f"workspace must be a uint8 tensor of >= {need} bytes")
                 ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
-        st = lib.dcn1d_forward_ws(*refs[:5], stride, padding, dilation, groups, offset_groups,
+        st = lib.dcn1d_forward_lr(*refs[:5], stride, pl, pr, dilation, groups, offset_groups,
                                   int(bool(unconstrained)), refs[5], _P(ws_ptr), ws_bytes,
                                   _P(_stream_ptr(stream, dev)))
     if st != 0:
@@ -236,9 +270,10 @@ def dcn1d_backward(x, offsets, mask, weight, grad_out, stride=1, padding=0, dila
     gd = [_desc(out.get(n)) for n in GRADS]
     lib = load()
     refs = [_ref(d) for d in ins] + [_ref(d) for d in gd]
-    args = (stride, padding, dilation, groups, offset_groups, int(bool(unconstrained)))
+    pl, pr = resolve_padding(padding, weight.shape[2], stride, dilation)
+    args = (stride, pl, pr, dilation, groups, offset_groups, int(bool(unconstrained)))
     with torch.cuda.device(dev):
-        need = int(lib.dcn1d_backward_workspace_size(*refs[:5], *args, *refs[5:]))
+        need = int(lib.dcn1d_backward_lr_workspace_size(*refs[:5], *args, *refs[5:]))
         if need < 0:
             raise Dcn1dError(-need, "dcn1d_backward_workspace_size")
         ws_ptr, ws_bytes = None, 0
@@ -248,8 +283,8 @@ def dcn1d_backward(x, offsets, mask, weight, grad_out, stride=1, padding=0, dila
             if workspace.numel() < need or workspace.dtype != torch.uint8:
                 raise ValueError(f"workspace must be a uint8 tensor of >= {need} bytes")
             ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
-        st = lib.dcn1d_backward(*refs[:5], *args, *refs[5:], _P(ws_ptr), ws_bytes,
-                                _P(_stream_ptr(stream, dev)))
+        st = lib.dcn1d_backward_lr(*refs[:5], *args, *refs[5:], _P(ws_ptr), ws_bytes,
+                                   _P(_stream_ptr(stream, dev)))
     if st != 0:
         raise Dcn1dError(st, "dcn1d_backward")
     return {n: out[n] for n in wanted}
@@ -263,27 +298,15 @@ def dcn1d_backward_workspace_size(x, offsets, mask, weight, grad_out, stride=1, 
     like = {"x": x, "offsets": offsets, "mask": mask, "weight": weight}
     probe = {n: torch.empty((weight.shape[0],) if n == "bias" else like[n].shape,
                             dtype=x.dtype, device="meta") for n in wanted}
-    gd = [_desc_meta(probe.get(n)) for n in GRADS]
+    gd = [None if probe.get(n) is None else _meta_desc(probe[n]) for n in GRADS]
     ins = [_desc(t) for t in (x, offsets, mask, weight, grad_out)]
-    need = int(load().dcn1d_backward_workspace_size(
-        *(_ref(d) for d in ins), stride, padding, dilation, groups, offset_groups,
+    pl, pr = resolve_padding(padding, weight.shape[2], stride, dilation)
+    need = int(load().dcn1d_backward_lr_workspace_size(
+        *(_ref(d) for d in ins), stride, pl, pr, dilation, groups, offset_groups,
         int(bool(unconstrained)), *(_ref(d) for d in gd)))
     if need < 0:
         raise Dcn1dError(-need, "dcn1d_backward_workspace_size")
     return need
-
-
-def _desc_meta(t):
-    """Descriptor of a shape-only tensor (a non-NULL placeholder pointer: sizing only)."""
-    if t is None:
-        return None
-    d = Dcn1dTensor()
-    d.data = ctypes.c_void_p(256)
-    d.dtype = _DTYPES.get(t.dtype, _BAD_DTYPE)
-    d.ndim = t.ndim
-    for i, n in enumerate(t.shape):
-        d.shape[i] = n
-    return d
 
 
 def dcn1d_forward_noalloc(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=1,
@@ -293,6 +316,10 @@ def dcn1d_forward_noalloc(x, offsets, mask, weight, bias, stride=1, padding=0, d
     allocates nothing).  Calls whose GPU work overlaps share the scratch and race."""
     if out is None:
         raise ValueError("dcn1d_forward_noalloc allocates nothing: pass out")
+    pl, pr = resolve_padding(padding, weight.shape[2], stride, dilation)
+    if pl != pr:
+        raise ValueError("dcn1d_forward_noalloc takes symmetric padding only")
+    padding = pl
     dev = _check_device((x, offsets, mask, weight, bias, out))
     descs = [_desc(t) for t in (x, offsets, mask, weight, bias, out)]
     lib = load()
@@ -312,10 +339,12 @@ def dcn1d_forward_workspace_size(x, offsets, mask, weight, bias, stride=1, paddi
     """Bytes of scratch the fastest path needs for these arguments (0 if none)."""
     if out is None:
         out = _out_for(x, weight, offsets)
+    pl, pr = resolve_padding(padding, weight.shape[2], stride, dilation)
     descs = [_desc(t) for t in (x, offsets, mask, weight, bias, out)]
-    need = int(load().dcn1d_forward_workspace_size(*(_ref(d) for d in descs[:5]), stride,
-                                                   padding, dilation, groups, offset_groups,
-                                                   int(bool(unconstrained)), _ref(descs[5])))
+    need = int(load().dcn1d_forward_lr_workspace_size(*(_ref(d) for d in descs[:5]), stride,
+                                                      pl, pr, dilation, groups, offset_groups,
+                                                      int(bool(unconstrained)),
+                                                      _ref(descs[5])))
     if need < 0:
         raise Dcn1dError(-need, "dcn1d_forward_workspace_size")
     return need
@@ -324,14 +353,15 @@ def dcn1d_forward_workspace_size(x, offsets, mask, weight, bias, stride=1, paddi
 def dcn1d_forward_kernel_name(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=1,
                               groups=1, offset_groups=1, unconstrained=False, out=None):
     """Name of the kernel dcn1d_forward would launch, or None for invalid arguments."""
+    pl, pr = resolve_padding(padding, weight.shape[2], stride, dilation)
     if out is None:
         out = torch.empty((x.shape[0], weight.shape[0], offsets.shape[2]), dtype=x.dtype,
                           device="meta")
     descs = [_desc(t) if t is None or t.device.type != "meta" else _meta_desc(t)
              for t in (x, offsets, mask, weight, bias, out)]
-    r = load().dcn1d_forward_kernel_name(*(_ref(d) for d in descs[:5]), stride, padding,
-                                         dilation, groups, offset_groups,
-                                         int(bool(unconstrained)), _ref(descs[5]))
+    r = load().dcn1d_forward_lr_kernel_name(*(_ref(d) for d in descs[:5]), stride, pl, pr,
+                                            dilation, groups, offset_groups,
+                                            int(bool(unconstrained)), _ref(descs[5]))
     return None if r is None else r.decode()
 
 

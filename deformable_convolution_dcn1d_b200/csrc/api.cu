@@ -70,6 +70,7 @@ size_t workspace_bytes(const Problem &P) {
 // Full validation; fills P and the chosen kernel on success.
 int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor *mask,
              const dcn1d_tensor *w, const dcn1d_tensor *bias, int64_t stride, int64_t padding,
+             int64_t padding_right,
              int64_t dilation, int64_t groups, int64_t offset_groups, int unconstrained,
              const dcn1d_tensor *out, Problem *P) {
     int st;
@@ -87,7 +88,8 @@ int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor 
         (bias && bias->dtype != dt))
         return DCN1D_ERR_DTYPE;
 
-    if (stride < 1 || padding < 0 || dilation < 1 || groups < 1 || offset_groups < 1)
+    if (stride < 1 || padding < 0 || padding_right < 0 || dilation < 1 || groups < 1 ||
+        offset_groups < 1)
         return DCN1D_ERR_ARG;
     const int64_t B = x->shape[0], C_in = x->shape[1], L_in = x->shape[2];
     const int64_t C_out = w->shape[0], K = w->shape[2];
@@ -97,10 +99,10 @@ int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor 
         return DCN1D_ERR_ARG;
     if (w->shape[1] * groups != C_in)
         return DCN1D_ERR_SHAPE;
-    if (stride >= kMaxPos || padding >= kMaxPos || dilation >= kMaxPos || K >= kMaxPos ||
-        L_in >= kMaxPos)
+    if (stride >= kMaxPos || padding >= kMaxPos || padding_right >= kMaxPos ||
+        dilation >= kMaxPos || K >= kMaxPos || L_in >= kMaxPos)
         return DCN1D_ERR_UNSUPPORTED;
-    const int64_t L_out = dcn1d_out_length(L_in, K, stride, padding, dilation);
+    const int64_t L_out = dcn1d_out_length_lr(L_in, K, stride, padding, padding_right, dilation);
     if (L_out < 1)
         return DCN1D_ERR_ARG;
     if (!shape_is(off, B, offset_groups, L_out, K))
@@ -127,6 +129,7 @@ int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor 
     P->L_out = (int)L_out;
     P->stride = (int)stride;
     P->padding = (int)padding;
+    P->padding_right = (int)padding_right;
     P->dilation = (int)dilation;
     P->groups = (int)groups;
     P->offset_groups = (int)offset_groups;
@@ -148,12 +151,13 @@ int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor 
 // of out, then every wanted gradient against its input's dtype and shape.
 int validate_backward(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor *mask,
                       const dcn1d_tensor *w, const dcn1d_tensor *gout, int64_t stride,
-                      int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
+                      int64_t padding,
+                      int64_t padding_right, int64_t dilation, int64_t groups, int64_t offset_groups,
                       int unconstrained, const dcn1d_tensor *gx, const dcn1d_tensor *goff,
                       const dcn1d_tensor *gmask, const dcn1d_tensor *gw, const dcn1d_tensor *gbias,
                       Problem *P, BackwardGrads *G) {
-    int st = validate(x, off, mask, w, nullptr, stride, padding, dilation, groups, offset_groups,
-                      unconstrained, gout, P);
+    int st = validate(x, off, mask, w, nullptr, stride, padding, padding_right, dilation, groups,
+                      offset_groups, unconstrained, gout, P);
     if (st != DCN1D_OK)
         return st;
     auto like = [&](const dcn1d_tensor *g, const dcn1d_tensor *in, int nd) -> int {
@@ -237,18 +241,25 @@ using namespace dcn1d;
 
 extern "C" {
 
-int64_t dcn1d_out_length(int64_t L_in, int64_t K, int64_t stride, int64_t padding,
-                         int64_t dilation) {
-    if (L_in < 1 || K < 1 || stride < 1 || padding < 0 || dilation < 1)
+int64_t dcn1d_out_length_lr(int64_t L_in, int64_t K, int64_t stride, int64_t padding_left,
+                            int64_t padding_right, int64_t dilation) {
+    if (L_in < 1 || K < 1 || stride < 1 || padding_left < 0 || padding_right < 0 ||
+        dilation < 1)
         return -1;
     // Arguments past 2^31 are refused so the products below cannot overflow.
     const int64_t lim = (int64_t)1 << 31;
-    if (L_in > lim || K > lim || stride > lim || padding > lim || dilation > lim)
+    if (L_in > lim || K > lim || stride > lim || padding_left > lim || padding_right > lim ||
+        dilation > lim)
         return -1;
-    const int64_t num = L_in + 2 * padding - dilation * (K - 1) - 1;
+    const int64_t num = L_in + padding_left + padding_right - dilation * (K - 1) - 1;
     if (num < 0)
         return -1;
     return num / stride + 1;
+}
+
+int64_t dcn1d_out_length(int64_t L_in, int64_t K, int64_t stride, int64_t padding,
+                         int64_t dilation) {
+    return dcn1d_out_length_lr(L_in, K, stride, padding, padding, dilation);
 }
 
 const char *dcn1d_status_string(int status) {
@@ -266,15 +277,16 @@ const char *dcn1d_status_string(int status) {
     }
 }
 
-int dcn1d_forward_ws(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+int dcn1d_forward_lr(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
                      const dcn1d_tensor *mask, const dcn1d_tensor *weight,
-                     const dcn1d_tensor *bias, int64_t stride, int64_t padding, int64_t dilation,
-                     int64_t groups, int64_t offset_groups, int unconstrained, dcn1d_tensor *out,
+                     const dcn1d_tensor *bias, int64_t stride, int64_t padding_left,
+                     int64_t padding_right, int64_t dilation, int64_t groups,
+                     int64_t offset_groups, int unconstrained, dcn1d_tensor *out,
                      void *workspace, size_t workspace_bytes, void *stream) {
     g_last_launches = 0;
     Problem P;
-    int st = validate(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
-                      offset_groups, unconstrained, out, &P);
+    int st = validate(x, offsets, mask, weight, bias, stride, padding_left, padding_right,
+                      dilation, groups, offset_groups, unconstrained, out, &P);
     if (st != DCN1D_OK)
         return st;
     if (workspace_bytes > 0 && !workspace)
@@ -310,6 +322,16 @@ int dcn1d_forward_ws(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
     return DCN1D_OK;
 }
 
+int dcn1d_forward_ws(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                     const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                     const dcn1d_tensor *bias, int64_t stride, int64_t padding, int64_t dilation,
+                     int64_t groups, int64_t offset_groups, int unconstrained, dcn1d_tensor *out,
+                     void *workspace, size_t workspace_bytes, void *stream) {
+    return dcn1d_forward_lr(x, offsets, mask, weight, bias, stride, padding, padding, dilation,
+                            groups, offset_groups, unconstrained, out, workspace, workspace_bytes,
+                            stream);
+}
+
 int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
                   const dcn1d_tensor *weight, const dcn1d_tensor *bias, int64_t stride,
                   int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
@@ -318,17 +340,46 @@ int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1
                             offset_groups, unconstrained, out, nullptr, 0, stream);
 }
 
+int64_t dcn1d_forward_lr_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                                        const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                                        const dcn1d_tensor *bias, int64_t stride,
+                                        int64_t padding_left, int64_t padding_right,
+                                        int64_t dilation, int64_t groups, int64_t offset_groups,
+                                        int unconstrained, const dcn1d_tensor *out) {
+    Problem P;
+    const int st = validate(x, offsets, mask, weight, bias, stride, padding_left, padding_right,
+                            dilation, groups, offset_groups, unconstrained, out, &P);
+    if (st != DCN1D_OK)
+        return -st;
+    return (int64_t)workspace_bytes(P);
+}
+
 int64_t dcn1d_forward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
                                      const dcn1d_tensor *mask, const dcn1d_tensor *weight,
                                      const dcn1d_tensor *bias, int64_t stride, int64_t padding,
                                      int64_t dilation, int64_t groups, int64_t offset_groups,
                                      int unconstrained, const dcn1d_tensor *out) {
+    return dcn1d_forward_lr_workspace_size(x, offsets, mask, weight, bias, stride, padding,
+                                           padding, dilation, groups, offset_groups,
+                                           unconstrained, out);
+}
+
+int64_t dcn1d_backward_lr_workspace_size(
+    const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
+    const dcn1d_tensor *weight, const dcn1d_tensor *grad_out, int64_t stride,
+    int64_t padding_left, int64_t padding_right, int64_t dilation, int64_t groups,
+    int64_t offset_groups, int unconstrained, const dcn1d_tensor *grad_x,
+    const dcn1d_tensor *grad_offsets, const dcn1d_tensor *grad_mask,
+    const dcn1d_tensor *grad_weight, const dcn1d_tensor *grad_bias) {
     Problem P;
-    const int st = validate(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
-                            offset_groups, unconstrained, out, &P);
+    BackwardGrads G;
+    const int st = validate_backward(x, offsets, mask, weight, grad_out, stride, padding_left,
+                                     padding_right, dilation, groups, offset_groups,
+                                     unconstrained, grad_x, grad_offsets, grad_mask, grad_weight,
+                                     grad_bias, &P, &G);
     if (st != DCN1D_OK)
-        return -st;
-    return (int64_t)workspace_bytes(P);
+        return -(int64_t)st;
+    return (int64_t)backward_workspace(P, G);
 }
 
 int64_t dcn1d_backward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
@@ -340,28 +391,27 @@ int64_t dcn1d_backward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor 
                                       const dcn1d_tensor *grad_mask,
                                       const dcn1d_tensor *grad_weight,
                                       const dcn1d_tensor *grad_bias) {
-    Problem P;
-    BackwardGrads G;
-    const int st = validate_backward(x, offsets, mask, weight, grad_out, stride, padding,
-                                     dilation, groups, offset_groups, unconstrained, grad_x,
-                                     grad_offsets, grad_mask, grad_weight, grad_bias, &P, &G);
-    if (st != DCN1D_OK)
-        return -(int64_t)st;
-    return (int64_t)backward_workspace(P, G);
+    return dcn1d_backward_lr_workspace_size(x, offsets, mask, weight, grad_out, stride, padding,
+                                            padding, dilation, groups, offset_groups,
+                                            unconstrained, grad_x, grad_offsets, grad_mask,
+                                            grad_weight, grad_bias);
 }
 
-int dcn1d_backward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
-                   const dcn1d_tensor *weight, const dcn1d_tensor *grad_out, int64_t stride,
-                   int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
-                   int unconstrained, dcn1d_tensor *grad_x, dcn1d_tensor *grad_offsets,
-                   dcn1d_tensor *grad_mask, dcn1d_tensor *grad_weight, dcn1d_tensor *grad_bias,
-                   void *workspace, size_t workspace_bytes, void *stream) {
+int dcn1d_backward_lr(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                      const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                      const dcn1d_tensor *grad_out, int64_t stride, int64_t padding_left,
+                      int64_t padding_right, int64_t dilation, int64_t groups,
+                      int64_t offset_groups, int unconstrained, dcn1d_tensor *grad_x,
+                      dcn1d_tensor *grad_offsets, dcn1d_tensor *grad_mask,
+                      dcn1d_tensor *grad_weight, dcn1d_tensor *grad_bias, void *workspace,
+                      size_t workspace_bytes, void *stream) {
     g_last_launches = 0;
     Problem P;
     BackwardGrads G;
-    const int st = validate_backward(x, offsets, mask, weight, grad_out, stride, padding,
-                                     dilation, groups, offset_groups, unconstrained, grad_x,
-                                     grad_offsets, grad_mask, grad_weight, grad_bias, &P, &G);
+    const int st = validate_backward(x, offsets, mask, weight, grad_out, stride, padding_left,
+                                     padding_right, dilation, groups, offset_groups,
+                                     unconstrained, grad_x, grad_offsets, grad_mask, grad_weight,
+                                     grad_bias, &P, &G);
     if (st != DCN1D_OK)
         return st;
     const size_t need = backward_workspace(P, G);
@@ -377,16 +427,38 @@ int dcn1d_backward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn
     return DCN1D_OK;
 }
 
+int dcn1d_backward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
+                   const dcn1d_tensor *weight, const dcn1d_tensor *grad_out, int64_t stride,
+                   int64_t padding, int64_t dilation, int64_t groups, int64_t offset_groups,
+                   int unconstrained, dcn1d_tensor *grad_x, dcn1d_tensor *grad_offsets,
+                   dcn1d_tensor *grad_mask, dcn1d_tensor *grad_weight, dcn1d_tensor *grad_bias,
+                   void *workspace, size_t workspace_bytes, void *stream) {
+    return dcn1d_backward_lr(x, offsets, mask, weight, grad_out, stride, padding, padding,
+                             dilation, groups, offset_groups, unconstrained, grad_x,
+                             grad_offsets, grad_mask, grad_weight, grad_bias, workspace,
+                             workspace_bytes, stream);
+}
+
+const char *dcn1d_forward_lr_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                                         const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                                         const dcn1d_tensor *bias, int64_t stride,
+                                         int64_t padding_left, int64_t padding_right,
+                                         int64_t dilation, int64_t groups, int64_t offset_groups,
+                                         int unconstrained, const dcn1d_tensor *out) {
+    Problem P;
+    if (validate(x, offsets, mask, weight, bias, stride, padding_left, padding_right, dilation,
+                 groups, offset_groups, unconstrained, out, &P) != DCN1D_OK)
+        return nullptr;
+    return kernel_names[select_kernel(P, SIZE_MAX)];
+}
+
 const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
                                       const dcn1d_tensor *mask, const dcn1d_tensor *weight,
                                       const dcn1d_tensor *bias, int64_t stride, int64_t padding,
                                       int64_t dilation, int64_t groups, int64_t offset_groups,
                                       int unconstrained, const dcn1d_tensor *out) {
-    Problem P;
-    if (validate(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
-                 offset_groups, unconstrained, out, &P) != DCN1D_OK)
-        return nullptr;
-    return kernel_names[select_kernel(P, SIZE_MAX)];
+    return dcn1d_forward_lr_kernel_name(x, offsets, mask, weight, bias, stride, padding, padding,
+                                        dilation, groups, offset_groups, unconstrained, out);
 }
 
 int dcn1d_last_launch_count(void) { return g_last_launches; }

@@ -12,7 +12,8 @@ namespace dcn1d {
 // A validated forward problem.  All sizes fit in int32 (checked on the host).
 struct Problem {
     int B, C_in, L_in, C_out, K, L_out;
-    int stride, padding, dilation, groups, offset_groups;
+    int stride, padding, dilation, groups, offset_groups;   // padding: zeros before the signal
+    int padding_right;                                      // zeros after it
     int unconstrained;
     int dtype;                 // dcn1d_dtype
     int cin_g, cout_g;         // channels per conv group (input, output)
@@ -38,7 +39,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // exact, and the bit patterns it yields for larger |pos| cannot alias a
 // window index.
 inline bool fast_floor_ok(const Problem &P) {
-    return (int64_t)P.L_in + 2 * (int64_t)P.padding < (1 << 21);
+    return (int64_t)P.L_in + (int64_t)P.padding + P.padding_right < (1 << 21);
 }
 
 // Benchmark timing hook (dcn1d_set_timing_events): launchers call these right

@@ -1,6 +1,6 @@
 /*
- * dcn1d.h -- C ABI of the B200 (sm_100a) forward pass of 1D deformable
- * convolution (DeformConv1d), with optional DCNv2 modulation mask.
+ * dcn1d.h -- C ABI of the B200 (sm_100a) forward and backward passes of 1D
+ * deformable convolution (DeformConv1d), with optional DCNv2 modulation mask.
  *
  * What the forward computes (sources: the "conv1d" operator page, sections
  * "Description", "Shape" and "Axis convention"; the dc1d page "dc1d
@@ -82,6 +82,45 @@ typedef struct dcn1d_tensor {
  */
 int64_t dcn1d_out_length(int64_t L_in, int64_t kernel_size, int64_t stride, int64_t padding,
                          int64_t dilation);
+
+/*
+ * Padding given per side: `padding_left` zeros before the signal and
+ * `padding_right` after it (the symmetric functions pass the same value for
+ * both).  The dc1d page passes padding="valid" (0) and padding="same"; "same"
+ * is read as nn.Conv1d reads it, whose output-length closed form the page
+ * uses: stride 1, d(K-1)/2 zeros on the left and the rest on the right, so
+ * L_out = L_in (asymmetric when dilation*(kernel_size-1) is odd).  Only the
+ * left side moves the receptive fields, l*stride - padding_left + k*dilation;
+ * both sides enter the length:
+ *   L_out = floor((L_in + padding_left + padding_right - dilation*(K-1) - 1)/stride) + 1.
+ * Returns -1 as dcn1d_out_length does.
+ */
+int64_t dcn1d_out_length_lr(int64_t L_in, int64_t kernel_size, int64_t stride,
+                            int64_t padding_left, int64_t padding_right, int64_t dilation);
+
+/* dcn1d_forward_ws with padding per side (see dcn1d_out_length_lr); otherwise identical. */
+int dcn1d_forward_lr(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                     const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                     const dcn1d_tensor *bias, int64_t stride, int64_t padding_left,
+                     int64_t padding_right, int64_t dilation, int64_t groups,
+                     int64_t offset_groups, int unconstrained, dcn1d_tensor *out,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* dcn1d_forward_kernel_name with padding per side. */
+const char *dcn1d_forward_lr_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                                         const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                                         const dcn1d_tensor *bias, int64_t stride,
+                                         int64_t padding_left, int64_t padding_right,
+                                         int64_t dilation, int64_t groups, int64_t offset_groups,
+                                         int unconstrained, const dcn1d_tensor *out);
+
+/* dcn1d_forward_workspace_size with padding per side. */
+int64_t dcn1d_forward_lr_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                                        const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                                        const dcn1d_tensor *bias, int64_t stride,
+                                        int64_t padding_left, int64_t padding_right,
+                                        int64_t dilation, int64_t groups, int64_t offset_groups,
+                                        int unconstrained, const dcn1d_tensor *out);
 
 /*
  * The deformable convolution forward (formula at the top of this file).
@@ -227,6 +266,24 @@ int dcn1d_backward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn
                    int unconstrained, dcn1d_tensor *grad_x, dcn1d_tensor *grad_offsets,
                    dcn1d_tensor *grad_mask, dcn1d_tensor *grad_weight, dcn1d_tensor *grad_bias,
                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* dcn1d_backward and its workspace size with padding per side (see dcn1d_out_length_lr). */
+int64_t dcn1d_backward_lr_workspace_size(
+    const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
+    const dcn1d_tensor *weight, const dcn1d_tensor *grad_out, int64_t stride,
+    int64_t padding_left, int64_t padding_right, int64_t dilation, int64_t groups,
+    int64_t offset_groups, int unconstrained, const dcn1d_tensor *grad_x,
+    const dcn1d_tensor *grad_offsets, const dcn1d_tensor *grad_mask,
+    const dcn1d_tensor *grad_weight, const dcn1d_tensor *grad_bias);
+
+int dcn1d_backward_lr(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                      const dcn1d_tensor *mask, const dcn1d_tensor *weight,
+                      const dcn1d_tensor *grad_out, int64_t stride, int64_t padding_left,
+                      int64_t padding_right, int64_t dilation, int64_t groups,
+                      int64_t offset_groups, int unconstrained, dcn1d_tensor *grad_x,
+                      dcn1d_tensor *grad_offsets, dcn1d_tensor *grad_mask,
+                      dcn1d_tensor *grad_weight, dcn1d_tensor *grad_bias, void *workspace,
+                      size_t workspace_bytes, void *stream);
 
 /* A static, human-readable name of a status code ("DCN1D_OK", ...). Never NULL. */
 const char *dcn1d_status_string(int status);
