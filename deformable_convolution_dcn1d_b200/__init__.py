@@ -5,6 +5,7 @@ The computation lives in the C-ABI CUDA library ``libdcn1d.so`` (declared in
 """
 from ._binding import (  # noqa: F401
     DCN1D_BF16,
+    DCN1D_F16,
     DCN1D_F32,
     Dcn1dError,
     Dcn1dTensor,

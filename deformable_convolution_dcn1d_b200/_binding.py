@@ -22,7 +22,8 @@ _P = ctypes.c_void_p
 
 DCN1D_F32 = 0
 DCN1D_BF16 = 1
-_DTYPES = {torch.float32: DCN1D_F32, torch.bfloat16: DCN1D_BF16}
+DCN1D_F16 = 2
+_DTYPES = {torch.float32: DCN1D_F32, torch.bfloat16: DCN1D_BF16, torch.float16: DCN1D_F16}
 _BAD_DTYPE = 99   # any other torch dtype: the library rejects it with DCN1D_ERR_DTYPE
 
 STATUS = {0: "DCN1D_OK", 1: "DCN1D_ERR_NULL", 2: "DCN1D_ERR_DTYPE", 3: "DCN1D_ERR_SHAPE",
@@ -204,7 +205,7 @@ def dcn1d_forward(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=
 
     x [B, C_in, L_in]; offsets and mask [B, offset_groups, L_out, K] (mask may be None);
     weight [C_out, C_in/groups, K]; bias [C_out] or None.  All CUDA, contiguous, one dtype
-    (float32 or bfloat16).  ``padding``: an int, a (left, right) pair, "valid" or "same"
+    (float32, bfloat16 or float16).  ``padding``: an int, a (left, right) pair, "valid" or "same"
     (see resolve_padding).  ``out`` is allocated with torch when not given.  The scratch the
     fastest path needs (``dcn1d_forward_workspace_size``) is allocated with torch unless a
     uint8 CUDA tensor ``workspace`` is given; ``workspace=False`` asks for the path without

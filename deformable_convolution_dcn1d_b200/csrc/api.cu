@@ -26,7 +26,7 @@ int64_t numel(const dcn1d_tensor *t) {
 int check_desc(const dcn1d_tensor *t, int ndim) {
     if (!t)
         return DCN1D_ERR_NULL;
-    if (t->dtype != DCN1D_F32 && t->dtype != DCN1D_BF16)
+    if (t->dtype != DCN1D_F32 && t->dtype != DCN1D_BF16 && t->dtype != DCN1D_F16)
         return DCN1D_ERR_DTYPE;
     if (t->ndim != ndim)
         return DCN1D_ERR_SHAPE;
@@ -449,7 +449,10 @@ const char *dcn1d_forward_lr_kernel_name(const dcn1d_tensor *x, const dcn1d_tens
     if (validate(x, offsets, mask, weight, bias, stride, padding_left, padding_right, dilation,
                  groups, offset_groups, unconstrained, out, &P) != DCN1D_OK)
         return nullptr;
-    return kernel_names[select_kernel(P, SIZE_MAX)];
+    const Kernel k = select_kernel(P, SIZE_MAX);
+    if (k == kTcBf16 && P.dtype == DCN1D_F16)
+        return "tcgen05_f16";   // the same 16-bit tensor-core kernel with fp16 operands
+    return kernel_names[k];
 }
 
 const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor *offsets,

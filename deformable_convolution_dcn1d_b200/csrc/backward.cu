@@ -434,9 +434,11 @@ size_t backward_workspace(const Problem &P, const BackwardGrads &G) {
 cudaError_t launch_backward(const Problem &P, const BackwardGrads &G, void *workspace,
                             cudaStream_t stream, int *launches) {
     *launches = 0;
-    return P.dtype == DCN1D_BF16
-               ? run_backward<__nv_bfloat16>(P, G, workspace, stream, launches)
-               : run_backward<float>(P, G, workspace, stream, launches);
+    if (P.dtype == DCN1D_BF16)
+        return run_backward<__nv_bfloat16>(P, G, workspace, stream, launches);
+    if (P.dtype == DCN1D_F16)
+        return run_backward<__half>(P, G, workspace, stream, launches);
+    return run_backward<float>(P, G, workspace, stream, launches);
 }
 
 }  // namespace dcn1d

@@ -366,6 +366,8 @@ cudaError_t launch_t(const Problem &P, cudaStream_t stream) {
 }  // namespace
 
 bool depthwise_supported(const Problem &P) {
+    if (P.dtype == DCN1D_F16)   // the window packing reads bf16 bit patterns
+        return false;
     if (!(P.groups == P.C_in && P.C_out == P.C_in))
         return false;
     if (!(P.K == 1 || P.K == 2 || P.K == 3 || P.K == 4 || P.K == 5 || P.K == 7 || P.K == 9))

@@ -59,6 +59,8 @@ cudaError_t launch_direct(const Problem &P, cudaStream_t stream) {
     const int64_t blocks = (total + threads - 1) / threads;
     if (P.dtype == DCN1D_F32)
         direct_kernel<float><<<(unsigned)blocks, threads, 0, stream>>>(P, total);
+    else if (P.dtype == DCN1D_F16)
+        direct_kernel<__half><<<(unsigned)blocks, threads, 0, stream>>>(P, total);
     else
         direct_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, stream>>>(P, total);
     return cudaGetLastError();

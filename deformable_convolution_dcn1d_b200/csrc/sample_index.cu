@@ -40,6 +40,10 @@ cudaError_t launch_sample_index(const void *off, int dtype, int B, int G, int L_
         sample_index_kernel<float><<<blocks, threads, 0, stream>>>(
             static_cast<const float *>(off), total, L_out, K, stride, padding, dilation,
             unconstrained, i0, frac);
+    else if (dtype == DCN1D_F16)
+        sample_index_kernel<__half><<<blocks, threads, 0, stream>>>(
+            static_cast<const __half *>(off), total, L_out, K, stride, padding, dilation,
+            unconstrained, i0, frac);
     else
         sample_index_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(
             static_cast<const __nv_bfloat16 *>(off), total, L_out, K, stride, padding, dilation,

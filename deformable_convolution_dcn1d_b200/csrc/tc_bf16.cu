@@ -1,5 +1,6 @@
-// Fused deformable-im2col + tcgen05 tensor-core contraction, bf16 inputs and
-// fp32 accumulation (conv groups with C_out/groups <= 256).
+// Fused deformable-im2col + tcgen05 tensor-core contraction, 16-bit inputs (bf16,
+// or fp16: the same kernel with the element type a template parameter) and fp32
+// accumulation (conv groups with C_out/groups <= 256).
 //
 // Per conv group g the forward is a GEMM over the reduction index kk = (ci, k)
 // of the group (k fastest, the weight's own order):
@@ -100,34 +101,72 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t u) {
-    return *reinterpret_cast<__nv_bfloat162 *>(&u);
-}
-__device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 h) {
-    return *reinterpret_cast<uint32_t *>(&h);
-}
+// The 16-bit element type E of a problem (bf16 or fp16): its pair type, packing,
+// unpacking, TMA data type and MMA instruction descriptor (kind::f16 takes both).
+template <class E>
+struct Elem;
 
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+template <>
+struct Elem<__nv_bfloat16> {
+    using E2 = __nv_bfloat162;
+    static constexpr CUtensorMapDataType kTma = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    static __host__ __device__ constexpr uint32_t idesc(int M, int N) {
+        return idesc_bf16_f32(M, N);
+    }
+    static __device__ __forceinline__ uint32_t pack(float a, float b) {
+        E2 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+    static __device__ __forceinline__ float lo(uint32_t u) { return __uint_as_float(u << 16); }
+    static __device__ __forceinline__ float hi(uint32_t u) {
+        return __uint_as_float(u & 0xFFFF0000u);
+    }
+};
+
+template <>
+struct Elem<__half> {
+    using E2 = __half2;
+    static constexpr CUtensorMapDataType kTma = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    static __host__ __device__ constexpr uint32_t idesc(int M, int N) {
+        return idesc_f16_f32(M, N);
+    }
+    static __device__ __forceinline__ uint32_t pack(float a, float b) {
+        E2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+    static __device__ __forceinline__ float lo(uint32_t u) {
+        return __half2float(__ushort_as_half((unsigned short)(u & 0xFFFFu)));
+    }
+    static __device__ __forceinline__ float hi(uint32_t u) {
+        return __half2float(__ushort_as_half((unsigned short)(u >> 16)));
+    }
+};
+
+template <class E>
+__device__ __forceinline__ typename Elem<E>::E2 as_e2(uint32_t u) {
+    return *reinterpret_cast<typename Elem<E>::E2 *>(&u);
+}
+template <class E>
+__device__ __forceinline__ uint32_t as_u32(typename Elem<E>::E2 h) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
 // Per-row tap state of one offset group.  Elements come in pairs (kk, kk+1),
 // i.e. taps (k, (k+1) % K), so fractions and mask values are kept pre-packed
-// as bf16x2 pairs indexed by the first tap of the pair.
+// as 16-bit pairs indexed by the first tap of the pair.
 template <int K>
 struct Taps {
     uint32_t addr[K];    // byte offset of the tap's neighbour pair in a stage row
-    uint32_t fpair[K];   // bf16x2 (f_k, f_{(k+1)%K})
-    uint32_t mpair[K];   // bf16x2 (m_k, m_{(k+1)%K})
+    uint32_t fpair[K];   // E x2 (f_k, f_{(k+1)%K})
+    uint32_t mpair[K];   // E x2 (m_k, m_{(k+1)%K})
     float pos[K];        // position, for taps outside the window (slow path)
     uint32_t slow;       // bit k: tap k outside the staged window
 };
 
 // The col value of one element by the slow path: exact floor, global loads.
-template <int K, bool MASK>
+template <class E, int K, bool MASK>
 __device__ __forceinline__ float slow_element(const Taps<K> &tp, int kidx, int hi,
-                                              const __nv_bfloat16 *row, int L_in) {
+                                              const E *row, int L_in) {
     const Tap e = tap_floor_exact(tp.pos[kidx]);
     const float x0 = (e.i0 >= 0 && e.i0 < L_in) ? ld_f32(row + e.i0) : 0.0f;
     const float x1 = (e.i0 >= -1 && e.i0 < L_in - 1) ? ld_f32(row + e.i0 + 1) : 0.0f;
@@ -135,15 +174,15 @@ __device__ __forceinline__ float slow_element(const Taps<K> &tp, int kidx, int h
     if (!MASK)
         return r;
     const uint32_t mp = tp.mpair[(kidx + K - hi) % K];
-    return __fmul_rn(r, __uint_as_float(hi ? (mp & 0xFFFF0000u) : (mp << 16)));
+    return __fmul_rn(r, hi ? Elem<E>::hi(mp) : Elem<E>::lo(mp));
 }
 
 // Col values 2I and 2I+1 of a segment whose first element has phase K0 = kk0 % K:
 // taps (k0, k1) of channel rows (c0, c1) relative to the segment's first channel.
 // The lerp x0 + f (x1 - x0) runs on the two elements in bf16x2 arithmetic.
-template <int K, int K0, bool MASK, bool SLOW, int I>
+template <class E, int K, int K0, bool MASK, bool SLOW, int I>
 __device__ __forceinline__ void produce_pair(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
-                                             const uint32_t (&base)[K], const __nv_bfloat16 *xg,
+                                             const uint32_t (&base)[K], const E *xg,
                                              int64_t xg_row_stride, int L_in) {
     constexpr int k0 = (K0 + 2 * I) % K, c0 = (K0 + 2 * I) / K;
     constexpr int k1 = (K0 + 2 * I + 1) % K, c1 = (K0 + 2 * I + 1) / K;
@@ -152,52 +191,53 @@ __device__ __forceinline__ void produce_pair(uint32_t (&out)[kSeg / 2], const Ta
         __byte_perm(lds_u16<o0>(base[k0]), lds_u16<o1>(base[k1]), 0x5410);
     const uint32_t x1 =
         __byte_perm(lds_u16<o0 + 2>(base[k0]), lds_u16<o1 + 2>(base[k1]), 0x5410);
-    __nv_bfloat162 v = __hfma2(as_bf2(tp.fpair[k0]), __hsub2(as_bf2(x1), as_bf2(x0)), as_bf2(x0));
+    typename Elem<E>::E2 v = __hfma2(as_e2<E>(tp.fpair[k0]),
+                                     __hsub2(as_e2<E>(x1), as_e2<E>(x0)), as_e2<E>(x0));
     if (MASK)
-        v = __hmul2(v, as_bf2(tp.mpair[k0]));
-    out[I] = as_u32(v);
+        v = __hmul2(v, as_e2<E>(tp.mpair[k0]));
+    out[I] = as_u32<E>(v);
     if (SLOW && (((tp.slow >> k0) | (tp.slow >> k1)) & 1u)) {
         float lo = __low2float(v), hi = __high2float(v);
         if ((tp.slow >> k0) & 1u)
-            lo = slow_element<K, MASK>(tp, k0, 0, xg + c0 * xg_row_stride, L_in);
+            lo = slow_element<E, K, MASK>(tp, k0, 0, xg + c0 * xg_row_stride, L_in);
         if ((tp.slow >> k1) & 1u)
-            hi = slow_element<K, MASK>(tp, k1, 1, xg + c1 * xg_row_stride, L_in);
-        out[I] = pack2(lo, hi);
+            hi = slow_element<E, K, MASK>(tp, k1, 1, xg + c1 * xg_row_stride, L_in);
+        out[I] = Elem<E>::pack(lo, hi);
     }
 }
 
-template <int K, int K0, bool MASK, bool SLOW, int... Is>
+template <class E, int K, int K0, bool MASK, bool SLOW, int... Is>
 __device__ __forceinline__ void produce_pairs(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
-                                              const uint32_t (&base)[K], const __nv_bfloat16 *xg,
+                                              const uint32_t (&base)[K], const E *xg,
                                               int64_t xg_row_stride, int L_in,
                                               std::integer_sequence<int, Is...>) {
-    (produce_pair<K, K0, MASK, SLOW, Is>(out, tp, base, xg, xg_row_stride, L_in), ...);
+    (produce_pair<E, K, K0, MASK, SLOW, Is>(out, tp, base, xg, xg_row_stride, L_in), ...);
 }
 
 // kSeg col values of one row for the reduction elements kk0 .. kk0+kSeg-1 of a k-block,
 // packed bf16x2 (element 2i in the low half of out[i]).  Phase K0 = kk0 % K is a
 // compile-time constant, so every tap index and row offset below is static.
-template <int K, int K0, bool MASK, bool SLOW>
+template <class E, int K, int K0, bool MASK, bool SLOW>
 __device__ __forceinline__ void produce_segment(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
-                                                uint32_t xrow_addr, const __nv_bfloat16 *xg,
+                                                uint32_t xrow_addr, const E *xg,
                                                 int64_t xg_row_stride, int L_in) {
     uint32_t base[K];
 #pragma unroll
     for (int k = 0; k < K; ++k)
         base[k] = xrow_addr + tp.addr[k];
-    produce_pairs<K, K0, MASK, SLOW>(out, tp, base, xg, xg_row_stride, L_in,
+    produce_pairs<E, K, K0, MASK, SLOW>(out, tp, base, xg, xg_row_stride, L_in,
                                      std::make_integer_sequence<int, kSeg / 2>{});
 }
 
 // Jump to the segment code of phase k0 (a switch, so one indirect branch).
-template <int K, bool MASK, bool SLOW>
+template <class E, int K, bool MASK, bool SLOW>
 __device__ __forceinline__ void produce_dispatch(int k0, uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
-                                                 uint32_t xrow_addr, const __nv_bfloat16 *xg,
+                                                 uint32_t xrow_addr, const E *xg,
                                                  int64_t xg_row_stride, int L_in) {
 #define DCN1D_PHASE(P_)                                                                          \
     case P_:                                                                                    \
         if constexpr (P_ < K)                                                                   \
-            produce_segment<K, (P_ < K ? P_ : 0), MASK, SLOW>(out, tp, xrow_addr, xg,             \
+            produce_segment<E, K, (P_ < K ? P_ : 0), MASK, SLOW>(out, tp, xrow_addr, xg,          \
                                                               xg_row_stride, L_in);             \
         break;
     switch (k0) {
@@ -208,7 +248,7 @@ __device__ __forceinline__ void produce_dispatch(int k0, uint32_t (&out)[kSeg / 
 #undef DCN1D_PHASE
 }
 
-template <int K, bool MASK>
+template <class E, int K, bool MASK>
 // 18 warps: 5 land on some SM sub-partitions, each of which holds 16K registers,
 // so a thread may use at most 16384 / (5 * 32) -> 96 registers.
 __global__ void __maxnreg__(96)
@@ -229,7 +269,7 @@ __global__ void __maxnreg__(96)
     const uint32_t bar0 = sbase + A.off_bar;
     float *bias_s = reinterpret_cast<float *>(smem + A.off_bias);
     for (int i = threadIdx.x; i < P.C_out; i += kThreads)
-        bias_s[i] = P.bias ? ld_f32(static_cast<const __nv_bfloat16 *>(P.bias) + i) : 0.0f;
+        bias_s[i] = P.bias ? ld_f32(static_cast<const E *>(P.bias) + i) : 0.0f;
     auto bar_full = [&](int s) { return bar0 + 8u * s; };
     auto bar_empty = [&](int s) { return bar0 + 8u * (kStages + s); };
     auto bar_afull = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
@@ -298,7 +338,7 @@ __global__ void __maxnreg__(96)
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, A.N);
+            const uint32_t idesc = Elem<E>::idesc(128, A.N);
             uint32_t it = 0, tc = 0;
             for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
                 if (!wait(bar_dempty, (tc & 1u) ^ 1u))
@@ -344,7 +384,7 @@ __global__ void __maxnreg__(96)
             if (!__all_sync(0xffffffffu, wait(bar_dfull, tcnt & 1u)))
                 return false;
             tc_fence_after();
-            __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(P.out) +
+            E *outp = static_cast<E *>(P.out) +
                                   ((int64_t)T.b * P.C_out + (int64_t)T.g * P.cout_g) * P.L_out + l;
             for (int cc = h; cc < A.N / 16; cc += 4) {
                 uint32_t v[16];
@@ -355,7 +395,7 @@ __global__ void __maxnreg__(96)
                     for (int i = 0; i < 16; ++i) {
                         const int co = 16 * cc + i;
                         outp[(int64_t)co * P.L_out] =
-                            __float2bfloat16_rn(__uint_as_float(v[i]) + biasg[co]);
+                            from_f32<E>(__uint_as_float(v[i]) + biasg[co]);
                     }
                 }
             }
@@ -383,8 +423,8 @@ __global__ void __maxnreg__(96)
                 (((int64_t)T.b * P.offset_groups + og) * P.L_out + (l < P.L_out ? l : 0)) * K;
 #pragma unroll
             for (int k = 0; k < K; ++k) {
-                raw_off[k] = ld_f32(static_cast<const __nv_bfloat16 *>(P.off) + obase + k);
-                raw_m[k] = MASK ? ld_f32(static_cast<const __nv_bfloat16 *>(P.mask) + obase + k) : 1.0f;
+                raw_off[k] = ld_f32(static_cast<const E *>(P.off) + obase + k);
+                raw_m[k] = MASK ? ld_f32(static_cast<const E *>(P.mask) + obase + k) : 1.0f;
             }
         };
         if ((int)blockIdx.x < A.num_tiles) {
@@ -399,8 +439,7 @@ __global__ void __maxnreg__(96)
             const float start = (float)(l * P.stride - P.padding);
             const uint32_t win_bits = kFloorMagicBits + (uint32_t)T.wx0;
             const int og_last = (T.g * P.cin_g + P.cin_g - 1) / P.cin_per_og;
-            const __nv_bfloat16 *xb =
-                static_cast<const __nv_bfloat16 *>(P.x) + (int64_t)T.b * P.C_in * P.L_in;
+            const E *xb = static_cast<const E *>(P.x) + (int64_t)T.b * P.C_in * P.L_in;
             Taps<K> tp;
             // Offset group of the first channel of this warp's first segment; it only
             // grows with the channel, so it is tracked against the next boundary.
@@ -453,8 +492,8 @@ __global__ void __maxnreg__(96)
                     }
 #pragma unroll
                     for (int k = 0; k < K; ++k) {
-                        tp.fpair[k] = pack2(f[k], f[(k + 1) % K]);
-                        tp.mpair[k] = pack2(m[k], m[(k + 1) % K]);
+                        tp.fpair[k] = Elem<E>::pack(f[k], f[(k + 1) % K]);
+                        tp.mpair[k] = Elem<E>::pack(m[k], m[(k + 1) % K]);
                     }
                     // next group: the following offset group of this tile, else the
                     // first one of the next tile
@@ -470,14 +509,14 @@ __global__ void __maxnreg__(96)
                 {
                     const uint32_t xrow_addr =
                         x_st0 + s * A.x_stage_bytes + (uint32_t)(c_first - c_lo) * kRowBytes;
-                    const __nv_bfloat16 *xg =
+                    const E *xg =
                         xb + (int64_t)(T.g * P.cin_g + c_first) * P.L_in;
                     uint32_t packed[kSeg / 2];
                     if (__any_sync(0xffffffffu, tp.slow != 0))
-                        produce_dispatch<K, MASK, true>(k0, packed, tp, xrow_addr, xg, P.L_in,
+                        produce_dispatch<E, K, MASK, true>(k0, packed, tp, xrow_addr, xg, P.L_in,
                                                         P.L_in);
                     else
-                        produce_dispatch<K, MASK, false>(k0, packed, tp, xrow_addr, xg, P.L_in,
+                        produce_dispatch<E, K, MASK, false>(k0, packed, tp, xrow_addr, xg, P.L_in,
                                                          P.L_in);
                     tmem_st16(tmem + ((uint32_t)(32 * q) << 16) + kColA + 32u * s + 16u * half,
                               packed);
@@ -559,18 +598,18 @@ bool make_plan(const Problem &P, Plan *out) {
     return true;
 }
 
-template <int K, bool MASK>
+template <class E, int K, bool MASK>
 cudaError_t launch_km(const Plan &pl, cudaStream_t stream) {
     const Problem &P = pl.A.P;
     alignas(64) CUtensorMap wmap, xmap;
     const int Kg = P.cin_g * P.K;
-    if (!encode_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P.w, (uint64_t)Kg, (uint64_t)P.C_out,
+    if (!encode_2d(&wmap, Elem<E>::kTma, P.w, (uint64_t)Kg, (uint64_t)P.C_out,
                    2, kBK, (uint32_t)pl.A.N, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    if (!encode_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P.x, (uint64_t)P.L_in,
+    if (!encode_2d(&xmap, Elem<E>::kTma, P.x, (uint64_t)P.L_in,
                    (uint64_t)P.B * P.C_in, 2, kBox, (uint32_t)pl.A.nch, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    auto kern = tc_bf16_kernel<K, MASK>;
+    auto kern = tc_bf16_kernel<E, K, MASK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)pl.smem);
     if (e != cudaSuccess)
@@ -585,16 +624,28 @@ cudaError_t launch_km(const Plan &pl, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <int K>
+template <class E, int K>
 cudaError_t launch_k(const Plan &pl, cudaStream_t stream) {
-    return pl.A.P.mask ? launch_km<K, true>(pl, stream) : launch_km<K, false>(pl, stream);
+    return pl.A.P.mask ? launch_km<E, K, true>(pl, stream) : launch_km<E, K, false>(pl, stream);
+}
+
+template <class E>
+cudaError_t launch_e(const Plan &pl, cudaStream_t stream) {
+    switch (pl.A.P.K) {
+    case 3: return launch_k<E, 3>(pl, stream);
+    case 4: return launch_k<E, 4>(pl, stream);
+    case 5: return launch_k<E, 5>(pl, stream);
+    case 7: return launch_k<E, 7>(pl, stream);
+    case 9: return launch_k<E, 9>(pl, stream);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
 
 
 bool tc_bf16_supported(const Problem &P) {
-    if (P.dtype != DCN1D_BF16 || !fast_floor_ok(P))
+    if ((P.dtype != DCN1D_BF16 && P.dtype != DCN1D_F16) || !fast_floor_ok(P))
         return false;
     if (!(P.K == 3 || P.K == 4 || P.K == 5 || P.K == 7 || P.K == 9))
         return false;
@@ -623,14 +674,8 @@ cudaError_t launch_tc_bf16(const Problem &P, cudaStream_t stream) {
     pl.A.status = device_status_ptr();
     if (!pl.A.status)
         return cudaErrorInvalidDevice;
-    switch (P.K) {
-    case 3: return launch_k<3>(pl, stream);
-    case 4: return launch_k<4>(pl, stream);
-    case 5: return launch_k<5>(pl, stream);
-    case 7: return launch_k<7>(pl, stream);
-    case 9: return launch_k<9>(pl, stream);
-    default: return cudaErrorInvalidValue;
-    }
+    return P.dtype == DCN1D_F16 ? launch_e<__half>(pl, stream)
+                                : launch_e<__nv_bfloat16>(pl, stream);
 }
 
 }  // namespace dcn1d

@@ -62,7 +62,8 @@ typedef enum dcn1d_status {
 
 typedef enum dcn1d_dtype {
     DCN1D_F32 = 0,             /* IEEE float32                                             */
-    DCN1D_BF16 = 1             /* bfloat16                                                 */
+    DCN1D_BF16 = 1,            /* bfloat16                                                 */
+    DCN1D_F16 = 2              /* IEEE float16 (binary16)                                  */
 } dcn1d_dtype;
 
 /* A dense, contiguous, row-major device array of `ndim` (<= 4) dimensions. */

@@ -9,8 +9,8 @@ oracle), so no closed form lives here.
 
 Recipe (applies to every workload): one CPU ``torch.Generator`` seeded with
 ``seed`` (default 0); tensors are drawn in float32 in the fixed order
-x, weight, bias, offsets, mask, and cast to bfloat16 afterwards where the
-workload is bf16.  ``N(0, s)`` means mean 0 and standard deviation ``s``.
+x, weight, bias, offsets, mask, and cast to bfloat16 (float16) afterwards where the
+workload is bf16 (f16).  ``N(0, s)`` means mean 0 and standard deviation ``s``.
 """
 from __future__ import annotations
 
@@ -37,7 +37,7 @@ class Workload:
     offset_groups: int
     L_in: int
     L_out: int                # stated with the workload, not computed here
-    dtype: str                # "f32" or "bf16"
+    dtype: str                # "f32", "bf16" or "f16"
     x_dist: tuple             # ("uniform", lo, hi) | ("normal", std)
     w_dist: tuple             # ("normal", std) | ("kaiming_uniform",) | ("kaiming_normal",)
     bias_dist: Optional[tuple]
@@ -47,7 +47,7 @@ class Workload:
 
     @property
     def torch_dtype(self) -> torch.dtype:
-        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+        return {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[self.dtype]
 
     @property
     def fan_in(self) -> int:
