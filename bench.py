@@ -310,21 +310,15 @@ def run_ours(args, w: W.Workload, peaks: dict, want_cpu: bool):
     torch.cuda.synchronize(dev)
     launches_per_step = dcn.dcn1d_last_launch_count()
 
-    # ---- device-resident timing
+    # ---- device-resident timing: K steps, events around each whole step
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    # The library records these around its main kernel (helper kernels stay outside).
-    k_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    k_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    for e in k_starts + k_ends:
-        e.record(stream)   # creates the CUDA event (torch creates events lazily)
     barrier(ws)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)
-            dcn.dcn1d_set_timing_events(k_starts[i], k_ends[i])
             step(dev_in, out)
             ends[i].record(stream)
         torch.cuda.synchronize(dev)
@@ -332,6 +326,22 @@ def run_ours(args, w: W.Workload, peaks: dict, want_cpu: bool):
     ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     ms = max_over_ranks(ms, ws)
     ms_step = ms / args.steps
+
+    # ---- the main kernel's own time: a second run of the same K steps in which the
+    # library records events right around its main kernel (the events add a few us to
+    # each step, so they stay out of the run that gives the step time above)
+    k_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for e in k_starts + k_ends:
+        e.record(stream)   # creates the CUDA event (torch creates events lazily)
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        dcn.dcn1d_set_timing_events(k_starts[i], k_ends[i])
+        step(dev_in, out)
+    torch.cuda.synchronize(dev)
+    barrier(ws)
     ms_kernel = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(k_starts, k_ends)),
                                ws) / args.steps
     value, unit = unit_value(w, kernel, ms_step / 1e3, ws)
@@ -374,7 +384,8 @@ def run_ours(args, w: W.Workload, peaks: dict, want_cpu: bool):
             "frac": achieved / peak, "traffic": load_traffic(kernel, w), "kernel": kernel,
             "peak_source": note, "launches_per_step": launches_per_step,
             "kernel_ms": ms_kernel,
-            "timing": "CUDA events the library records around its main kernel, per step"}
+            "timing": "CUDA events the library records around its main kernel, per step, "
+                      "in a second timed run of the same K steps"}
 
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,

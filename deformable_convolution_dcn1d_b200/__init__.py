@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     Dcn1dTensor,
     GRADS,
     SIGNATURES,
+    clear_workspace_cache,
     dcn1d_backward,
     dcn1d_backward_workspace_size,
     dcn1d_device_status,

@@ -7,6 +7,7 @@ is no Python or CPU fallback, and a missing or unbuildable library raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -33,6 +34,9 @@ STATUS = {0: "DCN1D_OK", 1: "DCN1D_ERR_NULL", 2: "DCN1D_ERR_DTYPE", 3: "DCN1D_ER
 
 class Dcn1dTensor(ctypes.Structure):
     _fields_ = [("data", _P), ("dtype", _I32), ("ndim", _I32), ("shape", _I64 * 4)]
+
+
+_SHAPE4 = _I64 * 4
 
 
 class Dcn1dError(RuntimeError):
@@ -107,6 +111,8 @@ def lib_path() -> str:
 def load():
     """Load libdcn1d.so, building it from csrc/ with nvcc if it is missing or stale."""
     global _lib
+    if _lib is not None:
+        return _lib
     with _lock:
         if _lib is None:
             path = _build.build()
@@ -131,13 +137,9 @@ def _desc(t):
         raise ValueError("at most 4 dimensions")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
-    d = Dcn1dTensor()
-    d.data = t.data_ptr() if t.numel() > 0 else None
-    d.dtype = _DTYPES.get(t.dtype, _BAD_DTYPE)
-    d.ndim = t.ndim
-    for i, s in enumerate(t.shape):
-        d.shape[i] = s
-    return d
+    shape = t.shape
+    return Dcn1dTensor(t.data_ptr() if t.numel() > 0 else None,
+                       _DTYPES.get(t.dtype, _BAD_DTYPE), len(shape), _SHAPE4(*shape))
 
 
 def _ref(d):
@@ -209,36 +211,63 @@ def dcn1d_forward(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=
     (see resolve_padding).  ``out`` is allocated with torch when not given.  The scratch the
     fastest path needs (``dcn1d_forward_workspace_size``) is allocated with torch unless a
     uint8 CUDA tensor ``workspace`` is given; ``workspace=False`` asks for the path without
-    scratch.  Runs on ``stream`` (default: the current torch stream of x's device); does not
-    synchronise.
+    scratch.  Without ``workspace`` the scratch is kept for later calls on the same device
+    and stream (see clear_workspace_cache).  Runs on ``stream`` (default: the current torch
+    stream of x's device); does not synchronise.
     """
     pl, pr = resolve_padding(padding, weight.shape[2], stride, dilation)
     dev = _check_device((x, offsets, mask, weight, bias, out))
     if out is None:
         out = _out_for(x, weight, offsets)
-    descs = [_desc(t) for t in (x, offsets, mask, weight, bias, out)]
+    tensors = (x, offsets, mask, weight, bias, out)
+    refs = [_ref(_desc(t)) for t in tensors]
     lib = load()
-    refs = [_ref(d) for d in descs]
-    with torch.cuda.device(dev):
+    args = (stride, pl, pr, dilation, groups, offset_groups, int(bool(unconstrained)))
+    ctx = (contextlib.nullcontext() if torch.cuda.current_device() == dev.index
+           else torch.cuda.device(dev))
+    with ctx:
+        sptr = _stream_ptr(stream, dev)
         ws_ptr, ws_bytes = None, 0
         if workspace is not False:
-            need = int(lib.dcn1d_forward_lr_workspace_size(*refs[:5], stride, pl, pr, dilation,
-                                                           groups, offset_groups,
-                                                           int(bool(unconstrained)), refs[5]))
-            if need < 0:
-                raise Dcn1dError(-need, "dcn1d_forward_workspace_size")
+            key = (dev.index, args, tuple(None if t is None else
+                                          (tuple(t.shape), t.dtype, t.data_ptr() % 256)
+                                          for t in tensors))
+            need = _need_cache.get(key)
+            if need is None:
+                need = int(lib.dcn1d_forward_lr_workspace_size(*refs[:5], *args, refs[5]))
+                if need < 0:
+                    raise Dcn1dError(-need, "dcn1d_forward_workspace_size")
+                if len(_need_cache) > 4096:
+                    _need_cache.clear()
+                _need_cache[key] = need
             if need > 0:
                 if workspace is None:
-                    workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+                    workspace = _ws_cache.get((dev.index, sptr))
+                    if workspace is None or workspace.numel() < need:
+                        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+                        if isinstance(stream, torch.cuda.Stream):
+                            workspace.record_stream(stream)
+                        _ws_cache[(dev.index, sptr)] = workspace
                 if workspace.numel() < need or workspace.dtype != torch.uint8:
                     raise ValueError(f"workspace must be a uint8 tensor of >= {need} bytes")
                 ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
-        st = lib.dcn1d_forward_lr(*refs[:5], stride, pl, pr, dilation, groups, offset_groups,
-                                  int(bool(unconstrained)), refs[5], _P(ws_ptr), ws_bytes,
-                                  _P(_stream_ptr(stream, dev)))
+        st = lib.dcn1d_forward_lr(*refs[:5], *args, refs[5], _P(ws_ptr), ws_bytes, _P(sptr))
     if st != 0:
         raise Dcn1dError(st, "dcn1d_forward")
     return out
+
+
+# Scratch reused by dcn1d_forward calls that pass no workspace: one uint8 tensor per
+# (device, stream), grown when a call needs more (calls on one stream run in order, so
+# they can share it); and the scratch size of each call signature seen.
+_ws_cache = {}
+_need_cache = {}
+
+
+def clear_workspace_cache() -> None:
+    """Drop the scratch tensors dcn1d_forward keeps between calls."""
+    _ws_cache.clear()
+    _need_cache.clear()
 
 
 GRADS = ("x", "offsets", "mask", "weight", "bias")

@@ -1,36 +1,66 @@
-// Host helpers shared by the tensor-core kernels: the tensor-map encoder and the
-// SM count, both queried from the runtime once per process / device.
+// Host helpers shared by the tensor-core kernels: the tensor-map encoder, the SM
+// count and the kernels' shared-memory limits, each queried or set once per process /
+// device.
+#include <atomic>
+#include <mutex>
+
 #include "sm100.cuh"
 
 namespace dcn1d {
 
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    static const EncodeTiledFn fn = [] {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return static_cast<EncodeTiledFn>(nullptr);
+    }();
     return fn;
 }
 
 int sm_count() {
-    static int counts[64] = {};
+    static std::atomic<int> counts[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return 0;
-    if (counts[dev] == 0) {
+    if (counts[dev].load(std::memory_order_relaxed) == 0) {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return 0;
-        counts[dev] = n;
+        counts[dev].store(n, std::memory_order_relaxed);
     }
-    return counts[dev];
+    return counts[dev].load(std::memory_order_relaxed);
+}
+
+cudaError_t ensure_smem(const void *kernel, int bytes) {
+    struct Entry {
+        const void *fn;
+        int dev, bytes;
+    };
+    static std::mutex mu;
+    static Entry table[256];
+    static int n = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lock(mu);
+    int i = 0;
+    while (i < n && !(table[i].fn == kernel && table[i].dev == dev))
+        ++i;
+    if (i < n && table[i].bytes >= bytes)
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess)
+        return e;
+    if (i < n)
+        table[i].bytes = bytes;
+    else if (n < 256)
+        table[n++] = Entry{kernel, dev, bytes};
+    return cudaSuccess;
 }
 
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t cols,

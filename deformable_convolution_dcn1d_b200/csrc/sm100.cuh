@@ -255,6 +255,9 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
 EncodeTiledFn encode_fn();
 // Number of SMs of the current device (0 on failure).
 int sm_count();
+// Raises a kernel's dynamic shared-memory limit on the current device, once per size
+// increase (the runtime call costs microseconds; every launch would repeat it).
+cudaError_t ensure_smem(const void *kernel, int bytes);
 // A 2D tiled tensor map over a row-major [rows][cols] array (elements of `elem_bytes`).
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t cols,
                uint64_t rows, uint32_t elem_bytes, uint32_t box_cols, uint32_t box_rows,

@@ -610,8 +610,7 @@ cudaError_t launch_km(const Plan &pl, cudaStream_t stream) {
                    (uint64_t)P.B * P.C_in, 2, kBox, (uint32_t)pl.A.nch, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     auto kern = tc_bf16_kernel<E, K, MASK>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)pl.smem);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), (int)pl.smem);
     if (e != cudaSuccess)
         return e;
     const int sms = sm_count();

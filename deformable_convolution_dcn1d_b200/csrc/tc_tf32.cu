@@ -739,7 +739,7 @@ cudaError_t launch_tf_km(const TfPlan &pl, void *ws, cudaStream_t stream) {
     if (e != cudaSuccess)
         return e;
     auto kern = tc_tf32_kernel<K, MASK>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+    e = ensure_smem(reinterpret_cast<const void *>(kern), (int)pl.smem);
     if (e != cudaSuccess)
         return e;
     const int grid = A.num_units < sms ? A.num_units : sms;
