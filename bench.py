@@ -18,6 +18,7 @@ gradients of one batch per step; the work counted is its two contractions).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -70,6 +71,9 @@ def roofline_for(kernel: str, w: W.Workload, peaks: dict):
         return "hbm", "GB/s", peaks["hbm_gbs"], gbytes, f"HBM copy bandwidth ({src})"
     if kernel.startswith("tcgen05_bf16"):
         return "tensor", "TFLOP/s", peaks["bf16_tflops"], flops, f"bf16 dense GEMM burst ({src})"
+    if kernel.startswith("tcgen05_f16"):
+        return ("tensor", "TFLOP/s", peaks["bf16_tflops"], flops,
+                f"bf16 dense GEMM burst ({src}) x 1 (fp16 and bf16 share the nominal dense rate)")
     if kernel.startswith("tcgen05_3xtf32"):
         pk = peaks["bf16_tflops"] * TF32_OVER_BF16 / 3.0
         return ("tensor", "TFLOP/s", pk, flops,
@@ -99,7 +103,9 @@ def load_traffic(kernel: str, w: W.Workload):
             return None
         if want is not None and h != want:
             return None   # the kernel changed since the counters were taken
-        return float(parts[2])
+        full = W.WORKLOADS.get(w.name)
+        # the recorded figure is per launch of the named workload; a batch override scales it
+        return float(parts[2]) * (w.B / full.B if full is not None else 1.0)
     return None
 
 
@@ -505,6 +511,8 @@ def main():
                     help="time the forward (the default line) or the backward pass")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (small cases for profiling)")
+    ap.add_argument("--dtype", default=None, choices=["f16"],
+                    help="run a bf16 workload's shapes and distributions in float16 instead")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -513,6 +521,10 @@ def main():
 
     def pick(name):
         w = W.WORKLOADS[name]
+        if args.dtype:
+            if w.dtype != "bf16":
+                raise SystemExit("--dtype f16 applies to the bf16 workloads only")
+            w = dataclasses.replace(w, name=w.name.replace("bf16", args.dtype), dtype=args.dtype)
         return w.with_batch(args.batch) if args.batch else w
 
     if args.impl == "reference":
