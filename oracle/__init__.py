@@ -10,7 +10,9 @@ widened to float32 exactly before they reach the C code.
 
 Parity status: every function is pinned by ``tests/test_oracle_pins.py`` (forward)
 and ``tests/test_oracle_backward_pins.py`` (backward: finite differences of the
-forward, conv1d autograd for zero offsets) except the exact clamp bounds of
+forward, conv1d autograd for zero offsets) and ``tests/test_oracle_packed_pins.py``
+(PackedDeformConv1d's offset and mask trunk: torch's float64 conv1d composition, a worked
+example by hand, the zero-initialised mask halving the output) except the exact clamp bounds of
 constrained mode, which no page fixes; those are checked only through invariants
 (locality, saturation) and are "parity unpinned" as to the bounds themselves.
 """
@@ -67,6 +69,8 @@ class Oracle:
         lib.oracle_backward.restype = _int
         lib.oracle_backward.argtypes = [_p] * 5 + [_i64] * 12 + [_int] + [_p] * 5
         lib.oracle_threads.restype = _int
+        lib.oracle_packed_trunk.argtypes = [_p] * 7 + [_i64] * 10 + [_p, _p]
+        lib.oracle_packed_trunk.restype = _int
         lib.oracle_threads.argtypes = []
         lib.oracle_set_threads.restype = None
         lib.oracle_set_threads.argtypes = [_int]
@@ -144,6 +148,48 @@ class Oracle:
             raise ValueError(f"oracle_backward rejected the shapes (code {rc})")
         return g
 
+    def packed_trunk(self, x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias,
+                     kernel_size, stride, padding, dilation, offset_groups):
+        """PackedDeformConv1d's predicted offsets (and mask, None without a mask branch),
+        float64 [B, offset_groups, L_out, K].  dw_weight is [C_in, 1, K] (or [C_in, K]);
+        off_weight and mask_weight are [offset_groups*K, C_in] (or with a trailing 1)."""
+        xs, dws, dbs, ows, obs, mws, mbs = (_f32(t) for t in (x, dw_weight, dw_bias, off_weight,
+                                                              off_bias, mask_weight, mask_bias))
+        B, C_in, L_in = xs.shape
+        K = int(kernel_size)
+        pl, pr = _pads(padding)
+        if dws.size != C_in * K or ows.size != offset_groups * K * C_in:
+            raise ValueError("trunk weight shapes disagree with C_in, K and offset_groups")
+        if mws is not None and mws.size != ows.size:
+            raise ValueError("mask_weight must have off_weight's shape")
+        L_out = self.out_length(L_in, K, stride, (pl, pr), dilation)
+        off = np.empty((B, offset_groups, L_out, K), dtype=np.float64)
+        mask = np.empty_like(off) if mws is not None else None
+        rc = self.lib.oracle_packed_trunk(_ptr(xs), _ptr(dws), _ptr(dbs), _ptr(ows), _ptr(obs),
+                                          _ptr(mws), _ptr(mbs), B, C_in, L_in, K, L_out, stride,
+                                          pl, pr, dilation, offset_groups, _ptr(off), _ptr(mask))
+        if rc != 0:
+            raise ValueError(f"oracle_packed_trunk rejected the arguments (code {rc})")
+        return off, mask
+
+    def packed_forward(self, x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias,
+                       weight, bias, stride, padding, dilation, groups, offset_groups,
+                       unconstrained, dtype=None):
+        """PackedDeformConv1d's output: the trunk's offsets (and mask), rounded to ``dtype``
+        (x's own dtype by default: the tensor the layer passes on), then the forward.
+        Returns (out float64, offsets float64, mask float64 or None), the latter two
+        before that rounding."""
+        K = weight.shape[2]
+        off, mask = self.packed_trunk(x, dw_weight, dw_bias, off_weight, off_bias, mask_weight,
+                                      mask_bias, K, stride, padding, dilation, offset_groups)
+        dt = dtype if dtype is not None else (x.dtype if isinstance(x, torch.Tensor)
+                                              else torch.float32)
+        off_r = torch.from_numpy(off).to(dt)
+        mask_r = torch.from_numpy(mask).to(dt) if mask is not None else None
+        out = self.forward(x, off_r, mask_r, weight, bias, stride, padding, dilation, groups,
+                           offset_groups, unconstrained)
+        return out, off, mask
+
     def sample_index(self, offsets, L_in, K, stride, padding, dilation, unconstrained):
         """(i0 int32, frac float32) for every tap, each shaped like ``offsets``."""
         os_ = _f32(offsets)
@@ -190,6 +236,14 @@ def sample_index(*a, **k):
 
 def backward(*a, **k):
     return get().backward(*a, **k)
+
+
+def packed_trunk(*a, **k):
+    return get().packed_trunk(*a, **k)
+
+
+def packed_forward(*a, **k):
+    return get().packed_forward(*a, **k)
 
 
 def threads():

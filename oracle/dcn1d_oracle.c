@@ -365,3 +365,71 @@ int oracle_backward(const float *x, const float *off, const float *mask, const f
         }
     return 0;
 }
+
+/* ------------------------------------------------------------------ packed trunk
+ *
+ * The offset (and mask) predictor of PackedDeformConv1d.  Sources: "dc1d
+ * (DeformConv1d)" page, "PackedDeformConv1d": the layer computes its offsets
+ * itself with a depthwise-separable convolution block; "Modulation (DCNv2)":
+ * with modulated=True a second pointwise branch off the same depthwise trunk
+ * predicts the mask and ends in a sigmoid.  The deformable-convolution article,
+ * "Step 1: Offset Generation", makes the offset stage an ordinary convolution
+ * over the input whose output channels are the offsets of every tap.
+ *
+ *   t[b,c,l]      = dw_b[c] + sum_k dw_w[c,k] * X(b, c, l*s - pl + k*d)
+ *   off[b,g,l,k]  = off_b[g*K+k]  + sum_c off_w[g*K+k, c]  * t[b,c,l]
+ *   mask[b,g,l,k] = sigmoid(mask_b[g*K+k] + sum_c mask_w[g*K+k, c] * t[b,c,l])
+ *
+ * Readings where the pages are silent (listed in the design notes): the
+ * depthwise convolution takes the layer's own kernel size, stride, padding and
+ * dilation (so it yields one offset vector per output position); nothing sits
+ * between the depthwise and the pointwise convolution; pointwise output channel
+ * g*K + k is the offset (mask) of tap k of offset group g.  Every bias may be NULL
+ * (none); mask_w NULL means no mask branch.  Outputs are float64
+ * [B, offset_groups, L_out, K].
+ */
+int oracle_packed_trunk(const float *x, const float *dw_w, const float *dw_b,
+                        const float *off_w, const float *off_b, const float *mask_w,
+                        const float *mask_b, int64_t B, int64_t C_in, int64_t L_in, int64_t K,
+                        int64_t L_out, int64_t stride, int64_t padding, int64_t padding_right,
+                        int64_t dilation, int64_t offset_groups, double *off_out,
+                        double *mask_out)
+{
+    if (B < 0 || C_in < 1 || L_in < 0 || K < 1 || stride < 1 || dilation < 1 || padding < 0 ||
+        padding_right < 0 || offset_groups < 1 || C_in % offset_groups != 0)
+        return 1;
+    if (L_out != out_length_lr(L_in, K, stride, padding, padding_right, dilation))
+        return 1;
+    const int64_t J = offset_groups * K;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t l = 0; l < L_out; ++l) {
+            double t[C_in];
+            /* the depthwise stage at output position l */
+            for (int64_t c = 0; c < C_in; ++c) {
+                double acc = dw_b ? (double)dw_b[c] : 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    int64_t i = l * stride - padding + k * dilation;
+                    double xv = (i >= 0 && i < L_in) ? (double)x[(b * C_in + c) * L_in + i] : 0.0;
+                    acc += (double)dw_w[c * K + k] * xv;
+                }
+                t[c] = acc;
+            }
+            /* the pointwise projections */
+            for (int64_t j = 0; j < J; ++j) {
+                int64_t g = j / K, k = j % K;
+                int64_t oidx = ((b * offset_groups + g) * L_out + l) * K + k;
+                double z = off_b ? (double)off_b[j] : 0.0;
+                for (int64_t c = 0; c < C_in; ++c)
+                    z += (double)off_w[j * C_in + c] * t[c];
+                off_out[oidx] = z;
+                if (mask_w && mask_out) {
+                    double zm = mask_b ? (double)mask_b[j] : 0.0;
+                    for (int64_t c = 0; c < C_in; ++c)
+                        zm += (double)mask_w[j * C_in + c] * t[c];
+                    mask_out[oidx] = 1.0 / (1.0 + exp(-zm));
+                }
+            }
+        }
+    return 0;
+}
