@@ -1,4 +1,5 @@
-"""B200 (sm_100a) forward and backward passes of 1D deformable convolution (DeformConv1d).
+"""B200 (sm_100a) forward and backward passes of 1D deformable convolution (DeformConv1d)
+and PackedDeformConv1d's forward (offsets and mask predicted inside the layer).
 
 The computation lives in the C-ABI CUDA library ``libdcn1d.so`` (declared in
 ``include/dcn1d.h``); this package is its thin Python binding.
@@ -21,6 +22,9 @@ from ._binding import (  # noqa: F401
     dcn1d_forward_kernel_name,
     dcn1d_last_launch_count,
     dcn1d_out_length,
+    dcn1d_packed_forward,
+    dcn1d_packed_trunk,
+    dcn1d_packed_trunk_kernel_name,
     dcn1d_sample_index,
     dcn1d_set_timing_events,
     dcn1d_status_string,

@@ -80,6 +80,12 @@ SIGNATURES = [
      [_T, _T, _T, _T, _T] + [_I64] * 6 + [_INT] + [_T] * 5),
     ("dcn1d_backward_lr", _INT,
      [_T, _T, _T, _T, _T] + [_I64] * 6 + [_INT] + [_T] * 5 + [_P, ctypes.c_size_t, _P]),
+    ("dcn1d_packed_trunk", _INT, [_T] * 7 + [_I64] * 5 + [_T, _T, _P]),
+    ("dcn1d_packed_trunk_kernel_name", ctypes.c_char_p, [_T] * 7 + [_I64] * 5 + [_T, _T]),
+    ("dcn1d_packed_forward_workspace_size", _I64,
+     [_T] * 9 + [_I64] * 6 + [_INT] + [_T] * 3),
+    ("dcn1d_packed_forward", _INT,
+     [_T] * 9 + [_I64] * 6 + [_INT] + [_T] * 3 + [_P, ctypes.c_size_t, _P]),
 ]
 
 
@@ -420,3 +426,118 @@ def dcn1d_sample_index(offsets, L_in, stride=1, padding=0, dilation=1, unconstra
     if st != 0:
         raise Dcn1dError(st, "dcn1d_sample_index")
     return i0, fr
+
+
+# ------------------------------------------------------------------ PackedDeformConv1d
+
+
+def _trunk_outputs(x, dw_weight, mask_weight, stride, pl, pr, dilation, offset_groups):
+    K = dw_weight.shape[2]
+    L_out = int(load().dcn1d_out_length_lr(x.shape[2], K, stride, pl, pr, dilation))
+    shape = (x.shape[0], offset_groups, max(L_out, 0), K)
+    off = torch.empty(shape, dtype=x.dtype, device=x.device)
+    mask = torch.empty(shape, dtype=x.dtype, device=x.device) if mask_weight is not None else None
+    return off, mask
+
+
+def dcn1d_packed_trunk(x, dw_weight, dw_bias, off_weight, off_bias, mask_weight=None,
+                       mask_bias=None, stride=1, padding=0, dilation=1, offset_groups=1,
+                       offsets_out=None, mask_out=None, stream=None):
+    """PackedDeformConv1d's offset (and mask) predictor through the C ABI.
+
+    x [B, C_in, L_in]; dw_weight [C_in, 1, K] and dw_bias [C_in] (the depthwise trunk);
+    off_weight [offset_groups*K, C_in(, 1)] and off_bias (the offset head); mask_weight and
+    mask_bias likewise for the sigmoid mask head, or None.  Returns (offsets, mask) as
+    [B, offset_groups, L_out, K] tensors (mask None without a mask head).  Does not
+    synchronise.
+    """
+    K = dw_weight.shape[2]
+    pl, pr = resolve_padding(padding, K, stride, dilation)
+    dev = _check_device((x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias,
+                         offsets_out, mask_out))
+    if offsets_out is None or (mask_weight is not None and mask_out is None):
+        o, m = _trunk_outputs(x, dw_weight, mask_weight, stride, pl, pr, dilation,
+                              offset_groups)
+        offsets_out = o if offsets_out is None else offsets_out
+        mask_out = m if mask_out is None else mask_out
+    tensors = (x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias,
+               offsets_out, mask_out)
+    refs = [_ref(_desc(t)) for t in tensors]
+    lib = load()
+    with torch.cuda.device(dev):
+        st = lib.dcn1d_packed_trunk(*refs[:7], stride, pl, pr, dilation, offset_groups,
+                                    refs[7], refs[8], _P(_stream_ptr(stream, dev)))
+    if st != 0:
+        raise Dcn1dError(st, "dcn1d_packed_trunk")
+    return offsets_out, mask_out
+
+
+def dcn1d_packed_trunk_kernel_name(x, dw_weight, dw_bias, off_weight, off_bias,
+                                   mask_weight=None, mask_bias=None, stride=1, padding=0,
+                                   dilation=1, offset_groups=1):
+    """Name of the trunk kernel these arguments select (None if invalid)."""
+    K = dw_weight.shape[2]
+    pl, pr = resolve_padding(padding, K, stride, dilation)
+    o, m = _trunk_outputs(x, dw_weight, mask_weight, stride, pl, pr, dilation, offset_groups)
+    tensors = (x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias, o, m)
+    refs = [_ref(_desc(t)) for t in tensors]
+    r = load().dcn1d_packed_trunk_kernel_name(*refs[:7], stride, pl, pr, dilation,
+                                              offset_groups, refs[7], refs[8])
+    return r.decode() if r else None
+
+
+def dcn1d_packed_forward(x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias,
+                         weight, bias, stride=1, padding=0, dilation=1, groups=1,
+                         offset_groups=1, unconstrained=False, with_offsets=False, out=None,
+                         stream=None, workspace=None):
+    """PackedDeformConv1d's forward through the C ABI: the trunk predicts the offsets (and,
+    with mask_weight, the sigmoid mask), then the deformable convolution runs with them.
+
+    Returns ``out`` [B, C_out, L_out]; with ``with_offsets`` the dc1d page's forms:
+    (out, offsets), or (out, (offsets, mask)) when the layer is modulated.  Without
+    ``with_offsets`` the predicted tensors live in the call's workspace (a uint8 CUDA
+    tensor of ``dcn1d_packed_forward_workspace_size`` bytes, allocated with torch and kept
+    per device and stream when not given).  Does not synchronise.
+    """
+    K = weight.shape[2]
+    pl, pr = resolve_padding(padding, K, stride, dilation)
+    dev = _check_device((x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias,
+                         weight, bias, out))
+    off_t = mask_t = None
+    if with_offsets:
+        off_t, mask_t = _trunk_outputs(x, dw_weight, mask_weight, stride, pl, pr, dilation,
+                                       offset_groups)
+    if out is None:
+        L_out = int(load().dcn1d_out_length_lr(x.shape[2], K, stride, pl, pr, dilation))
+        out = torch.empty((x.shape[0], weight.shape[0], max(L_out, 0)), dtype=x.dtype,
+                          device=x.device)
+    tensors = (x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias, weight,
+               bias, off_t, mask_t, out)
+    refs = [_ref(_desc(t)) for t in tensors]
+    lib = load()
+    args = (stride, pl, pr, dilation, groups, offset_groups, int(bool(unconstrained)))
+    with torch.cuda.device(dev):
+        sptr = _stream_ptr(stream, dev)
+        need = int(lib.dcn1d_packed_forward_workspace_size(*refs[:9], *args, *refs[9:]))
+        if need < 0:
+            raise Dcn1dError(-need, "dcn1d_packed_forward_workspace_size")
+        ws_ptr, ws_bytes = None, 0
+        if need > 0:
+            if workspace is None:
+                key = ("packed", dev.index, sptr)
+                workspace = _ws_cache.get(key)
+                if workspace is None or workspace.numel() < need:
+                    workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+                    if isinstance(stream, torch.cuda.Stream):
+                        workspace.record_stream(stream)
+                    _ws_cache[key] = workspace
+            if workspace.dtype != torch.uint8 or workspace.numel() < need:
+                raise ValueError(f"workspace must be a uint8 tensor of >= {need} bytes")
+            ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+        st = lib.dcn1d_packed_forward(*refs[:9], *args, *refs[9:], _P(ws_ptr), ws_bytes,
+                                      _P(sptr))
+    if st != 0:
+        raise Dcn1dError(st, "dcn1d_packed_forward")
+    if not with_offsets:
+        return out
+    return (out, (off_t, mask_t)) if mask_weight is not None else (out, off_t)

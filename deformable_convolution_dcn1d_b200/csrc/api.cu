@@ -197,6 +197,189 @@ int validate_backward(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1
     return DCN1D_OK;
 }
 
+// Launches the forward of a validated problem with the fastest kernel that
+// `ws_bytes` of workspace allows; *launches receives the kernel launches made.
+cudaError_t run_forward(const Problem &P, void *workspace, size_t ws_bytes, cudaStream_t s,
+                        int *launches) {
+    cudaError_t err = cudaSuccess;
+    *launches = 1;
+    switch (select_kernel(P, ws_bytes)) {
+    case kDirect:
+        timing_begin(s);
+        err = launch_direct(P, s);
+        timing_end(s);
+        break;
+    case kDepthwise:
+        timing_begin(s);
+        err = launch_depthwise(P, s);
+        timing_end(s);
+        break;
+    case kTcBf16:
+        err = launch_tc_bf16(P, s);
+        break;
+    case kTcTf32:
+        err = launch_tc_tf32(P, workspace, s);
+        *launches = tc_tf32_launches(P);
+        break;
+    }
+    return err;
+}
+
+// A pointwise weight: [J, C_in] or conv1d's [J, C_in, 1].
+bool pointwise_shape(const dcn1d_tensor *w, int64_t J, int64_t C_in) {
+    if (w->ndim == 2)
+        return w->shape[0] == J && w->shape[1] == C_in;
+    return w->ndim == 3 && w->shape[0] == J && w->shape[1] == C_in && w->shape[2] == 1;
+}
+
+// Validation of PackedDeformConv1d's trunk: x [B, C_in, L_in], dw_w [C_in, 1, K],
+// dw_b [C_in], off_w / mask_w [J, C_in(, 1)], off_b / mask_b [J] with J = offset_groups*K,
+// outputs [B, offset_groups, L_out, K].  A NULL output descriptor is allowed only when
+// `outputs_optional` (the packed forward keeps such a tensor in its workspace); its
+// data pointer is then left NULL in T.
+int validate_trunk(const dcn1d_tensor *x, const dcn1d_tensor *dw_w, const dcn1d_tensor *dw_b,
+                   const dcn1d_tensor *off_w, const dcn1d_tensor *off_b,
+                   const dcn1d_tensor *mask_w, const dcn1d_tensor *mask_b, int64_t stride,
+                   int64_t padding, int64_t padding_right, int64_t dilation,
+                   int64_t offset_groups, const dcn1d_tensor *off_out,
+                   const dcn1d_tensor *mask_out, bool outputs_optional, TrunkProblem *T) {
+    int st;
+    if (!x || !dw_w || !off_w)
+        return DCN1D_ERR_NULL;
+    if (!outputs_optional && (!off_out || (mask_w && !mask_out)))
+        return DCN1D_ERR_NULL;
+    if (mask_out && !mask_w)
+        return DCN1D_ERR_ARG;   // a mask output without a mask head
+    if (mask_b && !mask_w)
+        return DCN1D_ERR_ARG;
+    if ((st = check_desc(x, 3)) || (st = check_desc(dw_w, 3)))
+        return st;
+    if ((st = check_desc(off_w, off_w->ndim == 2 ? 2 : 3)))
+        return st;
+    if (mask_w && (st = check_desc(mask_w, mask_w->ndim == 2 ? 2 : 3)))
+        return st;
+    if ((dw_b && (st = check_desc(dw_b, 1))) || (off_b && (st = check_desc(off_b, 1))) ||
+        (mask_b && (st = check_desc(mask_b, 1))))
+        return st;
+    if ((off_out && (st = check_desc(off_out, 4))) || (mask_out && (st = check_desc(mask_out, 4))))
+        return st;
+    const int dt = x->dtype;
+    const dcn1d_tensor *all[] = {dw_w, dw_b, off_w, off_b, mask_w, mask_b, off_out, mask_out};
+    for (const dcn1d_tensor *t : all)
+        if (t && t->dtype != dt)
+            return DCN1D_ERR_DTYPE;
+    if (stride < 1 || padding < 0 || padding_right < 0 || dilation < 1 || offset_groups < 1)
+        return DCN1D_ERR_ARG;
+    const int64_t B = x->shape[0], C_in = x->shape[1], L_in = x->shape[2];
+    const int64_t K = dw_w->shape[2];
+    if (C_in < 1 || L_in < 1 || K < 1)
+        return DCN1D_ERR_SHAPE;
+    if (C_in % offset_groups)
+        return DCN1D_ERR_ARG;
+    if (dw_w->shape[0] != C_in || dw_w->shape[1] != 1)
+        return DCN1D_ERR_SHAPE;
+    if (stride >= kMaxPos || padding >= kMaxPos || padding_right >= kMaxPos ||
+        dilation >= kMaxPos || K >= kMaxPos || L_in >= kMaxPos || offset_groups >= kMaxPos)
+        return DCN1D_ERR_UNSUPPORTED;
+    const int64_t J = offset_groups * K;
+    if (!pointwise_shape(off_w, J, C_in) || (mask_w && !pointwise_shape(mask_w, J, C_in)))
+        return DCN1D_ERR_SHAPE;
+    if ((dw_b && dw_b->shape[0] != C_in) || (off_b && off_b->shape[0] != J) ||
+        (mask_b && mask_b->shape[0] != J))
+        return DCN1D_ERR_SHAPE;
+    const int64_t L_out = dcn1d_out_length_lr(L_in, K, stride, padding, padding_right, dilation);
+    if (L_out < 1)
+        return DCN1D_ERR_ARG;
+    if ((off_out && !shape_is(off_out, B, offset_groups, L_out, K)) ||
+        (mask_out && !shape_is(mask_out, B, offset_groups, L_out, K)))
+        return DCN1D_ERR_SHAPE;
+    if ((L_out - 1) * stride + dilation * (K - 1) >= kMaxPos)
+        return DCN1D_ERR_UNSUPPORTED;
+    if (numel(x) >= kMaxElems || B * J * L_out >= kMaxElems || J * C_in >= kMaxElems ||
+        B > 65535)
+        return DCN1D_ERR_UNSUPPORTED;
+    T->B = (int)B;
+    T->C_in = (int)C_in;
+    T->L_in = (int)L_in;
+    T->K = (int)K;
+    T->L_out = (int)L_out;
+    T->stride = (int)stride;
+    T->padding = (int)padding;
+    T->dilation = (int)dilation;
+    T->offset_groups = (int)offset_groups;
+    T->J = (int)J;
+    T->dtype = dt;
+    T->x = x->data;
+    T->dw_w = dw_w->data;
+    T->dw_b = dw_b ? dw_b->data : nullptr;
+    T->off_w = off_w->data;
+    T->off_b = off_b ? off_b->data : nullptr;
+    T->mask_w = mask_w ? mask_w->data : nullptr;
+    T->mask_b = mask_b ? mask_b->data : nullptr;
+    T->off_out = off_out ? off_out->data : nullptr;
+    T->mask_out = mask_out ? mask_out->data : nullptr;
+    return DCN1D_OK;
+}
+
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+// Workspace of the packed forward: the predicted tensors the caller did not supply,
+// then the forward's own scratch.
+struct PackedLayout {
+    size_t off_bytes, mask_bytes, fwd_offset, total;
+};
+
+// Validation and layout shared by the packed forward and its workspace query.
+// `ws_base` NULL (a size query) places the predicted tensors at a placeholder
+// address; the descriptors are then used for shape checks only.
+int packed_prepare(const dcn1d_tensor *x, const dcn1d_tensor *dw_w, const dcn1d_tensor *dw_b,
+                   const dcn1d_tensor *off_w, const dcn1d_tensor *off_b,
+                   const dcn1d_tensor *mask_w, const dcn1d_tensor *mask_b,
+                   const dcn1d_tensor *weight, const dcn1d_tensor *bias, int64_t stride,
+                   int64_t padding, int64_t padding_right, int64_t dilation, int64_t groups,
+                   int64_t offset_groups, int unconstrained, const dcn1d_tensor *off_out,
+                   const dcn1d_tensor *mask_out, const dcn1d_tensor *out, char *ws_base,
+                   TrunkProblem *T, dcn1d_tensor *off_d, dcn1d_tensor *mask_d, Problem *P,
+                   PackedLayout *lay) {
+    int st = validate_trunk(x, dw_w, dw_b, off_w, off_b, mask_w, mask_b, stride, padding,
+                            padding_right, dilation, offset_groups, off_out, mask_out, true, T);
+    if (st != DCN1D_OK)
+        return st;
+    if (!weight)
+        return DCN1D_ERR_NULL;
+    if ((st = check_desc(weight, 3)) != DCN1D_OK)
+        return st;
+    if (weight->shape[2] != T->K)
+        return DCN1D_ERR_SHAPE;
+    const size_t es = x->dtype == DCN1D_F32 ? 4 : 2;
+    const size_t n = (size_t)T->B * T->J * T->L_out;
+    lay->off_bytes = off_out ? 0 : round256(n * es);
+    lay->mask_bytes = (mask_w && !mask_out) ? round256(n * es) : 0;
+    lay->fwd_offset = lay->off_bytes + lay->mask_bytes;
+    char *base = ws_base ? ws_base : reinterpret_cast<char *>((uintptr_t)256);
+    auto predicted = [&](char *data) {
+        dcn1d_tensor d;
+        memset(&d, 0, sizeof(d));
+        d.data = data;
+        d.dtype = x->dtype;
+        d.ndim = 4;
+        d.shape[0] = T->B;
+        d.shape[1] = T->offset_groups;
+        d.shape[2] = T->L_out;
+        d.shape[3] = T->K;
+        return d;
+    };
+    *off_d = off_out ? *off_out : predicted(base);
+    if (mask_w)
+        *mask_d = mask_out ? *mask_out : predicted(base + lay->off_bytes);
+    st = validate(x, off_d, mask_w ? mask_d : nullptr, weight, bias, stride, padding,
+                  padding_right, dilation, groups, offset_groups, unconstrained, out, P);
+    if (st != DCN1D_OK)
+        return st;
+    lay->total = lay->fwd_offset + round256(workspace_bytes(*P));
+    return DCN1D_OK;
+}
+
 }  // namespace
 
 void timing_begin(cudaStream_t stream) {
@@ -293,30 +476,9 @@ int dcn1d_forward_lr(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
         return DCN1D_ERR_NULL;
     if (P.B == 0)
         return DCN1D_OK;   // empty batch: nothing to compute
-    const Kernel kern = select_kernel(P, workspace ? workspace_bytes : 0);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t err = cudaSuccess;
-    int launches = 1;
-    switch (kern) {
-    case kDirect:
-        timing_begin(s);
-        err = launch_direct(P, s);
-        timing_end(s);
-        break;
-    case kDepthwise:
-        timing_begin(s);
-        err = launch_depthwise(P, s);
-        timing_end(s);
-        break;
-    case kTcBf16:
-        err = launch_tc_bf16(P, s);
-        break;
-    case kTcTf32:
-        err = launch_tc_tf32(P, workspace, s);
-        launches = tc_tf32_launches(P);
-        break;
-    }
-    if (err != cudaSuccess)
+    int launches = 0;
+    if (run_forward(P, workspace, workspace ? workspace_bytes : 0,
+                    static_cast<cudaStream_t>(stream), &launches) != cudaSuccess)
         return DCN1D_ERR_LAUNCH;
     g_last_launches = launches;
     return DCN1D_OK;
@@ -510,6 +672,104 @@ int dcn1d_sample_index(const dcn1d_tensor *offsets, int64_t L_in, int64_t stride
                                           (int)padding, (int)dilation, unconstrained,
                                           i0, frac, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? DCN1D_OK : DCN1D_ERR_LAUNCH;
+}
+
+int dcn1d_packed_trunk(const dcn1d_tensor *x, const dcn1d_tensor *dw_weight,
+                       const dcn1d_tensor *dw_bias, const dcn1d_tensor *off_weight,
+                       const dcn1d_tensor *off_bias, const dcn1d_tensor *mask_weight,
+                       const dcn1d_tensor *mask_bias, int64_t stride, int64_t padding_left,
+                       int64_t padding_right, int64_t dilation, int64_t offset_groups,
+                       dcn1d_tensor *offsets_out, dcn1d_tensor *mask_out, void *stream) {
+    g_last_launches = 0;
+    TrunkProblem T;
+    int st = validate_trunk(x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias,
+                            stride, padding_left, padding_right, dilation, offset_groups,
+                            offsets_out, mask_out, false, &T);
+    if (st != DCN1D_OK)
+        return st;
+    if (T.B == 0)
+        return DCN1D_OK;
+    const char *name = nullptr;
+    if (launch_trunk(T, static_cast<cudaStream_t>(stream), &name) != cudaSuccess)
+        return DCN1D_ERR_LAUNCH;
+    g_last_launches = 1;
+    return DCN1D_OK;
+}
+
+const char *dcn1d_packed_trunk_kernel_name(
+    const dcn1d_tensor *x, const dcn1d_tensor *dw_weight, const dcn1d_tensor *dw_bias,
+    const dcn1d_tensor *off_weight, const dcn1d_tensor *off_bias,
+    const dcn1d_tensor *mask_weight, const dcn1d_tensor *mask_bias, int64_t stride,
+    int64_t padding_left, int64_t padding_right, int64_t dilation, int64_t offset_groups,
+    const dcn1d_tensor *offsets_out, const dcn1d_tensor *mask_out) {
+    TrunkProblem T;
+    if (validate_trunk(x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias,
+                       stride, padding_left, padding_right, dilation, offset_groups, offsets_out,
+                       mask_out, false, &T) != DCN1D_OK)
+        return nullptr;
+    return trunk_tc_supported(T) ? "trunk_tcgen05" : "trunk_simt";
+}
+
+int64_t dcn1d_packed_forward_workspace_size(
+    const dcn1d_tensor *x, const dcn1d_tensor *dw_weight, const dcn1d_tensor *dw_bias,
+    const dcn1d_tensor *off_weight, const dcn1d_tensor *off_bias,
+    const dcn1d_tensor *mask_weight, const dcn1d_tensor *mask_bias, const dcn1d_tensor *weight,
+    const dcn1d_tensor *bias, int64_t stride, int64_t padding_left, int64_t padding_right,
+    int64_t dilation, int64_t groups, int64_t offset_groups, int unconstrained,
+    const dcn1d_tensor *offsets_out, const dcn1d_tensor *mask_out, const dcn1d_tensor *out) {
+    TrunkProblem T;
+    Problem P;
+    dcn1d_tensor od, md;
+    PackedLayout lay;
+    const int st = packed_prepare(x, dw_weight, dw_bias, off_weight, off_bias, mask_weight,
+                                  mask_bias, weight, bias, stride, padding_left, padding_right,
+                                  dilation, groups, offset_groups, unconstrained, offsets_out,
+                                  mask_out, out, nullptr, &T, &od, &md, &P, &lay);
+    if (st != DCN1D_OK)
+        return -(int64_t)st;
+    return (int64_t)lay.total;
+}
+
+int dcn1d_packed_forward(const dcn1d_tensor *x, const dcn1d_tensor *dw_weight,
+                         const dcn1d_tensor *dw_bias, const dcn1d_tensor *off_weight,
+                         const dcn1d_tensor *off_bias, const dcn1d_tensor *mask_weight,
+                         const dcn1d_tensor *mask_bias, const dcn1d_tensor *weight,
+                         const dcn1d_tensor *bias, int64_t stride, int64_t padding_left,
+                         int64_t padding_right, int64_t dilation, int64_t groups,
+                         int64_t offset_groups, int unconstrained, dcn1d_tensor *offsets_out,
+                         dcn1d_tensor *mask_out, dcn1d_tensor *out, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    g_last_launches = 0;
+    if (workspace_bytes > 0 && !workspace)
+        return DCN1D_ERR_NULL;
+    TrunkProblem T;
+    Problem P;
+    dcn1d_tensor od, md;
+    PackedLayout lay;
+    char *ws = static_cast<char *>(workspace);
+    int st = packed_prepare(x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias,
+                            weight, bias, stride, padding_left, padding_right, dilation, groups,
+                            offset_groups, unconstrained, offsets_out, mask_out, out,
+                            ws ? ws : nullptr, &T, &od, &md, &P, &lay);
+    if (st != DCN1D_OK)
+        return st;
+    if (lay.fwd_offset > 0 && (!ws || workspace_bytes < lay.fwd_offset))
+        return ws ? DCN1D_ERR_ARG : DCN1D_ERR_NULL;   // no room for the predicted tensors
+    if (T.B == 0)
+        return DCN1D_OK;
+    T.off_out = od.data;
+    T.mask_out = mask_weight ? md.data : nullptr;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const char *name = nullptr;
+    if (launch_trunk(T, s, &name) != cudaSuccess)
+        return DCN1D_ERR_LAUNCH;
+    int launches = 0;
+    const size_t rest = workspace_bytes - lay.fwd_offset;
+    if (run_forward(P, rest > 0 ? ws + lay.fwd_offset : nullptr, rest, s, &launches) !=
+        cudaSuccess)
+        return DCN1D_ERR_LAUNCH;
+    g_last_launches = 1 + launches;
+    return DCN1D_OK;
 }
 
 }  // extern "C"

@@ -75,6 +75,20 @@ struct BackwardGrads {
 size_t backward_workspace(const Problem &P, const BackwardGrads &G);
 cudaError_t launch_backward(const Problem &P, const BackwardGrads &G, void *workspace,
                             cudaStream_t stream, int *launches);
+// PackedDeformConv1d's offset (and mask) predictor (trunk.cu): a depthwise convolution
+// of x with the layer's K, stride, padding and dilation, then pointwise projections
+// ("heads") to offset_groups*K channels: the offsets, and the mask through a sigmoid.
+struct TrunkProblem {
+    int B, C_in, L_in, K, L_out;
+    int stride, padding, dilation, offset_groups;
+    int J;                     // offset_groups * K channels per head
+    int dtype;                 // dcn1d_dtype of every tensor
+    const void *x, *dw_w, *dw_b, *off_w, *off_b, *mask_w, *mask_b;   // biases may be NULL
+    void *off_out, *mask_out;  // [B, offset_groups, L_out, K]; mask_out NULL: no mask head
+};
+bool trunk_tc_supported(const TrunkProblem &T);
+// Launches the trunk; *kernel receives the name of the kernel chosen.
+cudaError_t launch_trunk(const TrunkProblem &T, cudaStream_t stream, const char **kernel);
 cudaError_t launch_sample_index(const void *off, int dtype, int B, int G, int L_out, int K,
                                 int L_in, int stride, int padding, int dilation,
                                 int unconstrained, int32_t *i0, float *frac,

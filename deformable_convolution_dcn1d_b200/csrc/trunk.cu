@@ -1,0 +1,535 @@
+// PackedDeformConv1d's offset (and mask) predictor: the depthwise-separable
+// block of the "dc1d (DeformConv1d)" page ("PackedDeformConv1d"; "Modulation
+// (DCNv2)" for the second, sigmoid-terminated branch off the same trunk):
+//
+//   t[b,c,l]         = dw_b[c] + sum_k dw_w[c,k] * x[b, c, l*s - p + k*d]   (zero outside)
+//   offsets[b,g,l,k] = off_b[j] + sum_c off_w[j,c] * t[b,c,l],            j = g*K + k
+//   mask[b,g,l,k]    = sigmoid(mask_b[j] + sum_c mask_w[j,c] * t[b,c,l])
+//
+// t never leaves the chip: it is formed in fp32 and consumed by the pointwise
+// contraction in the same kernel.  Two kernels:
+//
+//  * trunk_tc_kernel (16-bit inputs, C_in a multiple of 64 up to 512): a tile is
+//    128 output positions of one batch element.  Sixteen producer warps compute
+//    the tile's t for every channel (fp32 FMAs over x read straight from global
+//    memory, rounded once to the input type) into shared memory in the 128-byte
+//    swizzled K-major layout the tensor core reads; then one thread issues
+//    tcgen05.mma (M=128, N up to 256, K=16) against pointwise-weight tiles that
+//    a TMA warp streams through a ring of stages, accumulating in tensor memory
+//    (two 256-column buffers, so the next column chunk's MMAs run while the
+//    producer warps drain the previous one).  The drain adds the bias, applies
+//    the sigmoid on the mask head and stores in the [B, G, L_out, K] layout.
+//  * trunk_simt_kernel (every dtype and shape): 64 positions x 64 head channels
+//    per block, t formed per 16-channel slice in shared memory, CUDA-core FMAs.
+#include <string.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace dcn1d {
+
+namespace {
+
+// ---------------------------------------------------------------- CUDA-core kernel
+
+constexpr int kSimtL = 64, kSimtJ = 64, kSimtC = 16, kSimtThreads = 256;
+
+// One output of a head: bias, sigmoid on the mask head, [B, G, L_out, K] address.
+template <class T>
+__device__ __forceinline__ void store_head(const TrunkProblem &P, int head, int j, int b, int l,
+                                           float z) {
+    const T *bias = static_cast<const T *>(head ? P.mask_b : P.off_b);
+    if (bias)
+        z += ld_f32(bias + j);
+    if (head)
+        z = 1.0f / (1.0f + expf(-z));
+    const int g = j / P.K, k = j - g * P.K;
+    T *out = static_cast<T *>(head ? P.mask_out : P.off_out);
+    out[(((int64_t)b * P.offset_groups + g) * P.L_out + l) * P.K + k] = from_f32<T>(z);
+}
+
+template <class T>
+__global__ void __launch_bounds__(kSimtThreads)
+    trunk_simt_kernel(const __grid_constant__ TrunkProblem P) {
+    __shared__ float ts[kSimtC][kSimtL + 4];
+    __shared__ float ws[kSimtC][kSimtJ + 4];
+    const int l0 = blockIdx.x * kSimtL;
+    const int jt0 = blockIdx.y * kSimtJ;   // over both heads: [0, J) offsets, [J, 2J) mask
+    const int b = blockIdx.z;
+    const int heads = P.mask_out ? 2 : 1;
+    const int Jt = heads * P.J;
+    const int tid = threadIdx.x;
+    const int tj = tid / 16, tl = tid % 16;
+    const T *x = static_cast<const T *>(P.x) + (int64_t)b * P.C_in * P.L_in;
+    const T *dww = static_cast<const T *>(P.dw_w);
+    const T *dwb = static_cast<const T *>(P.dw_b);
+    float acc[4][4] = {};
+    for (int c0 = 0; c0 < P.C_in; c0 += kSimtC) {
+        for (int i = tid; i < kSimtC * kSimtL; i += kSimtThreads) {
+            const int cc = i / kSimtL, ll = i % kSimtL;
+            const int c = c0 + cc, l = l0 + ll;
+            float t = 0.0f;
+            if (c < P.C_in && l < P.L_out) {
+                t = dwb ? ld_f32(dwb + c) : 0.0f;
+                for (int k = 0; k < P.K; ++k) {
+                    const int pos = l * P.stride - P.padding + k * P.dilation;
+                    if (pos >= 0 && pos < P.L_in)
+                        t = fmaf(ld_f32(dww + (int64_t)c * P.K + k),
+                                 ld_f32(x + (int64_t)c * P.L_in + pos), t);
+                }
+            }
+            ts[cc][ll] = t;
+        }
+        for (int i = tid; i < kSimtC * kSimtJ; i += kSimtThreads) {
+            const int jj = i / kSimtC, cc = i % kSimtC;
+            const int jt = jt0 + jj, c = c0 + cc;
+            float w = 0.0f;
+            if (jt < Jt && c < P.C_in) {
+                const int head = jt >= P.J, j = jt - head * P.J;
+                const T *W = static_cast<const T *>(head ? P.mask_w : P.off_w);
+                w = ld_f32(W + (int64_t)j * P.C_in + c);
+            }
+            ws[cc][jj] = w;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int cc = 0; cc < kSimtC; ++cc) {
+            float wv[4], tv[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                wv[a] = ws[cc][tj + 16 * a];
+                tv[a] = ts[cc][tl + 16 * a];
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc[a][e] = fmaf(wv[a], tv[e], acc[a][e]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int jt = jt0 + tj + 16 * a;
+        if (jt >= Jt)
+            continue;
+        const int head = jt >= P.J;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int l = l0 + tl + 16 * e;
+            if (l < P.L_out)
+                store_head<T>(P, head, jt - head * P.J, b, l, acc[a][e]);
+        }
+    }
+}
+
+template <class T>
+cudaError_t launch_simt(const TrunkProblem &P, cudaStream_t stream) {
+    const int heads = P.mask_out ? 2 : 1;
+    dim3 grid((P.L_out + kSimtL - 1) / kSimtL, (heads * P.J + kSimtJ - 1) / kSimtJ, P.B);
+    timing_begin(stream);
+    trunk_simt_kernel<T><<<grid, kSimtThreads, 0, stream>>>(P);
+    timing_end(stream);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- tensor-core kernel
+
+constexpr int kTRows = 128;                 // output positions per tile = TMEM lanes
+constexpr int kTBK = 64;                    // channels per k-block (128 bytes of 16-bit values)
+constexpr uint32_t kTABytes = kTRows * 128; // one k-block of the A tile (16 KB)
+constexpr int kTMaxN = 256;                 // head channels per column chunk (MMA N limit)
+constexpr int kTMaxCin = 512;               // the whole A tile stays in shared memory
+constexpr int kTProdWarps = 16, kTTmaWarp = 16, kTMmaWarp = 17, kTThreads = 18 * 32;
+constexpr uint32_t kTTmemCols = 512;        // two accumulator buffers of 256 columns
+constexpr uint64_t kTWaitNs = 2000000000ull;   // 2 s
+
+template <class E>
+struct TElem;
+
+template <>
+struct TElem<__nv_bfloat16> {
+    static constexpr CUtensorMapDataType kTma = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    static __host__ __device__ constexpr uint32_t idesc(int M, int N) {
+        return idesc_bf16_f32(M, N);
+    }
+    static __device__ __forceinline__ uint32_t pack(float a, float b) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+};
+
+template <>
+struct TElem<__half> {
+    static constexpr CUtensorMapDataType kTma = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    static __host__ __device__ constexpr uint32_t idesc(int M, int N) {
+        return idesc_f16_f32(M, N);
+    }
+    static __device__ __forceinline__ uint32_t pack(float a, float b) {
+        __half2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+};
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&v)[4]) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3])
+                 : "memory");
+}
+
+struct TcTrunkArgs {
+    TrunkProblem P;
+    int nkb;                 // k-blocks: C_in / 64
+    int nbox;                // MMA N = weight tile rows (multiple of 16, <= 256)
+    int chunks_per_head;     // column chunks of kTMaxN per head
+    int heads, chunks;       // heads (1 or 2) and chunks per tile
+    int tiles_l, num_tiles;
+    int stages;              // weight ring depth
+    uint32_t w_stage_bytes;
+    uint32_t off_a, off_w, off_dw, off_bar;   // shared-memory layout
+    unsigned int *status;    // device status word
+};
+
+template <class E>
+__global__ void __launch_bounds__(kTThreads, 1)
+    trunk_tc_kernel(const __grid_constant__ TcTrunkArgs A,
+                    const __grid_constant__ CUtensorMap map_off,
+                    const __grid_constant__ CUtensorMap map_mask) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const TrunkProblem &P = A.P;
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    // The 128-byte swizzle wants 1024-byte aligned tiles (1 KB of slack is reserved).
+    const uint32_t sraw = smem_u32(smem_raw);
+    const uint32_t sbase = (sraw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - sraw);
+    const uint32_t a_s = sbase + A.off_a;
+    const uint32_t w_s0 = sbase + A.off_w;
+    float *dw_s = reinterpret_cast<float *>(smem + A.off_dw);   // [C_in][K] weights, [C_in] biases
+    const uint32_t bar0 = sbase + A.off_bar;
+    const int S = A.stages;
+    auto w_full = [&](int s) { return bar0 + 8u * s; };
+    auto w_empty = [&](int s) { return bar0 + 8u * (S + s); };
+    const uint32_t a_full = bar0 + 16u * S;
+    const uint32_t a_empty = a_full + 8u;
+    const uint32_t d_full0 = a_full + 16u;    // + 8 d
+    const uint32_t d_empty0 = a_full + 32u;   // + 8 d
+    const uint32_t drain_bar = a_full + 48u;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + A.off_bar + 16 * S + 56);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    {
+        const E *dww = static_cast<const E *>(P.dw_w);
+        const E *dwb = static_cast<const E *>(P.dw_b);
+        for (int i = threadIdx.x; i < P.C_in * P.K; i += kTThreads)
+            dw_s[i] = ld_f32(dww + i);
+        for (int i = threadIdx.x; i < P.C_in; i += kTThreads)
+            dw_s[P.C_in * P.K + i] = dwb ? ld_f32(dwb + i) : 0.0f;
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(w_full(s), 1);
+            mbar_init(w_empty(s), 1);
+        }
+        mbar_init(a_full, kTProdWarps);
+        mbar_init(a_empty, 1);
+        for (int d = 0; d < 2; ++d) {
+            mbar_init(d_full0 + 8u * d, 1);
+            mbar_init(d_empty0 + 8u * d, kTProdWarps);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kTMmaWarp) {
+        tmem_alloc(smem_u32(tmem_holder), kTTmemCols);
+        tc_fence_before();
+    }
+    if (warp == kTTmaWarp && lane == 0) {
+        tma_prefetch_desc(&map_off);
+        if (A.heads > 1)
+            tma_prefetch_desc(&map_mask);
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const BoundedWait wait{abort_flag, kTWaitNs, A.status};
+
+    if (warp == kTTmaWarp) {
+        // ------------------------------------------------------------ weight tiles
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x)
+                for (int c = 0; c < A.chunks; ++c) {
+                    const int head = c / A.chunks_per_head;
+                    const int n0 = (c % A.chunks_per_head) * kTMaxN;
+                    const CUtensorMap *map = head ? &map_mask : &map_off;
+                    for (int kb = 0; kb < A.nkb; ++kb, ++it) {
+                        const int s = it % S;
+                        const uint32_t ph = (it / S) & 1u;
+                        if (!wait(w_empty(s), ph ^ 1u))
+                            goto tma_done;
+                        mbar_arrive_expect_tx(w_full(s), A.w_stage_bytes);
+                        tma_load_2d(w_s0 + s * A.w_stage_bytes, map, kb * kTBK, n0, w_full(s));
+                    }
+                }
+        tma_done:
+            // Let every load this thread issued land before the CTA can exit.
+            volatile int never = 0;
+            const BoundedWait drain{&never, kTWaitNs, A.status};
+            const uint32_t Su = (uint32_t)S;
+            for (uint32_t j = (it > Su ? it - Su : 0); j < it; ++j)
+                drain(w_full(j % Su), (j / Su) & 1u);
+        }
+    } else if (warp == kTMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = TElem<E>::idesc(kTRows, A.nbox);
+            uint32_t it = 0, cg = 0, tc = 0;
+            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
+                if (!wait(a_full, tc & 1u))
+                    goto mma_done;
+                tc_fence_after();
+                for (int c = 0; c < A.chunks; ++c, ++cg) {
+                    const uint32_t d = cg & 1u;
+                    if (!wait(d_empty0 + 8u * d, ((cg >> 1) & 1u) ^ 1u))
+                        goto mma_done;
+                    tc_fence_after();
+                    for (int kb = 0; kb < A.nkb; ++kb, ++it) {
+                        const int s = it % S;
+                        const uint32_t ph = (it / S) & 1u;
+                        if (!wait(w_full(s), ph))
+                            goto mma_done;
+                        tc_fence_after();
+                        const uint32_t wst = w_s0 + s * A.w_stage_bytes;
+                        const uint32_t ast = a_s + kb * kTABytes;
+#pragma unroll
+                        for (int kk = 0; kk < kTBK / 16; ++kk)
+                            mma_f16_ss(tmem + 256u * d, sw128_kmajor_desc(ast + 32u * kk),
+                                       sw128_kmajor_desc(wst + 32u * kk), idesc,
+                                       (kb > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(w_empty(s));
+                    }
+                    mma_commit(d_full0 + 8u * d);
+                }
+                mma_commit(a_empty);   // the tile's A may be overwritten once this arrives
+            }
+        mma_done:
+            // Every MMA issued has completed once this commit arrives.
+            mma_commit(drain_bar);
+            volatile int never = 0;
+            const BoundedWait drain{&never, kTWaitNs, A.status};
+            drain(drain_bar, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ depthwise + drain
+        const int q = warp % 4;          // TMEM lane quarter
+        const int h = warp / 4;          // k-blocks h, h+4, ...; drain columns 16h, 16(h+4), ...
+        const int r = 32 * q + lane;     // tile row
+        uint32_t cg = 0, tc = 0;
+        for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
+            const int b = t / A.tiles_l;
+            const int l = (t % A.tiles_l) * kTRows + r;
+            const bool valid = l < P.L_out;
+            if (!__all_sync(0xffffffffu, wait(a_empty, (tc & 1u) ^ 1u)))
+                goto prod_done;
+            {
+                const E *xb = static_cast<const E *>(P.x) + (int64_t)b * P.C_in * P.L_in;
+                const int pos0 = l * P.stride - P.padding;
+                for (int kb = h; kb < A.nkb; kb += 4) {
+                    const uint32_t row_addr = a_s + kb * kTABytes + r * 128;
+#pragma unroll 1
+                    for (int ch = 0; ch < 8; ++ch) {   // 8 channels = one 16-byte chunk
+                        const int c0 = kb * kTBK + ch * 8;
+                        float acc[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            acc[i] = dw_s[P.C_in * P.K + c0 + i];
+                        if (valid) {
+                            for (int k = 0; k < P.K; ++k) {
+                                const int pos = pos0 + k * P.dilation;
+                                if (pos >= 0 && pos < P.L_in) {
+                                    const E *xp = xb + (int64_t)c0 * P.L_in + pos;
+#pragma unroll
+                                    for (int i = 0; i < 8; ++i)
+                                        acc[i] = fmaf(dw_s[(c0 + i) * P.K + k],
+                                                      ld_f32(xp + (int64_t)i * P.L_in), acc[i]);
+                                }
+                            }
+                        }
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            pk[i] = TElem<E>::pack(acc[2 * i], acc[2 * i + 1]);
+                        // 128-byte swizzle: 16-byte chunk `ch` of row r sits at chunk ch ^ (r % 8)
+                        st_shared_v4(row_addr + ((uint32_t)(ch ^ (r & 7)) << 4), pk);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(a_full);
+            for (int c = 0; c < A.chunks; ++c, ++cg) {
+                const uint32_t d = cg & 1u;
+                if (!__all_sync(0xffffffffu, wait(d_full0 + 8u * d, (cg >> 1) & 1u)))
+                    goto prod_done;
+                tc_fence_after();
+                const int head = c / A.chunks_per_head;
+                const int n0 = (c % A.chunks_per_head) * kTMaxN;
+                E *outp = static_cast<E *>(head ? P.mask_out : P.off_out);
+                const E *biasp = static_cast<const E *>(head ? P.mask_b : P.off_b);
+                for (int cc = h; cc < A.nbox / 16; cc += 4) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 256u * d + 16u * cc, v);
+                    tmem_wait_ld();
+                    int j = n0 + 16 * cc;
+                    int g = j / P.K, k = j - g * P.K;
+                    if (valid) {
+                        E *orow = outp + (((int64_t)b * P.offset_groups) * P.L_out + l) * P.K;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            if (j < P.J) {
+                                float z = __uint_as_float(v[i]);
+                                if (biasp)
+                                    z += ld_f32(biasp + j);
+                                if (head)
+                                    z = 1.0f / (1.0f + __expf(-z));
+                                orow[(int64_t)g * P.L_out * P.K + k] = from_f32<E>(z);
+                            }
+                            ++j;
+                            if (++k == P.K) {
+                                k = 0;
+                                ++g;
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(d_empty0 + 8u * d);
+            }
+        }
+    prod_done:;
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kTMmaWarp) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+struct TcPlan {
+    TcTrunkArgs A;
+    size_t smem;
+};
+
+bool make_tc_plan(const TrunkProblem &P, TcPlan *out) {
+    TcTrunkArgs A;
+    memset(&A, 0, sizeof(A));
+    A.P = P;
+    if (P.C_in % kTBK != 0 || P.C_in > kTMaxCin || P.J < 1)
+        return false;
+    A.nkb = P.C_in / kTBK;
+    A.nbox = P.J >= kTMaxN ? kTMaxN : (P.J + 15) / 16 * 16;
+    A.chunks_per_head = (P.J + kTMaxN - 1) / kTMaxN;
+    A.heads = P.mask_out ? 2 : 1;
+    A.chunks = A.heads * A.chunks_per_head;
+    A.tiles_l = (P.L_out + kTRows - 1) / kTRows;
+    A.num_tiles = P.B * A.tiles_l;
+    A.w_stage_bytes = (uint32_t)A.nbox * 128u;
+    A.off_a = 0;
+    A.off_w = A.off_a + (uint32_t)A.nkb * kTABytes;
+    const size_t dw_bytes = ((size_t)P.C_in * (P.K + 1) * 4 + 15) / 16 * 16;
+    const size_t limit = 227 * 1024, fixed = 1024 + 16 * 8 + 64;   // slack, bars, holder
+    const size_t base = A.off_w + dw_bytes + fixed;
+    if (base >= limit)
+        return false;
+    int stages = (int)((limit - base) / (A.w_stage_bytes + 16));
+    if (stages > 4)
+        stages = 4;
+    if (stages < 2)
+        return false;
+    A.stages = stages;
+    A.off_dw = A.off_w + (uint32_t)stages * A.w_stage_bytes;
+    A.off_bar = A.off_dw + (uint32_t)dw_bytes;
+    size_t smem = A.off_bar + 16 * stages + 64 + 1024;
+    if (smem > limit)
+        return false;
+    // More than half the SM's shared memory: two CTAs (each holding all 512
+    // tensor-memory columns) never share an SM.
+    if (smem < 116 * 1024)
+        smem = 116 * 1024;
+    out->A = A;
+    out->smem = smem;
+    return true;
+}
+
+template <class E>
+cudaError_t launch_tc(TcPlan pl, cudaStream_t stream) {
+    const TrunkProblem &P = pl.A.P;
+    alignas(64) CUtensorMap moff, mmask;
+    if (!encode_2d(&moff, TElem<E>::kTma, P.off_w, (uint64_t)P.C_in, (uint64_t)P.J, 2, kTBK,
+                   (uint32_t)pl.A.nbox, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (P.mask_out) {
+        if (!encode_2d(&mmask, TElem<E>::kTma, P.mask_w, (uint64_t)P.C_in, (uint64_t)P.J, 2,
+                       kTBK, (uint32_t)pl.A.nbox, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    } else {
+        mmask = moff;   // never read
+    }
+    pl.A.status = device_status_ptr();
+    if (!pl.A.status)
+        return cudaErrorInvalidDevice;
+    auto kern = trunk_tc_kernel<E>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), (int)pl.smem);
+    if (e != cudaSuccess)
+        return e;
+    const int sms = sm_count();
+    if (sms <= 0)
+        return cudaErrorNoDevice;
+    const int grid = pl.A.num_tiles < sms ? pl.A.num_tiles : sms;
+    timing_begin(stream);
+    kern<<<grid, kTThreads, pl.smem, stream>>>(pl.A, moff, mmask);
+    timing_end(stream);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool trunk_tc_supported(const TrunkProblem &P) {
+    if (P.dtype != DCN1D_BF16 && P.dtype != DCN1D_F16)
+        return false;
+    if ((reinterpret_cast<uintptr_t>(P.off_w) & 15) ||
+        (P.mask_out && (reinterpret_cast<uintptr_t>(P.mask_w) & 15)))
+        return false;   // TMA sources start on 16 bytes
+    TcPlan pl;
+    return make_tc_plan(P, &pl);
+}
+
+cudaError_t launch_trunk(const TrunkProblem &P, cudaStream_t stream, const char **kernel) {
+    if (trunk_tc_supported(P)) {
+        TcPlan pl;
+        make_tc_plan(P, &pl);
+        *kernel = "trunk_tcgen05";
+        return P.dtype == DCN1D_F16 ? launch_tc<__half>(pl, stream)
+                                    : launch_tc<__nv_bfloat16>(pl, stream);
+    }
+    *kernel = "trunk_simt";
+    switch (P.dtype) {
+    case DCN1D_F32: return launch_simt<float>(P, stream);
+    case DCN1D_BF16: return launch_simt<__nv_bfloat16>(P, stream);
+    case DCN1D_F16: return launch_simt<__half>(P, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace dcn1d

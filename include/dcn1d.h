@@ -286,6 +286,87 @@ int dcn1d_backward_lr(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
                       dcn1d_tensor *grad_weight, dcn1d_tensor *grad_bias, void *workspace,
                       size_t workspace_bytes, void *stream);
 
+/*
+ * PackedDeformConv1d's offset (and mask) predictor ("dc1d (DeformConv1d)" page,
+ * "PackedDeformConv1d": a depthwise-separable convolution block computes the
+ * offsets inside the layer; "Modulation (DCNv2)": modulated=True adds a second
+ * pointwise branch off the same depthwise trunk, ending in a sigmoid, for the
+ * mask).  With J = offset_groups * K and j = g*K + k:
+ *
+ *   t[b,c,l]         = dw_bias[c] + sum_k dw_weight[c,0,k] * x[b, c, l*stride - padding_left + k*dilation]
+ *   offsets[b,g,l,k] = off_bias[j] + sum_c off_weight[j,c] * t[b,c,l]
+ *   mask[b,g,l,k]    = sigmoid(mask_bias[j] + sum_c mask_weight[j,c] * t[b,c,l])
+ *
+ * (x reads zero outside [0, L_in)).  The depthwise convolution takes the
+ * layer's kernel size, stride, padding and dilation, so it yields one offset
+ * vector per output position; nothing sits between the depthwise and the
+ * pointwise convolutions.
+ *
+ *   x            [B, C_in, L_in]                      required
+ *   dw_weight    [C_in, 1, K]                         required
+ *   dw_bias      [C_in] or NULL
+ *   off_weight   [J, C_in] or [J, C_in, 1]            required
+ *   off_bias     [J] or NULL
+ *   mask_weight  like off_weight, or NULL (no mask head)
+ *   mask_bias    [J] or NULL (NULL when mask_weight is NULL)
+ *   offsets_out  [B, offset_groups, L_out, K]          required, written entirely
+ *   mask_out     like offsets_out; required with mask_weight, else NULL
+ *
+ * All tensors share one dtype; t stays on chip in fp32 and the outputs are
+ * rounded to that dtype.  offset_groups must divide C_in.  Device memory
+ * owned by the caller; runs on `stream`, asynchronously, and allocates
+ * nothing.  Returns DCN1D_OK, or the validation codes of dcn1d_forward
+ * (nothing launched), DCN1D_ERR_LAUNCH if the launch failed.
+ */
+int dcn1d_packed_trunk(const dcn1d_tensor *x, const dcn1d_tensor *dw_weight,
+                       const dcn1d_tensor *dw_bias, const dcn1d_tensor *off_weight,
+                       const dcn1d_tensor *off_bias, const dcn1d_tensor *mask_weight,
+                       const dcn1d_tensor *mask_bias, int64_t stride, int64_t padding_left,
+                       int64_t padding_right, int64_t dilation, int64_t offset_groups,
+                       dcn1d_tensor *offsets_out, dcn1d_tensor *mask_out, void *stream);
+
+/* Which trunk kernel dcn1d_packed_trunk launches ("trunk_tcgen05" or "trunk_simt"),
+ * or NULL if the arguments are invalid.  Host only. */
+const char *dcn1d_packed_trunk_kernel_name(
+    const dcn1d_tensor *x, const dcn1d_tensor *dw_weight, const dcn1d_tensor *dw_bias,
+    const dcn1d_tensor *off_weight, const dcn1d_tensor *off_bias,
+    const dcn1d_tensor *mask_weight, const dcn1d_tensor *mask_bias, int64_t stride,
+    int64_t padding_left, int64_t padding_right, int64_t dilation, int64_t offset_groups,
+    const dcn1d_tensor *offsets_out, const dcn1d_tensor *mask_out);
+
+/*
+ * The whole PackedDeformConv1d forward: dcn1d_packed_trunk, then the deformable
+ * convolution (dcn1d_forward_lr) of x with the predicted offsets and, when
+ * mask_weight is given, the predicted mask.  weight [C_out, C_in/groups, K]
+ * (K = dw_weight's), bias [C_out] or NULL, out [B, C_out, L_out].
+ * offsets_out / mask_out may be NULL: the predicted tensors then live in
+ * `workspace` (caller-owned device memory, 256-byte aligned, used only by the
+ * work this call enqueues).  dcn1d_packed_forward_workspace_size() gives the
+ * bytes for those tensors plus the forward's own scratch; a workspace smaller
+ * than the predicted tensors is DCN1D_ERR_ARG (NULL: DCN1D_ERR_NULL), and
+ * between that and the full size the forward runs a kernel without scratch.
+ * Enqueues the trunk kernel and the forward's kernels on `stream`.
+ */
+int dcn1d_packed_forward(const dcn1d_tensor *x, const dcn1d_tensor *dw_weight,
+                         const dcn1d_tensor *dw_bias, const dcn1d_tensor *off_weight,
+                         const dcn1d_tensor *off_bias, const dcn1d_tensor *mask_weight,
+                         const dcn1d_tensor *mask_bias, const dcn1d_tensor *weight,
+                         const dcn1d_tensor *bias, int64_t stride, int64_t padding_left,
+                         int64_t padding_right, int64_t dilation, int64_t groups,
+                         int64_t offset_groups, int unconstrained, dcn1d_tensor *offsets_out,
+                         dcn1d_tensor *mask_out, dcn1d_tensor *out, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/* Workspace bytes dcn1d_packed_forward wants for these arguments (see there), or
+ * minus the status code of invalid arguments.  Host only. */
+int64_t dcn1d_packed_forward_workspace_size(
+    const dcn1d_tensor *x, const dcn1d_tensor *dw_weight, const dcn1d_tensor *dw_bias,
+    const dcn1d_tensor *off_weight, const dcn1d_tensor *off_bias,
+    const dcn1d_tensor *mask_weight, const dcn1d_tensor *mask_bias, const dcn1d_tensor *weight,
+    const dcn1d_tensor *bias, int64_t stride, int64_t padding_left, int64_t padding_right,
+    int64_t dilation, int64_t groups, int64_t offset_groups, int unconstrained,
+    const dcn1d_tensor *offsets_out, const dcn1d_tensor *mask_out, const dcn1d_tensor *out);
+
 /* A static, human-readable name of a status code ("DCN1D_OK", ...). Never NULL. */
 const char *dcn1d_status_string(int status);
 

@@ -106,6 +106,17 @@ LARGE_BF16 = Workload(
     x_dist=("normal", 1.0), w_dist=("kaiming_normal",), bias_dist=("normal", 0.02),
     off_dist=("normal", 2.0), mask=False, unconstrained=True)
 
+# PackedDeformConv1d(modulated=True): the dc1d page's example layer (depthwise, one offset
+# group per channel, kernel 3, dilation 4, padding "same") at a long-signal size.  Its offsets
+# and mask come from the layer's own trunk; off_dist sets the spread of the predicted offsets.
+PACKED_MODULATED_BF16 = Workload(
+    name="packed_modulated_bf16", B=8, C_in=256, C_out=256, K=3, stride=1, padding=4,
+    dilation=4, groups=256, offset_groups=256, L_in=16384, L_out=16384, dtype="bf16",
+    x_dist=("normal", 1.0), w_dist=("normal", 0.3), bias_dist=("normal", 0.02),
+    off_dist=("normal", 2.0), mask=True, unconstrained=False)
+
+PACKED = {w.name: w for w in (PACKED_MODULATED_BF16,)}
+
 WORKLOADS = {w.name: w for w in (TINY_F32, USAGE_F32, DEPTHWISE_BF16, MODULATED_BF16, LARGE_BF16)}
 ORDERED = [TINY_F32, USAGE_F32, DEPTHWISE_BF16, MODULATED_BF16, LARGE_BF16]
 
@@ -157,3 +168,56 @@ def small_case(seed: int, *, B, C_in, C_out, K, stride, padding, dilation, group
         bias_dist=("normal", 0.5) if bias else None, off_dist=("normal", off_scale),
         mask=mask, unconstrained=unconstrained)
     return w, make_inputs(w, seed)
+
+
+def make_packed_inputs(w: Workload, seed: int = 0, modulated: Optional[bool] = None,
+                       biases: bool = True) -> dict:
+    """Draw PackedDeformConv1d's tensors on the CPU (same generator recipe as make_inputs).
+
+    Order: x [B, C_in, L_in] ~ x_dist; dw_weight [C_in, 1, K] ~ N(0, 1/sqrt(K)); dw_bias
+    [C_in] ~ N(0, 0.1); off_weight [G*K, C_in] ~ N(0, s/sqrt(C_in)) with s the std of
+    off_dist (so the predicted offsets spread about that much); off_bias [G*K] ~ N(0, 0.1);
+    mask_weight [G*K, C_in] ~ N(0, 1.5/sqrt(C_in)) and mask_bias ~ N(0, 0.1) when modulated
+    (default: the workload's mask flag); weight and bias as in make_inputs.  Biases are None
+    when ``biases`` is False.
+    """
+    if modulated is None:
+        modulated = w.mask
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    J = w.offset_groups * w.K
+    s_off = w.off_dist[1] if w.off_dist[0] == "normal" else 1.0
+
+    def normal(shape, std):
+        return torch.randn(shape, generator=gen, dtype=torch.float32) * std
+
+    x = _draw(gen, (w.B, w.C_in, w.L_in), w.x_dist, w.fan_in)
+    dw_weight = normal((w.C_in, 1, w.K), 1.0 / math.sqrt(w.K))
+    dw_bias = normal((w.C_in,), 0.1)
+    off_weight = normal((J, w.C_in), s_off / math.sqrt(w.C_in))
+    off_bias = normal((J,), 0.1)
+    mask_weight = normal((J, w.C_in), 1.5 / math.sqrt(w.C_in)) if modulated else None
+    mask_bias = normal((J,), 0.1) if modulated else None
+    weight = _draw(gen, (w.C_out, w.C_in // w.groups, w.K), w.w_dist, w.fan_in)
+    bias = _draw(gen, (w.C_out,), w.bias_dist, w.fan_in) if w.bias_dist is not None else None
+    out = {"x": x, "dw_weight": dw_weight, "dw_bias": dw_bias, "off_weight": off_weight,
+           "off_bias": off_bias, "mask_weight": mask_weight, "mask_bias": mask_bias,
+           "weight": weight, "bias": bias}
+    if not biases:
+        for k in ("dw_bias", "off_bias", "mask_bias", "bias"):
+            out[k] = None
+    dt = w.torch_dtype
+    return {k: (v.to(dt).contiguous() if v is not None else None) for k, v in out.items()}
+
+
+def packed_case(seed: int, *, B, C_in, C_out, K, stride, padding, dilation, groups,
+                offset_groups, L_in, L_out, dtype="f32", modulated=True, biases=True,
+                off_scale=2.0) -> tuple:
+    """A small random PackedDeformConv1d case (not one of the named workloads)."""
+    w = Workload(
+        name="packed_small", B=B, C_in=C_in, C_out=C_out, K=K, stride=stride, padding=padding,
+        dilation=dilation, groups=groups, offset_groups=offset_groups, L_in=L_in, L_out=L_out,
+        dtype=dtype, x_dist=("normal", 1.0), w_dist=("normal", 0.5),
+        bias_dist=("normal", 0.5) if biases else None, off_dist=("normal", off_scale),
+        mask=modulated, unconstrained=False)
+    return w, make_packed_inputs(w, seed, modulated, biases)
