@@ -35,6 +35,7 @@ import workloads as W  # noqa: E402
 
 METRIC = "DeformConv1d forward TFLOP/s (HBM GB/s if depthwise) as % of B200 roofline"
 METRIC_BACKWARD = "DeformConv1d backward TFLOP/s as % of B200 roofline"
+METRIC_PACKED = "PackedDeformConv1d forward TFLOP/s (trunk + deformable conv)"
 DEFAULT_WORKLOAD = "usage_f32"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -497,17 +498,202 @@ def run_backward_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
     return line if rank == 0 else None
 
 
+# ------------------------------------------------------------------ PackedDeformConv1d
+
+PACKED_KEYS = ("x", "dw_weight", "dw_bias", "off_weight", "off_bias", "mask_weight", "mask_bias",
+               "weight", "bias")
+
+
+def packed_flops(w: W.Workload, L_out: int = None, B: int = None) -> int:
+    """Multiply-adds x 2 of the layer: the trunk's depthwise (K per channel and position) and
+    pointwise heads (C_in per head channel and position), then the deformable convolution."""
+    L = w.L_out if L_out is None else L_out
+    b = w.B if B is None else B
+    heads = 2 if w.mask else 1
+    J = w.offset_groups * w.K
+    trunk = 2 * b * L * w.C_in * (w.K + heads * J)
+    return trunk + 2 * b * L * w.C_out * (w.C_in // w.groups) * w.K
+
+
+def packed_trunk_bytes(w: W.Workload) -> int:
+    """The trunk's tensors counted once: x and the trunk weights read, the predicted offsets
+    (and mask) written."""
+    es = 4 if w.dtype == "f32" else 2
+    heads = 2 if w.mask else 1
+    J = w.offset_groups * w.K
+    n = w.B * w.C_in * w.L_in + w.C_in * (w.K + 1) + heads * J * (w.C_in + 1)
+    n += heads * w.B * J * w.L_out
+    return n * es
+
+
+def time_oracle_packed(w: W.Workload, host: dict, target_s: float):
+    """The oracle layer on the first positions of batch element 0, grown to about target_s."""
+    import oracle
+    L = 64
+    while True:
+        Ls = min(w.L_in, L)
+        sl = dict(host)
+        sl["x"] = host["x"][:1, :, :Ls]
+        t0 = time.perf_counter()
+        _, _, _ = oracle.packed_forward(*[sl[k] for k in PACKED_KEYS], w.stride, w.padding,
+                                        w.dilation, w.groups, w.offset_groups,
+                                        w.unconstrained)
+        dt = time.perf_counter() - t0
+        L_out = oracle.out_length(Ls, w.K, w.stride, w.padding, w.dilation)
+        if dt > target_s / 4 or Ls >= w.L_in:
+            return packed_flops(w, L_out, 1) / dt / 1e12, L_out, dt, oracle.threads()
+        L = int(L * max(2.0, min(8.0, target_s / 4 / max(dt, 1e-3))))
+
+
+def run_packed_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
+    """One step = PackedDeformConv1d's forward of one batch: the fused trunk predicts the
+    offsets and mask (kept in the workspace), then the deformable convolution."""
+    import deformable_convolution_dcn1d_b200 as dcn
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dcn.load()
+    host = W.make_packed_inputs(w, seed=rank)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in host.items()}
+    out = torch.empty((w.B, w.C_out, w.L_out), dtype=w.torch_dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    pads = (w.padding, w.padding)
+
+    def step(t, o):
+        dcn.dcn1d_packed_forward(*[t[k] for k in PACKED_KEYS], w.stride, pads, w.dilation,
+                                 w.groups, w.offset_groups, w.unconstrained, out=o,
+                                 stream=stream)
+
+    trunk_kernel = dcn.dcn1d_packed_trunk_kernel_name(*[d[k] for k in PACKED_KEYS[:7]],
+                                                      w.stride, pads, w.dilation,
+                                                      w.offset_groups)
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step(d, out)
+    torch.cuda.synchronize(dev)
+    launches = dcn.dcn1d_last_launch_count()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step(d, out)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(ws)
+    ms_step = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), ws) / args.steps
+    # the trunk kernel's own time (the library's timing events go to the first launch)
+    k_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for e in k_starts + k_ends:
+        e.record(stream)
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        dcn.dcn1d_set_timing_events(k_starts[i], k_ends[i])
+        step(d, out)
+    torch.cuda.synchronize(dev)
+    barrier(ws)
+    ms_trunk = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(k_starts, k_ends)),
+                              ws) / args.steps
+    flops = packed_flops(w)
+    value = ws * flops / (ms_step / 1e3) / 1e12
+
+    # end to end: x and every weight from pinned host memory, the output back
+    pinned = {k: (v.pin_memory() if v is not None else None) for k, v in host.items()}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values() if v is not None)
+    d2h = out_host.numel() * out_host.element_size()
+    scratch = {k: (torch.empty_like(v) if v is not None else None) for k, v in d.items()}
+
+    def e2e_step():
+        for k, v in pinned.items():
+            if v is not None:
+                scratch[k].copy_(v, non_blocking=True)
+        step(scratch, out)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(args.warmup, 1)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        e2e_step()
+        e_ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(ws)
+    e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), ws)
+    e_value = ws * flops / (e_ms / args.steps / 1e3) / 1e12
+
+    # roofline of the trunk: the slower of its tensor-core time and its HBM time
+    heads = 2 if w.mask else 1
+    t_flops = 2 * w.B * w.L_out * w.C_in * (w.K + heads * w.offset_groups * w.K)
+    t_bytes = packed_trunk_bytes(w)
+    t_tensor = t_flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = t_bytes / (peaks["hbm_gbs"] * 1e9)
+    sec = ms_trunk / 1e3
+    if t_hbm >= t_tensor:
+        roof = {"bound": "hbm", "achieved": t_bytes / sec / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": t_flops / sec / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    roof.update({"frac": roof["achieved"] / roof["peak"],
+                 "traffic": load_traffic(trunk_kernel, w), "kernel": trunk_kernel,
+                 "peak_source": f"measured ({peaks['source']}); the bound is the slower of "
+                                f"{t_tensor * 1e6:.1f} us of tensor work and "
+                                f"{t_hbm * 1e6:.1f} us of HBM traffic",
+                 "algorithmic_flops": t_flops, "algorithmic_bytes": t_bytes,
+                 "tensor_frac": t_flops / sec / 1e12 / peaks["bf16_tflops"],
+                 "hbm_frac": t_bytes / sec / 1e9 / peaks["hbm_gbs"],
+                 "launches_per_step": launches, "kernel_ms": ms_trunk,
+                 "timing": "CUDA events the library records around the trunk kernel, per "
+                           "step, in a second timed run of the same K steps"})
+    line = {"metric": METRIC_PACKED, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded, shapes and distributions of the named "
+                                      "workload; random trunk weights)",
+            "config": workload_config(w, f"{trunk_kernel} + forward", ws,
+                                      l2="flushed between steps (256 MiB write outside the "
+                                         "timed events)"),
+            "roofline": roof, "clocks": clk.summary(),
+            "e2e": {"value": e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h,
+                    "note": "pinned host x and weights copied in, layer forward, output out"},
+            "gpu_launches": launches * args.steps}
+    line["config"]["modulated"] = w.mask
+    if want_cpu and ws == 1 and rank == 0:
+        v, n, dt, cores = time_oracle_packed(w, host, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": f"the layer on the first {n} output positions of "
+                                          f"batch element 0 ({dt:.1f} s)"}
+    return line if rank == 0 else None
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    help="one of %s, or 'all'" % ", ".join(W.WORKLOADS))
+                    help="one of %s, or 'all'; --pass packed takes %s"
+                         % (", ".join(W.WORKLOADS), ", ".join(W.PACKED)))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+    ap.add_argument("--pass", dest="which", default="forward",
+                    choices=["forward", "backward", "packed"],
                     help="time the forward (the default line) or the backward pass")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (small cases for profiling)")
@@ -519,8 +705,11 @@ def main():
     names = list(W.WORKLOADS) if args.workload == "all" else [args.workload]
     ws, rank, local = dist_env()
 
+    if args.which == "packed" and args.workload == DEFAULT_WORKLOAD:
+        names = ["packed_modulated_bf16"]
+
     def pick(name):
-        w = W.WORKLOADS[name]
+        w = W.WORKLOADS[name] if name in W.WORKLOADS else W.PACKED[name]
         if args.dtype:
             if w.dtype != "bf16":
                 raise SystemExit("--dtype f16 applies to the bf16 workloads only")
@@ -542,7 +731,8 @@ def main():
     peaks = load_peaks()
     try:
         for name in names:
-            run = run_backward_pass if args.which == "backward" else run_ours
+            run = {"backward": run_backward_pass, "packed": run_packed_pass}.get(args.which,
+                                                                                run_ours)
             line = run(args, pick(name), peaks, want_cpu=not args.no_cpu_baseline)
             if line is not None:
                 print(json.dumps(line), flush=True)

@@ -133,6 +133,7 @@ cudaError_t launch_simt(const TrunkProblem &P, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+
 // ---------------------------------------------------------------- tensor-core kernel
 
 constexpr int kTRows = 128;                 // output positions per tile = TMEM lanes
@@ -140,7 +141,9 @@ constexpr int kTBK = 64;                    // channels per k-block (128 bytes o
 constexpr uint32_t kTABytes = kTRows * 128; // one k-block of the A tile (16 KB)
 constexpr int kTMaxN = 256;                 // head channels per column chunk (MMA N limit)
 constexpr int kTMaxCin = 512;               // the whole A tile stays in shared memory
-constexpr int kTProdWarps = 16, kTTmaWarp = 16, kTMmaWarp = 17, kTThreads = 18 * 32;
+constexpr int kTBoxMax = 256;               // widest x window a TMA box holds (positions)
+constexpr int kTProdWarps = 16, kTWTmaWarp = 16, kTMmaWarp = 17, kTXTmaWarp = 18;
+constexpr int kTThreads = 19 * 32;
 constexpr uint32_t kTTmemCols = 512;        // two accumulator buffers of 256 columns
 constexpr uint64_t kTWaitNs = 2000000000ull;   // 2 s
 
@@ -157,6 +160,9 @@ struct TElem<__nv_bfloat16> {
         __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
         return *reinterpret_cast<uint32_t *>(&h);
     }
+    static __device__ __forceinline__ float widen(uint32_t bits16) {
+        return __uint_as_float(bits16 << 16);
+    }
 };
 
 template <>
@@ -169,12 +175,36 @@ struct TElem<__half> {
         __half2 h = __floats2half2_rn(a, b);
         return *reinterpret_cast<uint32_t *>(&h);
     }
+    static __device__ __forceinline__ float widen(uint32_t bits16) {
+        return __half2float(__ushort_as_half((unsigned short)bits16));
+    }
 };
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&v)[4]) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]),
                  "r"(v[2]), "r"(v[3])
                  : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ int2 ld_shared_v2(uint32_t addr) {
+    int2 v;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+// The logistic function through the hardware tanh: sigmoid(z) = (1 + tanh(z/2)) / 2.
+// tanh.approx.f32 is accurate to about 2^-11 relative, far inside a 16-bit output's
+// rounding (the tensor-core kernel writes bf16 or fp16 only).
+__device__ __forceinline__ float sigmoid_tanh(float z) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+    return fmaf(0.5f, t, 0.5f);
 }
 
 struct TcTrunkArgs {
@@ -184,17 +214,30 @@ struct TcTrunkArgs {
     int chunks_per_head;     // column chunks of kTMaxN per head
     int heads, chunks;       // heads (1 or 2) and chunks per tile
     int tiles_l, num_tiles;
-    int stages;              // weight ring depth
-    uint32_t w_stage_bytes;
-    uint32_t off_a, off_w, off_dw, off_bar;   // shared-memory layout
+    int wstages, xstages;    // weight and x ring depths
+    int boxw;                // x window width (positions, multiple of 8)
+    uint32_t w_stage_bytes, x_stage_bytes;
+    uint32_t off_a, off_w, off_x, off_dw, off_tab, off_bar;   // shared-memory layout
     unsigned int *status;    // device status word
 };
 
-template <class E>
+// First position of the x window of a tile: l*s - p for its first row, rounded down to a
+// multiple of 8 (a TMA box starts on 16 bytes); may be negative (zero fill).
+__device__ __forceinline__ int window_start(const TrunkProblem &P, int lbase) {
+    const int w = lbase * P.stride - P.padding;
+    return w >= 0 ? (w / 8) * 8 : -(((-w) + 7) / 8) * 8;
+}
+
+// kStageX: the x window of every (tile, k-block) is staged in shared memory by TMA (a
+// 19th warp issues those loads ahead of the producers); otherwise the producers read x
+// from global memory.  Every ring (weights, x windows) has exactly one consumer order:
+// a waiter is never more than one phase ahead of a barrier, which the parity waits need.
+template <class E, bool kStageX>
 __global__ void __launch_bounds__(kTThreads, 1)
     trunk_tc_kernel(const __grid_constant__ TcTrunkArgs A,
                     const __grid_constant__ CUtensorMap map_off,
-                    const __grid_constant__ CUtensorMap map_mask) {
+                    const __grid_constant__ CUtensorMap map_mask,
+                    const __grid_constant__ CUtensorMap map_x) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const TrunkProblem &P = A.P;
     const int warp = threadIdx.x / 32;
@@ -205,17 +248,23 @@ __global__ void __launch_bounds__(kTThreads, 1)
     unsigned char *smem = smem_raw + (sbase - sraw);
     const uint32_t a_s = sbase + A.off_a;
     const uint32_t w_s0 = sbase + A.off_w;
+    const uint32_t x_s0 = sbase + A.off_x;
     float *dw_s = reinterpret_cast<float *>(smem + A.off_dw);   // [C_in][K] weights, [C_in] biases
+    int2 *tab = reinterpret_cast<int2 *>(smem + A.off_tab);     // [heads][J] (offset, bias)
+    const uint32_t tab_s = sbase + A.off_tab;
     const uint32_t bar0 = sbase + A.off_bar;
-    const int S = A.stages;
+    const int SW = A.wstages, SX = A.xstages;
     auto w_full = [&](int s) { return bar0 + 8u * s; };
-    auto w_empty = [&](int s) { return bar0 + 8u * (S + s); };
-    const uint32_t a_full = bar0 + 16u * S;
+    auto w_empty = [&](int s) { return bar0 + 8u * (SW + s); };
+    auto x_full = [&](int s) { return bar0 + 8u * (2 * SW + s); };
+    auto x_empty = [&](int s) { return bar0 + 8u * (2 * SW + SX + s); };
+    const uint32_t a_full = bar0 + 8u * (2 * SW + 2 * SX);
     const uint32_t a_empty = a_full + 8u;
     const uint32_t d_full0 = a_full + 16u;    // + 8 d
     const uint32_t d_empty0 = a_full + 32u;   // + 8 d
     const uint32_t drain_bar = a_full + 48u;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + A.off_bar + 16 * S + 56);
+    uint32_t *tmem_holder =
+        reinterpret_cast<uint32_t *>(smem + A.off_bar + 8 * (2 * SW + 2 * SX) + 56);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     {
@@ -225,11 +274,24 @@ __global__ void __launch_bounds__(kTThreads, 1)
             dw_s[i] = ld_f32(dww + i);
         for (int i = threadIdx.x; i < P.C_in; i += kTThreads)
             dw_s[P.C_in * P.K + i] = dwb ? ld_f32(dwb + i) : 0.0f;
+        // Per head column j = g*K + k: its offset in the [G, L_out, K] block of one batch
+        // element (relative to row l's first value) and its bias.
+        const int LK = P.L_out * P.K;
+        for (int i = threadIdx.x; i < A.heads * P.J; i += kTThreads) {
+            const int head = i >= P.J, j = i - head * P.J;
+            const int g = j / P.K, k = j - g * P.K;
+            const E *bias = static_cast<const E *>(head ? P.mask_b : P.off_b);
+            tab[i] = make_int2(g * LK + k, __float_as_int(bias ? ld_f32(bias + j) : 0.0f));
+        }
     }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
+        for (int s = 0; s < SW; ++s) {
             mbar_init(w_full(s), 1);
             mbar_init(w_empty(s), 1);
+        }
+        for (int s = 0; s < SX; ++s) {
+            mbar_init(x_full(s), 1);
+            mbar_init(x_empty(s), kTProdWarps);   // every producer warp reads every stage
         }
         mbar_init(a_full, kTProdWarps);
         mbar_init(a_empty, 1);
@@ -245,17 +307,19 @@ __global__ void __launch_bounds__(kTThreads, 1)
         tmem_alloc(smem_u32(tmem_holder), kTTmemCols);
         tc_fence_before();
     }
-    if (warp == kTTmaWarp && lane == 0) {
+    if (warp == kTWTmaWarp && lane == 0) {
         tma_prefetch_desc(&map_off);
         if (A.heads > 1)
             tma_prefetch_desc(&map_mask);
+        if (kStageX)
+            tma_prefetch_desc(&map_x);
     }
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const BoundedWait wait{abort_flag, kTWaitNs, A.status};
 
-    if (warp == kTTmaWarp) {
+    if (warp == kTWTmaWarp) {
         // ------------------------------------------------------------ weight tiles
         if (lane == 0) {
             uint32_t it = 0;
@@ -265,21 +329,45 @@ __global__ void __launch_bounds__(kTThreads, 1)
                     const int n0 = (c % A.chunks_per_head) * kTMaxN;
                     const CUtensorMap *map = head ? &map_mask : &map_off;
                     for (int kb = 0; kb < A.nkb; ++kb, ++it) {
-                        const int s = it % S;
-                        const uint32_t ph = (it / S) & 1u;
+                        const int s = it % SW;
+                        const uint32_t ph = (it / SW) & 1u;
                         if (!wait(w_empty(s), ph ^ 1u))
-                            goto tma_done;
+                            goto wtma_done;
                         mbar_arrive_expect_tx(w_full(s), A.w_stage_bytes);
                         tma_load_2d(w_s0 + s * A.w_stage_bytes, map, kb * kTBK, n0, w_full(s));
                     }
                 }
-        tma_done:
+        wtma_done:
             // Let every load this thread issued land before the CTA can exit.
             volatile int never = 0;
             const BoundedWait drain{&never, kTWaitNs, A.status};
-            const uint32_t Su = (uint32_t)S;
-            for (uint32_t j = (it > Su ? it - Su : 0); j < it; ++j)
-                drain(w_full(j % Su), (j / Su) & 1u);
+            const uint32_t S = (uint32_t)SW;
+            for (uint32_t j = (it > S ? it - S : 0); j < it; ++j)
+                drain(w_full(j % S), (j / S) & 1u);
+        }
+    } else if (warp == kTXTmaWarp) {
+        // ------------------------------------------------------------ x windows
+        if (kStageX && lane == 0) {
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
+                const int b = t / A.tiles_l;
+                const int wx0 = window_start(P, (t % A.tiles_l) * kTRows);
+                for (int kb = 0; kb < A.nkb; ++kb, ++it) {
+                    const int s = it % SX;
+                    const uint32_t ph = (it / SX) & 1u;
+                    if (!wait(x_empty(s), ph ^ 1u))
+                        goto xtma_done;
+                    mbar_arrive_expect_tx(x_full(s), A.x_stage_bytes);
+                    tma_load_2d(x_s0 + s * A.x_stage_bytes, &map_x, wx0, b * P.C_in + kb * kTBK,
+                                x_full(s));
+                }
+            }
+        xtma_done:
+            volatile int never = 0;
+            const BoundedWait drain{&never, kTWaitNs, A.status};
+            const uint32_t S = (uint32_t)SX;
+            for (uint32_t j = (it > S ? it - S : 0); j < it; ++j)
+                drain(x_full(j % S), (j / S) & 1u);
         }
     } else if (warp == kTMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -296,8 +384,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
                         goto mma_done;
                     tc_fence_after();
                     for (int kb = 0; kb < A.nkb; ++kb, ++it) {
-                        const int s = it % S;
-                        const uint32_t ph = (it / S) & 1u;
+                        const int s = it % SW;
+                        const uint32_t ph = (it / SW) & 1u;
                         if (!wait(w_full(s), ph))
                             goto mma_done;
                         tc_fence_after();
@@ -324,22 +412,65 @@ __global__ void __launch_bounds__(kTThreads, 1)
     } else {
         // ------------------------------------------------------------ depthwise + drain
         const int q = warp % 4;          // TMEM lane quarter
-        const int h = warp / 4;          // k-blocks h, h+4, ...; drain columns 16h, 16(h+4), ...
+        const int h = warp / 4;          // k-blocks h, h+4, ... (global-load path); drain columns 16h, 16(h+4), ...
         const int r = 32 * q + lane;     // tile row
         uint32_t cg = 0, tc = 0;
         for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
             const int b = t / A.tiles_l;
-            const int l = (t % A.tiles_l) * kTRows + r;
+            const int lbase = (t % A.tiles_l) * kTRows;
+            const int l = lbase + r;
             const bool valid = l < P.L_out;
             if (!__all_sync(0xffffffffu, wait(a_empty, (tc & 1u) ^ 1u)))
                 goto prod_done;
-            {
+            if constexpr (kStageX) {
+                // Every warp takes 16 channels (two 16-byte chunks) of every k-block, so the
+                // x stages are consumed in ring order whatever the ring's depth.
+                // Window position of tap 0 of this row: l*s - p - window start (>= 0).
+                const uint32_t rel0 =
+                    (uint32_t)(r * P.stride + lbase * P.stride - P.padding -
+                               window_start(P, lbase));
+                for (int kb = 0; kb < A.nkb; ++kb) {
+                    const uint32_t itx = tc * (uint32_t)A.nkb + (uint32_t)kb;
+                    const int s = itx % SX;
+                    if (!__all_sync(0xffffffffu, wait(x_full(s), (itx / SX) & 1u)))
+                        goto prod_done;
+                    const uint32_t xst = x_s0 + s * A.x_stage_bytes + rel0 * 2u;
+                    const uint32_t row_addr = a_s + kb * kTABytes + r * 128;
+#pragma unroll 1
+                    for (int ch = 2 * h; ch < 2 * h + 2; ++ch) {   // 8 channels = 16 bytes
+                        const int c0 = kb * kTBK + ch * 8;
+                        float acc[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            acc[i] = dw_s[P.C_in * P.K + c0 + i];
+                        const uint32_t xrow = xst + (uint32_t)(ch * 8) * A.boxw * 2u;
+                        for (int k = 0; k < P.K; ++k) {
+                            const uint32_t xa = xrow + (uint32_t)(k * P.dilation) * 2u;
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                acc[i] = fmaf(dw_s[(c0 + i) * P.K + k],
+                                              TElem<E>::widen(ld_shared_u16(
+                                                  xa + (uint32_t)i * A.boxw * 2u)),
+                                              acc[i]);
+                        }
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            pk[i] = TElem<E>::pack(acc[2 * i], acc[2 * i + 1]);
+                        // 128-byte swizzle: 16-byte chunk `ch` of row r sits at chunk ch ^ (r % 8)
+                        st_shared_v4(row_addr + ((uint32_t)(ch ^ (r & 7)) << 4), pk);
+                    }
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(x_empty(s));
+                }
+            } else {
                 const E *xb = static_cast<const E *>(P.x) + (int64_t)b * P.C_in * P.L_in;
                 const int pos0 = l * P.stride - P.padding;
                 for (int kb = h; kb < A.nkb; kb += 4) {
                     const uint32_t row_addr = a_s + kb * kTABytes + r * 128;
 #pragma unroll 1
-                    for (int ch = 0; ch < 8; ++ch) {   // 8 channels = one 16-byte chunk
+                    for (int ch = 0; ch < 8; ++ch) {
                         const int c0 = kb * kTBK + ch * 8;
                         float acc[8];
 #pragma unroll
@@ -361,7 +492,6 @@ __global__ void __launch_bounds__(kTThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             pk[i] = TElem<E>::pack(acc[2 * i], acc[2 * i + 1]);
-                        // 128-byte swizzle: 16-byte chunk `ch` of row r sits at chunk ch ^ (r % 8)
                         st_shared_v4(row_addr + ((uint32_t)(ch ^ (r & 7)) << 4), pk);
                     }
                 }
@@ -370,45 +500,42 @@ __global__ void __launch_bounds__(kTThreads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(a_full);
-            for (int c = 0; c < A.chunks; ++c, ++cg) {
-                const uint32_t d = cg & 1u;
-                if (!__all_sync(0xffffffffu, wait(d_full0 + 8u * d, (cg >> 1) & 1u)))
-                    goto prod_done;
-                tc_fence_after();
-                const int head = c / A.chunks_per_head;
-                const int n0 = (c % A.chunks_per_head) * kTMaxN;
-                E *outp = static_cast<E *>(head ? P.mask_out : P.off_out);
-                const E *biasp = static_cast<const E *>(head ? P.mask_b : P.off_b);
-                for (int cc = h; cc < A.nbox / 16; cc += 4) {
-                    uint32_t v[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 256u * d + 16u * cc, v);
-                    tmem_wait_ld();
-                    int j = n0 + 16 * cc;
-                    int g = j / P.K, k = j - g * P.K;
-                    if (valid) {
-                        E *orow = outp + (((int64_t)b * P.offset_groups) * P.L_out + l) * P.K;
+            {
+                // offset of row l's first value in batch element b's [G, L_out, K] block
+                const int64_t rowoff =
+                    ((int64_t)b * P.offset_groups * P.L_out + (valid ? l : 0)) * P.K;
+                for (int c = 0; c < A.chunks; ++c, ++cg) {
+                    const uint32_t d = cg & 1u;
+                    if (!__all_sync(0xffffffffu, wait(d_full0 + 8u * d, (cg >> 1) & 1u)))
+                        goto prod_done;
+                    tc_fence_after();
+                    const int head = c / A.chunks_per_head;
+                    const int n0 = (c % A.chunks_per_head) * kTMaxN;
+                    E *orow = static_cast<E *>(head ? P.mask_out : P.off_out) + rowoff;
+                    const uint32_t tab_h = tab_s + (uint32_t)(head * P.J) * 8u;
+                    for (int cc = h; cc < A.nbox / 16; cc += 4) {
+                        uint32_t v[16];
+                        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 256u * d + 16u * cc, v);
+                        tmem_wait_ld();
+                        const int j0 = n0 + 16 * cc;
+                        if (valid) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            if (j < P.J) {
-                                float z = __uint_as_float(v[i]);
-                                if (biasp)
-                                    z += ld_f32(biasp + j);
-                                if (head)
-                                    z = 1.0f / (1.0f + __expf(-z));
-                                orow[(int64_t)g * P.L_out * P.K + k] = from_f32<E>(z);
-                            }
-                            ++j;
-                            if (++k == P.K) {
-                                k = 0;
-                                ++g;
+                            for (int i = 0; i < 16; ++i) {
+                                if (j0 + i < P.J) {
+                                    const int2 e = ld_shared_v2(tab_h + (uint32_t)(j0 + i) * 8u);
+                                    float z = __uint_as_float(v[i]) + __int_as_float(e.y);
+                                    if (head)
+                                        z = sigmoid_tanh(z);
+                                    orow[e.x] = from_f32<E>(z);
+                                }
                             }
                         }
                     }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(d_empty0 + 8u * d);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(d_empty0 + 8u * d);
             }
         }
     prod_done:;
@@ -429,7 +556,48 @@ __global__ void __launch_bounds__(kTThreads, 1)
 struct TcPlan {
     TcTrunkArgs A;
     size_t smem;
+    bool stage_x;
 };
+
+// Shared-memory layout: A tile, weight ring, x ring (staged only), depthwise weights,
+// column table, barriers.  Prefers deeper weight rings, then x rings of 2..4 stages.
+bool layout_tc(TcTrunkArgs &A, bool stage_x, size_t *smem_out) {
+    const TrunkProblem &P = A.P;
+    const size_t limit = 227 * 1024;
+    const size_t dw_bytes = ((size_t)P.C_in * (P.K + 1) * 4 + 15) / 16 * 16;
+    const size_t tab_bytes = ((size_t)A.heads * P.J * 8 + 15) / 16 * 16;
+    for (int sw = 4; sw >= 2; --sw) {
+        const size_t fixed = (size_t)A.off_w + (size_t)sw * A.w_stage_bytes + dw_bytes +
+                             tab_bytes + 64 + 1024;
+        int sx = 1;
+        if (stage_x) {
+            if (fixed + 8 * (2 * sw + 2 * 2) >= limit)
+                continue;
+            const size_t rest = limit - fixed - 8 * (2 * sw + 2 * 4);
+            sx = (int)(rest / A.x_stage_bytes);
+            if (sx > 4)
+                sx = 4;
+            if (sx < 2)
+                continue;
+        }
+        A.wstages = sw;
+        A.xstages = sx;
+        A.off_x = A.off_w + (uint32_t)sw * A.w_stage_bytes;
+        A.off_dw = A.off_x + (stage_x ? (uint32_t)sx * A.x_stage_bytes : 0u);
+        A.off_tab = A.off_dw + (uint32_t)dw_bytes;
+        A.off_bar = A.off_tab + (uint32_t)tab_bytes;
+        size_t smem = (size_t)A.off_bar + 8 * (2 * sw + 2 * sx) + 64 + 1024;
+        if (smem > limit)
+            continue;
+        // More than half the SM's shared memory: two CTAs (each holding all 512
+        // tensor-memory columns) never share an SM.
+        if (smem < 116 * 1024)
+            smem = 116 * 1024;
+        *smem_out = smem;
+        return true;
+    }
+    return false;
+}
 
 bool make_tc_plan(const TrunkProblem &P, TcPlan *out) {
     TcTrunkArgs A;
@@ -445,37 +613,30 @@ bool make_tc_plan(const TrunkProblem &P, TcPlan *out) {
     A.tiles_l = (P.L_out + kTRows - 1) / kTRows;
     A.num_tiles = P.B * A.tiles_l;
     A.w_stage_bytes = (uint32_t)A.nbox * 128u;
+    // The x window of a tile: 128 rows of taps, plus up to 7 positions of alignment.
+    const int64_t need = (int64_t)(kTRows - 1) * P.stride + (int64_t)P.dilation * (P.K - 1) + 1 + 7;
+    A.boxw = (int)((need + 7) / 8 * 8);
+    A.x_stage_bytes = (uint32_t)kTBK * (uint32_t)(A.boxw > 0 ? A.boxw : 8) * 2u;
     A.off_a = 0;
     A.off_w = A.off_a + (uint32_t)A.nkb * kTABytes;
-    const size_t dw_bytes = ((size_t)P.C_in * (P.K + 1) * 4 + 15) / 16 * 16;
-    const size_t limit = 227 * 1024, fixed = 1024 + 16 * 8 + 64;   // slack, bars, holder
-    const size_t base = A.off_w + dw_bytes + fixed;
-    if (base >= limit)
-        return false;
-    int stages = (int)((limit - base) / (A.w_stage_bytes + 16));
-    if (stages > 4)
-        stages = 4;
-    if (stages < 2)
-        return false;
-    A.stages = stages;
-    A.off_dw = A.off_w + (uint32_t)stages * A.w_stage_bytes;
-    A.off_bar = A.off_dw + (uint32_t)dw_bytes;
-    size_t smem = A.off_bar + 16 * stages + 64 + 1024;
-    if (smem > limit)
-        return false;
-    // More than half the SM's shared memory: two CTAs (each holding all 512
-    // tensor-memory columns) never share an SM.
-    if (smem < 116 * 1024)
-        smem = 116 * 1024;
+    bool stage_x = need <= kTBoxMax && P.L_in % 8 == 0 &&
+                   (reinterpret_cast<uintptr_t>(P.x) & 15) == 0;
+    size_t smem = 0;
+    if (!(stage_x && layout_tc(A, true, &smem))) {
+        stage_x = false;
+        if (!layout_tc(A, false, &smem))
+            return false;
+    }
     out->A = A;
     out->smem = smem;
+    out->stage_x = stage_x;
     return true;
 }
 
-template <class E>
+template <class E, bool kStageX>
 cudaError_t launch_tc(TcPlan pl, cudaStream_t stream) {
     const TrunkProblem &P = pl.A.P;
-    alignas(64) CUtensorMap moff, mmask;
+    alignas(64) CUtensorMap moff, mmask, mx;
     if (!encode_2d(&moff, TElem<E>::kTma, P.off_w, (uint64_t)P.C_in, (uint64_t)P.J, 2, kTBK,
                    (uint32_t)pl.A.nbox, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
@@ -486,10 +647,17 @@ cudaError_t launch_tc(TcPlan pl, cudaStream_t stream) {
     } else {
         mmask = moff;   // never read
     }
+    if (kStageX) {
+        if (!encode_2d(&mx, TElem<E>::kTma, P.x, (uint64_t)P.L_in, (uint64_t)P.B * P.C_in, 2,
+                       (uint32_t)pl.A.boxw, kTBK, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    } else {
+        mx = moff;      // never read
+    }
     pl.A.status = device_status_ptr();
     if (!pl.A.status)
         return cudaErrorInvalidDevice;
-    auto kern = trunk_tc_kernel<E>;
+    auto kern = trunk_tc_kernel<E, kStageX>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), (int)pl.smem);
     if (e != cudaSuccess)
         return e;
@@ -498,9 +666,14 @@ cudaError_t launch_tc(TcPlan pl, cudaStream_t stream) {
         return cudaErrorNoDevice;
     const int grid = pl.A.num_tiles < sms ? pl.A.num_tiles : sms;
     timing_begin(stream);
-    kern<<<grid, kTThreads, pl.smem, stream>>>(pl.A, moff, mmask);
+    kern<<<grid, kTThreads, pl.smem, stream>>>(pl.A, moff, mmask, mx);
     timing_end(stream);
     return cudaGetLastError();
+}
+
+template <class E>
+cudaError_t launch_tc_e(const TcPlan &pl, cudaStream_t stream) {
+    return pl.stage_x ? launch_tc<E, true>(pl, stream) : launch_tc<E, false>(pl, stream);
 }
 
 }  // namespace
@@ -511,6 +684,8 @@ bool trunk_tc_supported(const TrunkProblem &P) {
     if ((reinterpret_cast<uintptr_t>(P.off_w) & 15) ||
         (P.mask_out && (reinterpret_cast<uintptr_t>(P.mask_w) & 15)))
         return false;   // TMA sources start on 16 bytes
+    if ((int64_t)P.offset_groups * P.L_out * P.K >= ((int64_t)1 << 31))
+        return false;   // column offsets are int32
     TcPlan pl;
     return make_tc_plan(P, &pl);
 }
@@ -520,8 +695,8 @@ cudaError_t launch_trunk(const TrunkProblem &P, cudaStream_t stream, const char 
         TcPlan pl;
         make_tc_plan(P, &pl);
         *kernel = "trunk_tcgen05";
-        return P.dtype == DCN1D_F16 ? launch_tc<__half>(pl, stream)
-                                    : launch_tc<__nv_bfloat16>(pl, stream);
+        return P.dtype == DCN1D_F16 ? launch_tc_e<__half>(pl, stream)
+                                    : launch_tc_e<__nv_bfloat16>(pl, stream);
     }
     *kernel = "trunk_simt";
     switch (P.dtype) {
