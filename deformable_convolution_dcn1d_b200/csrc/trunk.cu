@@ -192,12 +192,6 @@ __device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ int2 ld_shared_v2(uint32_t addr) {
-    int2 v;
-    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-    return v;
-}
-
 // The logistic function through the hardware tanh: sigmoid(z) = (1 + tanh(z/2)) / 2.
 // tanh.approx.f32 is accurate to about 2^-11 relative, far inside a 16-bit output's
 // rounding (the tensor-core kernel writes bf16 or fp16 only).
@@ -205,6 +199,36 @@ __device__ __forceinline__ float sigmoid_tanh(float z) {
     float t;
     asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
     return fmaf(0.5f, t, 0.5f);
+}
+
+__device__ __forceinline__ int4 ld_shared_v4i(uint32_t addr) {
+    int4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+// Bias, sigmoid (mask head) and store of up to 32 consecutive head columns of one row:
+// column i's (offset, bias) pair sits at tab_addr + 8 i (two pairs per 16-byte load).
+template <class E, bool kMaskHead>
+__device__ __forceinline__ void drain32(const uint32_t (&v)[32], uint32_t tab_addr, E *orow,
+                                        int n_valid) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        if (i < n_valid) {
+            const int4 e = ld_shared_v4i(tab_addr + (uint32_t)i * 8u);
+            float z0 = __uint_as_float(v[i]) + __int_as_float(e.y);
+            float z1 = __uint_as_float(v[i + 1]) + __int_as_float(e.w);
+            if (kMaskHead) {
+                z0 = sigmoid_tanh(z0);
+                z1 = sigmoid_tanh(z1);
+            }
+            orow[e.x] = from_f32<E>(z0);
+            if (i + 1 < n_valid)
+                orow[e.z] = from_f32<E>(z1);
+        }
+    }
 }
 
 struct TcTrunkArgs {
@@ -216,6 +240,8 @@ struct TcTrunkArgs {
     int tiles_l, num_tiles;
     int wstages, xstages;    // weight and x ring depths
     int boxw;                // x window width (positions, multiple of 8)
+    int tabj;                // column-table entries per head (J rounded up to even: each
+                             // head's table starts on 16 bytes for the paired loads)
     uint32_t w_stage_bytes, x_stage_bytes;
     uint32_t off_a, off_w, off_x, off_dw, off_tab, off_bar;   // shared-memory layout
     unsigned int *status;    // device status word
@@ -277,11 +303,13 @@ __global__ void __launch_bounds__(kTThreads, 1)
         // Per head column j = g*K + k: its offset in the [G, L_out, K] block of one batch
         // element (relative to row l's first value) and its bias.
         const int LK = P.L_out * P.K;
-        for (int i = threadIdx.x; i < A.heads * P.J; i += kTThreads) {
-            const int head = i >= P.J, j = i - head * P.J;
+        for (int i = threadIdx.x; i < A.heads * A.tabj; i += kTThreads) {
+            const int head = i >= A.tabj, j = i - head * A.tabj;
             const int g = j / P.K, k = j - g * P.K;
             const E *bias = static_cast<const E *>(head ? P.mask_b : P.off_b);
-            tab[i] = make_int2(g * LK + k, __float_as_int(bias ? ld_f32(bias + j) : 0.0f));
+            tab[i] = j < P.J ? make_int2(g * LK + k,
+                                         __float_as_int(bias ? ld_f32(bias + j) : 0.0f))
+                             : make_int2(0, 0);
         }
     }
     if (threadIdx.x == 0) {
@@ -412,7 +440,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     } else {
         // ------------------------------------------------------------ depthwise + drain
         const int q = warp % 4;          // TMEM lane quarter
-        const int h = warp / 4;          // k-blocks h, h+4, ... (global-load path); drain columns 16h, 16(h+4), ...
+        const int h = warp / 4;          // k-blocks h, h+4, ... (global-load path); columns 64h..64h+63
         const int r = 32 * q + lane;     // tile row
         uint32_t cg = 0, tc = 0;
         for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
@@ -512,23 +540,22 @@ __global__ void __launch_bounds__(kTThreads, 1)
                     const int head = c / A.chunks_per_head;
                     const int n0 = (c % A.chunks_per_head) * kTMaxN;
                     E *orow = static_cast<E *>(head ? P.mask_out : P.off_out) + rowoff;
-                    const uint32_t tab_h = tab_s + (uint32_t)(head * P.J) * 8u;
-                    for (int cc = h; cc < A.nbox / 16; cc += 4) {
-                        uint32_t v[16];
-                        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 256u * d + 16u * cc, v);
+                    const uint32_t tab_h = tab_s + (uint32_t)(head * A.tabj) * 8u;
+                    // this warp's 64 columns of the chunk, 32 per tensor-memory load
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const int col = 64 * h + 32 * blk;
+                        if (col >= A.nbox)
+                            break;
+                        uint32_t v[32];
+                        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 256u * d + (uint32_t)col, v);
                         tmem_wait_ld();
-                        const int j0 = n0 + 16 * cc;
+                        const int j0 = n0 + col;
+                        const int n_valid = P.J - j0 < 32 ? P.J - j0 : 32;
                         if (valid) {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                if (j0 + i < P.J) {
-                                    const int2 e = ld_shared_v2(tab_h + (uint32_t)(j0 + i) * 8u);
-                                    float z = __uint_as_float(v[i]) + __int_as_float(e.y);
-                                    if (head)
-                                        z = sigmoid_tanh(z);
-                                    orow[e.x] = from_f32<E>(z);
-                                }
-                            }
+                            if (head)
+                                drain32<E, true>(v, tab_h + (uint32_t)j0 * 8u, orow, n_valid);
+                            else
+                                drain32<E, false>(v, tab_h + (uint32_t)j0 * 8u, orow, n_valid);
                         }
                     }
                     tc_fence_before();
@@ -565,7 +592,7 @@ bool layout_tc(TcTrunkArgs &A, bool stage_x, size_t *smem_out) {
     const TrunkProblem &P = A.P;
     const size_t limit = 227 * 1024;
     const size_t dw_bytes = ((size_t)P.C_in * (P.K + 1) * 4 + 15) / 16 * 16;
-    const size_t tab_bytes = ((size_t)A.heads * P.J * 8 + 15) / 16 * 16;
+    const size_t tab_bytes = (size_t)A.heads * A.tabj * 8 + 16;   // + one pair read past the end
     for (int sw = 4; sw >= 2; --sw) {
         const size_t fixed = (size_t)A.off_w + (size_t)sw * A.w_stage_bytes + dw_bytes +
                              tab_bytes + 64 + 1024;
@@ -610,6 +637,7 @@ bool make_tc_plan(const TrunkProblem &P, TcPlan *out) {
     A.chunks_per_head = (P.J + kTMaxN - 1) / kTMaxN;
     A.heads = P.mask_out ? 2 : 1;
     A.chunks = A.heads * A.chunks_per_head;
+    A.tabj = (P.J + 1) & ~1;
     A.tiles_l = (P.L_out + kTRows - 1) / kTRows;
     A.num_tiles = P.B * A.tiles_l;
     A.w_stage_bytes = (uint32_t)A.nbox * 128u;
