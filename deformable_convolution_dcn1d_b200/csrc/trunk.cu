@@ -209,14 +209,15 @@ __device__ __forceinline__ int4 ld_shared_v4i(uint32_t addr) {
     return v;
 }
 
-// Bias, sigmoid (mask head) and store of up to 32 consecutive head columns of one row:
-// column i's (offset, bias) pair sits at tab_addr + 8 i (two pairs per 16-byte load).
-template <class E, bool kMaskHead>
+// Bias, sigmoid (mask head) and store of 32 consecutive head columns of one row (the
+// first n_valid of them when kFull is false): column i's (offset, bias) pair sits at
+// tab_addr + 8 i, two pairs per 16-byte load.  The full form has no per-column test.
+template <class E, bool kMaskHead, bool kFull>
 __device__ __forceinline__ void drain32(const uint32_t (&v)[32], uint32_t tab_addr, E *orow,
                                         int n_valid) {
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
-        if (i < n_valid) {
+        if (kFull || i < n_valid) {
             const int4 e = ld_shared_v4i(tab_addr + (uint32_t)i * 8u);
             float z0 = __uint_as_float(v[i]) + __int_as_float(e.y);
             float z1 = __uint_as_float(v[i + 1]) + __int_as_float(e.w);
@@ -225,10 +226,19 @@ __device__ __forceinline__ void drain32(const uint32_t (&v)[32], uint32_t tab_ad
                 z1 = sigmoid_tanh(z1);
             }
             orow[e.x] = from_f32<E>(z0);
-            if (i + 1 < n_valid)
+            if (kFull || i + 1 < n_valid)
                 orow[e.z] = from_f32<E>(z1);
         }
     }
+}
+
+template <class E, bool kMaskHead>
+__device__ __forceinline__ void drain32_any(const uint32_t (&v)[32], uint32_t tab_addr,
+                                            E *orow, int n_valid) {
+    if (n_valid >= 32)
+        drain32<E, kMaskHead, true>(v, tab_addr, orow, 32);
+    else
+        drain32<E, kMaskHead, false>(v, tab_addr, orow, n_valid);
 }
 
 struct TcTrunkArgs {
@@ -553,9 +563,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
                         const int n_valid = P.J - j0 < 32 ? P.J - j0 : 32;
                         if (valid) {
                             if (head)
-                                drain32<E, true>(v, tab_h + (uint32_t)j0 * 8u, orow, n_valid);
+                                drain32_any<E, true>(v, tab_h + (uint32_t)j0 * 8u, orow, n_valid);
                             else
-                                drain32<E, false>(v, tab_h + (uint32_t)j0 * 8u, orow, n_valid);
+                                drain32_any<E, false>(v, tab_h + (uint32_t)j0 * 8u, orow, n_valid);
                         }
                     }
                     tc_fence_before();
