@@ -201,24 +201,18 @@ __device__ __forceinline__ float sigmoid_tanh(float z) {
     return fmaf(0.5f, t, 0.5f);
 }
 
-__device__ __forceinline__ int4 ld_shared_v4i(uint32_t addr) {
-    int4 v;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr));
-    return v;
-}
-
 // Bias, sigmoid (mask head) and store of 32 consecutive head columns of one row (the
-// first n_valid of them when kFull is false): column i's (offset, bias) pair sits at
-// tab_addr + 8 i, two pairs per 16-byte load.  The full form has no per-column test.
+// first n_valid of them when kFull is false): column i's (offset, bias) pair is tab[i],
+// read two pairs per 16-byte load.  The table is written once before the CTA's first
+// barrier, so these are ordinary loads the compiler may schedule ahead of their use.
+// The full form has no per-column test.
 template <class E, bool kMaskHead, bool kFull>
-__device__ __forceinline__ void drain32(const uint32_t (&v)[32], uint32_t tab_addr, E *orow,
+__device__ __forceinline__ void drain32(const uint32_t (&v)[32], const int4 *tab, E *orow,
                                         int n_valid) {
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
         if (kFull || i < n_valid) {
-            const int4 e = ld_shared_v4i(tab_addr + (uint32_t)i * 8u);
+            const int4 e = tab[i / 2];
             float z0 = __uint_as_float(v[i]) + __int_as_float(e.y);
             float z1 = __uint_as_float(v[i + 1]) + __int_as_float(e.w);
             if (kMaskHead) {
@@ -233,12 +227,12 @@ __device__ __forceinline__ void drain32(const uint32_t (&v)[32], uint32_t tab_ad
 }
 
 template <class E, bool kMaskHead>
-__device__ __forceinline__ void drain32_any(const uint32_t (&v)[32], uint32_t tab_addr,
+__device__ __forceinline__ void drain32_any(const uint32_t (&v)[32], const int4 *tab,
                                             E *orow, int n_valid) {
     if (n_valid >= 32)
-        drain32<E, kMaskHead, true>(v, tab_addr, orow, 32);
+        drain32<E, kMaskHead, true>(v, tab, orow, 32);
     else
-        drain32<E, kMaskHead, false>(v, tab_addr, orow, n_valid);
+        drain32<E, kMaskHead, false>(v, tab, orow, n_valid);
 }
 
 struct TcTrunkArgs {
@@ -287,7 +281,6 @@ __global__ void __launch_bounds__(kTThreads, 1)
     const uint32_t x_s0 = sbase + A.off_x;
     float *dw_s = reinterpret_cast<float *>(smem + A.off_dw);   // [C_in][K] weights, [C_in] biases
     int2 *tab = reinterpret_cast<int2 *>(smem + A.off_tab);     // [heads][J] (offset, bias)
-    const uint32_t tab_s = sbase + A.off_tab;
     const uint32_t bar0 = sbase + A.off_bar;
     const int SW = A.wstages, SX = A.xstages;
     auto w_full = [&](int s) { return bar0 + 8u * s; };
@@ -550,7 +543,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
                     const int head = c / A.chunks_per_head;
                     const int n0 = (c % A.chunks_per_head) * kTMaxN;
                     E *orow = static_cast<E *>(head ? P.mask_out : P.off_out) + rowoff;
-                    const uint32_t tab_h = tab_s + (uint32_t)(head * A.tabj) * 8u;
+                    const int2 *tab_h = tab + head * A.tabj;
                     // this warp's 64 columns of the chunk, 32 per tensor-memory load
                     for (int blk = 0; blk < 2; ++blk) {
                         const int col = 64 * h + 32 * blk;
@@ -562,10 +555,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
                         const int j0 = n0 + col;
                         const int n_valid = P.J - j0 < 32 ? P.J - j0 : 32;
                         if (valid) {
+                            // j0 is even and every head's table starts on 16 bytes
+                            const int4 *t4 = reinterpret_cast<const int4 *>(tab_h + j0);
                             if (head)
-                                drain32_any<E, true>(v, tab_h + (uint32_t)j0 * 8u, orow, n_valid);
+                                drain32_any<E, true>(v, t4, orow, n_valid);
                             else
-                                drain32_any<E, false>(v, tab_h + (uint32_t)j0 * 8u, orow, n_valid);
+                                drain32_any<E, false>(v, t4, orow, n_valid);
                         }
                     }
                     tc_fence_before();
