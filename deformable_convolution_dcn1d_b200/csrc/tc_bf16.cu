@@ -65,6 +65,8 @@ struct TcArgs {
     Problem P;
     int N;             // MMA N = Cg_out (multiple of 32, <= 256)
     int num_kb;        // k-blocks per tile
+    int half_kb;       // > 0: producer groups take contiguous halves [0, half_kb) and
+                       // [half_kb, num_kb); 0: they take the even and the odd k-blocks
     int tiles_l;       // tiles per (g, b)
     int num_tiles;
     int nch;           // x rows per stage
@@ -75,6 +77,14 @@ struct TcArgs {
     uint32_t off_w, off_x, off_bias, off_bar;   // shared-memory layout
     unsigned int *status;                       // device status word
 };
+
+// The k-block at pipeline position i of a tile.  Positions alternate between the two
+// producer groups (group = i % 2), so each group owns every other stage of the ring (the
+// ring depth is even).  With contiguous halves a group walks its channels in order and
+// meets each offset group once; the parity split is the fallback for odd counts.
+__device__ __forceinline__ int kb_at(const TcArgs &A, int i) {
+    return A.half_kb ? ((i & 1) ? A.half_kb + (i >> 1) : (i >> 1)) : i;
+}
 
 struct Tile {
     int g, b, lbase, wx0;
@@ -311,7 +321,8 @@ __global__ void __maxnreg__(96)
             for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
                 const Tile T = decode_tile(A, t);
                 const int xrow0 = T.b * P.C_in + T.g * P.cin_g;
-                for (int kb = 0; kb < A.num_kb; ++kb, ++it) {
+                for (int pos = 0; pos < A.num_kb; ++pos, ++it) {
+                    const int kb = kb_at(A, pos);
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
                     if (!wait(bar_empty(s), ph ^ 1u))
@@ -344,7 +355,7 @@ __global__ void __maxnreg__(96)
                 if (!wait(bar_dempty, (tc & 1u) ^ 1u))
                     goto mma_done;
                 tc_fence_after();
-                for (int kb = 0; kb < A.num_kb; ++kb, ++it) {
+                for (int pos = 0; pos < A.num_kb; ++pos, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
                     if (!wait(bar_full(s), ph) || !wait(bar_afull(s), ph))
@@ -355,7 +366,7 @@ __global__ void __maxnreg__(96)
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         mma_bf16_ts(tmem + kColD, tmem + kColA + 32u * s + 8u * kk,
                                     sw128_kmajor_desc(wst + 32u * kk), idesc,
-                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                                    (pos > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(bar_empty(s));
                 }
@@ -427,9 +438,20 @@ __global__ void __maxnreg__(96)
                 raw_m[k] = MASK ? ld_f32(static_cast<const E *>(P.mask) + obase + k) : 1.0f;
             }
         };
-        if ((int)blockIdx.x < A.num_tiles) {
+        // offset group of this warp's segment at position `pos` of a tile of group Tt.g
+        auto seg_og = [&](const Tile &Tt, int pos) {
+            const int c = (kb_at(A, pos) * kBK + kSeg * half) / K;
+            return (Tt.g * P.cin_g + c) / P.cin_per_og;
+        };
+        // This warp's group takes the positions whose ring index tcount*num_kb + pos has
+        // its parity, so each ring stage always has the same consumer group, even when a
+        // tile has an odd number of k-blocks (a parity wait is never a phase ahead).
+        auto first_pos = [&](uint32_t tcnt) {
+            return (int)(((uint32_t)par ^ (tcnt * (uint32_t)A.num_kb)) & 1u);
+        };
+        if ((int)blockIdx.x < A.num_tiles && first_pos(0) < A.num_kb) {
             const Tile T0 = decode_tile(A, blockIdx.x);
-            prefetch(blockIdx.x, T0, (T0.g * P.cin_g) / P.cin_per_og);
+            prefetch(blockIdx.x, T0, seg_og(T0, first_pos(0)));
         }
         for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
             const Tile T = decode_tile(A, t);
@@ -438,7 +460,10 @@ __global__ void __maxnreg__(96)
             const bool valid = l < P.L_out;
             const float start = (float)(l * P.stride - P.padding);
             const uint32_t win_bits = kFloorMagicBits + (uint32_t)T.wx0;
-            const int og_last = (T.g * P.cin_g + P.cin_g - 1) / P.cin_per_og;
+            const int pos_first = first_pos(tcount);
+            const int pos_last =
+                pos_first < A.num_kb ? pos_first + ((A.num_kb - 1 - pos_first) / 2) * 2 : 0;
+            const int og_last = pos_first < A.num_kb ? seg_og(T, pos_last) : 0;   // this warp's last
             const E *xb = static_cast<const E *>(P.x) + (int64_t)T.b * P.C_in * P.L_in;
             Taps<K> tp;
             // Offset group of the first channel of this warp's first segment; it only
@@ -446,9 +471,10 @@ __global__ void __maxnreg__(96)
             int og_cur = -1;
             int og = (T.g * P.cin_g) / P.cin_per_og;
             int og_next_c = (og + 1) * P.cin_per_og - T.g * P.cin_g;   // group-relative
-            const int kb_first = par, kb_first_stage = (A.num_kb < kStages ? A.num_kb : kStages);
-            for (int kb = kb_first; kb < A.num_kb; kb += 2) {
-                const uint32_t it = tcount * (uint32_t)A.num_kb + (uint32_t)kb;
+            const int kb_first_stage = (A.num_kb < kStages ? A.num_kb : kStages);
+            for (int pos = pos_first; pos < A.num_kb; pos += 2) {
+                const int kb = kb_at(A, pos);
+                const uint32_t it = tcount * (uint32_t)A.num_kb + (uint32_t)pos;
                 const int s = it % kStages;
                 const uint32_t ph = (it / kStages) & 1u;
                 const int kk0 = kb * kBK + kSeg * half;
@@ -501,7 +527,8 @@ __global__ void __maxnreg__(96)
                         prefetch(t, T, og + 1);
                     else if (t_next < A.num_tiles) {
                         const Tile Tn = decode_tile(A, t_next);   // once per tile
-                        prefetch(t_next, Tn, (Tn.g * P.cin_g) / P.cin_per_og);
+                        if (first_pos(tcount + 1) < A.num_kb)
+                            prefetch(t_next, Tn, seg_og(Tn, first_pos(tcount + 1)));
                     }
                 }
                 if (!__all_sync(0xffffffffu, wait(bar_full(s), ph)))
@@ -526,7 +553,7 @@ __global__ void __maxnreg__(96)
                     if (lane == 0)
                         mbar_arrive(bar_afull(s));
                 }
-                if (pend_t >= 0 && kb + 2 >= kb_first_stage) {
+                if (pend_t >= 0 && pos + 2 >= kb_first_stage) {
                     if (!epilogue(pend_t, pend_cnt))
                         goto prod_done;
                     pend_t = -1;
@@ -570,6 +597,11 @@ bool make_plan(const Problem &P, Plan *out) {
     const int Kg = P.cin_g * P.K;
     A.N = P.cout_g;
     A.num_kb = Kg / kBK;
+    // Contiguous halves pay off when offset groups change inside a conv group (each
+    // warp then meets every offset group of its half once instead of every group of the
+    // tile); with one offset group per conv group the k-block parities measure faster.
+    A.half_kb = (A.num_kb % 2 == 0 && A.num_kb >= 4 && P.cin_per_og < P.cin_g) ? A.num_kb / 2
+                                                                                 : 0;
     A.tiles_l = (P.L_out + kRows - 1) / kRows;
     A.num_tiles = P.groups * P.B * A.tiles_l;
     A.nch = (kBK - 1) / P.K + 2;
