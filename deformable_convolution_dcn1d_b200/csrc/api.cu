@@ -3,7 +3,9 @@
 #include <stdint.h>
 #include <string.h>
 
-#include "common.cuh"
+#include <mutex>
+
+#include "sm100.cuh"
 
 namespace dcn1d {
 namespace {
@@ -396,16 +398,23 @@ void timing_end(cudaStream_t stream) {
 // One status word per device (a __device__ variable exists once per device).
 __device__ unsigned int g_device_status = 0;
 
+// Cached per device and context (a device reset starts a new context, in which the
+// variable may live elsewhere).
 unsigned int *device_status_ptr() {
+    static std::mutex mu;
     static unsigned int *ptrs[64] = {};
+    static void *ctx_of[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return nullptr;
-    if (!ptrs[dev]) {
+    void *ctx = current_context();
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev] || ctx_of[dev] != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess)
             return nullptr;
         ptrs[dev] = static_cast<unsigned int *>(p);
+        ctx_of[dev] = ctx;
     }
     return ptrs[dev];
 }

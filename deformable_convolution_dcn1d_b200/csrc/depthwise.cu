@@ -228,11 +228,14 @@ __global__ void __launch_bounds__(kThreads) depthwise_kernel(DwArgs A) {
                 const uint32_t lim = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rz(off_limit));
                 inside = ((amax & 0xFFFFu) <= lim) && ((amax >> 16) <= lim);
             } else {
-                float amax = 0.0f;
+                // On the bits of |offset|: NaN and inf patterns exceed every finite
+                // one, so a NaN offset sends the warp to the checked path (a float
+                // max would drop the NaN).
+                uint32_t amax = 0;
 #pragma unroll
                 for (int j = 0; j < NW; ++j)
-                    amax = fmaxf(amax, fabsf(__uint_as_float(ow[j])));
-                inside = amax <= off_limit;   // false for NaN
+                    amax = max(amax, ow[j] & 0x7FFFFFFFu);
+                inside = amax <= __float_as_uint(off_limit);
             }
         }
         const float s0 = (float)(lg * P.stride - P.padding);

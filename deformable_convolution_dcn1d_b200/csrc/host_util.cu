@@ -21,6 +21,23 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+void *current_context() {
+    using GetCtxFn = CUresult (*)(CUcontext *);
+    static const GetCtxFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<GetCtxFn>(p);
+        return static_cast<GetCtxFn>(nullptr);
+    }();
+    CUcontext ctx = nullptr;
+    if (!fn || fn(&ctx) != CUDA_SUCCESS)
+        return nullptr;
+    return ctx;
+}
+
 int sm_count() {
     static std::atomic<int> counts[64] = {};
     int dev = 0;

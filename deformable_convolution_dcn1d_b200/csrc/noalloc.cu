@@ -11,7 +11,7 @@
 // device with cudaGetSymbolAddress.
 #include <mutex>
 
-#include "common.cuh"
+#include "sm100.cuh"
 
 namespace {
 
@@ -20,19 +20,25 @@ constexpr size_t kNoAllocScratchBytes = size_t(48) << 20;   // 48 MiB
 // Shared by every call on a device; it keeps the last call's contents.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of the scratch array on the current device (NULL on failure).
+// Device address of the scratch array on the current device (NULL on failure).  It is
+// looked up once per device and context: a device reset (cudaDeviceReset) ends the
+// context the cached address belongs to, so a new context triggers a new lookup.
 void *scratch_address() {
     static std::mutex mu;
     static void *addr[64] = {};
+    static void *ctx_of[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return nullptr;
+    // The first runtime call above made the device's primary context current.
+    void *ctx = dcn1d::current_context();
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (!addr[dev] || ctx_of[dev] != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess)
             return nullptr;
         addr[dev] = p;
+        ctx_of[dev] = ctx;
     }
     return addr[dev];
 }

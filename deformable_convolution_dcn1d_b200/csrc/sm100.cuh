@@ -270,6 +270,10 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (NULL if unavailable).
 EncodeTiledFn encode_fn();
+// The driver context current on this thread (NULL on failure).  Device addresses of
+// the library's static device variables belong to a context: a device reset ends it,
+// and the next context may place the variables elsewhere.
+void *current_context();
 // Number of SMs of the current device (0 on failure).
 int sm_count();
 // Raises a kernel's dynamic shared-memory limit on the current device, once per size

@@ -197,7 +197,9 @@ int dcn1d_forward_ws(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const d
  *
  * Set-up: the first call on each device looks up the array's device address
  * (with that device current) and caches it; make that first call before any
- * stream capture.
+ * stream capture.  The cached address belongs to the device's current driver
+ * context: after a device reset (cudaDeviceReset) the next call sees a new
+ * context and looks the address up again (that call is then a set-up call too).
  *
  * Scratch limit: arguments whose fastest path needs more than 48 MiB
  * (dcn1d_forward_workspace_size) are rejected with DCN1D_ERR_UNSUPPORTED and

@@ -62,5 +62,11 @@ def test_each_kernel_is_held_to_its_own_roofline():
     assert bench.roofline_for("tcgen05_f16", w, peaks)[:3] == ("tensor", "TFLOP/s", 1600.0)
     bound, unit, peak = bench.roofline_for("tcgen05_3xtf32", w, peaks)[:3]
     assert (bound, unit) == ("tensor", "TFLOP/s")
-    assert peak == pytest.approx(1600.0 * 1.1 / 2.25 / 3)
+    # the TF32 dense peak with the flops counted once, not divided by the three passes
+    assert peak == pytest.approx(1600.0 * 1.1 / 2.25)
     assert bench.roofline_for("direct", w, peaks)[0] == "alu"
+
+
+def test_default_line_is_the_largest_single_gpu_workload():
+    """The bench's default line runs the workload with the most contraction work."""
+    assert bench.DEFAULT_WORKLOAD == max(W.WORKLOADS.values(), key=lambda w: w.flops()).name
