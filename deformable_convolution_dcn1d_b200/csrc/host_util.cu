@@ -80,6 +80,33 @@ cudaError_t ensure_smem(const void *kernel, int bytes) {
     return cudaSuccess;
 }
 
+int resident_clusters(const void *kernel, const cudaLaunchConfig_t *cfg) {
+    struct Entry {
+        const void *fn;
+        int dev;
+        size_t smem;
+        int n;
+    };
+    static std::mutex mu;
+    static Entry table[64];
+    static int n = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+        if (table[i].fn == kernel && table[i].dev == dev && table[i].smem == cfg->dynamicSmemBytes)
+            return table[i].n;
+    cudaLaunchConfig_t q = *cfg;
+    q.gridDim = dim3(2 * 1024);   // any grid: the query counts resident clusters
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &q) != cudaSuccess)
+        return 0;
+    if (n < 64)
+        table[n++] = Entry{kernel, dev, cfg->dynamicSmemBytes, clusters};
+    return clusters;
+}
+
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t cols,
                uint64_t rows, uint32_t elem_bytes, uint32_t box_cols, uint32_t box_rows,
                CUtensorMapSwizzle swizzle) {
