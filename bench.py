@@ -227,9 +227,9 @@ def time_oracle(w: W.Workload, inputs: dict, target_s: float, seed: int = 0):
     n = int(min(total_points, max(n, n * target_s / max(dt, 1e-9))))
     p = pts(n)
     t0 = time.perf_counter()
-    oracle.forward_points(*args, p)
+    r = oracle.forward_points(*args, p)
     dt = time.perf_counter() - t0
-    return n * per_point_flops / dt / 1e12, n, dt, oracle.threads()
+    return n * per_point_flops / dt / 1e12, n, dt, oracle.threads(), (p, r)
 
 
 def unit_value(w: W.Workload, kernel: str, seconds: float, ranks: int = 1):
@@ -249,7 +249,7 @@ def run_reference(args, w: W.Workload):
     inputs = W.make_inputs(w, seed=0)
     per_point_flops = 2 * (w.C_in // w.groups) * w.K
     # Calibrate one step to about 1 s of oracle work.
-    _, n_step, _, cores = time_oracle(w, inputs, target_s=1.0)
+    _, n_step, _, cores, _ = time_oracle(w, inputs, target_s=1.0)
     import numpy as np
     rng = np.random.default_rng(1)
     a = (inputs["x"], inputs["offsets"], inputs["mask"], inputs["weight"], inputs["bias"],
@@ -417,12 +417,18 @@ def run_ours(args, w: W.Workload, peaks: dict, want_cpu: bool):
                     "note": "pinned host inputs copied in, forward, output copied out, per step"},
             "gpu_launches": launches_per_step * args.steps}
     if want_cpu and ws == 1 and rank == 0:
-        v, n, dt, cores = time_oracle(w, host, target_s=args.cpu_seconds)
+        v, n, dt, cores, (pts, r) = time_oracle(w, host, target_s=args.cpu_seconds)
         if kernel.startswith("depthwise"):
             v = n / (w.B * w.C_out * w.L_out) * w.algorithmic_bytes() / dt / 1e9
+        # the same sampled outputs of the timed path (out holds the last step's result, on
+        # the same inputs): max|y - r| / max|r| over the sample
+        y = out.double().cpu().numpy()[pts[:, 0], pts[:, 1], pts[:, 2]]
+        den = float(abs(r).max()) if len(r) else 0.0
+        err = float(abs(y - r).max()) / den if den > 0 else float(abs(y).max())
         line["cpu_baseline"] = {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
                                 "sample": f"{n} random outputs of {w.B * w.C_out * w.L_out} "
-                                          f"({dt:.1f} s)"}
+                                          f"({dt:.1f} s)",
+                                "max_rel_err_of_timed_path": err}
     return line if rank == 0 else None
 
 
@@ -537,6 +543,18 @@ def packed_trunk_bytes(w: W.Workload) -> int:
     return n * es
 
 
+def packed_layer_bytes(w: W.Workload) -> int:
+    """The fused layer's tensors counted once: x, the trunk weights and the deformable
+    weight and bias read, the output written (the predicted offsets and mask stay on chip)."""
+    es = 4 if w.dtype == "f32" else 2
+    heads = 2 if w.mask else 1
+    J = w.offset_groups * w.K
+    n = w.B * w.C_in * w.L_in + w.C_in * (w.K + 1) + heads * J * (w.C_in + 1)
+    n += w.C_out * (w.C_in // w.groups) * w.K + (w.C_out if w.bias_dist is not None else 0)
+    n += w.B * w.C_out * w.L_out
+    return n * es
+
+
 def time_oracle_packed(w: W.Workload, host: dict, target_s: float):
     """The oracle layer on the first positions of batch element 0, grown to about target_s."""
     import oracle
@@ -557,8 +575,9 @@ def time_oracle_packed(w: W.Workload, host: dict, target_s: float):
 
 
 def run_packed_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
-    """One step = PackedDeformConv1d's forward of one batch: the fused trunk predicts the
-    offsets and mask (kept in the workspace), then the deformable convolution."""
+    """One step = PackedDeformConv1d's forward of one batch: for the depthwise layer one
+    kernel whose predicted offsets and mask never leave the chip, otherwise the trunk
+    (predicted tensors in the workspace) and then the deformable convolution."""
     import deformable_convolution_dcn1d_b200 as dcn
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -579,6 +598,10 @@ def run_packed_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
     trunk_kernel = dcn.dcn1d_packed_trunk_kernel_name(*[d[k] for k in PACKED_KEYS[:7]],
                                                       w.stride, pads, w.dilation,
                                                       w.offset_groups)
+    layer_kernel = dcn.dcn1d_packed_forward_kernel_name(*[d[k] for k in PACKED_KEYS], w.stride,
+                                                        pads, w.dilation, w.groups,
+                                                        w.offset_groups, w.unconstrained)
+    fused = layer_kernel == "packed_fused_tcgen05"
     for _ in range(max(args.warmup, 0)):
         flush.zero_()
         step(d, out)
@@ -646,10 +669,11 @@ def run_packed_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
     e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), ws)
     e_value = ws * flops / (e_ms / args.steps / 1e3) / 1e12
 
-    # roofline of the trunk: the slower of its tensor-core time and its HBM time
+    # roofline of the timed kernel (the fused layer, else the trunk): the slower of its
+    # tensor-core time (the trunk's contraction) and its HBM time
     heads = 2 if w.mask else 1
     t_flops = 2 * w.B * w.L_out * w.C_in * (w.K + heads * w.offset_groups * w.K)
-    t_bytes = packed_trunk_bytes(w)
+    t_bytes = packed_layer_bytes(w) if fused else packed_trunk_bytes(w)
     t_tensor = t_flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = t_bytes / (peaks["hbm_gbs"] * 1e9)
     sec = ms_trunk / 1e3
@@ -659,8 +683,9 @@ def run_packed_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
     else:
         roof = {"bound": "tensor", "achieved": t_flops / sec / 1e12,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    timed = layer_kernel if fused else trunk_kernel
     roof.update({"frac": roof["achieved"] / roof["peak"],
-                 "traffic": load_traffic(trunk_kernel, w), "kernel": trunk_kernel,
+                 "traffic": load_traffic(timed, w), "kernel": timed,
                  "peak_source": f"measured ({peaks['source']}); the bound is the slower of "
                                 f"{t_tensor * 1e6:.1f} us of tensor work and "
                                 f"{t_hbm * 1e6:.1f} us of HBM traffic",
@@ -668,14 +693,15 @@ def run_packed_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
                  "tensor_frac": t_flops / sec / 1e12 / peaks["bf16_tflops"],
                  "hbm_frac": t_bytes / sec / 1e9 / peaks["hbm_gbs"],
                  "launches_per_step": launches, "kernel_ms": ms_trunk,
-                 "timing": "CUDA events the library records around the trunk kernel, per "
-                           "step, in a second timed run of the same K steps"})
+                 "timing": "CUDA events the library records around the "
+                           + ("fused layer kernel" if fused else "trunk kernel")
+                           + ", per step, in a second timed run of the same K steps"})
     line = {"metric": METRIC_PACKED, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic (seeded, shapes and distributions of the named "
                                       "workload; random trunk weights)",
-            "config": workload_config(w, f"{trunk_kernel} + forward", ws,
+            "config": workload_config(w, layer_kernel, ws,
                                       l2="flushed between steps (256 MiB write outside the "
                                          "timed events)"),
             "roofline": roof, "clocks": clk.summary(),

@@ -23,6 +23,7 @@ from ._binding import (  # noqa: F401
     dcn1d_last_launch_count,
     dcn1d_out_length,
     dcn1d_packed_forward,
+    dcn1d_packed_forward_kernel_name,
     dcn1d_packed_trunk,
     dcn1d_packed_trunk_kernel_name,
     dcn1d_sample_index,

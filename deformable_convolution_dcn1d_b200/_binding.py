@@ -86,6 +86,10 @@ SIGNATURES = [
      [_T] * 9 + [_I64] * 6 + [_INT] + [_T] * 3),
     ("dcn1d_packed_forward", _INT,
      [_T] * 9 + [_I64] * 6 + [_INT] + [_T] * 3 + [_P, ctypes.c_size_t, _P]),
+    ("dcn1d_packed_forward_kernel_name", ctypes.c_char_p,
+     [_T] * 9 + [_I64] * 6 + [_INT] + [_T] * 3),
+    ("dcn1d_test_forward_stalled", _INT,
+     [_T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _I64, _P]),
 ]
 
 
@@ -369,6 +373,23 @@ def dcn1d_forward_noalloc(x, offsets, mask, weight, bias, stride=1, padding=0, d
     return out
 
 
+def dcn1d_test_forward_stalled(x, offsets, weight, stride=1, padding=0, dilation=1, groups=1,
+                               offset_groups=1, unconstrained=False, out=None,
+                               wait_limit_ns=1_000_000, stream=None):
+    """Test hook of the failure path (include/dcn1d.h): the bf16 tensor-core kernel with its
+    loader switched off and a short wait limit.  Returns the call's status code (no raise);
+    the timeout itself is reported by the next dcn1d_device_status()."""
+    dev = _check_device((x, offsets, weight, out))
+    if out is None:
+        out = _out_for(x, weight, offsets)
+    descs = [_desc(t) for t in (x, offsets, weight, out)]
+    with torch.cuda.device(dev):
+        return int(load().dcn1d_test_forward_stalled(
+            _ref(descs[0]), _ref(descs[1]), _ref(descs[2]), stride, int(padding), dilation,
+            groups, offset_groups, int(bool(unconstrained)), _ref(descs[3]), int(wait_limit_ns),
+            _P(_stream_ptr(stream, dev))))
+
+
 def dcn1d_forward_workspace_size(x, offsets, mask, weight, bias, stride=1, padding=0,
                                  dilation=1, groups=1, offset_groups=1, unconstrained=False,
                                  out=None) -> int:
@@ -483,6 +504,32 @@ def dcn1d_packed_trunk_kernel_name(x, dw_weight, dw_bias, off_weight, off_bias,
     refs = [_ref(_desc(t)) for t in tensors]
     r = load().dcn1d_packed_trunk_kernel_name(*refs[:7], stride, pl, pr, dilation,
                                               offset_groups, refs[7], refs[8])
+    return r.decode() if r else None
+
+
+def dcn1d_packed_forward_kernel_name(x, dw_weight, dw_bias, off_weight, off_bias, mask_weight,
+                                     mask_bias, weight, bias, stride=1, padding=0, dilation=1,
+                                     groups=1, offset_groups=1, unconstrained=False,
+                                     with_offsets=False):
+    """Which form dcn1d_packed_forward takes ("packed_fused_tcgen05", or "<trunk>+<forward>"
+    for two launches); None for invalid arguments."""
+    K = weight.shape[2]
+    pl, pr = resolve_padding(padding, K, stride, dilation)
+    off_t = mask_t = None
+    if with_offsets:
+        off_t, mask_t = _trunk_outputs(x, dw_weight, mask_weight, stride, pl, pr, dilation,
+                                       offset_groups)
+    L_out = int(load().dcn1d_out_length_lr(x.shape[2], K, stride, pl, pr, dilation))
+    out = torch.empty((x.shape[0], weight.shape[0], max(L_out, 0)), dtype=x.dtype,
+                      device="meta")
+    tensors = (x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias, weight,
+               bias, off_t, mask_t)
+    descs = [_desc(t) if t is None or t.device.type != "meta" else _meta_desc(t)
+             for t in tensors] + [_meta_desc(out)]
+    r = load().dcn1d_packed_forward_kernel_name(*[_ref(d) for d in descs[:9]], stride, pl, pr,
+                                                dilation, groups, offset_groups,
+                                                int(bool(unconstrained)),
+                                                *[_ref(d) for d in descs[9:]])
     return r.decode() if r else None
 
 

@@ -329,6 +329,7 @@ size_t round256(size_t n) { return (n + 255) / 256 * 256; }
 // then the forward's own scratch.
 struct PackedLayout {
     size_t off_bytes, mask_bytes, fwd_offset, total;
+    bool fused;   // one kernel: the predicted tensors stay on chip, no workspace
 };
 
 // Validation and layout shared by the packed forward and its workspace query.
@@ -378,6 +379,13 @@ int packed_prepare(const dcn1d_tensor *x, const dcn1d_tensor *dw_w, const dcn1d_
                   padding_right, dilation, groups, offset_groups, unconstrained, out, P);
     if (st != DCN1D_OK)
         return st;
+    // The caller asked for neither predicted tensor and the layer is the depthwise one the
+    // fused kernel takes: nothing goes through global memory between the two stages.
+    lay->fused = !off_out && !mask_out && packed_fused_supported(*T, *P);
+    if (lay->fused) {
+        lay->off_bytes = lay->mask_bytes = lay->fwd_offset = lay->total = 0;
+        return DCN1D_OK;
+    }
     lay->total = lay->fwd_offset + round256(workspace_bytes(*P));
     return DCN1D_OK;
 }
@@ -509,6 +517,28 @@ int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1
                   int unconstrained, dcn1d_tensor *out, void *stream) {
     return dcn1d_forward_ws(x, offsets, mask, weight, bias, stride, padding, dilation, groups,
                             offset_groups, unconstrained, out, nullptr, 0, stream);
+}
+
+int dcn1d_test_forward_stalled(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                               const dcn1d_tensor *weight, int64_t stride, int64_t padding,
+                               int64_t dilation, int64_t groups, int64_t offset_groups,
+                               int unconstrained, dcn1d_tensor *out, int64_t wait_limit_ns,
+                               void *stream) {
+    g_last_launches = 0;
+    Problem P;
+    int st = validate(x, offsets, nullptr, weight, nullptr, stride, padding, padding, dilation,
+                      groups, offset_groups, unconstrained, out, &P);
+    if (st != DCN1D_OK)
+        return st;
+    if (wait_limit_ns < 1000 || wait_limit_ns > 100000000)   // 1 us .. 100 ms
+        return DCN1D_ERR_ARG;
+    if (P.B == 0 || !tc_bf16_stalled_supported(P))
+        return DCN1D_ERR_UNSUPPORTED;
+    if (launch_tc_bf16_stalled(P, (uint64_t)wait_limit_ns, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return DCN1D_ERR_LAUNCH;
+    g_last_launches = 1;
+    return DCN1D_OK;
 }
 
 int64_t dcn1d_forward_lr_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
@@ -719,6 +749,33 @@ const char *dcn1d_packed_trunk_kernel_name(
     return trunk_tc_supported(T) ? "trunk_tcgen05" : "trunk_simt";
 }
 
+const char *dcn1d_packed_forward_kernel_name(
+    const dcn1d_tensor *x, const dcn1d_tensor *dw_weight, const dcn1d_tensor *dw_bias,
+    const dcn1d_tensor *off_weight, const dcn1d_tensor *off_bias,
+    const dcn1d_tensor *mask_weight, const dcn1d_tensor *mask_bias, const dcn1d_tensor *weight,
+    const dcn1d_tensor *bias, int64_t stride, int64_t padding_left, int64_t padding_right,
+    int64_t dilation, int64_t groups, int64_t offset_groups, int unconstrained,
+    const dcn1d_tensor *offsets_out, const dcn1d_tensor *mask_out, const dcn1d_tensor *out) {
+    TrunkProblem T;
+    Problem P;
+    dcn1d_tensor od, md;
+    PackedLayout lay;
+    if (packed_prepare(x, dw_weight, dw_bias, off_weight, off_bias, mask_weight, mask_bias,
+                       weight, bias, stride, padding_left, padding_right, dilation, groups,
+                       offset_groups, unconstrained, offsets_out, mask_out, out, nullptr, &T, &od,
+                       &md, &P, &lay) != DCN1D_OK)
+        return nullptr;
+    if (lay.fused)
+        return "packed_fused_tcgen05";
+    // two launches: the trunk, then the forward on the predicted tensors
+    static const char *names[2][4] = {
+        {"trunk_simt+direct", "trunk_simt+depthwise", "trunk_simt+tcgen05_bf16",
+         "trunk_simt+tcgen05_3xtf32"},
+        {"trunk_tcgen05+direct", "trunk_tcgen05+depthwise", "trunk_tcgen05+tcgen05_bf16",
+         "trunk_tcgen05+tcgen05_3xtf32"}};
+    return names[trunk_tc_supported(T) ? 1 : 0][select_kernel(P, SIZE_MAX)];
+}
+
 int64_t dcn1d_packed_forward_workspace_size(
     const dcn1d_tensor *x, const dcn1d_tensor *dw_weight, const dcn1d_tensor *dw_bias,
     const dcn1d_tensor *off_weight, const dcn1d_tensor *off_bias,
@@ -766,6 +823,12 @@ int dcn1d_packed_forward(const dcn1d_tensor *x, const dcn1d_tensor *dw_weight,
         return ws ? DCN1D_ERR_ARG : DCN1D_ERR_NULL;   // no room for the predicted tensors
     if (T.B == 0)
         return DCN1D_OK;
+    if (lay.fused) {
+        if (launch_packed_fused(T, P, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return DCN1D_ERR_LAUNCH;
+        g_last_launches = 1;
+        return DCN1D_OK;
+    }
     T.off_out = od.data;
     T.mask_out = mask_weight ? md.data : nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -66,6 +66,10 @@ int tc_tf32_launches(const Problem &P);
 cudaError_t launch_tc_tf32(const Problem &P, void *workspace, cudaStream_t stream);
 bool tc_bf16_supported(const Problem &P);
 cudaError_t launch_tc_bf16(const Problem &P, cudaStream_t stream);
+// Test of the failure path: the tensor-core kernel with its loader switched off at
+// compile time and every wait limited to wait_ns (bf16, K = 3, no mask only).
+bool tc_bf16_stalled_supported(const Problem &P);
+cudaError_t launch_tc_bf16_stalled(const Problem &P, uint64_t wait_ns, cudaStream_t stream);
 // Backward (backward.cu): the upstream gradient and the wanted gradients (each
 // output NULL when not wanted), all in the problem's dtype and its inputs' shapes.
 struct BackwardGrads {
@@ -87,6 +91,11 @@ struct TrunkProblem {
     void *off_out, *mask_out;  // [B, offset_groups, L_out, K]; mask_out NULL: no mask head
 };
 bool trunk_tc_supported(const TrunkProblem &T);
+// PackedDeformConv1d's whole forward as one kernel (packed_fused.cu) for the depthwise
+// layer (groups == offset_groups == C_in == C_out, 16-bit): the trunk T feeds the
+// deformable forward P (whose offset and mask pointers are not used) on chip.
+bool packed_fused_supported(const TrunkProblem &T, const Problem &P);
+cudaError_t launch_packed_fused(const TrunkProblem &T, const Problem &P, cudaStream_t stream);
 // Launches the trunk; *kernel receives the name of the kernel chosen.
 cudaError_t launch_trunk(const TrunkProblem &T, cudaStream_t stream, const char **kernel);
 cudaError_t launch_sample_index(const void *off, int dtype, int B, int G, int L_out, int K,

@@ -348,6 +348,16 @@ const char *dcn1d_packed_trunk_kernel_name(
  * than the predicted tensors is DCN1D_ERR_ARG (NULL: DCN1D_ERR_NULL), and
  * between that and the full size the forward runs a kernel without scratch.
  * Enqueues the trunk kernel and the forward's kernels on `stream`.
+ *
+ * One kernel instead, with no workspace at all, for the depthwise layer of the
+ * dc1d page's PackedDeformConv1d example: when offsets_out and mask_out are
+ * both NULL, groups == offset_groups == C_in == C_out, the dtype is BF16 or
+ * F16, K <= 4 (K <= 3 with a mask head when C_in is 256), C_in a multiple of
+ * 64 up to 256, L_in a multiple of 8 and x and the head weights 16-byte
+ * aligned.  The trunk's output, the predicted offsets and the mask then stay
+ * on chip: each tile's offsets and mask (rounded to the dtype, as the tensors
+ * the two-launch path hands on) feed the deformable convolution inside the
+ * kernel.  dcn1d_packed_forward_kernel_name() says which form runs.
  */
 int dcn1d_packed_forward(const dcn1d_tensor *x, const dcn1d_tensor *dw_weight,
                          const dcn1d_tensor *dw_bias, const dcn1d_tensor *off_weight,
@@ -362,6 +372,17 @@ int dcn1d_packed_forward(const dcn1d_tensor *x, const dcn1d_tensor *dw_weight,
 /* Workspace bytes dcn1d_packed_forward wants for these arguments (see there), or
  * minus the status code of invalid arguments.  Host only. */
 int64_t dcn1d_packed_forward_workspace_size(
+    const dcn1d_tensor *x, const dcn1d_tensor *dw_weight, const dcn1d_tensor *dw_bias,
+    const dcn1d_tensor *off_weight, const dcn1d_tensor *off_bias,
+    const dcn1d_tensor *mask_weight, const dcn1d_tensor *mask_bias, const dcn1d_tensor *weight,
+    const dcn1d_tensor *bias, int64_t stride, int64_t padding_left, int64_t padding_right,
+    int64_t dilation, int64_t groups, int64_t offset_groups, int unconstrained,
+    const dcn1d_tensor *offsets_out, const dcn1d_tensor *mask_out, const dcn1d_tensor *out);
+
+/* Which form dcn1d_packed_forward takes for these arguments: "packed_fused_tcgen05"
+ * (one kernel, no workspace) or "<trunk kernel>+<forward kernel>" (two launches,
+ * e.g. "trunk_tcgen05+depthwise"); NULL if the arguments are invalid.  Host only. */
+const char *dcn1d_packed_forward_kernel_name(
     const dcn1d_tensor *x, const dcn1d_tensor *dw_weight, const dcn1d_tensor *dw_bias,
     const dcn1d_tensor *off_weight, const dcn1d_tensor *off_bias,
     const dcn1d_tensor *mask_weight, const dcn1d_tensor *mask_bias, const dcn1d_tensor *weight,
@@ -423,6 +444,26 @@ int dcn1d_device_status(void *stream);
  * this host thread enqueued (0 if none).  For counting launches in benchmarks.
  */
 int dcn1d_last_launch_count(void);
+
+/*
+ * TEST HOOK of the failure path of dcn1d_device_status (no counterpart on the
+ * pages; not part of the forward).  Runs the bf16 tensor-core kernel of
+ * dcn1d_forward on these arguments (bf16, kernel size 3, no mask, no bias,
+ * shapes that kernel takes) in a build whose loader never issues a load, with
+ * every on-chip wait limited to `wait_limit_ns` (1 us .. 100 ms).  No stage
+ * ever fills, so the waits run out: the kernel records the timeout in the
+ * device status word, lets nothing it issued stay in flight, frees its tensor
+ * memory and exits; `out` is left unwritten.  The next dcn1d_device_status on
+ * this device returns DCN1D_ERR_TIMEOUT.  No GPU fault, trap or hang is
+ * involved.  Returns DCN1D_ERR_UNSUPPORTED for other shapes or dtypes,
+ * DCN1D_ERR_ARG for a limit outside the range, else the codes of
+ * dcn1d_forward.
+ */
+int dcn1d_test_forward_stalled(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
+                               const dcn1d_tensor *weight, int64_t stride, int64_t padding,
+                               int64_t dilation, int64_t groups, int64_t offset_groups,
+                               int unconstrained, dcn1d_tensor *out, int64_t wait_limit_ns,
+                               void *stream);
 
 #ifdef __cplusplus
 }

@@ -51,6 +51,9 @@ def test_packed_flops_and_trunk_bytes(modulated):
                                           "mask_weight", "mask_bias") if t[k] is not None)
     predicted = heads * w.B * w.offset_groups * w.L_out * w.K
     assert bench.packed_trunk_bytes(w) == (trunk_in + predicted) * 2
+    # the fused layer: every input once, the output once, the predicted tensors not at all
+    every_input = sum(v.numel() for v in t.values() if v is not None)
+    assert bench.packed_layer_bytes(w) == (every_input + w.B * w.C_out * w.L_out) * 2
 
 
 def test_each_kernel_is_held_to_its_own_roofline():
