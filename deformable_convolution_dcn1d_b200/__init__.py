@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     SIGNATURES,
     clear_workspace_cache,
     dcn1d_backward,
+    dcn1d_backward_kernel_name,
     dcn1d_backward_workspace_size,
     dcn1d_device_status,
     dcn1d_forward,

@@ -88,6 +88,8 @@ SIGNATURES = [
      [_T] * 9 + [_I64] * 6 + [_INT] + [_T] * 3 + [_P, ctypes.c_size_t, _P]),
     ("dcn1d_packed_forward_kernel_name", ctypes.c_char_p,
      [_T] * 9 + [_I64] * 6 + [_INT] + [_T] * 3),
+    ("dcn1d_backward_kernel_name", ctypes.c_char_p,
+     [_T, _T, _T, _T, _T] + [_I64] * 6 + [_INT] + [_T] * 5),
     ("dcn1d_test_forward_stalled", _INT,
      [_T, _T, _T, _I64, _I64, _I64, _I64, _I64, _INT, _T, _I64, _P]),
 ]
@@ -328,6 +330,24 @@ def dcn1d_backward(x, offsets, mask, weight, grad_out, stride=1, padding=0, dila
     if st != 0:
         raise Dcn1dError(st, "dcn1d_backward")
     return {n: out[n] for n in wanted}
+
+
+def dcn1d_backward_kernel_name(x, offsets, mask, weight, grad_out, stride=1, padding=0,
+                               dilation=1, groups=1, offset_groups=1, unconstrained=False,
+                               wanted=GRADS):
+    """Which contraction kernels dcn1d_backward runs ("tcgen05_gemm" or "cuda_core_gemm")."""
+    wanted = tuple(n for n in wanted if n != "mask" or mask is not None)
+    like = {"x": x, "offsets": offsets, "mask": mask, "weight": weight}
+    probe = {n: torch.empty((weight.shape[0],) if n == "bias" else like[n].shape,
+                            dtype=x.dtype, device="meta") for n in wanted}
+    gd = [None if probe.get(n) is None else _meta_desc(probe[n]) for n in GRADS]
+    ins = [_desc(t) if t is None or t.device.type != "meta" else _meta_desc(t)
+           for t in (x, offsets, mask, weight, grad_out)]
+    pl, pr = resolve_padding(padding, weight.shape[2], stride, dilation)
+    r = load().dcn1d_backward_kernel_name(*(_ref(d) for d in ins), stride, pl, pr, dilation,
+                                          groups, offset_groups, int(bool(unconstrained)),
+                                          *(_ref(d) for d in gd))
+    return None if r is None else r.decode()
 
 
 def dcn1d_backward_workspace_size(x, offsets, mask, weight, grad_out, stride=1, padding=0,

@@ -565,6 +565,22 @@ int64_t dcn1d_forward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *
                                            unconstrained, out);
 }
 
+const char *dcn1d_backward_kernel_name(
+    const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
+    const dcn1d_tensor *weight, const dcn1d_tensor *grad_out, int64_t stride,
+    int64_t padding_left, int64_t padding_right, int64_t dilation, int64_t groups,
+    int64_t offset_groups, int unconstrained, const dcn1d_tensor *grad_x,
+    const dcn1d_tensor *grad_offsets, const dcn1d_tensor *grad_mask,
+    const dcn1d_tensor *grad_weight, const dcn1d_tensor *grad_bias) {
+    Problem P;
+    BackwardGrads G;
+    if (validate_backward(x, offsets, mask, weight, grad_out, stride, padding_left, padding_right,
+                          dilation, groups, offset_groups, unconstrained, grad_x, grad_offsets,
+                          grad_mask, grad_weight, grad_bias, &P, &G) != DCN1D_OK)
+        return nullptr;
+    return backward_uses_tensor_cores(P, G) ? "tcgen05_gemm" : "cuda_core_gemm";
+}
+
 int64_t dcn1d_backward_lr_workspace_size(
     const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
     const dcn1d_tensor *weight, const dcn1d_tensor *grad_out, int64_t stride,

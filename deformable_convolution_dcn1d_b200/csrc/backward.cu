@@ -13,17 +13,21 @@
 //                          constrained clamp moved the position)
 //   grad_bias[co]         = sum_{b,l} grad_out[b, co, l]
 //
-// Kernels, all fp32 arithmetic whatever the input type:
+// Kernels, fp32 arithmetic whatever the input type (16-bit problems contract 16-bit
+// operands on the tensor cores with fp32 accumulation):
 //  1. dcols[b, (c,k), l] = sum_co W[co, (c,k)] grad_out[b, co, l]: a batched GEMM
-//     per (batch, conv group) on CUDA cores (64x64 tiles, 4x4 per thread);
+//     per (batch, conv group); 16-bit problems: the tensor-core GEMM of gemm_tc.cu on
+//     K-major copies (grad_out transposed to [b][l][co], W per group to [(c,k)][co]),
+//     otherwise on CUDA cores (64x64 tiles, 4x4 per thread);
 //  2. the sampling gradient: one thread per (batch, 16-channel chunk, offset
 //     group, tap, position) recomputes the tap's position once, then for its
 //     channels scatters grad_x, sums the offset and mask gradients (atomics
 //     into fp32 scratch: the order of those sums is not fixed) and writes the
 //     sampled columns m*v that the weight gradient needs;
 //  3. grad_weight = sum_b grad_out[b] cols[b]^T: the same GEMM kernel, summing
-//     over the batch inside the tile loop; when that grid is small the batch sum
-//     is split across CTAs into fp32 slices added in split order (a fixed order);
+//     over the batch inside the tile loop (16-bit problems: the tensor-core GEMM on
+//     16-bit columns); when that grid is small the batch sum is split across CTAs
+//     into fp32 slices added in split order (a fixed order);
 //  4. grad_bias: one block per channel, a fixed-order tree reduction;
 //  5. the fp32 scratch of grad_x / grad_offsets / grad_mask is written out in
 //     the input type.
@@ -139,6 +143,7 @@ struct SampArgs {
     int nchunk;                  // channel chunks per offset group
     const float *dcols;          // [B][C_in*K][L_out] or NULL
     float *cols;                 // [B][C_in*K][L_out] or NULL
+    void *cols16;                // the same columns in the input's 16-bit type, or NULL
     float *gx, *goff, *gmask;    // fp32 scratch, each may be NULL
 };
 
@@ -184,6 +189,8 @@ __global__ void __launch_bounds__(256) sample_grad_kernel(const SampArgs a) {
         const int64_t cidx = (((int64_t)b * P.C_in + ci) * P.K + k) * P.L_out + l;
         if (a.cols)
             a.cols[cidx] = __fmul_rn(m, v);
+        if (sizeof(T) == 2 && a.cols16)
+            static_cast<T *>(a.cols16)[cidx] = from_f32<T>(__fmul_rn(m, v));
         if (a.dcols) {
             const float dv = a.dcols[cidx];
             if (a.gx) {
@@ -201,6 +208,28 @@ __global__ void __launch_bounds__(256) sample_grad_kernel(const SampArgs a) {
         atomicAdd(a.goff + oidx, s_off);
     if (a.gmask)
         atomicAdd(a.gmask + oidx, s_mask);
+}
+
+// dst[z][c][r] = src[z][r][c] for z < nz, r < R, c < Cc (16-bit elements): 32 x 32 tiles
+// through shared memory, both sides coalesced.  Source rows are ld_src elements apart,
+// destination rows ld_dst; z strides in elements.
+template <class T>
+__global__ void __launch_bounds__(256) transpose_kernel(const T *src, T *dst, int R, int Cc,
+                                                        int64_t ld_src, int64_t ld_dst,
+                                                        int64_t sz_src, int64_t sz_dst) {
+    __shared__ T tile[32][33];
+    const int z = blockIdx.z;
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+    const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;   // 32 x 8
+    const T *s = src + (int64_t)z * sz_src;
+    T *d = dst + (int64_t)z * sz_dst;
+    for (int i = ty; i < 32; i += 8)
+        if (r0 + i < R && c0 + tx < Cc)
+            tile[i][tx] = s[(int64_t)(r0 + i) * ld_src + c0 + tx];
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8)
+        if (c0 + i < Cc && r0 + tx < R)
+            d[(int64_t)(c0 + i) * ld_dst + r0 + tx] = tile[tx][i];
 }
 
 // grad_bias[co] = sum over (b, l) of grad_out[b, co, l]: one block per channel,
@@ -251,30 +280,70 @@ int wgrad_splits(const Problem &P) {
     return S;
 }
 
+// The tensor-core GEMMs serve 16-bit problems whose K-major operands TMA can read: rows
+// of grad_out and of the columns (L_out elements), of grad_out transposed (C_out) and of
+// W transposed per group (C_out / groups) all multiples of 16 bytes.
+bool tc_backward(const Problem &P, const BackwardGrads &G) {
+    if (P.dtype != DCN1D_BF16 && P.dtype != DCN1D_F16)
+        return false;
+    if (P.L_out % 8 || P.C_out % 8 || P.cout_g % 8)
+        return false;
+    if ((reinterpret_cast<uintptr_t>(G.gout) & 15) || (reinterpret_cast<uintptr_t>(P.w) & 15))
+        return false;
+    const int64_t rows = (int64_t)P.B * (P.C_in * P.K > P.C_out ? P.C_in * P.K : P.C_out);
+    return (int64_t)P.B * P.L_out < (1LL << 31) && rows < (1LL << 31);
+}
+
+// Splits of the tensor-core weight-gradient GEMM's batch sum: the largest divisor of B
+// that brings its 128 x N tiles to about one or two waves of the SMs.
+int wgrad_splits_tc(const Problem &P) {
+    const int sms = sm_count() > 0 ? sm_count() : 148;
+    const int nt = P.cout_g <= 128 ? (P.cout_g <= 64 ? 64 : 128) : 256;
+    const int64_t tiles = (int64_t)((P.cin_g * P.K + 127) / 128) * ((P.cout_g + nt - 1) / nt) *
+                          P.groups;
+    int want = (int)((2 * sms + tiles - 1) / tiles);
+    if (want > P.B)
+        want = P.B;
+    int S = 1;
+    for (int d = 1; d <= want; ++d)
+        if (P.B % d == 0)
+            S = d;
+    return S;
+}
+
 struct WsLayout {
     size_t dcols, cols, gx, goff, gmask, wpart, total;   // byte offsets (SIZE_MAX: not used)
+    size_t goutT, wT;    // tensor-core path: grad_out and W transposed (16-bit)
     int wsplits;
+    bool tc;
 };
 
 WsLayout ws_layout(const Problem &P, const BackwardGrads &G) {
     WsLayout w;
+    w.tc = tc_backward(P, G);
     const size_t ncol = (size_t)P.B * P.C_in * P.K * P.L_out * 4;
     const size_t noff = (size_t)P.B * P.offset_groups * P.L_out * P.K * 4;
     const bool need_dcols = G.x || G.off || G.mask;
     size_t at = 0;
     w.dcols = need_dcols ? at : SIZE_MAX;
     at += need_dcols ? align256(ncol) : 0;
-    w.cols = G.w ? at : SIZE_MAX;
-    at += G.w ? align256(ncol) : 0;
+    w.cols = G.w ? at : SIZE_MAX;   // the tensor-core path keeps them in 16 bits
+    at += G.w ? align256(w.tc ? ncol / 2 : ncol) : 0;
+    w.goutT = (w.tc && need_dcols) ? at : SIZE_MAX;
+    at += (w.tc && need_dcols) ? align256((size_t)P.B * P.C_out * P.L_out * 2) : 0;
+    w.wT = (w.tc && need_dcols) ? at : SIZE_MAX;
+    at += (w.tc && need_dcols) ? align256((size_t)P.C_out * P.cin_g * P.K * 2) : 0;
     w.gx = G.x ? at : SIZE_MAX;
     at += G.x ? align256((size_t)P.B * P.C_in * P.L_in * 4) : 0;
     w.goff = G.off ? at : SIZE_MAX;
     at += G.off ? align256(noff) : 0;
     w.gmask = G.mask ? at : SIZE_MAX;
     at += G.mask ? align256(noff) : 0;
-    w.wsplits = G.w ? wgrad_splits(P) : 1;
-    w.wpart = w.wsplits > 1 ? at : SIZE_MAX;
-    at += w.wsplits > 1 ? align256((size_t)w.wsplits * P.C_out * P.cin_g * P.K * 4) : 0;
+    w.wsplits = G.w ? (w.tc ? wgrad_splits_tc(P) : wgrad_splits(P)) : 1;
+    // the tensor-core GEMM writes fp32 slices even unsplit (then converted)
+    const bool parts = G.w && (w.wsplits > 1 || w.tc);
+    w.wpart = parts ? at : SIZE_MAX;
+    at += parts ? align256((size_t)w.wsplits * P.C_out * P.cin_g * P.K * 4) : 0;
     w.total = at;
     return w;
 }
@@ -290,7 +359,11 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
     const WsLayout L = ws_layout(P, G);
     unsigned char *wsb = static_cast<unsigned char *>(ws);
     float *dcols = L.dcols != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.dcols) : nullptr;
-    float *cols = L.cols != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.cols) : nullptr;
+    float *cols = (L.cols != SIZE_MAX && !L.tc) ? reinterpret_cast<float *>(wsb + L.cols)
+                                                : nullptr;
+    T *cols16 = (L.cols != SIZE_MAX && L.tc) ? reinterpret_cast<T *>(wsb + L.cols) : nullptr;
+    T *goutT = L.goutT != SIZE_MAX ? reinterpret_cast<T *>(wsb + L.goutT) : nullptr;
+    T *wT = L.wT != SIZE_MAX ? reinterpret_cast<T *>(wsb + L.wT) : nullptr;
     float *gx = L.gx != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.gx) : nullptr;
     float *goff = L.goff != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.goff) : nullptr;
     float *gmask = L.gmask != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.gmask) : nullptr;
@@ -311,7 +384,29 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
     if (gmask && (e = cudaMemsetAsync(gmask, 0, noff * 4, s)) != cudaSuccess)
         return e;
 
-    if (want_dcols && P.B > 0) {
+    if (want_dcols && P.B > 0 && L.tc) {
+        // 1. on the tensor cores: D[l][m] = sum_co goutT[b][l][g*cout_g + co] * wT[g][m][co],
+        // stored to dcols[b][g*Kg + m][l] (lanes = consecutive l)
+        const dim3 tb(256);
+        transpose_kernel<T><<<dim3((P.L_out + 31) / 32, (P.C_out + 31) / 32, P.B), tb, 0, s>>>(
+            gout, goutT, P.C_out, P.L_out, P.L_out, P.C_out, (int64_t)P.C_out * P.L_out,
+            (int64_t)P.L_out * P.C_out);
+        transpose_kernel<T><<<dim3((Kg + 31) / 32, (P.cout_g + 31) / 32, P.groups), tb, 0, s>>>(
+            w, wT, P.cout_g, Kg, Kg, P.cout_g, (int64_t)P.cout_g * Kg, (int64_t)Kg * P.cout_g);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+        n += 2;
+        for (int gi = 0; gi < P.groups; ++gi) {
+            if ((e = launch_gemm_tc(P.dtype, goutT + (int64_t)gi * P.cout_g,
+                                    (int64_t)P.B * P.L_out, P.C_out, 0, P.L_out, 0,
+                                    wT + (int64_t)gi * Kg * P.cout_g, Kg, P.cout_g, 0, 0, 0,
+                                    P.L_out, Kg, P.cout_g, 1, P.B,
+                                    dcols + (int64_t)gi * Kg * P.L_out, 1, P.L_out,
+                                    (int64_t)P.C_in * P.K * P.L_out, s)) != cudaSuccess)
+                return e;
+            ++n;
+        }
+    } else if (want_dcols && P.B > 0) {
         // 1. dcols[b][g*Kg + m][l] = sum_co W[g*cout_g + co][m] * gout[b][g*cout_g + co][l]
         GemmArgs g;
         memset(&g, 0, sizeof(g));
@@ -343,6 +438,7 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
         a.nchunk = (P.cin_per_og + kChunk - 1) / kChunk;
         a.dcols = dcols;
         a.cols = cols;
+        a.cols16 = cols16;
         a.gx = gx;
         a.goff = goff;
         a.gmask = gmask;
@@ -358,7 +454,32 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
             return e;
         n += nt > 0;
     }
-    if (want_cols) {
+    if (want_cols && L.tc) {
+        // 3. on the tensor cores, per split z of the batch sum: D[m][co] = sum over the
+        // split's batches b and l of cols16[b][g*Kg + m][l] * gout[b][g*cout_g + co][l],
+        // stored to wpart[z][g*cout_g + co][m]; then the slices added in split order
+        const int S = L.wsplits, rps = P.B / S;
+        if (P.B > 0) {
+            for (int gi = 0; gi < P.groups; ++gi) {
+                if ((e = launch_gemm_tc(P.dtype, cols16, (int64_t)P.B * P.C_in * P.K, P.L_out,
+                                        gi * Kg, rps * P.C_in * P.K, P.C_in * P.K, gout,
+                                        (int64_t)P.B * P.C_out, P.L_out, gi * P.cout_g,
+                                        rps * P.C_out, P.C_out, Kg, P.cout_g, P.L_out, rps, S,
+                                        wpart + (int64_t)gi * P.cout_g * Kg, 1, Kg,
+                                        (int64_t)P.C_out * Kg, s)) != cudaSuccess)
+                    return e;
+                ++n;
+            }
+        }
+        const int64_t nw = (int64_t)P.C_out * Kg;
+        if (P.B > 0)
+            sum_splits_kernel<T><<<grid_1d(nw), 256, 0, s>>>(wpart, static_cast<T *>(G.w), S, nw);
+        else if ((e = cudaMemsetAsync(G.w, 0, nw * sizeof(T), s)) != cudaSuccess)
+            return e;
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+        n += P.B > 0;
+    } else if (want_cols) {
         // 3. gW[g*cout_g + co][m] = sum_b sum_l gout[b][g*cout_g + co][l] * cols[b][g*Kg + m][l]
         // (zeros for an empty batch).  Split s of the batch sum covers batches
         // [s * rps, (s + 1) * rps) (blockIdx.z = s * groups + group) and writes its own
@@ -429,6 +550,10 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
 
 size_t backward_workspace(const Problem &P, const BackwardGrads &G) {
     return ws_layout(P, G).total;
+}
+
+bool backward_uses_tensor_cores(const Problem &P, const BackwardGrads &G) {
+    return tc_backward(P, G);
 }
 
 cudaError_t launch_backward(const Problem &P, const BackwardGrads &G, void *workspace,

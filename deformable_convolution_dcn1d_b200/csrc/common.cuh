@@ -72,11 +72,22 @@ bool tc_bf16_stalled_supported(const Problem &P);
 cudaError_t launch_tc_bf16_stalled(const Problem &P, uint64_t wait_ns, cudaStream_t stream);
 // Backward (backward.cu): the upstream gradient and the wanted gradients (each
 // output NULL when not wanted), all in the problem's dtype and its inputs' shapes.
+// The tensor-core GEMM of the backward pass (gemm_tc.cu): C[z][m*c_sm + n*c_sn] (fp32) =
+// sum over r < R and k < K of A[row_a(z, r) + m][k] * B[row_b(z, r) + n][k], A and B
+// 16-bit K-major row-major arrays with `*_ld` elements per row and `*_rows` rows.
+bool gemm_tc_supported(int dtype, const void *A, int64_t a_rows, int64_t a_ld, const void *B,
+                       int64_t b_rows, int64_t b_ld);
+cudaError_t launch_gemm_tc(int dtype, const void *A, int64_t a_rows, int64_t a_ld, int a_row0,
+                           int a_row_z, int a_row_r, const void *B, int64_t b_rows, int64_t b_ld,
+                           int b_row0, int b_row_z, int b_row_r, int M, int N, int K, int R,
+                           int nz, float *C, int64_t c_sm, int64_t c_sn, int64_t c_sz,
+                           cudaStream_t stream);
 struct BackwardGrads {
     const void *gout;                    // [B, C_out, L_out]
     void *x, *off, *mask, *w, *bias;     // outputs
 };
 size_t backward_workspace(const Problem &P, const BackwardGrads &G);
+bool backward_uses_tensor_cores(const Problem &P, const BackwardGrads &G);
 cudaError_t launch_backward(const Problem &P, const BackwardGrads &G, void *workspace,
                             cudaStream_t stream, int *launches);
 // PackedDeformConv1d's offset (and mask) predictor (trunk.cu): a depthwise convolution

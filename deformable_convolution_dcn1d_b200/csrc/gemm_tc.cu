@@ -1,0 +1,247 @@
+// A tensor-core GEMM for the backward pass's two contractions (16-bit operands, fp32
+// accumulation and output):
+//
+//   C[z][m * c_sm + n * c_sn] = sum_{r < R} sum_{k < K} A_zr[m][k] * B_zr[n][k]
+//
+// Both operands are K-major 16-bit row-major arrays read by TMA (128-byte swizzle):
+// A_zr's row m is row a_row0 + z * a_row_z + r * a_row_r + m of the A tensor map, B's
+// likewise; K runs along the rows (the tensor maps' column extent ends the reduction,
+// reading zeros past it).  One CTA per 128 x NT output tile and z: a TMA warp feeds a
+// ring of stages, one thread issues tcgen05.mma (M = 128, N = NT, K = 16, both operands
+// from shared memory) into a tensor-memory accumulator, four warps drain it (lanes =
+// consecutive m, so with c_sm = 1 each warp store covers 128 contiguous bytes).
+#include <string.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace dcn1d {
+
+namespace {
+
+constexpr int kGM = 128;                  // tile rows = TMEM lanes
+constexpr int kGBK = 64;                  // reduction elements per stage (128 bytes)
+constexpr int kGStages = 4;
+constexpr int kGTma = 0, kGMma = 1;       // warps 2..5 drain
+constexpr int kGThreads = 6 * 32;
+constexpr uint64_t kGWaitNs = 2000000000ull;
+
+struct GemmTcArgs {
+    int M, N, K, R, NT;
+    int tiles_m, tiles_n;
+    int a_row0, a_row_z, a_row_r;
+    int b_row0, b_row_z, b_row_r;
+    float *C;
+    int64_t c_sm, c_sn, c_sz;
+    uint32_t a_bytes, b_bytes;            // one stage's A and B tiles
+    unsigned int *status;
+};
+
+template <class E>
+struct GElem;
+template <>
+struct GElem<__nv_bfloat16> {
+    static __host__ __device__ constexpr uint32_t idesc(int M, int N) { return idesc_bf16_f32(M, N); }
+};
+template <>
+struct GElem<__half> {
+    static __host__ __device__ constexpr uint32_t idesc(int M, int N) { return idesc_f16_f32(M, N); }
+};
+
+template <class E>
+__global__ void __launch_bounds__(kGThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ GemmTcArgs G, const __grid_constant__ CUtensorMap amap,
+                   const __grid_constant__ CUtensorMap bmap) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int tile = blockIdx.x;
+    const int tn = tile % G.tiles_n;
+    const int tm = (tile / G.tiles_n) % G.tiles_m;
+    const int z = tile / (G.tiles_n * G.tiles_m);
+    const int m0 = tm * kGM, n0 = tn * G.NT;
+
+    const uint32_t sraw = smem_u32(smem_raw);
+    const uint32_t sbase = (sraw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - sraw);
+    const uint32_t a_s0 = sbase;
+    const uint32_t b_s0 = sbase + kGStages * G.a_bytes;
+    const uint32_t bar0 = b_s0 + kGStages * G.b_bytes;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (kGStages + s); };
+    const uint32_t dfull = bar0 + 8u * (2 * kGStages);
+    uint32_t *tmem_holder =
+        reinterpret_cast<uint32_t *>(smem + (bar0 - sbase) + 8 * (2 * kGStages + 2));
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGStages; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(dfull, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kGMma) {
+        tmem_alloc(smem_u32(tmem_holder), 256);
+        tc_fence_before();
+    }
+    if (warp == kGTma && lane == 0) {
+        tma_prefetch_desc(&amap);
+        tma_prefetch_desc(&bmap);
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const BoundedWait wait{abort_flag, kGWaitNs, G.status};
+    const int nkb = (G.K + kGBK - 1) / kGBK;
+    const int total = nkb * G.R;
+
+    if (warp == kGTma) {
+        if (lane == 0) {
+            int it = 0;
+            for (; it < total; ++it) {
+                const int r = it / nkb, kb = it - r * nkb;
+                const int s = it % kGStages;
+                const uint32_t ph = (uint32_t)(it / kGStages) & 1u;
+                if (!wait(empty(s), ph ^ 1u))
+                    break;
+                mbar_arrive_expect_tx(full(s), G.a_bytes + G.b_bytes);
+                tma_load_2d(a_s0 + s * G.a_bytes, &amap, kb * kGBK,
+                            G.a_row0 + z * G.a_row_z + r * G.a_row_r + m0, full(s));
+                tma_load_2d(b_s0 + s * G.b_bytes, &bmap, kb * kGBK,
+                            G.b_row0 + z * G.b_row_z + r * G.b_row_r + n0, full(s));
+            }
+            volatile int never = 0;
+            const BoundedWait drain{&never, kGWaitNs, G.status};
+            for (int j = (it > kGStages ? it - kGStages : 0); j < it; ++j)
+                drain(full(j % kGStages), (uint32_t)(j / kGStages) & 1u);
+        }
+    } else if (warp == kGMma) {
+        if (lane == 0) {
+            const uint32_t idesc = GElem<E>::idesc(kGM, G.NT);
+            for (int it = 0; it < total; ++it) {
+                const int s = it % kGStages;
+                if (!wait(full(s), (uint32_t)(it / kGStages) & 1u))
+                    break;
+                tc_fence_after();
+                const uint32_t as = a_s0 + s * G.a_bytes, bs = b_s0 + s * G.b_bytes;
+#pragma unroll
+                for (int kk = 0; kk < kGBK / 16; ++kk)
+                    mma_f16_ss(tmem, sw128_kmajor_desc(as + 32u * kk),
+                               sw128_kmajor_desc(bs + 32u * kk), idesc,
+                               (it > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(empty(s));
+            }
+            mma_commit(dfull);       // also the drain point: every MMA issued is complete
+            volatile int never = 0;
+            const BoundedWait drain{&never, kGWaitNs, G.status};
+            drain(dfull, 0);
+        }
+    } else {
+        // drain: warp w reads TMEM lanes 32 (w % 4) ..
+        const int q = warp % 4;
+        const int m = m0 + 32 * q + lane;
+        if (__all_sync(0xffffffffu, wait(dfull, 0))) {
+            tc_fence_after();
+            float *Cz = G.C + (int64_t)z * G.c_sz;
+            for (int c = 0; c < G.NT; c += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c, v);
+                tmem_wait_ld();
+                if (m < G.M) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int n = n0 + c + i;
+                        if (n < G.N)
+                            Cz[(int64_t)m * G.c_sm + (int64_t)n * G.c_sn] = __uint_as_float(v[i]);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kGMma) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace
+
+// The A and B operands as 16-bit row-major [rows][cols] arrays (row strides in
+// elements, multiples of 8), the reduction over their first `K` columns.
+bool gemm_tc_supported(int dtype, const void *A, int64_t a_rows, int64_t a_ld, const void *B,
+                       int64_t b_rows, int64_t b_ld) {
+    if (dtype != DCN1D_BF16 && dtype != DCN1D_F16)
+        return false;
+    if ((reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(B) & 15))
+        return false;
+    if (a_ld % 8 || b_ld % 8 || a_rows < 1 || b_rows < 1 || a_rows >= (1LL << 31) ||
+        b_rows >= (1LL << 31))
+        return false;
+    return true;
+}
+
+cudaError_t launch_gemm_tc(int dtype, const void *A, int64_t a_rows, int64_t a_ld, int a_row0,
+                           int a_row_z, int a_row_r, const void *B, int64_t b_rows, int64_t b_ld,
+                           int b_row0, int b_row_z, int b_row_r, int M, int N, int K, int R,
+                           int nz, float *C, int64_t c_sm, int64_t c_sn, int64_t c_sz,
+                           cudaStream_t stream) {
+    GemmTcArgs G;
+    memset(&G, 0, sizeof(G));
+    G.M = M;
+    G.N = N;
+    G.K = K;
+    G.R = R;
+    G.NT = N <= 128 ? (N <= 64 ? 64 : 128) : 256;
+    G.tiles_m = (M + kGM - 1) / kGM;
+    G.tiles_n = (N + G.NT - 1) / G.NT;
+    G.a_row0 = a_row0;
+    G.a_row_z = a_row_z;
+    G.a_row_r = a_row_r;
+    G.b_row0 = b_row0;
+    G.b_row_z = b_row_z;
+    G.b_row_r = b_row_r;
+    G.C = C;
+    G.c_sm = c_sm;
+    G.c_sn = c_sn;
+    G.c_sz = c_sz;
+    G.a_bytes = kGM * kGBK * 2;
+    G.b_bytes = (uint32_t)G.NT * kGBK * 2;
+    G.status = device_status_ptr();
+    if (!G.status)
+        return cudaErrorInvalidDevice;
+    const int64_t blocks = (int64_t)G.tiles_m * G.tiles_n * nz;
+    if (blocks < 1 || blocks >= (1LL << 31))
+        return cudaErrorInvalidValue;
+    const CUtensorMapDataType ty = dtype == DCN1D_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                      : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    alignas(64) CUtensorMap amap, bmap;
+    // the maps' column extent is the reduction length: TMA reads zeros past it
+    if (!encode_2d_ld(&amap, ty, A, (uint64_t)K, (uint64_t)a_rows, (uint64_t)a_ld, 2, kGBK, kGM,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d_ld(&bmap, ty, B, (uint64_t)K, (uint64_t)b_rows, (uint64_t)b_ld, 2, kGBK,
+                      (uint32_t)G.NT, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const size_t smem = (size_t)kGStages * (G.a_bytes + G.b_bytes) + 8 * (2 * kGStages + 2) + 16 +
+                        1024;
+    const void *kern = dtype == DCN1D_F16 ? reinterpret_cast<const void *>(gemm_tc_kernel<__half>)
+                                          : reinterpret_cast<const void *>(
+                                                gemm_tc_kernel<__nv_bfloat16>);
+    cudaError_t e = ensure_smem(kern, (int)(smem < 116 * 1024 ? 116 * 1024 : smem));
+    if (e != cudaSuccess)
+        return e;
+    const size_t smem_launch = smem < 116 * 1024 ? 116 * 1024 : smem;   // one CTA per SM
+    if (dtype == DCN1D_F16)
+        gemm_tc_kernel<__half><<<(unsigned)blocks, kGThreads, smem_launch, stream>>>(G, amap, bmap);
+    else
+        gemm_tc_kernel<__nv_bfloat16><<<(unsigned)blocks, kGThreads, smem_launch, stream>>>(G, amap,
+                                                                                            bmap);
+    return cudaGetLastError();
+}
+
+}  // namespace dcn1d

@@ -80,31 +80,19 @@ cudaError_t ensure_smem(const void *kernel, int bytes) {
     return cudaSuccess;
 }
 
-int resident_clusters(const void *kernel, const cudaLaunchConfig_t *cfg) {
-    struct Entry {
-        const void *fn;
-        int dev;
-        size_t smem;
-        int n;
-    };
-    static std::mutex mu;
-    static Entry table[64];
-    static int n = 0;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess)
-        return 0;
-    std::lock_guard<std::mutex> lock(mu);
-    for (int i = 0; i < n; ++i)
-        if (table[i].fn == kernel && table[i].dev == dev && table[i].smem == cfg->dynamicSmemBytes)
-            return table[i].n;
-    cudaLaunchConfig_t q = *cfg;
-    q.gridDim = dim3(2 * 1024);   // any grid: the query counts resident clusters
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &q) != cudaSuccess)
-        return 0;
-    if (n < 64)
-        table[n++] = Entry{kernel, dev, cfg->dynamicSmemBytes, clusters};
-    return clusters;
+bool encode_2d_ld(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t cols,
+                  uint64_t rows, uint64_t ld, uint32_t elem_bytes, uint32_t box_cols,
+                  uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * elem_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t cols,

@@ -4,7 +4,9 @@
 //
 // Per tile of 128 output positions of one batch element (TMEM lane = position):
 //   1. the x window of every channel (the tile's receptive fields, plus a margin when
-//      unconstrained) is staged in shared memory by TMA, double-buffered across tiles;
+//      unconstrained) is staged in shared memory by TMA, one 64-channel block per stage
+//      of a ring one block deeper than a tile needs (a block's stage is refilled for the
+//      next tile as soon as the chunks reading it are drained);
 //   2. sixteen producer warps form the trunk's depthwise output
 //        t[c, l] = dw_b[c] + sum_k dw_w[c, k] * x[c, l*s - p + k*d]
 //      in fp32 from that window, round it once to the input type and write it straight
@@ -56,7 +58,8 @@ struct FusedArgs {
     int boxw, margin;        // x window width (positions) and its margin per side
     int wstages;
     uint32_t colD1, colA;    // tensor-memory columns: D buffers at 0 and colD1, A at colA
-    uint32_t w_stage_bytes, x_buf_bytes;
+    int xstages;             // x ring depth (>= nkb + 1)
+    uint32_t w_stage_bytes, x_stage_bytes;
     uint32_t off_x, off_w, off_par, off_bar;   // shared-memory layout
     unsigned int *status;
 };
@@ -168,14 +171,16 @@ __global__ void __launch_bounds__(kFThreads, 1)
     const int SW = A.wstages;
     auto w_full = [&](int s) { return bar0 + 8u * s; };
     auto w_empty = [&](int s) { return bar0 + 8u * (SW + s); };
-    auto x_full = [&](int b) { return bar0 + 8u * (2 * SW + b); };
-    auto x_empty = [&](int b) { return bar0 + 8u * (2 * SW + 2 + b); };
-    const uint32_t a_full = bar0 + 8u * (2 * SW + 4);
+    const int SX = A.xstages;
+    auto x_full = [&](int s) { return bar0 + 8u * (2 * SW + s); };
+    auto x_empty = [&](int s) { return bar0 + 8u * (2 * SW + SX + s); };
+    const uint32_t a_full = bar0 + 8u * (2 * SW + 2 * SX);
     const uint32_t a_empty = a_full + 8u;
     const uint32_t d_full0 = a_full + 16u;    // + 8 d
     const uint32_t d_empty0 = a_full + 32u;   // + 8 d
     const uint32_t drain_bar = a_full + 48u;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + A.off_bar + 8 * (2 * SW + 4) + 56);
+    uint32_t *tmem_holder =
+        reinterpret_cast<uint32_t *>(smem + A.off_bar + 8 * (2 * SW + 2 * SX) + 56);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     {   // parameters, widened to fp32 once per CTA
@@ -202,9 +207,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
             mbar_init(w_full(s), 1);
             mbar_init(w_empty(s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(x_full(b), 1);
-            mbar_init(x_empty(b), kFProd);    // every drain warp reads the whole window
+        for (int s = 0; s < SX; ++s) {
+            mbar_init(x_full(s), 1);
+            mbar_init(x_empty(s), kFProd);    // every producer warp reads every block
         }
         mbar_init(a_full, kFProd);
         mbar_init(a_empty, 1);
@@ -261,25 +266,26 @@ __global__ void __launch_bounds__(kFThreads, 1)
     } else if (warp == kFXTma) {
         // ------------------------------------------------------------ x windows
         if (lane == 0) {
-            uint32_t tc = 0;
-            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
                 const int b = t / A.tiles_l;
                 const int lbase = (t % A.tiles_l) * kFRows;
                 const int wx0 = floor8(lbase * T.stride - T.padding - A.margin);
-                const int buf = tc & 1;
-                if (!wait(x_empty(buf), ((tc >> 1) & 1u) ^ 1u))
-                    goto xtma_done;
-                mbar_arrive_expect_tx(x_full(buf), A.x_buf_bytes);
-                const uint32_t dst = x_s0 + buf * A.x_buf_bytes;
-                for (int kb = 0; kb < A.nkb; ++kb)
-                    tma_load_2d(dst + (uint32_t)(kb * kFBK * A.boxw * 2), &map_x, wx0,
-                                b * C + kb * kFBK, x_full(buf));
+                for (int kb = 0; kb < A.nkb; ++kb, ++it) {
+                    const int s = it % SX;
+                    if (!wait(x_empty(s), ((it / SX) & 1u) ^ 1u))
+                        goto xtma_done;
+                    mbar_arrive_expect_tx(x_full(s), A.x_stage_bytes);
+                    tma_load_2d(x_s0 + s * A.x_stage_bytes, &map_x, wx0, b * C + kb * kFBK,
+                                x_full(s));
+                }
             }
         xtma_done:
             volatile int never = 0;
             const BoundedWait drain{&never, kFWaitNs, A.status};
-            for (uint32_t j = (tc > 2 ? tc - 2 : 0); j < tc; ++j)
-                drain(x_full(j & 1), (j >> 1) & 1u);
+            const uint32_t S = (uint32_t)SX;
+            for (uint32_t j = (it > S ? it - S : 0); j < it; ++j)
+                drain(x_full(j % S), (j / S) & 1u);
         }
     } else if (warp == kFMma) {
         // ------------------------------------------------------------ MMA issuer
@@ -334,18 +340,22 @@ __global__ void __launch_bounds__(kFThreads, 1)
             const int l = lbase + r;
             const bool valid = l < T.L_out;
             const int wx0 = floor8(lbase * T.stride - T.padding - A.margin);
-            const int buf = tc & 1;
-            const uint32_t xbuf = x_s0 + buf * A.x_buf_bytes;
+            const uint32_t it0 = tc * (uint32_t)A.nkb;       // ring index of block 0
+            // stage address of channel block kb's window
+            auto xblock = [&](int kb) {
+                return x_s0 + ((it0 + (uint32_t)kb) % (uint32_t)SX) * A.x_stage_bytes;
+            };
             const uint32_t rowb = (uint32_t)A.boxw * 2u;     // bytes per channel row
             const int start = l * T.stride - T.padding;      // first tap of row l
             const uint32_t rel0 = (uint32_t)(start - wx0);   // its window index (>= margin)
             if (!__all_sync(0xffffffffu, wait(a_empty, (tc & 1u) ^ 1u)))
                 goto prod_done;
-            if (!__all_sync(0xffffffffu, wait(x_full(buf), (tc >> 1) & 1u)))
-                goto prod_done;
-            tc_fence_after();
             // ---- trunk: this warp's 16 channels of every k-block into tensor memory
             for (int kb = 0; kb < A.nkb; ++kb) {
+                const uint32_t itx = it0 + (uint32_t)kb;
+                if (!__all_sync(0xffffffffu, wait(x_full(itx % SX), (itx / SX) & 1u)))
+                    goto prod_done;
+                const uint32_t xbuf = xblock(kb) - (uint32_t)(kb * kFBK) * rowb;
                 uint32_t pk[8];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -381,6 +391,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
             const float startf = (float)start;
             for (int c = 0; c < A.chunks; ++c, ++cg) {
                 const uint32_t d = cg & 1u;
+                const int kbc = (c * A.cpc) / kFBK;     // the channel block this chunk reads
+                const uint32_t xbuf = xblock(kbc) - (uint32_t)(kbc * kFBK) * rowb;
                 const uint32_t dcol = d ? A.colD1 : 0u;
                 if (!__all_sync(0xffffffffu, wait(d_full0 + 8u * d, (cg >> 1) & 1u)))
                     goto prod_done;
@@ -401,49 +413,85 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 if (lane == 0)
                     mbar_arrive(d_empty0 + 8u * d);   // the buffer is free for chunk c + 2
                 const int ch0 = c * A.cpc + h * kFCw;
+                // two channels at a time: packed f32x2 arithmetic, the same roundings per
+                // element as the scalar forms (and as the depthwise kernel's)
 #pragma unroll
-                for (int i = 0; i < kFCw; ++i) {
-                    const int ch = ch0 + i;
-                    const uint32_t xr = xbuf + (uint32_t)ch * rowb;
-                    float acc = p.fb[ch];
+                for (int ip = 0; ip < kFCw / 2; ++ip) {
+                    const int cA = ch0 + 2 * ip, cB = cA + 1;
+                    const uint32_t xrA = xbuf + (uint32_t)cA * rowb, xrB = xrA + rowb;
+                    float2 acc = make_float2(p.fb[cA], p.fb[cB]);
 #pragma unroll
                     for (int k = 0; k < K; ++k) {
-                        const int e = i * K + k;      // a compile-time register index
-                        const int jh = ch * K + k;    // head column (offset group ch, tap k)
-                        const float off =
-                            FElem<E>::round(__uint_as_float(vo[e]) + p.offb[jh]);
-                        float m = 1.0f;
-                        if (MASKHEAD)
-                            m = FElem<E>::round(
-                                fsigmoid(__uint_as_float(vm[MASKHEAD ? e : 0]) + p.maskb[jh]));
-                        float pos = __fadd_rn(__fadd_rn(startf, (float)(k * T.dilation)), off);
-                        if (!UNC)
-                            pos = fminf(fmaxf(pos, startf), __fadd_rn(startf, spanf));
-                        Tap tp = tap_floor_fast(pos);
-                        const uint32_t rel = (uint32_t)(tp.i0 - wx0);
-                        float x0, x1;
-                        if (rel < (uint32_t)(A.boxw - 1)) {
-                            x0 = FElem<E>::widen(lds_u16(xr + rel * 2u));
-                            x1 = FElem<E>::widen(lds_u16(xr + rel * 2u + 2u));
-                        } else {   // outside the staged window: exact floor, global loads
-                            tp = tap_floor_exact(pos);
-                            const E *xg = xrow_g + (int64_t)ch * T.L_in;
-                            x0 = (tp.i0 >= 0 && tp.i0 < T.L_in) ? ld_f32(xg + tp.i0) : 0.0f;
-                            x1 = (tp.i0 >= -1 && tp.i0 < T.L_in - 1) ? ld_f32(xg + tp.i0 + 1)
-                                                                     : 0.0f;
+                        const int eA = (2 * ip) * K + k, eB = eA + K;   // register indices
+                        const float2 z = __fadd2_rn(
+                            make_float2(__uint_as_float(vo[eA]), __uint_as_float(vo[eB])),
+                            make_float2(p.offb[cA * K + k], p.offb[cB * K + k]));
+                        const float2 off = make_float2(FElem<E>::round(z.x), FElem<E>::round(z.y));
+                        float2 m = make_float2(1.0f, 1.0f);
+                        if (MASKHEAD) {
+                            const float2 zm = __fadd2_rn(
+                                make_float2(__uint_as_float(vm[MASKHEAD ? eA : 0]),
+                                            __uint_as_float(vm[MASKHEAD ? eB : 0])),
+                                make_float2(p.maskb[cA * K + k], p.maskb[cB * K + k]));
+                            m = make_float2(FElem<E>::round(fsigmoid(zm.x)),
+                                            FElem<E>::round(fsigmoid(zm.y)));
                         }
-                        float v = __fmaf_rn(tp.f, __fsub_rn(x1, x0), x0);
+                        const float bk = __fadd_rn(startf, (float)(k * T.dilation));
+                        float2 pos = __fadd2_rn(make_float2(bk, bk), off);
+                        if (!UNC) {
+                            const float hi = __fadd_rn(startf, spanf);
+                            pos.x = fminf(fmaxf(pos.x, startf), hi);
+                            pos.y = fminf(fmaxf(pos.y, startf), hi);
+                        }
+                        const float2 tt = __fadd2_rd(pos, make_float2(kFloorMagic, kFloorMagic));
+                        float2 f = __ffma2_rn(
+                            __fadd2_rn(tt, make_float2(-kFloorMagic, -kFloorMagic)),
+                            make_float2(-1.0f, -1.0f), pos);
+                        const uint32_t wbits = kFloorMagicBits + (uint32_t)wx0;
+                        const uint32_t relA = __float_as_uint(tt.x) - wbits;   // i0 - wx0
+                        const uint32_t relB = __float_as_uint(tt.y) - wbits;
+                        const uint32_t lim = (uint32_t)(A.boxw - 1);
+                        float2 x0, x1;
+                        if (relA < lim) {
+                            x0.x = FElem<E>::widen(lds_u16(xrA + relA * 2u));
+                            x1.x = FElem<E>::widen(lds_u16(xrA + relA * 2u + 2u));
+                        } else {   // outside the staged window: exact floor, global loads
+                            const Tap e = tap_floor_exact(pos.x);
+                            const E *xg = xrow_g + (int64_t)cA * T.L_in;
+                            x0.x = (e.i0 >= 0 && e.i0 < T.L_in) ? ld_f32(xg + e.i0) : 0.0f;
+                            x1.x = (e.i0 >= -1 && e.i0 < T.L_in - 1) ? ld_f32(xg + e.i0 + 1)
+                                                                     : 0.0f;
+                            f.x = e.f;
+                        }
+                        if (relB < lim) {
+                            x0.y = FElem<E>::widen(lds_u16(xrB + relB * 2u));
+                            x1.y = FElem<E>::widen(lds_u16(xrB + relB * 2u + 2u));
+                        } else {
+                            const Tap e = tap_floor_exact(pos.y);
+                            const E *xg = xrow_g + (int64_t)cB * T.L_in;
+                            x0.y = (e.i0 >= 0 && e.i0 < T.L_in) ? ld_f32(xg + e.i0) : 0.0f;
+                            x1.y = (e.i0 >= -1 && e.i0 < T.L_in - 1) ? ld_f32(xg + e.i0 + 1)
+                                                                     : 0.0f;
+                            f.y = e.f;
+                        }
+                        float2 v = __ffma2_rn(f, __ffma2_rn(x0, make_float2(-1.0f, -1.0f), x1),
+                                              x0);
                         if (MASKHEAD)
-                            v = __fmul_rn(v, m);
-                        acc = __fmaf_rn(p.fw[ch * K + k], v, acc);
+                            v = __fmul2_rn(v, m);
+                        acc = __ffma2_rn(make_float2(p.fw[cA * K + k], p.fw[cB * K + k]), v, acc);
                     }
-                    if (valid)
-                        orow[(int64_t)ch * T.L_out] = from_f32<E>(acc);
+                    if (valid) {
+                        orow[(int64_t)cA * T.L_out] = from_f32<E>(acc.x);
+                        orow[(int64_t)cB * T.L_out] = from_f32<E>(acc.y);
+                    }
+                }
+                // the chunk that finishes a channel block releases its stage
+                if ((((c + 1) * A.cpc) % kFBK) == 0) {
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(x_empty((it0 + (uint32_t)kbc) % (uint32_t)SX));
                 }
             }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(x_empty(buf));    // this tile's x window is no longer read
         }
     prod_done:;
     }
@@ -497,16 +545,17 @@ bool make_fused_plan(const TrunkProblem &T, const Problem &P, FusedPlan *out) {
     A.boxw = (int)((need + 7) / 8 * 8);
     if (A.boxw > kFBoxMax)
         return false;
-    A.x_buf_bytes = (uint32_t)C * (uint32_t)A.boxw * 2u;
+    A.x_stage_bytes = (uint32_t)kFBK * (uint32_t)A.boxw * 2u;   // multiple of 1024
+    A.xstages = A.nkb + 1;
     A.w_stage_bytes = (uint32_t)A.N * 128u;
     const size_t par_bytes = ((size_t)(4 * C * K + 2 * C) * 4 + 15) / 16 * 16;
     for (int sw = 4; sw >= 2; --sw) {
         A.wstages = sw;
         A.off_x = 0;
-        A.off_w = (2 * A.x_buf_bytes + 1023u) / 1024u * 1024u;
+        A.off_w = (uint32_t)A.xstages * A.x_stage_bytes;
         A.off_par = A.off_w + (uint32_t)sw * A.w_stage_bytes;
         A.off_bar = A.off_par + (uint32_t)par_bytes;
-        size_t smem = (size_t)A.off_bar + 8 * (2 * sw + 4) + 64 + 1024;
+        size_t smem = (size_t)A.off_bar + 8 * (2 * sw + 2 * A.xstages) + 64 + 1024;
         if (smem > 227 * 1024)
             continue;
         if (smem < 116 * 1024)

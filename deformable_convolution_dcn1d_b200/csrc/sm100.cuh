@@ -72,52 +72,6 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
     return ok != 0;
 }
 
-// try_wait at cluster scope: the phase may have been completed by arrivals from
-// the peer CTA of a CTA pair, whose prior writes (tensor memory, shared memory)
-// this thread must then observe.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity,
-                                                      uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
-
-// ---------------------------------------------------------------- clusters (CTA pairs)
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Address, in the cluster's shared window, of the variable at shared::cta address
-// `addr` in the CTA of rank `rank`.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-
-// Arrival on an mbarrier given by its cluster-window address (possibly in the peer
-// CTA), releasing this thread's prior writes at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
-                 : "memory");
-}
-
-// Every thread of both CTAs of the cluster: all prior writes are visible to the
-// other CTA afterwards.  No timeout: only reached on paths whose waits are bounded.
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 // A wait on an mbarrier phase that gives up after `limit_ns` of wall time or as
 // soon as another role of the CTA has given up (shared abort flag).  On giving
 // up it records kStatusTimeout in the device status word and raises the abort
@@ -128,20 +82,13 @@ struct BoundedWait {
     volatile int *abort;   // shared-memory flag of this CTA
     uint64_t limit_ns;
     unsigned int *status;  // device status word
-    bool cluster = false;  // acquire at cluster scope (barriers the peer CTA arrives on)
-
-    __device__ __forceinline__ bool try_once(uint32_t bar, uint32_t parity, uint32_t hint) const {
-        return cluster ? mbar_try_wait_cluster(bar, parity, hint)
-                       : (hint ? mbar_try_wait_sleep(bar, parity, hint)
-                               : mbar_try_wait(bar, parity));
-    }
 
     __device__ __forceinline__ bool operator()(uint32_t bar, uint32_t parity) const {
-        if (try_once(bar, parity, 0u))
+        if (mbar_try_wait(bar, parity))
             return true;
         const uint64_t t0 = globaltimer_ns();
         for (;;) {
-            if (try_once(bar, parity, 20000u))
+            if (mbar_try_wait_sleep(bar, parity, 20000u))
                 return true;
             if (*abort)
                 return false;
@@ -165,18 +112,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-// The load of a CTA pair's half of an MMA operand (tcgen05 cta_group::2): the tile
-// lands in this CTA's shared memory at `dst`; the completed bytes are counted on
-// the mbarrier at cluster-window address `cluster_bar` (the pair's first CTA).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map,
-                                                 int32_t c0, int32_t c1, uint32_t cluster_bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(cluster_bar)
-        : "memory");
-}
-
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -190,21 +125,6 @@ __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
                  "r"(ncols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-// CTA-pair forms (tcgen05 cta_group::2): one warp with the same warp index in
-// each CTA of the pair executes them together; the allocation covers the same
-// columns in both CTAs' tensor memory.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-                 "r"(ncols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
@@ -227,31 +147,6 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// The CTA pair's MMA (issued by the first CTA): M = 256 rows, 128 in each CTA's
-// tensor memory (A and D at the same addresses in both); B's N rows are split,
-// the first N/2 in the first CTA's shared memory, the rest at the same address
-// in the second's.
-__device__ __forceinline__ void mma_bf16_ts_pair(uint32_t d_tmem, uint32_t a_tmem,
-                                                 uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Completion of the pair's MMAs issued so far arrives on the mbarrier at this
-// shared::cta address in every CTA of `cta_mask`.
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t cta_mask) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], %1;" ::"r"(bar),
-        "h"(cta_mask)
         : "memory");
 }
 
@@ -381,13 +276,14 @@ EncodeTiledFn encode_fn();
 void *current_context();
 // Number of SMs of the current device (0 on failure).
 int sm_count();
-// Clusters of this launch configuration (cluster dimension attribute included) that
-// the current device holds at once; cached per kernel, device and shared-memory size
-// (0 on failure).
-int resident_clusters(const void *kernel, const cudaLaunchConfig_t *cfg);
 // Raises a kernel's dynamic shared-memory limit on the current device, once per size
 // increase (the runtime call costs microseconds; every launch would repeat it).
 cudaError_t ensure_smem(const void *kernel, int bytes);
+// A 2D tiled tensor map over the first `cols` columns of a row-major array whose rows are
+// `ld` elements apart (reads past `cols` return zeros).
+bool encode_2d_ld(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t cols,
+                  uint64_t rows, uint64_t ld, uint32_t elem_bytes, uint32_t box_cols,
+                  uint32_t box_rows, CUtensorMapSwizzle swizzle);
 // A 2D tiled tensor map over a row-major [rows][cols] array (elements of `elem_bytes`).
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t cols,
                uint64_t rows, uint32_t elem_bytes, uint32_t box_cols, uint32_t box_rows,

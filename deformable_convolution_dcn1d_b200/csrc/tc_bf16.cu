@@ -1,6 +1,6 @@
 // Fused deformable-im2col + tcgen05 tensor-core contraction, 16-bit inputs (bf16,
 // or fp16: the same kernel with the element type a template parameter) and fp32
-// accumulation (conv groups with C_out/groups <= 256).
+// accumulation.
 //
 // Per conv group g the forward is a GEMM over the reduction index kk = (ci, k)
 // of the group (k fastest, the weight's own order):
@@ -9,8 +9,9 @@
 // ("conv1d" page, "Description", with the sampling of the deformable-
 // convolution article, "Step 2").  The cols never exist in global memory:
 //
-//  * a TILE is 128 consecutive output positions of one (g, b) and all
-//    Cg_out output channels; the CTA is persistent over tiles;
+//  * a TILE is 128 consecutive output positions of one (g, b) and one block of
+//    N output channels (all Cg_out of them when Cg_out <= 256); the CTA is
+//    persistent over tiles;
 //  * TMA warp: per 64-wide k-block, one TMA load of the weight tile
 //    W[co 0..N-1][kk block] (128-byte swizzle, K-major: the MMA's B operand)
 //    and one or two TMA loads of the x window [channels of the block][up to
@@ -22,7 +23,7 @@
 //    once and each warp computes 32 col values per k-block from the staged
 //    window in bf16x2 arithmetic, written straight into TENSOR MEMORY with
 //    tcgen05.st (the MMA's A operand) -- no shared-memory round trip;
-//  * MMA warp: one thread issues 4 tcgen05.mma (M=128, N=Cg_out, K=16) per
+//  * MMA warp: one thread issues 4 tcgen05.mma (M=128, N, K=16) per
 //    k-block, A from tensor memory, B from shared memory, D (fp32) in tensor
 //    memory, and commits completion to the stage's "empty" barrier;
 //  * epilogue, by the same 16 warps (each drains a quarter of its lane
@@ -32,7 +33,6 @@
 //    staged the first kStages k-blocks of their next tile, so the MMA resumes
 //    on ready stages as soon as the accumulator is free.
 // Stages are chained by mbarriers; every wait is bounded (sm100.cuh).
-#include <stdlib.h>
 #include <string.h>
 
 #include <utility>
@@ -45,9 +45,7 @@ namespace dcn1d {
 
 namespace {
 
-constexpr int kStages = 4;         // ring depth of the one-SM kernel (even: see kb_at)
-constexpr int kStagesPair = 6;     // ring depth of the SM-pair kernel (half the weight bytes)
-__host__ __device__ constexpr int stages_of(int cg) { return cg == 2 ? kStagesPair : kStages; }
+constexpr int kStages = 4;
 constexpr int kRows = 128;         // output positions per tile = TMEM lanes
 constexpr int kBK = 64;            // reduction elements per k-block
 constexpr int kSeg = 32;           // reduction elements per producer warp and k-block
@@ -66,11 +64,12 @@ constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s
 
 struct TcArgs {
     Problem P;
-    int N;             // MMA N = Cg_out (multiple of 32, <= 256)
+    int N;             // MMA N: output channels per block (multiple of 32, <= 256)
+    int n_cob;         // channel blocks per conv group (Cg_out / N)
     int num_kb;        // k-blocks per tile
     int half_kb;       // > 0: producer groups take contiguous halves [0, half_kb) and
                        // [half_kb, num_kb); 0: they take the even and the odd k-blocks
-    int tiles_l;       // tiles per (g, b)
+    int tiles_l;       // tiles per (g, channel block, b)
     int num_tiles;
     int nch;           // x rows per stage
     int nbox;          // x boxes per stage (1 or 2)
@@ -92,18 +91,21 @@ __device__ __forceinline__ int kb_at(const TcArgs &A, int i) {
 
 struct Tile {
     int g, b, lbase, wx0;
+    int co0;           // first output channel of the tile's block
 };
 
-// Tile t of the CTA of rank `rank` in its pair: tiles are 128 * CG positions long,
-// and each CTA of a pair owns 128 of them.
-template <int CG>
-__device__ __forceinline__ Tile decode_tile(const TcArgs &A, int t, uint32_t rank) {
+__device__ __forceinline__ Tile decode_tile(const TcArgs &A, int t) {
     Tile r;
-    const int lt = t % A.tiles_l;
-    const int gb = t / A.tiles_l;
+    // channel blocks of one (g, b, positions) are consecutive tiles: they run at the
+    // same time on neighbouring CTAs and share the x window through L2
+    const int cob = t % A.n_cob;
+    const int t2 = t / A.n_cob;
+    const int lt = t2 % A.tiles_l;
+    const int gb = t2 / A.tiles_l;
     r.b = gb % A.P.B;
     r.g = gb / A.P.B;
-    r.lbase = lt * kRows * CG + kRows * (int)rank;
+    r.co0 = r.g * A.P.cout_g + cob * A.N;
+    r.lbase = lt * kRows;
     int w = r.lbase * A.P.stride - A.P.padding - A.margin;
     r.wx0 = (w >= 0) ? (w / 8) * 8 : -(((-w) + 7) / 8) * 8;
     return r;
@@ -134,8 +136,10 @@ struct Elem<__nv_bfloat16> {
         E2 h = __floats2bfloat162_rn(a, b);
         return *reinterpret_cast<uint32_t *>(&h);
     }
-    // a 16-bit pattern zero-extended in a register, as a float
-    static __device__ __forceinline__ float widen(uint32_t u) { return __uint_as_float(u << 16); }
+    static __device__ __forceinline__ float lo(uint32_t u) { return __uint_as_float(u << 16); }
+    static __device__ __forceinline__ float hi(uint32_t u) {
+        return __uint_as_float(u & 0xFFFF0000u);
+    }
 };
 
 template <>
@@ -149,17 +153,31 @@ struct Elem<__half> {
         E2 h = __floats2half2_rn(a, b);
         return *reinterpret_cast<uint32_t *>(&h);
     }
-    static __device__ __forceinline__ float widen(uint32_t u) {
-        return __half2float(__ushort_as_half((unsigned short)u));
+    static __device__ __forceinline__ float lo(uint32_t u) {
+        return __half2float(__ushort_as_half((unsigned short)(u & 0xFFFFu)));
+    }
+    static __device__ __forceinline__ float hi(uint32_t u) {
+        return __half2float(__ushort_as_half((unsigned short)(u >> 16)));
     }
 };
 
-// Per-row tap state of one offset group (fp32 fractions and mask values).
+template <class E>
+__device__ __forceinline__ typename Elem<E>::E2 as_e2(uint32_t u) {
+    return *reinterpret_cast<typename Elem<E>::E2 *>(&u);
+}
+template <class E>
+__device__ __forceinline__ uint32_t as_u32(typename Elem<E>::E2 h) {
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Per-row tap state of one offset group.  Elements come in pairs (kk, kk+1),
+// i.e. taps (k, (k+1) % K), so fractions and mask values are kept pre-packed
+// as 16-bit pairs indexed by the first tap of the pair.
 template <int K>
 struct Taps {
     uint32_t addr[K];    // byte offset of the tap's neighbour pair in a stage row
-    float f[K];          // fraction of the position
-    float m[K];          // mask value (1 without a mask)
+    uint32_t fpair[K];   // E x2 (f_k, f_{(k+1)%K})
+    uint32_t mpair[K];   // E x2 (m_k, m_{(k+1)%K})
     float pos[K];        // position, for taps outside the window (slow path)
     uint32_t slow;       // bit k: tap k outside the staged window
 };
@@ -172,13 +190,15 @@ __device__ __forceinline__ float slow_element(const Taps<K> &tp, int kidx, int h
     const float x0 = (e.i0 >= 0 && e.i0 < L_in) ? ld_f32(row + e.i0) : 0.0f;
     const float x1 = (e.i0 >= -1 && e.i0 < L_in - 1) ? ld_f32(row + e.i0 + 1) : 0.0f;
     const float r = __fmaf_rn(e.f, __fsub_rn(x1, x0), x0);
-    return MASK ? __fmul_rn(r, tp.m[kidx]) : r;
+    if (!MASK)
+        return r;
+    const uint32_t mp = tp.mpair[(kidx + K - hi) % K];
+    return __fmul_rn(r, hi ? Elem<E>::hi(mp) : Elem<E>::lo(mp));
 }
 
 // Col values 2I and 2I+1 of a segment whose first element has phase K0 = kk0 % K:
 // taps (k0, k1) of channel rows (c0, c1) relative to the segment's first channel.
-// The lerp x0 + f (x1 - x0) and the mask run in fp32 on the two elements at once
-// (packed f32x2 instructions); the pair is rounded once, to the 16-bit operand.
+// The lerp x0 + f (x1 - x0) runs on the two elements in bf16x2 arithmetic.
 template <class E, int K, int K0, bool MASK, bool SLOW, int I>
 __device__ __forceinline__ void produce_pair(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
                                              const uint32_t (&base)[K], const E *xg,
@@ -186,17 +206,17 @@ __device__ __forceinline__ void produce_pair(uint32_t (&out)[kSeg / 2], const Ta
     constexpr int k0 = (K0 + 2 * I) % K, c0 = (K0 + 2 * I) / K;
     constexpr int k1 = (K0 + 2 * I + 1) % K, c1 = (K0 + 2 * I + 1) / K;
     constexpr uint32_t o0 = c0 * kRowBytes, o1 = c1 * kRowBytes;
-    const float2 x0 = make_float2(Elem<E>::widen(lds_u16<o0>(base[k0])),
-                                  Elem<E>::widen(lds_u16<o1>(base[k1])));
-    const float2 x1 = make_float2(Elem<E>::widen(lds_u16<o0 + 2>(base[k0])),
-                                  Elem<E>::widen(lds_u16<o1 + 2>(base[k1])));
-    float2 v = __ffma2_rn(make_float2(tp.f[k0], tp.f[k1]),
-                          __ffma2_rn(x0, make_float2(-1.0f, -1.0f), x1), x0);
+    const uint32_t x0 =
+        __byte_perm(lds_u16<o0>(base[k0]), lds_u16<o1>(base[k1]), 0x5410);
+    const uint32_t x1 =
+        __byte_perm(lds_u16<o0 + 2>(base[k0]), lds_u16<o1 + 2>(base[k1]), 0x5410);
+    typename Elem<E>::E2 v = __hfma2(as_e2<E>(tp.fpair[k0]),
+                                     __hsub2(as_e2<E>(x1), as_e2<E>(x0)), as_e2<E>(x0));
     if (MASK)
-        v = __fmul2_rn(v, make_float2(tp.m[k0], tp.m[k1]));
-    out[I] = Elem<E>::pack(v.x, v.y);
+        v = __hmul2(v, as_e2<E>(tp.mpair[k0]));
+    out[I] = as_u32<E>(v);
     if (SLOW && (((tp.slow >> k0) | (tp.slow >> k1)) & 1u)) {
-        float lo = v.x, hi = v.y;
+        float lo = __low2float(v), hi = __high2float(v);
         if ((tp.slow >> k0) & 1u)
             lo = slow_element<E, K, MASK>(tp, k0, 0, xg + c0 * xg_row_stride, L_in);
         if ((tp.slow >> k1) & 1u)
@@ -250,28 +270,16 @@ __device__ __forceinline__ void produce_dispatch(int k0, uint32_t (&out)[kSeg / 
 // STALL (test builds of the failure path only): the loader issues nothing, so the
 // first wait of every other role runs out; the kernel must then record the timeout,
 // drain and exit on its own.  Every forward launch uses STALL = false.
-//
-// CG = 2: a cluster of two CTAs on a pair of SMs works as one M = 256 tile (128
-// output positions in each CTA, A and D in each CTA's tensor memory); each CTA
-// loads HALF of the weight tile (N/2 output channels) and the first CTA issues
-// one tcgen05.mma.cta_group::2 for both.  Each SM thus moves half the weight
-// bytes through its shared memory per k-block.  Barriers the MMA waits on live in
-// the first CTA; the second CTA's producers and drain arrive on them remotely,
-// and the MMA's commits arrive on both CTAs' barriers.
-template <class E, int K, bool MASK, bool STALL, int CG>
+template <class E, int K, bool MASK, bool STALL>
 // 18 warps: 5 land on some SM sub-partitions, each of which holds 16K registers,
 // so a thread may use at most 16384 / (5 * 32) -> 96 registers.
 __global__ void __maxnreg__(96)
     tc_bf16_kernel(const __grid_constant__ TcArgs A, const __grid_constant__ CUtensorMap wmap,
                    const __grid_constant__ CUtensorMap xmap) {
-    constexpr int ST = stages_of(CG);
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const Problem &P = A.P;
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;   // 0: the pair's first CTA
-    const int unit0 = (int)blockIdx.x / CG;                   // this CTA's first tile
-    const int nunits = (int)gridDim.x / CG;
 
     // The 128-byte swizzle needs 1024-byte aligned stages: align the base by hand
     // (the launch reserves 1 KB of slack for this).
@@ -284,44 +292,29 @@ __global__ void __maxnreg__(96)
     float *bias_s = reinterpret_cast<float *>(smem + A.off_bias);
     for (int i = threadIdx.x; i < P.C_out; i += kThreads)
         bias_s[i] = P.bias ? ld_f32(static_cast<const E *>(P.bias) + i) : 0.0f;
-    // wfull: the stage's weight tile (both halves for CG = 2, counted on the first
-    // CTA's barrier); xfull: this CTA's x window (CG = 1: the same barrier as wfull)
-    auto bar_wfull = [&](int s) { return bar0 + 8u * s; };
-    auto bar_empty = [&](int s) { return bar0 + 8u * (ST + s); };
-    auto bar_afull = [&](int s) { return bar0 + 8u * (2 * ST + s); };
-    auto bar_xfull = [&](int s) { return CG == 2 ? bar0 + 8u * (3 * ST + s) : bar0 + 8u * s; };
-    const uint32_t bar_dfull = bar0 + 8u * (4 * ST);
-    const uint32_t bar_dempty = bar0 + 8u * (4 * ST + 1);
-    const uint32_t bar_drain = bar0 + 8u * (4 * ST + 2);
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + A.off_bar + 8 * (4 * ST + 3));
+    auto bar_full = [&](int s) { return bar0 + 8u * s; };
+    auto bar_empty = [&](int s) { return bar0 + 8u * (kStages + s); };
+    auto bar_afull = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+    const uint32_t bar_dfull = bar0 + 8u * (3 * kStages);
+    const uint32_t bar_dempty = bar0 + 8u * (3 * kStages + 1);
+    const uint32_t bar_drain = bar0 + 8u * (3 * kStages + 2);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + A.off_bar + 8 * (3 * kStages + 3));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-    // arrivals on the first CTA's barriers (remote from the second CTA)
-    auto arrive_first = [&](uint32_t bar) {
-        if (CG == 2)
-            mbar_arrive_cluster(mapa_shared(bar, 0));
-        else
-            mbar_arrive(bar);
-    };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < ST; ++s) {
-            mbar_init(bar_wfull(s), 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full(s), 1);
             mbar_init(bar_empty(s), 1);
-            mbar_init(bar_afull(s), (kProdWarps / 2) * CG);
-            if (CG == 2)
-                mbar_init(bar_xfull(s), 1);
+            mbar_init(bar_afull(s), kProdWarps / 2);
         }
         mbar_init(bar_dfull, 1);
-        mbar_init(bar_dempty, kProdWarps * CG);
+        mbar_init(bar_dempty, kProdWarps);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == kMmaWarp) {
-        if (CG == 2)
-            tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
-        else
-            tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+        tmem_alloc(smem_u32(tmem_holder), kTmemCols);
         tc_fence_before();
     }
     if (warp == kTmaWarp && lane == 0) {
@@ -329,100 +322,71 @@ __global__ void __maxnreg__(96)
         tma_prefetch_desc(&xmap);
     }
     __syncthreads();
-    if (CG == 2)
-        cluster_sync();   // the peer's barriers are initialised before any remote arrival
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    BoundedWait wait{abort_flag, A.wait_ns, A.status};
-    wait.cluster = (CG == 2);
+    const BoundedWait wait{abort_flag, A.wait_ns, A.status};
 
     if (warp == kTmaWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && !STALL) {
             uint32_t it = 0;
-            for (int t = unit0; t < A.num_tiles; t += nunits) {
-                const Tile T = decode_tile<CG>(A, t, rank);
+            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
+                const Tile T = decode_tile(A, t);
                 const int xrow0 = T.b * P.C_in + T.g * P.cin_g;
-                const int wrow0 = T.g * P.cout_g + (int)rank * (A.N / CG);
                 for (int pos = 0; pos < A.num_kb; ++pos, ++it) {
                     const int kb = kb_at(A, pos);
-                    const int s = it % ST;
-                    const uint32_t ph = (it / ST) & 1u;
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
                     if (!wait(bar_empty(s), ph ^ 1u))
                         goto tma_done;
+                    mbar_arrive_expect_tx(bar_full(s), A.w_stage_bytes + A.x_stage_bytes);
+                    tma_load_2d(w_st0 + s * A.w_stage_bytes, &wmap, kb * kBK, T.co0,
+                                bar_full(s));
                     const int c_lo = (kb * kBK) / K;
                     const uint32_t xdst = x_st0 + s * A.x_stage_bytes;
-                    if (CG == 2) {
-                        if (rank == 0)   // both halves' bytes land on the first CTA's barrier
-                            mbar_arrive_expect_tx(bar_wfull(s), 2u * A.w_stage_bytes);
-                        tma_load_2d_pair(w_st0 + s * A.w_stage_bytes, &wmap, kb * kBK, wrow0,
-                                         mapa_shared(bar_wfull(s), 0));
-                        mbar_arrive_expect_tx(bar_xfull(s), A.x_stage_bytes);
-                    } else {
-                        mbar_arrive_expect_tx(bar_wfull(s), A.w_stage_bytes + A.x_stage_bytes);
-                        tma_load_2d(w_st0 + s * A.w_stage_bytes, &wmap, kb * kBK, wrow0,
-                                    bar_wfull(s));
-                    }
-                    tma_load_2d(xdst, &xmap, T.wx0, xrow0 + c_lo, bar_xfull(s));
+                    tma_load_2d(xdst, &xmap, T.wx0, xrow0 + c_lo, bar_full(s));
                     if (A.nbox == 2)
                         tma_load_2d(xdst + A.x_box_bytes, &xmap, T.wx0 + kBoxStep, xrow0 + c_lo,
-                                    bar_xfull(s));
+                                    bar_full(s));
                 }
             }
         tma_done:
             // Let every load this thread issued land before the CTA can exit
             // (bounded; on the normal path they have all been consumed already).
             volatile int never = 0;
-            BoundedWait drain{&never, A.wait_ns, A.status};
-            drain.cluster = (CG == 2);
-            for (uint32_t j = (it > ST ? it - ST : 0); j < it; ++j) {
-                drain(bar_xfull(j % ST), (j / ST) & 1u);
-                if (CG == 2 && rank == 0)   // the pair's weight halves
-                    drain(bar_wfull(j % ST), (j / ST) & 1u);
-            }
+            const BoundedWait drain{&never, A.wait_ns, A.status};
+            for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
+                drain(bar_full(j % kStages), (j / kStages) & 1u);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && rank == 0) {
-            const uint32_t idesc = Elem<E>::idesc(128 * CG, A.N);
+        if (lane == 0) {
+            const uint32_t idesc = Elem<E>::idesc(128, A.N);
             uint32_t it = 0, tc = 0;
-            for (int t = unit0; t < A.num_tiles; t += nunits, ++tc) {
+            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
                 if (!wait(bar_dempty, (tc & 1u) ^ 1u))
                     goto mma_done;
                 tc_fence_after();
                 for (int pos = 0; pos < A.num_kb; ++pos, ++it) {
-                    const int s = it % ST;
-                    const uint32_t ph = (it / ST) & 1u;
-                    if (!wait(bar_wfull(s), ph) || !wait(bar_afull(s), ph))
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!wait(bar_full(s), ph) || !wait(bar_afull(s), ph))
                         goto mma_done;
                     tc_fence_after();
                     const uint32_t wst = w_st0 + s * A.w_stage_bytes;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
-                        const uint32_t acc = (pos > 0 || kk > 0) ? 1u : 0u;
-                        if (CG == 2)
-                            mma_bf16_ts_pair(tmem + kColD, tmem + kColA + 32u * s + 8u * kk,
-                                             sw128_kmajor_desc(wst + 32u * kk), idesc, acc);
-                        else
-                            mma_bf16_ts(tmem + kColD, tmem + kColA + 32u * s + 8u * kk,
-                                        sw128_kmajor_desc(wst + 32u * kk), idesc, acc);
+                        mma_bf16_ts(tmem + kColD, tmem + kColA + 32u * s + 8u * kk,
+                                    sw128_kmajor_desc(wst + 32u * kk), idesc,
+                                    (pos > 0 || kk > 0) ? 1u : 0u);
                     }
-                    if (CG == 2)
-                        mma_commit_pair(bar_empty(s), 0x3);
-                    else
-                        mma_commit(bar_empty(s));
+                    mma_commit(bar_empty(s));
                 }
-                if (CG == 2)
-                    mma_commit_pair(bar_dfull, 0x3);
-                else
-                    mma_commit(bar_dfull);
+                mma_commit(bar_dfull);
             }
         mma_done:
             // Every MMA issued has completed once this commit arrives.
-            if (CG == 2)
-                mma_commit_pair(bar_drain, 0x1);
-            else
-                mma_commit(bar_drain);
+            mma_commit(bar_drain);
             volatile int never = 0;
             const BoundedWait drain{&never, A.wait_ns, A.status};
             drain(bar_drain, 0);
@@ -436,15 +400,15 @@ __global__ void __maxnreg__(96)
         const int row = 32 * q + lane;
         // Epilogue of tile t (tile count tcnt): this warp's share of the accumulator columns.
         auto epilogue = [&](int t, uint32_t tcnt) -> bool {
-            const Tile T = decode_tile<CG>(A, t, rank);
+            const Tile T = decode_tile(A, t);
             const int l = T.lbase + row;
             const bool valid = l < P.L_out;
-            const float *biasg = bias_s + T.g * P.cout_g;
+            const float *biasg = bias_s + T.co0;
             if (!__all_sync(0xffffffffu, wait(bar_dfull, tcnt & 1u)))
                 return false;
             tc_fence_after();
             E *outp = static_cast<E *>(P.out) +
-                                  ((int64_t)T.b * P.C_out + (int64_t)T.g * P.cout_g) * P.L_out + l;
+                                  ((int64_t)T.b * P.C_out + (int64_t)T.co0) * P.L_out + l;
             for (int cc = h; cc < A.N / 16; cc += 4) {
                 uint32_t v[16];
                 tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + kColD + 16u * cc, v);
@@ -461,7 +425,7 @@ __global__ void __maxnreg__(96)
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                arrive_first(bar_dempty);
+                mbar_arrive(bar_dempty);
             return true;
         };
         int pend_t = -1;        // tile whose epilogue is still to do
@@ -497,13 +461,13 @@ __global__ void __maxnreg__(96)
         auto first_pos = [&](uint32_t tcnt) {
             return (int)(((uint32_t)par ^ (tcnt * (uint32_t)A.num_kb)) & 1u);
         };
-        if (unit0 < A.num_tiles && first_pos(0) < A.num_kb) {
-            const Tile T0 = decode_tile<CG>(A, unit0, rank);
-            prefetch(unit0, T0, seg_og(T0, first_pos(0)));
+        if ((int)blockIdx.x < A.num_tiles && first_pos(0) < A.num_kb) {
+            const Tile T0 = decode_tile(A, blockIdx.x);
+            prefetch(blockIdx.x, T0, seg_og(T0, first_pos(0)));
         }
-        for (int t = unit0; t < A.num_tiles; t += nunits) {
-            const Tile T = decode_tile<CG>(A, t, rank);
-            const int t_next = t + nunits;
+        for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
+            const Tile T = decode_tile(A, t);
+            const int t_next = t + (int)gridDim.x;
             const int l = T.lbase + row;
             const bool valid = l < P.L_out;
             const float start = (float)(l * P.stride - P.padding);
@@ -519,12 +483,12 @@ __global__ void __maxnreg__(96)
             int og_cur = -1;
             int og = (T.g * P.cin_g) / P.cin_per_og;
             int og_next_c = (og + 1) * P.cin_per_og - T.g * P.cin_g;   // group-relative
-            const int kb_first_stage = (A.num_kb < ST ? A.num_kb : ST);
+            const int kb_first_stage = (A.num_kb < kStages ? A.num_kb : kStages);
             for (int pos = pos_first; pos < A.num_kb; pos += 2) {
                 const int kb = kb_at(A, pos);
                 const uint32_t it = tcount * (uint32_t)A.num_kb + (uint32_t)pos;
-                const int s = it % ST;
-                const uint32_t ph = (it / ST) & 1u;
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1u;
                 const int kk0 = kb * kBK + kSeg * half;
                 const int c_first = kk0 / K;             // group-relative channel
                 const int k0 = kk0 - c_first * K;
@@ -566,20 +530,20 @@ __global__ void __maxnreg__(96)
                     }
 #pragma unroll
                     for (int k = 0; k < K; ++k) {
-                        tp.f[k] = f[k];
-                        tp.m[k] = m[k];
+                        tp.fpair[k] = Elem<E>::pack(f[k], f[(k + 1) % K]);
+                        tp.mpair[k] = Elem<E>::pack(m[k], m[(k + 1) % K]);
                     }
                     // next group: the following offset group of this tile, else the
                     // first one of the next tile
                     if (og < og_last)
                         prefetch(t, T, og + 1);
                     else if (t_next < A.num_tiles) {
-                        const Tile Tn = decode_tile<CG>(A, t_next, rank);   // once per tile
+                        const Tile Tn = decode_tile(A, t_next);   // once per tile
                         if (first_pos(tcount + 1) < A.num_kb)
                             prefetch(t_next, Tn, seg_og(Tn, first_pos(tcount + 1)));
                     }
                 }
-                if (!__all_sync(0xffffffffu, wait(bar_xfull(s), ph)))
+                if (!__all_sync(0xffffffffu, wait(bar_full(s), ph)))
                     goto prod_done;
                 {
                     const uint32_t xrow_addr =
@@ -599,7 +563,7 @@ __global__ void __maxnreg__(96)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
-                        arrive_first(bar_afull(s));
+                        mbar_arrive(bar_afull(s));
                 }
                 if (pend_t >= 0 && pos + 2 >= kb_first_stage) {
                     if (!epilogue(pend_t, pend_cnt))
@@ -623,15 +587,10 @@ __global__ void __maxnreg__(96)
     // ---------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
-    if (CG == 2)
-        cluster_sync();   // the pair's MMAs no longer read this CTA's memory
     if (warp == kMmaWarp) {
         __syncwarp();
         tc_fence_after();
-        if (CG == 2)
-            tmem_dealloc_pair(tmem, kTmemCols);
-        else
-            tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -640,37 +599,33 @@ __global__ void __maxnreg__(96)
 struct Plan {
     TcArgs A;
     size_t smem;
-    int cg;          // CTAs per tile: 1, or 2 (an SM pair)
 };
 
-// Kernel form: DCN1D_TC_PAIR=1 in the environment selects the SM-pair kernel wherever
-// it fits, anything else (or nothing) the one-SM kernel.
-int pair_mode() {
-    static const int mode = [] {
-        const char *e = getenv("DCN1D_TC_PAIR");
-        if (!e || !*e)
-            return -1;
-        return e[0] == '0' ? 0 : 1;
-    }();
-    return mode;
-}
-
-bool make_plan_cg(const Problem &P, int cg, Plan *out) {
+bool make_plan(const Problem &P, Plan *out) {
     TcArgs A;
     memset(&A, 0, sizeof(A));
     A.P = P;
     A.status = nullptr;
     const int Kg = P.cin_g * P.K;
-    const int st = stages_of(cg);
-    A.N = P.cout_g;
+    // the widest block of output channels (a multiple of 32, at most 256) that divides
+    // the conv group's; each block re-forms the columns it contracts
+    A.N = 0;
+    for (int n = 256; n >= 32; n -= 32)
+        if (P.cout_g % n == 0) {
+            A.N = n;
+            break;
+        }
+    if (A.N == 0)
+        return false;
+    A.n_cob = P.cout_g / A.N;
     A.num_kb = Kg / kBK;
     // Contiguous halves pay off when offset groups change inside a conv group (each
     // warp then meets every offset group of its half once instead of every group of the
     // tile); with one offset group per conv group the k-block parities measure faster.
     A.half_kb = (A.num_kb % 2 == 0 && A.num_kb >= 4 && P.cin_per_og < P.cin_g) ? A.num_kb / 2
                                                                                  : 0;
-    A.tiles_l = (P.L_out + kRows * cg - 1) / (kRows * cg);
-    A.num_tiles = P.groups * P.B * A.tiles_l;
+    A.tiles_l = (P.L_out + kRows - 1) / kRows;
+    A.num_tiles = P.groups * A.n_cob * P.B * A.tiles_l;
     A.nch = (kBK - 1) / P.K + 2;
     A.margin = P.unconstrained ? 32 : 0;
     const int64_t need = (int64_t)(kRows - 1) * P.stride + (int64_t)P.dilation * (P.K - 1) + 2 +
@@ -678,87 +633,48 @@ bool make_plan_cg(const Problem &P, int cg, Plan *out) {
     if (need > kWinMax)
         return false;
     A.nbox = need > kBox - 1 ? 2 : 1;
-    A.w_stage_bytes = (uint32_t)(A.N / cg) * 128u;   // this CTA's rows of the weight tile
+    A.w_stage_bytes = (uint32_t)A.N * 128u;
     A.x_box_bytes = (uint32_t)A.nch * kRowBytes;
     A.x_stage_bytes = A.x_box_bytes * A.nbox;
     A.off_w = 0;
-    A.off_x = A.off_w + st * A.w_stage_bytes;
-    A.off_bias = A.off_x + st * A.x_stage_bytes;
+    A.off_x = A.off_w + kStages * A.w_stage_bytes;
+    A.off_bias = A.off_x + kStages * A.x_stage_bytes;
     A.off_bar = A.off_bias + (uint32_t)((P.C_out * 4 + 15) / 16 * 16);
-    size_t smem = A.off_bar + 8 * (4 * st + 3) + 16 + 1024;   // + alignment slack
+    size_t smem = A.off_bar + 8 * (3 * kStages + 3) + 16 + 1024;   // + alignment slack
     if (smem > 227 * 1024)
         return false;
     // At least half the SM's shared memory, so two CTAs (each allocating all 512
     // tensor-memory columns) never share an SM.
     if (smem < 116 * 1024)
         smem = 116 * 1024;
-    if (kColA + 32u * st > kTmemCols)
-        return false;
     out->A = A;
     out->smem = smem;
-    out->cg = cg;
     return true;
-}
-
-bool make_plan(const Problem &P, Plan *out) {
-    const int mode = pair_mode();
-    const bool pair = mode == 1;
-    if (pair && make_plan_cg(P, 2, out))
-        return true;
-    return make_plan_cg(P, 1, out);
-}
-
-template <class E, int K, bool MASK, bool STALL, int CG>
-cudaError_t launch_kmc(const Plan &pl, cudaStream_t stream) {
-    const Problem &P = pl.A.P;
-    alignas(64) CUtensorMap wmap, xmap;
-    const int Kg = P.cin_g * P.K;
-    if (!encode_2d(&wmap, Elem<E>::kTma, P.w, (uint64_t)Kg, (uint64_t)P.C_out,
-                   2, kBK, (uint32_t)(pl.A.N / CG), CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    if (!encode_2d(&xmap, Elem<E>::kTma, P.x, (uint64_t)P.L_in,
-                   (uint64_t)P.B * P.C_in, 2, kBox, (uint32_t)pl.A.nch, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-    auto kern = tc_bf16_kernel<E, K, MASK, STALL, CG>;
-    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), (int)pl.smem);
-    if (e != cudaSuccess)
-        return e;
-    const int sms = sm_count();
-    if (sms < CG)
-        return cudaErrorNoDevice;
-    int units = sms / CG;   // persistent: one CTA (pair) per SM (pair)
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = pl.smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1] = {};
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CG;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = CG > 1 ? 1 : 0;   // the one-SM kernel is an ordinary launch
-    if (CG > 1) {
-        // SM pairs that can hold a cluster at once (a GPC with an odd number of free SMs
-        // leaves one out): the persistent grid should not exceed them
-        const int pairs = resident_clusters(reinterpret_cast<const void *>(kern), &cfg);
-        if (pairs > 0 && pairs < units)
-            units = pairs;
-    }
-    const int grid = CG * (pl.A.num_tiles < units ? pl.A.num_tiles : units);
-    cfg.gridDim = dim3((unsigned)grid);
-    timing_begin(stream);
-    e = cudaLaunchKernelEx(&cfg, kern, pl.A, wmap, xmap);
-    timing_end(stream);
-    if (e != cudaSuccess)
-        return e;
-    return cudaGetLastError();
 }
 
 template <class E, int K, bool MASK, bool STALL = false>
 cudaError_t launch_km(const Plan &pl, cudaStream_t stream) {
-    return pl.cg == 2 ? launch_kmc<E, K, MASK, STALL, 2>(pl, stream)
-                      : launch_kmc<E, K, MASK, STALL, 1>(pl, stream);
+    const Problem &P = pl.A.P;
+    alignas(64) CUtensorMap wmap, xmap;
+    const int Kg = P.cin_g * P.K;
+    if (!encode_2d(&wmap, Elem<E>::kTma, P.w, (uint64_t)Kg, (uint64_t)P.C_out,
+                   2, kBK, (uint32_t)pl.A.N, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!encode_2d(&xmap, Elem<E>::kTma, P.x, (uint64_t)P.L_in,
+                   (uint64_t)P.B * P.C_in, 2, kBox, (uint32_t)pl.A.nch, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    auto kern = tc_bf16_kernel<E, K, MASK, STALL>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), (int)pl.smem);
+    if (e != cudaSuccess)
+        return e;
+    const int sms = sm_count();
+    if (sms <= 0)
+        return cudaErrorNoDevice;
+    const int grid = pl.A.num_tiles < sms ? pl.A.num_tiles : sms;
+    timing_begin(stream);
+    kern<<<grid, kThreads, pl.smem, stream>>>(pl.A, wmap, xmap);
+    timing_end(stream);
+    return cudaGetLastError();
 }
 
 template <class E, int K>
@@ -786,7 +702,7 @@ bool tc_bf16_supported(const Problem &P) {
         return false;
     if (!(P.K == 3 || P.K == 4 || P.K == 5 || P.K == 7 || P.K == 9))
         return false;
-    if (P.cout_g % 32 != 0 || P.cout_g > 256)
+    if (P.cout_g % 32 != 0)
         return false;
     if ((P.cin_g * P.K) % kBK != 0)
         return false;

@@ -239,16 +239,21 @@ int dcn1d_forward_noalloc(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
  * L_out] in their dtype, and the gradients wanted, each NULL when not wanted
  * and otherwise shaped like its input in the same dtype (grad_mask needs a
  * mask: DCN1D_ERR_ARG otherwise).  Every wanted gradient is overwritten.
- * Arithmetic is fp32 for both dtypes; grad_x, grad_offsets and grad_mask are
- * sums of atomic fp32 additions, so their low bits may differ between calls;
- * grad_weight and grad_bias are summed in a fixed order.
+ * Arithmetic is fp32; for 16-bit dtypes the two contractions run on the tensor
+ * cores with 16-bit operands (grad_out, W, and the sampled columns rounded to
+ * the dtype) and fp32 accumulation, when L_out, C_out and C_out/groups are
+ * multiples of 8 (dcn1d_backward_kernel_name says which).  grad_x,
+ * grad_offsets and grad_mask are sums of atomic fp32 additions, so their low
+ * bits may differ between calls; grad_weight and grad_bias are summed in a
+ * fixed order.
  *
  * Scratch: `workspace` (256-byte aligned, owned by the caller, used only by the
  * work enqueued on `stream`) of at least dcn1d_backward_workspace_size() bytes:
- * fp32 column buffers of B * C_in * K * L_out floats (one for the gradient
- * sampled columns when any of grad_x / grad_offsets / grad_mask is wanted, one
- * for the sampled columns when grad_weight is wanted) plus fp32 accumulators of
- * grad_x, grad_offsets and grad_mask.  Too small or misaligned:
+ * column buffers of B * C_in * K * L_out values (fp32 gradient columns when any
+ * of grad_x / grad_offsets / grad_mask is wanted; the sampled columns, fp32 or
+ * 16-bit on the tensor-core path, when grad_weight is wanted), on the
+ * tensor-core path grad_out and W transposed, fp32 slices of grad_weight, and
+ * fp32 accumulators of grad_x, grad_offsets and grad_mask.  Too small or misaligned:
  * DCN1D_ERR_ARG; NULL with a non-zero need: DCN1D_ERR_NULL.
  * Other errors as for dcn1d_forward; B * groups above 65535 is
  * DCN1D_ERR_UNSUPPORTED.
@@ -271,6 +276,17 @@ int dcn1d_backward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn
                    void *workspace, size_t workspace_bytes, void *stream);
 
 /* dcn1d_backward and its workspace size with padding per side (see dcn1d_out_length_lr). */
+/* Which contraction kernels dcn1d_backward_lr runs for these arguments
+ * ("tcgen05_gemm": 16-bit operands on the tensor cores, or "cuda_core_gemm"), or
+ * NULL if the arguments are invalid.  Host only. */
+const char *dcn1d_backward_kernel_name(
+    const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
+    const dcn1d_tensor *weight, const dcn1d_tensor *grad_out, int64_t stride,
+    int64_t padding_left, int64_t padding_right, int64_t dilation, int64_t groups,
+    int64_t offset_groups, int unconstrained, const dcn1d_tensor *grad_x,
+    const dcn1d_tensor *grad_offsets, const dcn1d_tensor *grad_mask,
+    const dcn1d_tensor *grad_weight, const dcn1d_tensor *grad_bias);
+
 int64_t dcn1d_backward_lr_workspace_size(
     const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
     const dcn1d_tensor *weight, const dcn1d_tensor *grad_out, int64_t stride,

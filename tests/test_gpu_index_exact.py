@@ -36,6 +36,8 @@ CASES = [
      2, 2, 2, True, False, False),
     ("tc_f16_k3_unconstrained", "tcgen05_f16", "f16", 2, 64, 192, 3, 264, 1, 1, 1, 1, 2,
      True, True, False),
+    ("tc_k3_cout_512_two_blocks", "tcgen05_bf16", "bf16", 1, 64, 512, 3, 264, 1, 1, 1, 1, 1,
+     False, True, False),
     ("tf32_k16_d3_constrained", "tcgen05_3xtf32", "f32", 2, 32, 512, 16, 128, 1, 0, 3, 1, 1,
      False, False, False),
     ("tf32_k4_strided_groups_mask_unconstrained", "tcgen05_3xtf32", "f32", 2, 64, 128, 4, 160,
@@ -148,6 +150,9 @@ PACKED = [
     ("packed_dense_unmodulated_k3", 64, 192, 3, 264, 1, (1, 1), 1, 1, 2, False,
      "tcgen05_bf16"),
 ]
+# unconstrained forms of the depthwise layers (the probe's offsets include values past
+# the window margin and far past the signal): name suffix "_unc"
+PACKED += [(c[0] + "_unc",) + c[1:] for c in PACKED if c[0].startswith("packed_depthwise")]
 KEYS = ("x", "dw_weight", "dw_bias", "off_weight", "off_bias", "mask_weight", "mask_bias",
         "weight", "bias")
 
@@ -155,6 +160,7 @@ KEYS = ("x", "dw_weight", "dw_bias", "off_weight", "off_bias", "mask_weight", "m
 @pytest.mark.parametrize("case", PACKED, ids=[c[0] for c in PACKED])
 def test_packed_layer_bit_exact(case):
     name, Ci, Co, K, L, s, pad, d, G, og, modulated, fwd = case
+    unc = name.endswith("_unc")
     pl, pr = dcn.resolve_padding(pad, K, s, d)
     t = _packed_probe(Ci, Co, K, L, s, (pl, pr), d, G, og, modulated,
                       seed=zlib.crc32(name.encode()) % 1000)
@@ -171,15 +177,15 @@ def test_packed_layer_bit_exact(case):
         t["weight"] = w.to(torch.bfloat16)
         t["bias"] = None
         td = {k: (v.cuda() if v is not None else None) for k, v in t.items()}
-        y, pred = dcn.dcn1d_packed_forward(*[td[k] for k in KEYS], s, pad, d, G, og, False,
+        y, pred = dcn.dcn1d_packed_forward(*[td[k] for k in KEYS], s, pad, d, G, og, unc,
                                            with_offsets=True)
         off, mask = pred if modulated else (pred, None)
         torch.cuda.synchronize()
         assert dcn.dcn1d_device_status() == 0
         kern = dcn.dcn1d_forward_kernel_name(td["x"], off, mask, td["weight"], None, s, pad, d,
-                                             G, og, False)
+                                             G, og, unc)
         assert kern == fwd, (name, kern)
-        r, roff, _ = oracle.packed_forward(*[t[k] for k in KEYS], s, (pl, pr), d, G, og, False)
+        r, roff, _ = oracle.packed_forward(*[t[k] for k in KEYS], s, (pl, pr), d, G, og, unc)
         # the predicted offsets are exact too: compare them bit for bit first
         assert torch.equal(off.cpu(), torch.from_numpy(np.ascontiguousarray(roff)).to(
             torch.bfloat16)), name
@@ -188,7 +194,7 @@ def test_packed_layer_bit_exact(case):
         ref = torch.from_numpy(np.ascontiguousarray(r)).to(torch.bfloat16)
         assert torch.equal(y.cpu(), ref), (name, int((y.cpu() != ref).sum()))
         # the same layer without the predicted tensors: one fused kernel where it applies
-        y1 = dcn.dcn1d_packed_forward(*[td[k] for k in KEYS], s, pad, d, G, og, False)
+        y1 = dcn.dcn1d_packed_forward(*[td[k] for k in KEYS], s, pad, d, G, og, unc)
         torch.cuda.synchronize()
         assert dcn.dcn1d_device_status() == 0
         assert torch.equal(y1.cpu(), ref), (name, "fused", int((y1.cpu() != ref).sum()))

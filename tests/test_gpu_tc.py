@@ -20,6 +20,9 @@ CASES = [
     ("g1_k7_og_per_32", 1, 64, 64, 7, 136, 1, 3, 1, 1, 2, False, False, 2.5),
     ("far_offsets_slow_taps", 2, 64, 64, 5, 256, 1, 2, 1, 1, 1, False, True, 80.0),
     ("l_out_below_one_tile", 2, 128, 256, 5, 64, 1, 2, 1, 1, 4, True, False, 3.0),
+    # more than 256 output channels per conv group: blocks of 256, and of 192
+    ("cout_512_two_blocks", 2, 128, 512, 5, 256, 1, 2, 1, 1, 4, True, False, 3.0),
+    ("g2_cout_g384_blocks_of_192", 1, 128, 768, 3, 200, 1, 1, 1, 2, 2, False, True, 2.0),
 ]
 
 
