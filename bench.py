@@ -467,6 +467,8 @@ def run_backward_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
     args_c = (w.stride, w.padding, w.dilation, w.groups, w.offset_groups, w.unconstrained)
     need = dcn.dcn1d_backward_workspace_size(d["x"], d["offsets"], d["mask"], d["weight"], gout,
                                              *args_c, wanted=wanted)
+    gemm_kernel = dcn.dcn1d_backward_kernel_name(d["x"], d["offsets"], d["mask"], d["weight"],
+                                                 gout, *args_c, wanted=wanted)
     scratch = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -494,18 +496,26 @@ def run_backward_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
     barrier(ws)
     ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), ws) / args.steps
     per_gpu = 2 * w.flops() / (ms / 1e3) / 1e12
+    if gemm_kernel == "tcgen05_gemm":   # 16-bit operands on the tensor cores
+        roof = {"bound": "tensor", "achieved": per_gpu, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": per_gpu / peaks["bf16_tflops"], "traffic": None,
+                "kernel": "backward: two tcgen05 GEMMs (16-bit operands, fp32 accumulation) "
+                          "+ sampling gradient + transposes",
+                "peak_source": f"bf16 dense GEMM burst ({peaks['source']})"}
+    else:
+        roof = {"bound": "alu", "achieved": per_gpu, "peak": ALU_F32_TFLOPS,
+                "unit": "TFLOP/s", "frac": per_gpu / ALU_F32_TFLOPS, "traffic": None,
+                "kernel": "backward: two CUDA-core fp32 GEMMs + sampling gradient",
+                "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz"}
+    roof.update({"launches_per_step": launches,
+                 "timing": "CUDA events around the whole backward call, per step"})
     line = {"metric": METRIC_BACKWARD, "value": per_gpu * ws, "unit": "TFLOP/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic (seeded, shapes and distributions of the named workload)",
-            "config": workload_config(w, "backward", ws,
+            "config": workload_config(w, f"backward ({gemm_kernel})", ws,
                                       l2="flushed between steps (256 MiB write outside the timed events)"),
-            "roofline": {"bound": "alu", "achieved": per_gpu, "peak": ALU_F32_TFLOPS,
-                         "unit": "TFLOP/s", "frac": per_gpu / ALU_F32_TFLOPS, "traffic": None,
-                         "kernel": "backward: two CUDA-core fp32 GEMMs + sampling gradient",
-                         "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz",
-                         "launches_per_step": launches,
-                         "timing": "CUDA events around the whole backward call, per step"},
+            "roofline": roof,
             "clocks": clk.summary(), "gpu_launches": launches * args.steps,
             "workspace_bytes": need}
     if want_cpu and ws == 1 and rank == 0:
