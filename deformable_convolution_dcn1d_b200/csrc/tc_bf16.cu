@@ -76,7 +76,9 @@ struct TcArgs {
     int margin;        // staged positions beyond the receptive fields (unconstrained)
     uint32_t w_stage_bytes, x_stage_bytes, x_box_bytes;
     int pair_store;    // 1: L_out even and out 4-byte aligned (32-bit epilogue stores)
-    uint32_t off_w, off_x, off_bias, off_bar;   // shared-memory layout
+    int xtma;          // 1: x windows by TMA; 0 (L_in not a multiple of 8, even): by the
+                       // loader warp's 4-byte cp.async copies into the same layout
+    uint32_t off_w, off_x, off_bias, off_pos, off_bar;   // shared-memory layout
     unsigned int *status;                       // device status word
     uint64_t wait_ns;                           // limit of every mbarrier wait
 };
@@ -98,8 +100,9 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs &A, int t) {
     Tile r;
     // channel blocks of one (g, b, positions) are consecutive tiles: they run at the
     // same time on neighbouring CTAs and share the x window through L2
-    const int cob = t % A.n_cob;
-    const int t2 = t / A.n_cob;
+    // (one block per group is the common case: no division then)
+    const int cob = A.n_cob == 1 ? 0 : t % A.n_cob;
+    const int t2 = A.n_cob == 1 ? t : t / A.n_cob;
     const int lt = t2 % A.tiles_l;
     const int gb = t2 / A.tiles_l;
     r.b = gb % A.P.B;
@@ -118,6 +121,23 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared.u16 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
     return v;
+}
+
+// 4-byte asynchronous global -> shared copy; `bytes` (4 or 0) are read, the rest of the
+// 4 bytes zero-filled.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(bytes)
+                 : "memory");
+}
+
+// One arrival on `bar` once every cp.async this thread issued so far has landed (the
+// arrival counts against the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // The 16-bit element type E of a problem (bf16 or fp16): its pair type, packing,
@@ -173,20 +193,42 @@ __device__ __forceinline__ uint32_t as_u32(typename Elem<E>::E2 h) {
 // Per-row tap state of one offset group.  Elements come in pairs (kk, kk+1),
 // i.e. taps (k, (k+1) % K), so fractions and mask values are kept pre-packed
 // as 16-bit pairs indexed by the first tap of the pair.
+//
+// Register budget (96 a thread): from K = kPosSmemMinK on, the taps' positions, which
+// only the slow path reads, live in shared memory instead (`pos_s`, this thread's column
+// of a [K][512] array); past K = 7 a group's offsets are loaded when they are needed
+// instead of one group ahead.  Both measured faster (K = 9: no spills, K = 5 with a mask:
+// fewer registers).
+constexpr int kPosSmemMinK = 4;
+template <int K>
+constexpr bool kWideK = K >= kPosSmemMinK;
+template <int K>
+constexpr bool kAheadK = K <= 7;
+
 template <int K>
 struct Taps {
     uint32_t addr[K];    // byte offset of the tap's neighbour pair in a stage row
     uint32_t fpair[K];   // E x2 (f_k, f_{(k+1)%K})
     uint32_t mpair[K];   // E x2 (m_k, m_{(k+1)%K})
-    float pos[K];        // position, for taps outside the window (slow path)
+    float pos[kWideK<K> ? 1 : K];   // position, for taps outside the window (slow path)
     uint32_t slow;       // bit k: tap k outside the staged window
 };
 
+constexpr int kProdThreads = kProdWarps * 32;
+
+template <int K>
+__device__ __forceinline__ float tap_pos(const Taps<K> &tp, const float *pos_s, int k) {
+    if constexpr (kWideK<K>)
+        return pos_s[k * kProdThreads];
+    else
+        return tp.pos[k];
+}
+
 // The col value of one element by the slow path: exact floor, global loads.
 template <class E, int K, bool MASK>
-__device__ __forceinline__ float slow_element(const Taps<K> &tp, int kidx, int hi,
-                                              const E *row, int L_in) {
-    const Tap e = tap_floor_exact(tp.pos[kidx]);
+__device__ __forceinline__ float slow_element(const Taps<K> &tp, const float *pos_s, int kidx,
+                                              int hi, const E *row, int L_in) {
+    const Tap e = tap_floor_exact(tap_pos<K>(tp, pos_s, kidx));
     const float x0 = (e.i0 >= 0 && e.i0 < L_in) ? ld_f32(row + e.i0) : 0.0f;
     const float x1 = (e.i0 >= -1 && e.i0 < L_in - 1) ? ld_f32(row + e.i0 + 1) : 0.0f;
     const float r = __fmaf_rn(e.f, __fsub_rn(x1, x0), x0);
@@ -201,8 +243,8 @@ __device__ __forceinline__ float slow_element(const Taps<K> &tp, int kidx, int h
 // The lerp x0 + f (x1 - x0) runs on the two elements in bf16x2 arithmetic.
 template <class E, int K, int K0, bool MASK, bool SLOW, int I>
 __device__ __forceinline__ void produce_pair(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
-                                             const uint32_t (&base)[K], const E *xg,
-                                             int64_t xg_row_stride, int L_in) {
+                                             const float *pos_s, const uint32_t (&base)[K],
+                                             const E *xg, int64_t xg_row_stride, int L_in) {
     constexpr int k0 = (K0 + 2 * I) % K, c0 = (K0 + 2 * I) / K;
     constexpr int k1 = (K0 + 2 * I + 1) % K, c1 = (K0 + 2 * I + 1) / K;
     constexpr uint32_t o0 = c0 * kRowBytes, o1 = c1 * kRowBytes;
@@ -218,19 +260,20 @@ __device__ __forceinline__ void produce_pair(uint32_t (&out)[kSeg / 2], const Ta
     if (SLOW && (((tp.slow >> k0) | (tp.slow >> k1)) & 1u)) {
         float lo = __low2float(v), hi = __high2float(v);
         if ((tp.slow >> k0) & 1u)
-            lo = slow_element<E, K, MASK>(tp, k0, 0, xg + c0 * xg_row_stride, L_in);
+            lo = slow_element<E, K, MASK>(tp, pos_s, k0, 0, xg + c0 * xg_row_stride, L_in);
         if ((tp.slow >> k1) & 1u)
-            hi = slow_element<E, K, MASK>(tp, k1, 1, xg + c1 * xg_row_stride, L_in);
+            hi = slow_element<E, K, MASK>(tp, pos_s, k1, 1, xg + c1 * xg_row_stride, L_in);
         out[I] = Elem<E>::pack(lo, hi);
     }
 }
 
 template <class E, int K, int K0, bool MASK, bool SLOW, int... Is>
 __device__ __forceinline__ void produce_pairs(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
-                                              const uint32_t (&base)[K], const E *xg,
-                                              int64_t xg_row_stride, int L_in,
+                                              const float *pos_s, const uint32_t (&base)[K],
+                                              const E *xg, int64_t xg_row_stride, int L_in,
                                               std::integer_sequence<int, Is...>) {
-    (produce_pair<E, K, K0, MASK, SLOW, Is>(out, tp, base, xg, xg_row_stride, L_in), ...);
+    (produce_pair<E, K, K0, MASK, SLOW, Is>(out, tp, pos_s, base, xg, xg_row_stride, L_in),
+     ...);
 }
 
 // kSeg col values of one row for the reduction elements kk0 .. kk0+kSeg-1 of a k-block,
@@ -238,33 +281,38 @@ __device__ __forceinline__ void produce_pairs(uint32_t (&out)[kSeg / 2], const T
 // compile-time constant, so every tap index and row offset below is static.
 template <class E, int K, int K0, bool MASK, bool SLOW>
 __device__ __forceinline__ void produce_segment(uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
-                                                uint32_t xrow_addr, const E *xg,
-                                                int64_t xg_row_stride, int L_in) {
+                                                const float *pos_s, uint32_t xrow_addr,
+                                                const E *xg, int64_t xg_row_stride, int L_in) {
     uint32_t base[K];
 #pragma unroll
     for (int k = 0; k < K; ++k)
         base[k] = xrow_addr + tp.addr[k];
-    produce_pairs<E, K, K0, MASK, SLOW>(out, tp, base, xg, xg_row_stride, L_in,
+    produce_pairs<E, K, K0, MASK, SLOW>(out, tp, pos_s, base, xg, xg_row_stride, L_in,
                                      std::make_integer_sequence<int, kSeg / 2>{});
 }
 
 // Jump to the segment code of phase k0 (a switch, so one indirect branch).
 template <class E, int K, bool MASK, bool SLOW>
 __device__ __forceinline__ void produce_dispatch(int k0, uint32_t (&out)[kSeg / 2], const Taps<K> &tp,
-                                                 uint32_t xrow_addr, const E *xg,
-                                                 int64_t xg_row_stride, int L_in) {
+                                                 const float *pos_s, uint32_t xrow_addr,
+                                                 const E *xg, int64_t xg_row_stride, int L_in) {
+    if constexpr (kSeg % K == 0) {   // segments start on a channel: phase 0 only
+        produce_segment<E, K, 0, MASK, SLOW>(out, tp, pos_s, xrow_addr, xg, xg_row_stride,
+                                            L_in);
+    } else {
 #define DCN1D_PHASE(P_)                                                                          \
     case P_:                                                                                    \
         if constexpr (P_ < K)                                                                   \
-            produce_segment<E, K, (P_ < K ? P_ : 0), MASK, SLOW>(out, tp, xrow_addr, xg,          \
+            produce_segment<E, K, (P_ < K ? P_ : 0), MASK, SLOW>(out, tp, pos_s, xrow_addr, xg,   \
                                                               xg_row_stride, L_in);             \
         break;
-    switch (k0) {
-        DCN1D_PHASE(0) DCN1D_PHASE(1) DCN1D_PHASE(2) DCN1D_PHASE(3) DCN1D_PHASE(4)
-        DCN1D_PHASE(5) DCN1D_PHASE(6) DCN1D_PHASE(7) DCN1D_PHASE(8)
-        default: break;
-    }
+        switch (k0) {
+            DCN1D_PHASE(0) DCN1D_PHASE(1) DCN1D_PHASE(2) DCN1D_PHASE(3) DCN1D_PHASE(4)
+            DCN1D_PHASE(5) DCN1D_PHASE(6) DCN1D_PHASE(7) DCN1D_PHASE(8)
+            default: break;
+        }
 #undef DCN1D_PHASE
+    }
 }
 
 // STALL (test builds of the failure path only): the loader issues nothing, so the
@@ -303,7 +351,9 @@ __global__ void __maxnreg__(96)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar_full(s), 1);
+            // TMA mode: the loader's expect-tx arrival; copy mode: also one arrival per
+            // loader lane when its copies have landed
+            mbar_init(bar_full(s), A.xtma ? 1 : 33);
             mbar_init(bar_empty(s), 1);
             mbar_init(bar_afull(s), kProdWarps / 2);
         }
@@ -319,14 +369,71 @@ __global__ void __maxnreg__(96)
     }
     if (warp == kTmaWarp && lane == 0) {
         tma_prefetch_desc(&wmap);
-        tma_prefetch_desc(&xmap);
+        if (A.xtma)
+            tma_prefetch_desc(&xmap);
     }
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const BoundedWait wait{abort_flag, A.wait_ns, A.status};
+    // the limit is a constant except in the STALL test build
+    const uint64_t wait_ns = STALL ? A.wait_ns : kWaitNs;
+    const BoundedWait wait{abort_flag, wait_ns, A.status};
 
-    if (warp == kTmaWarp) {
+    if (warp == kTmaWarp && !A.xtma) {
+        // ------------------------------------------------------------ loader, copy mode
+        // The weight tile by TMA (lane 0); the x window [nch rows][nbox boxes] by 4-byte
+        // copies from all 32 lanes (L_in even, so every copied pair starts on an even
+        // element and lies inside its row or outside the signal, zero-filled).
+        uint32_t it = 0;
+        const int rows_total = P.B * P.C_in;
+        const E *xbase = static_cast<const E *>(P.x);
+        const int words = A.nbox * (kBox / 2);   // 4-byte words per staged row
+        if (!STALL) {
+            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
+                const Tile T = decode_tile(A, t);
+                const int xrow0 = T.b * P.C_in + T.g * P.cin_g;
+                for (int pos = 0; pos < A.num_kb; ++pos, ++it) {
+                    const int kb = kb_at(A, pos);
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!__all_sync(0xffffffffu, wait(bar_empty(s), ph ^ 1u)))
+                        goto copy_done;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar_full(s), A.w_stage_bytes);
+                        tma_load_2d(w_st0 + s * A.w_stage_bytes, &wmap, kb * kBK, T.co0,
+                                    bar_full(s));
+                    }
+                    const int c_lo = (kb * kBK) / K;
+                    const uint32_t xdst = x_st0 + s * A.x_stage_bytes;
+                    for (int r = 0; r < A.nch; ++r) {
+                        const int xr = xrow0 + c_lo + r;
+                        const bool row_ok = xr < rows_total;
+                        const E *xrow = xbase + (int64_t)(row_ok ? xr : 0) * P.L_in;
+                        const uint32_t drow = xdst + (uint32_t)r * kRowBytes;
+                        for (int j = lane; j < words; j += 32) {
+                            const int bx = j >= kBox / 2 ? 1 : 0;
+                            const int w = j - bx * (kBox / 2);
+                            const int p = T.wx0 + bx * kBoxStep + 2 * w;
+                            const bool ok = row_ok && p >= 0 && p < P.L_in;
+                            cp_async4(drow + (uint32_t)bx * A.x_box_bytes + 4u * (uint32_t)w,
+                                      ok ? static_cast<const void *>(xrow + p)
+                                         : static_cast<const void *>(xbase),
+                                      ok ? 4u : 0u);
+                        }
+                    }
+                    cp_async_arrive(bar_full(s));
+                }
+            }
+        }
+    copy_done:
+        cp_async_wait_all();
+        if (lane == 0) {   // the weight tiles still in flight (bounded)
+            volatile int never = 0;
+            const BoundedWait drain{&never, wait_ns, A.status};
+            for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
+                drain(bar_full(j % kStages), (j / kStages) & 1u);
+        }
+    } else if (warp == kTmaWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && !STALL) {
             uint32_t it = 0;
@@ -354,7 +461,7 @@ __global__ void __maxnreg__(96)
             // Let every load this thread issued land before the CTA can exit
             // (bounded; on the normal path they have all been consumed already).
             volatile int never = 0;
-            const BoundedWait drain{&never, A.wait_ns, A.status};
+            const BoundedWait drain{&never, wait_ns, A.status};
             for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
                 drain(bar_full(j % kStages), (j / kStages) & 1u);
         }
@@ -388,7 +495,7 @@ __global__ void __maxnreg__(96)
             // Every MMA issued has completed once this commit arrives.
             mma_commit(bar_drain);
             volatile int never = 0;
-            const BoundedWait drain{&never, A.wait_ns, A.status};
+            const BoundedWait drain{&never, wait_ns, A.status};
             drain(bar_drain, 0);
         }
     } else if (warp < kProdWarps) {
@@ -433,7 +540,11 @@ __global__ void __maxnreg__(96)
         const float M = kFloorMagic;
         const float spanf = (float)(P.dilation * (K - 1));
         // Offsets (and mask) of the next (tile, offset group) this thread needs, loaded
-        // one group ahead so the global-load latency hides behind the current group.
+        // one group ahead so the global-load latency hides behind the current group
+        // (wide K: loaded when needed, to keep the registers).
+        constexpr bool kAhead = kAheadK<K>;
+        float *pos_s = kWideK<K> ? reinterpret_cast<float *>(smem + A.off_pos) + threadIdx.x
+                                 : nullptr;
         float raw_off[K], raw_m[K];
         int pf_t = -1, pf_og = -1;
         auto prefetch = [&](int t, const Tile &T, int og) {
@@ -461,15 +572,17 @@ __global__ void __maxnreg__(96)
         auto first_pos = [&](uint32_t tcnt) {
             return (int)(((uint32_t)par ^ (tcnt * (uint32_t)A.num_kb)) & 1u);
         };
-        if ((int)blockIdx.x < A.num_tiles && first_pos(0) < A.num_kb) {
+        if (kAhead && (int)blockIdx.x < A.num_tiles && first_pos(0) < A.num_kb) {
             const Tile T0 = decode_tile(A, blockIdx.x);
             prefetch(blockIdx.x, T0, seg_og(T0, first_pos(0)));
         }
         for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
             const Tile T = decode_tile(A, t);
             const int t_next = t + (int)gridDim.x;
+            // Rows past L_out (the last tile's) sample with row 0's offsets: their taps are
+            // finite and read the window or the bounds-checked slow path, and their
+            // accumulator rows (each depends on its own operand row only) are never stored.
             const int l = T.lbase + row;
-            const bool valid = l < P.L_out;
             const float start = (float)(l * P.stride - P.padding);
             const uint32_t win_bits = kFloorMagicBits + (uint32_t)T.wx0;
             const int pos_first = first_pos(tcount);
@@ -512,7 +625,10 @@ __global__ void __maxnreg__(96)
                         const uint32_t rel = __float_as_uint(tt) - win_bits;   // i0 - wx0
                         f[k] = __fsub_rn(pos, __fsub_rn(tt, M));
                         m[k] = raw_m[k];
-                        tp.pos[k] = pos;
+                        if constexpr (kWideK<K>)
+                            pos_s[k * kProdThreads] = pos;
+                        else
+                            tp.pos[k] = pos;
                         if (rel < (uint32_t)(kBox - 1)) {
                             tp.addr[k] = rel * 2u;
                         } else if (A.nbox == 2 && rel < (uint32_t)kWinMax) {
@@ -520,12 +636,6 @@ __global__ void __maxnreg__(96)
                         } else {
                             tp.addr[k] = 0;
                             tp.slow |= 1u << k;
-                        }
-                        if (!valid) {   // rows past L_out: finite zeros, never stored
-                            f[k] = 0.0f;
-                            m[k] = 0.0f;
-                            tp.addr[k] = 0;
-                            tp.slow &= ~(1u << k);
                         }
                     }
 #pragma unroll
@@ -535,12 +645,14 @@ __global__ void __maxnreg__(96)
                     }
                     // next group: the following offset group of this tile, else the
                     // first one of the next tile
-                    if (og < og_last)
-                        prefetch(t, T, og + 1);
-                    else if (t_next < A.num_tiles) {
-                        const Tile Tn = decode_tile(A, t_next);   // once per tile
-                        if (first_pos(tcount + 1) < A.num_kb)
-                            prefetch(t_next, Tn, seg_og(Tn, first_pos(tcount + 1)));
+                    if constexpr (kAhead) {
+                        if (og < og_last)
+                            prefetch(t, T, og + 1);
+                        else if (t_next < A.num_tiles) {
+                            const Tile Tn = decode_tile(A, t_next);   // once per tile
+                            if (first_pos(tcount + 1) < A.num_kb)
+                                prefetch(t_next, Tn, seg_og(Tn, first_pos(tcount + 1)));
+                        }
                     }
                 }
                 if (!__all_sync(0xffffffffu, wait(bar_full(s), ph)))
@@ -552,10 +664,12 @@ __global__ void __maxnreg__(96)
                         xb + (int64_t)(T.g * P.cin_g + c_first) * P.L_in;
                     uint32_t packed[kSeg / 2];
                     if (__any_sync(0xffffffffu, tp.slow != 0))
-                        produce_dispatch<E, K, MASK, true>(k0, packed, tp, xrow_addr, xg, P.L_in,
+                        produce_dispatch<E, K, MASK, true>(k0, packed, tp, pos_s, xrow_addr, xg,
+                                                        P.L_in,
                                                         P.L_in);
                     else
-                        produce_dispatch<E, K, MASK, false>(k0, packed, tp, xrow_addr, xg, P.L_in,
+                        produce_dispatch<E, K, MASK, false>(k0, packed, tp, pos_s, xrow_addr, xg,
+                                                         P.L_in,
                                                          P.L_in);
                     tmem_st16(tmem + ((uint32_t)(32 * q) << 16) + kColA + 32u * s + 16u * half,
                               packed);
@@ -624,6 +738,7 @@ bool make_plan(const Problem &P, Plan *out) {
     // tile); with one offset group per conv group the k-block parities measure faster.
     A.half_kb = (A.num_kb % 2 == 0 && A.num_kb >= 4 && P.cin_per_og < P.cin_g) ? A.num_kb / 2
                                                                                  : 0;
+    A.xtma = (P.L_in % 8 == 0 && (reinterpret_cast<uintptr_t>(P.x) & 15) == 0) ? 1 : 0;
     A.tiles_l = (P.L_out + kRows - 1) / kRows;
     A.num_tiles = P.groups * A.n_cob * P.B * A.tiles_l;
     A.nch = (kBK - 1) / P.K + 2;
@@ -639,7 +754,9 @@ bool make_plan(const Problem &P, Plan *out) {
     A.off_w = 0;
     A.off_x = A.off_w + kStages * A.w_stage_bytes;
     A.off_bias = A.off_x + kStages * A.x_stage_bytes;
-    A.off_bar = A.off_bias + (uint32_t)((P.C_out * 4 + 15) / 16 * 16);
+    A.off_pos = A.off_bias + (uint32_t)((P.C_out * 4 + 15) / 16 * 16);
+    // wide K: the producers' tap positions, [K][512] floats
+    A.off_bar = A.off_pos + (P.K >= kPosSmemMinK ? (uint32_t)(P.K * kProdThreads * 4) : 0u);
     size_t smem = A.off_bar + 8 * (3 * kStages + 3) + 16 + 1024;   // + alignment slack
     if (smem > 227 * 1024)
         return false;
@@ -660,8 +777,10 @@ cudaError_t launch_km(const Plan &pl, cudaStream_t stream) {
     if (!encode_2d(&wmap, Elem<E>::kTma, P.w, (uint64_t)Kg, (uint64_t)P.C_out,
                    2, kBK, (uint32_t)pl.A.N, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    if (!encode_2d(&xmap, Elem<E>::kTma, P.x, (uint64_t)P.L_in,
-                   (uint64_t)P.B * P.C_in, 2, kBox, (uint32_t)pl.A.nch, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!pl.A.xtma)
+        memset(&xmap, 0, sizeof(xmap));   // copy mode: not read
+    else if (!encode_2d(&xmap, Elem<E>::kTma, P.x, (uint64_t)P.L_in, (uint64_t)P.B * P.C_in, 2,
+                        kBox, (uint32_t)pl.A.nch, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     auto kern = tc_bf16_kernel<E, K, MASK, STALL>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), (int)pl.smem);
@@ -690,6 +809,7 @@ cudaError_t launch_e(const Plan &pl, cudaStream_t stream) {
     case 5: return launch_k<E, 5>(pl, stream);
     case 7: return launch_k<E, 7>(pl, stream);
     case 9: return launch_k<E, 9>(pl, stream);
+    case 16: return launch_k<E, 16>(pl, stream);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -700,19 +820,21 @@ cudaError_t launch_e(const Plan &pl, cudaStream_t stream) {
 bool tc_bf16_supported(const Problem &P) {
     if ((P.dtype != DCN1D_BF16 && P.dtype != DCN1D_F16) || !fast_floor_ok(P))
         return false;
-    if (!(P.K == 3 || P.K == 4 || P.K == 5 || P.K == 7 || P.K == 9))
+    if (!(P.K == 3 || P.K == 4 || P.K == 5 || P.K == 7 || P.K == 9 || P.K == 16))
         return false;
     if (P.cout_g % 32 != 0)
         return false;
     if ((P.cin_g * P.K) % kBK != 0)
         return false;
-    if (P.L_in % 8 != 0)   // TMA row stride must be a multiple of 16 bytes
+    // x windows: by TMA when the row pitch is a multiple of 16 bytes, else by 4-byte
+    // copies, which need an even L_in
+    if (P.L_in % 2 != 0)
         return false;
     // Offsets are uniform across each 32-element segment of the reduction.
     const bool og_whole_group = (P.cin_per_og % P.cin_g) == 0;
     if (!og_whole_group && (P.cin_per_og * P.K) % kSeg != 0)
         return false;
-    if ((reinterpret_cast<uintptr_t>(P.x) & 15) || (reinterpret_cast<uintptr_t>(P.w) & 15))
+    if ((reinterpret_cast<uintptr_t>(P.x) & 3) || (reinterpret_cast<uintptr_t>(P.w) & 15))
         return false;
     if (P.C_out > 8192)   // the bias is staged in shared memory
         return false;
@@ -733,7 +855,8 @@ cudaError_t launch_tc_bf16(const Problem &P, cudaStream_t stream) {
 }
 
 bool tc_bf16_stalled_supported(const Problem &P) {
-    return tc_bf16_supported(P) && P.dtype == DCN1D_BF16 && P.K == 3 && !P.mask;
+    return tc_bf16_supported(P) && P.dtype == DCN1D_BF16 && P.K == 3 && !P.mask &&
+           P.L_in % 8 == 0;
 }
 
 cudaError_t launch_tc_bf16_stalled(const Problem &P, uint64_t wait_ns, cudaStream_t stream) {

@@ -38,6 +38,14 @@ CASES = [
      True, True, False),
     ("tc_k3_cout_512_two_blocks", "tcgen05_bf16", "bf16", 1, 64, 512, 3, 264, 1, 1, 1, 1, 1,
      False, True, False),
+    ("tc_k16_d3_constrained", "tcgen05_bf16", "bf16", 2, 64, 128, 16, 128, 1, 0, 3, 1, 1,
+     False, False, False),
+    ("tc_k16_mask_og2_unconstrained", "tcgen05_bf16", "bf16", 2, 64, 64, 16, 200, 1, 8, 2, 1,
+     2, True, True, False),
+    ("tc_k5_mask_copy_mode_lin300", "tcgen05_bf16", "bf16", 2, 64, 128, 5, 300, 1, 2, 1, 1,
+     2, True, True, False),
+    ("tc_k9_strided_copy_mode_lin330", "tcgen05_bf16", "bf16", 1, 64, 128, 9, 330, 2, 4, 2, 1,
+     1, False, False, False),
     ("tf32_k16_d3_constrained", "tcgen05_3xtf32", "f32", 2, 32, 512, 16, 128, 1, 0, 3, 1, 1,
      False, False, False),
     ("tf32_k4_strided_groups_mask_unconstrained", "tcgen05_3xtf32", "f32", 2, 64, 128, 4, 160,

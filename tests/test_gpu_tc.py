@@ -23,6 +23,16 @@ CASES = [
     # more than 256 output channels per conv group: blocks of 256, and of 192
     ("cout_512_two_blocks", 2, 128, 512, 5, 256, 1, 2, 1, 1, 4, True, False, 3.0),
     ("g2_cout_g384_blocks_of_192", 1, 128, 768, 3, 200, 1, 1, 1, 2, 2, False, True, 2.0),
+    # the dc1d page's usage layer (kernel 16, dilation 3) in bf16: narrower, then its own
+    # 512 channels; tap positions of wide kernels live in shared memory
+    ("k16_d3_usage_like", 2, 128, 128, 16, 128, 1, 0, 3, 1, 1, False, False, 1.5),
+    ("k16_d3_usage_channels", 1, 512, 512, 16, 128, 1, 0, 3, 1, 1, False, False, 1.5),
+    ("k16_mask_og2_unc_far", 2, 64, 64, 16, 200, 1, 8, 2, 1, 2, True, True, 40.0),
+    # L_in not a multiple of 8: x windows by the loader's 4-byte copies (one box, two
+    # boxes, taps past the window)
+    ("lin300_copy_k5_mask", 2, 128, 128, 5, 300, 1, 2, 1, 1, 4, True, False, 3.0),
+    ("lin330_copy_k9_strided_two_boxes", 2, 128, 128, 9, 330, 2, 4, 2, 2, 2, False, True, 2.0),
+    ("lin202_copy_far_offsets", 3, 64, 64, 3, 202, 1, 1, 1, 1, 1, False, True, 80.0),
 ]
 
 
