@@ -220,11 +220,11 @@ def dcn1d_forward(x, offsets, mask, weight, bias, stride=1, padding=0, dilation=
     x [B, C_in, L_in]; offsets and mask [B, offset_groups, L_out, K] (mask may be None);
     weight [C_out, C_in/groups, K]; bias [C_out] or None.  All CUDA, contiguous, one dtype
     (float32, bfloat16 or float16).  ``padding``: an int, a (left, right) pair, "valid" or "same"
-    (see resolve_padding).  ``out`` is allocated with torch when not given.  The scratch the
-    fastest path needs (``dcn1d_forward_workspace_size``) is allocated with torch unless a
-    uint8 CUDA tensor ``workspace`` is given; ``workspace=False`` asks for the path without
-    scratch.  Without ``workspace`` the scratch is kept for later calls on the same device
-    and stream (see clear_workspace_cache).  Runs on ``stream`` (default: the current torch
+    (see resolve_padding).  ``out`` is allocated with torch when not given.  Scratch that a
+    path needs (``dcn1d_forward_workspace_size``; no present path needs any) is allocated
+    with torch unless a uint8 CUDA tensor ``workspace`` is given; ``workspace=False`` passes
+    none.  Without ``workspace`` such scratch is kept for later calls on the same device and
+    stream (see clear_workspace_cache).  Runs on ``stream`` (default: the current torch
     stream of x's device); does not synchronise.
     """
     pl, pr = resolve_padding(padding, weight.shape[2], stride, dilation)

@@ -50,24 +50,20 @@ enum Kernel { kDirect = 0, kDepthwise = 1, kTcBf16 = 2, kTcTf32 = 3 };
 
 const char *kernel_names[] = {"direct", "depthwise", "tcgen05_bf16", "tcgen05_3xtf32"};
 
-// The fastest kernel for P, given `ws_bytes` of caller workspace (SIZE_MAX: any amount).
-Kernel select_kernel(const Problem &P, size_t ws_bytes) {
+// The fastest kernel for P.  No forward kernel needs workspace; the workspace forms of
+// the entry points accept (and ignore) one, so that callers sized for a path that might
+// need scratch keep working.
+Kernel select_kernel(const Problem &P, size_t /*ws_bytes*/) {
     if (depthwise_supported(P))
         return kDepthwise;
     if (tc_bf16_supported(P))
         return kTcBf16;
-    if (tc_tf32_supported(P) && ws_bytes >= tc_tf32_workspace(P))
+    if (tc_tf32_supported(P))
         return kTcTf32;
     return kDirect;
 }
 
-size_t workspace_bytes(const Problem &P) {
-    if (depthwise_supported(P) || tc_bf16_supported(P))
-        return 0;
-    if (tc_tf32_supported(P))
-        return tc_tf32_workspace(P);
-    return 0;
-}
+size_t workspace_bytes(const Problem & /*P*/) { return 0; }
 
 // Full validation; fills P and the chosen kernel on success.
 int validate(const dcn1d_tensor *x, const dcn1d_tensor *off, const dcn1d_tensor *mask,
@@ -220,8 +216,7 @@ cudaError_t run_forward(const Problem &P, void *workspace, size_t ws_bytes, cuda
         err = launch_tc_bf16(P, s);
         break;
     case kTcTf32:
-        err = launch_tc_tf32(P, workspace, s);
-        *launches = tc_tf32_launches(P);
+        err = launch_tc_tf32(P, s);
         break;
     }
     return err;

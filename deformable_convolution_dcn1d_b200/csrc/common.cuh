@@ -61,9 +61,9 @@ cudaError_t launch_depthwise(const Problem &P, cudaStream_t stream);
 unsigned int *device_status_ptr();
 cudaError_t read_and_clear_device_status(unsigned int *word);
 bool tc_tf32_supported(const Problem &P);
-size_t tc_tf32_workspace(const Problem &P);
-int tc_tf32_launches(const Problem &P);
-cudaError_t launch_tc_tf32(const Problem &P, void *workspace, cudaStream_t stream);
+// One launch, no workspace; split-K problems run as clusters of tc_tf32_splits(P) CTAs.
+int tc_tf32_splits(const Problem &P);
+cudaError_t launch_tc_tf32(const Problem &P, cudaStream_t stream);
 bool tc_bf16_supported(const Problem &P);
 cudaError_t launch_tc_bf16(const Problem &P, cudaStream_t stream);
 // Test of the failure path: the tensor-core kernel with its loader switched off at

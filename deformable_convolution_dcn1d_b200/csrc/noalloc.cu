@@ -3,12 +3,13 @@
 // as a real-time loop that must not allocate, an embedding runtime that owns
 // every allocation, or a host that reserved all device memory up front.
 //
-// The fastest fp32 path needs scratch (the weight split into tf32 high and low
-// parts, and the per-split partial sums).  Here that scratch is a file-scope
-// device array of fixed size; the kernels receive its device address.  Host
-// code must not pass the array's name itself to a kernel: on the host it is a
-// stand-in symbol, not a device address, so the address is looked up once per
-// device with cudaGetSymbolAddress.
+// A path that needs scratch gets it here from a file-scope device array of fixed
+// size; the kernels receive its device address.  (No forward path needs scratch at
+// present -- the fp32 tensor-core path forms the weight's low tf32 part in shared
+// memory and adds its split-K partial sums on chip -- so every valid call runs as
+// dcn1d_forward without touching the array.)  Host code must not pass the array's
+// name itself to a kernel: on the host it is a stand-in symbol, not a device
+// address, so the address is looked up once per device with cudaGetSymbolAddress.
 #include <mutex>
 
 #include "sm100.cuh"

@@ -8,16 +8,21 @@
 // and the MMA accumulates hi*hi + hi*lo + lo*hi in fp32; the dropped lo*lo
 // term is about 2^-22 of the product.
 //
-//  * A one-pass kernel writes W_lo to the workspace; W itself serves as W_hi,
-//    since the tf32 MMA ignores the low 13 mantissa bits of an fp32 operand.
-//  * The main kernel has the bf16 kernel's roles: a TMA warp loads the W and
-//    W_lo tiles (128-byte swizzle) and the fp32 x window of each 32-wide
-//    k-block; 16 producer warps interpolate 16 columns each in fp32 and write
-//    their hi and lo parts straight into tensor memory (A operand); one thread
-//    issues 3 tcgen05.mma kind::tf32 per 8-wide k step; the producers drain D.
-//  * Small-N, large-K problems are split along the reduction (split-K) across
-//    CTAs; each split writes fp32 partial sums to the workspace and a third
-//    kernel adds them in a fixed order, plus the bias -- deterministic.
+// One launch, no workspace:
+//  * the bf16 kernel's roles: a TMA warp loads the W tile (128-byte swizzle) and
+//    the fp32 x window of each 32-wide k-block; W itself serves as W_hi, since the
+//    tf32 MMA ignores the low 13 mantissa bits of an fp32 operand.  The 8 producer
+//    warps that consume a stage first write W_lo = W - W_hi of an eighth of its W
+//    tile next to it (a second shared-memory tile, read by the MMA), then
+//    interpolate 16 columns each in fp32 and write their hi and lo parts straight
+//    into tensor memory (A operand); one thread issues 3 tcgen05.mma kind::tf32 per
+//    8-wide k step; the producers drain D.
+//  * Small-N, large-K problems are split along the reduction (split-K) across the
+//    CTAs of a thread-block cluster, one split per CTA.  When every split's D is
+//    complete, each CTA sends 16-column chunks of it through distributed shared
+//    memory to the chunk's owner CTA (its stage memory, free by then), which adds the
+//    splits in rank order plus the bias and stores the outputs -- deterministic,
+//    and the same sums in the same order as adding per-split partial tensors.
 #include <string.h>
 
 #include "common.cuh"
@@ -46,13 +51,16 @@ constexpr uint32_t kColA = 256;    // A stage s: hi [256 + 64 s, +32), lo [256 +
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kTf32Mask = 0xFFFFE000u;
 
+constexpr int kMaxSplits = 8;      // portable cluster size
+
 struct TfArgs {
     Problem P;
     int N;              // MMA N = output channels per block (multiple of 32, <= 256)
     int n_cob;          // channel blocks per conv group
     int num_kb;         // k-blocks of the whole reduction
     int kb_per_split;   // k-blocks per split
-    int splits;
+    int splits;         // > 1: cluster launch, one split per CTA of a cluster
+    int n_own;          // 16-column chunks of a tile each cluster CTA owns (at most)
     int flat;           // 1: tiles run over the flattened positions n = b * L_out + l
                         // 0: tiles stay inside one batch row (tiles_l per row)
     int tiles_l;
@@ -63,13 +71,13 @@ struct TfArgs {
     uint32_t w_stage_bytes, x_stage_bytes, x_box_bytes, x_slot_bytes;
     uint32_t off_w, off_wlo, off_x, off_bias, off_bar;
     unsigned int *status;
-    float *partial;     // [splits][B][C_out][L_out] when splits > 1
 };
 
 // A unit of work: one split of the reduction for one tile of up to 128
 // consecutive flattened output positions n = b * L_out + l in [nbase, n_end)
 // and one block of N output channels of conv group g.  A flat tile may span
-// several batch rows b_first ..; "slot" j is batch row b_first + j.
+// several batch rows b_first ..; "slot" j is batch row b_first + j.  The split is
+// the fastest-running index, so a cluster's CTAs hold the splits of one tile.
 struct Unit {
     int split, g, cob, nbase, n_end, b_first, nslots, kb0, kb1;
 };
@@ -78,12 +86,12 @@ __device__ __forceinline__ int floor8(int w) { return (w >= 0) ? (w / 8) * 8 : -
 
 __device__ __forceinline__ Unit decode_unit(const TfArgs &A, int u) {
     Unit r;
-    const int nt = u % A.n_tiles;
-    int t = u / A.n_tiles;
+    r.split = u % A.splits;
+    int t = u / A.splits;
+    const int nt = t % A.n_tiles;
+    t /= A.n_tiles;
     r.cob = t % A.n_cob;
-    t /= A.n_cob;
-    r.g = t % A.P.groups;
-    r.split = t / A.P.groups;
+    r.g = t / A.n_cob;
     if (A.flat) {
         r.nbase = nt * kRows;
         r.n_end = min(r.nbase + kRows, A.P.B * A.P.L_out);
@@ -111,6 +119,25 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
     float v;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
     return v;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// v - (v with its low 13 mantissa bits cleared), as bits: the operand's tf32 low part.
+__device__ __forceinline__ uint32_t lo_bits(uint32_t v) {
+    return __float_as_uint(__fsub_rn(__uint_as_float(v), __uint_as_float(v & kTf32Mask)));
 }
 
 // D[tmem] (+)= A[tmem] * B[smem desc], kind::tf32.
@@ -222,7 +249,6 @@ __device__ __forceinline__ void produce_dispatch(int k0, uint32_t tmem_hi, uint3
 template <int K, bool MASK>
 __global__ void __maxnreg__(96)
     tc_tf32_kernel(const __grid_constant__ TfArgs A, const __grid_constant__ CUtensorMap whimap,
-                   const __grid_constant__ CUtensorMap wlomap,
                    const __grid_constant__ CUtensorMap xmap) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const Problem &P = A.P;
@@ -266,7 +292,6 @@ __global__ void __maxnreg__(96)
     }
     if (warp == kTmaWarp && lane == 0) {
         tma_prefetch_desc(&whimap);
-        tma_prefetch_desc(&wlomap);
         tma_prefetch_desc(&xmap);
     }
     __syncthreads();
@@ -281,7 +306,7 @@ __global__ void __maxnreg__(96)
             for (int u = blockIdx.x; u < A.num_units; u += gridDim.x) {
                 const Unit U = decode_unit(A, u);
                 const int corow = U.g * P.cout_g + U.cob * A.N;
-                const uint32_t tx = 2 * A.w_stage_bytes + (uint32_t)U.nslots * A.x_slot_bytes;
+                const uint32_t tx = A.w_stage_bytes + (uint32_t)U.nslots * A.x_slot_bytes;
                 for (int kb = U.kb0; kb < U.kb1; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
@@ -289,7 +314,6 @@ __global__ void __maxnreg__(96)
                         goto tma_done;
                     mbar_arrive_expect_tx(bar_full(s), tx);
                     tma_load_2d(w_st0 + s * A.w_stage_bytes, &whimap, kb * kBK, corow, bar_full(s));
-                    tma_load_2d(wlo_st0 + s * A.w_stage_bytes, &wlomap, kb * kBK, corow, bar_full(s));
                     const int c_lo = (kb * kBK) / K;
                     for (int j = 0; j < U.nslots; ++j) {   // one window per batch row of the tile
                         const int xrow = (U.b_first + j) * P.C_in + U.g * P.cin_g + c_lo;
@@ -368,15 +392,7 @@ __global__ void __maxnreg__(96)
             if (!__all_sync(0xffffffffu, wait(bar_dfull, tcnt & 1u)))
                 return false;
             tc_fence_after();
-            float *dst;
-            bool add_bias;
-            if (A.splits > 1) {
-                dst = A.partial + ((((int64_t)U.split * P.B + b) * P.C_out + co0) * P.L_out + l);
-                add_bias = false;
-            } else {
-                dst = static_cast<float *>(P.out) + (((int64_t)b * P.C_out + co0) * P.L_out + l);
-                add_bias = true;
-            }
+            float *dst = static_cast<float *>(P.out) + (((int64_t)b * P.C_out + co0) * P.L_out + l);
             for (int cc = h; cc < A.N / 16; cc += 4) {
                 uint32_t v[16];
                 tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + kColD + 16u * cc, v);
@@ -385,8 +401,8 @@ __global__ void __maxnreg__(96)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int co = 16 * cc + i;
-                        const float bv = add_bias ? bias_s[co0 + co] : 0.0f;
-                        dst[(int64_t)co * P.L_out] = __fadd_rn(__uint_as_float(v[i]), bv);
+                        dst[(int64_t)co * P.L_out] =
+                            __fadd_rn(__uint_as_float(v[i]), bias_s[co0 + co]);
                     }
                 }
             }
@@ -397,7 +413,9 @@ __global__ void __maxnreg__(96)
             return true;
         };
 
-        // Offsets (and mask) of the next (unit, offset group), loaded one group ahead.
+        // Offsets (and mask) of the next (unit, offset group), loaded one group ahead
+        // (past K = 7: when needed, to keep the registers).
+        constexpr bool kAhead = K <= 7;
         float raw_off[K], raw_m[K];
         int pf_u = -1, pf_og = -1;
         auto prefetch = [&](int u, const Unit &U, int og) {
@@ -418,7 +436,7 @@ __global__ void __maxnreg__(96)
         auto og_of = [&](const Unit &U, int kb) {
             return (U.g * P.cin_g + (kb * kBK) / K) / P.cin_per_og;
         };
-        if ((int)blockIdx.x < A.num_units) {
+        if (kAhead && (int)blockIdx.x < A.num_units) {
             const Unit U0 = decode_unit(A, blockIdx.x);
             prefetch(blockIdx.x, U0, og_of(U0, U0.kb0));
         }
@@ -485,15 +503,35 @@ __global__ void __maxnreg__(96)
                             tp.slow &= ~(1u << k);
                         }
                     }
-                    if (og < og_last) {
-                        prefetch(u, U, og + 1);
-                    } else if (u_next < A.num_units) {
-                        const Unit Un = decode_unit(A, u_next);
-                        prefetch(u_next, Un, og_of(Un, Un.kb0));
+                    if constexpr (kAhead) {
+                        if (og < og_last) {
+                            prefetch(u, U, og + 1);
+                        } else if (u_next < A.num_units) {
+                            const Unit Un = decode_unit(A, u_next);
+                            prefetch(u_next, Un, og_of(Un, Un.kb0));
+                        }
                     }
                 }
                 if (!__all_sync(0xffffffffu, wait(bar_full(s), ph)))
                     goto prod_done;
+                {
+                    // this warp's eighth of the stage's W_lo tile (any layout: elementwise);
+                    // the proxy fence orders it before the tensor core's reads, which
+                    // follow this warp's arrival on the stage's A barrier
+                    const uint32_t share = A.w_stage_bytes / 8u;
+                    const uint32_t w0 = (uint32_t)(2 * q + half) * share;
+                    const uint32_t whi_s = w_st0 + s * A.w_stage_bytes;
+                    const uint32_t wlo_s = wlo_st0 + s * A.w_stage_bytes;
+                    for (uint32_t o = w0 + 16u * lane; o < w0 + share; o += 512u) {
+                        uint4 v = lds_v4(whi_s + o);
+                        v.x = lo_bits(v.x);
+                        v.y = lo_bits(v.y);
+                        v.z = lo_bits(v.z);
+                        v.w = lo_bits(v.w);
+                        sts_v4(wlo_s + o, v);
+                    }
+                    fence_proxy_async_smem();
+                }
                 {
                     const uint32_t xrow_addr =
                         x_st0 + s * A.x_stage_bytes + (uint32_t)(c_first - c_lo) * kRowBytes;
@@ -530,9 +568,95 @@ __global__ void __maxnreg__(96)
             pend_cnt = ucount++;
             it_base += (uint32_t)nkb;
         }
-        if (pend_u >= 0)
+        if (pend_u >= 0 && A.splits == 1)
             epilogue(pend_u, pend_cnt);
     prod_done:;
+    }
+
+    if (A.splits > 1) {
+        // ------------------------------------------------------------ split-K reduction
+        // One unit per CTA.  Chunk c (16 accumulator columns) of the tile belongs to
+        // cluster rank c % S and lands in its receive area at slot [this rank][c / S]
+        // as [128 rows][16 columns] fp32, over the owner's stage memory; the four
+        // 16-byte column groups of row r sit in the order g ^ ((r >> 1) & 3), so the
+        // 16-byte accesses of eight consecutive rows cover all 32 banks.
+        const int S = A.splits;
+        const uint32_t rank = cluster_ctarank();
+        const int nchunk = A.N / 16;
+        const uint32_t slot_bytes = (uint32_t)A.n_own * 16u * 128u * 4u;
+        bool have_d = false;
+        if (warp < kProdWarps && (int)blockIdx.x < A.num_units) {
+            have_d = __all_sync(0xffffffffu, wait(bar_dfull, 0));
+            tc_fence_after();
+        }
+        // 1: every CTA's accumulator is complete and its stage memory idle (loads
+        //    landed, MMAs done)
+        cluster_barrier();
+        const int q = warp % 4, h = warp / 4, row = 32 * q + lane;
+        if (warp < kProdWarps && have_d) {
+            for (int c = h; c < nchunk; c += 4) {
+                uint32_t v[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + kColD + 16u * c, v);
+                tmem_wait_ld();
+                const uint32_t owner = (uint32_t)(c % S);
+                const uint32_t local = sbase + rank * slot_bytes +
+                                       (uint32_t)(c / S) * (16u * 128u * 4u) + 64u * row;
+                const uint32_t sw = ((uint32_t)row >> 1) & 3u;
+                if (owner == rank) {   // this CTA's own chunks stay local
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        sts_v4(local + 16u * ((uint32_t)g ^ sw),
+                               make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]));
+                } else {
+                    const uint32_t remote = cluster_map(local, owner);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        st_cluster_v4(remote + 16u * ((uint32_t)g ^ sw), v[4 * g], v[4 * g + 1],
+                                      v[4 * g + 2], v[4 * g + 3]);
+                }
+            }
+        }
+        // 2: every chunk has reached its owner
+        cluster_barrier();
+        if (warp < kProdWarps && have_d) {
+            const Unit U = decode_unit(A, blockIdx.x);
+            const int n = U.nbase + row;
+            const bool valid = n < U.n_end;
+            const int b = valid ? n / P.L_out : 0;
+            const int l = valid ? n - b * P.L_out : 0;
+            const int co0 = U.g * P.cout_g + U.cob * A.N;
+            float *dst = static_cast<float *>(P.out) + (((int64_t)b * P.C_out + co0) * P.L_out + l);
+            const uint32_t sw = ((uint32_t)row >> 1) & 3u;
+            for (int lc = h; lc < A.n_own; lc += 4) {   // owned chunks over the 4 warps
+                const int c = lc * S + (int)rank;
+                if (c >= nchunk)
+                    break;
+                const uint32_t a = sbase + (uint32_t)lc * (16u * 128u * 4u) + 64u * row;
+                float acc[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    acc[i] = 0.0f;
+                for (int sp = 0; sp < S; ++sp) {   // splits in rank order
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const uint4 p = lds_v4(a + (uint32_t)sp * slot_bytes +
+                                               16u * ((uint32_t)g ^ sw));
+                        acc[4 * g] = __fadd_rn(acc[4 * g], __uint_as_float(p.x));
+                        acc[4 * g + 1] = __fadd_rn(acc[4 * g + 1], __uint_as_float(p.y));
+                        acc[4 * g + 2] = __fadd_rn(acc[4 * g + 2], __uint_as_float(p.z));
+                        acc[4 * g + 3] = __fadd_rn(acc[4 * g + 3], __uint_as_float(p.w));
+                    }
+                }
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int co = 16 * c + i;
+                        const float r = P.bias ? __fadd_rn(acc[i], bias_s[co0 + co]) : acc[i];
+                        dst[(int64_t)co * P.L_out] = r;
+                    }
+                }
+            }
+        }
     }
 
     tc_fence_before();
@@ -544,91 +668,10 @@ __global__ void __maxnreg__(96)
     }
 }
 
-// W_lo = W - W_hi, W_hi = W with the low 13 mantissa bits cleared (a tf32 value).
-// W_hi itself is never stored: tcgen05.mma kind::tf32 ignores the low 13 mantissa
-// bits of an fp32 operand (its results on W are bit-identical to those on W_hi), so
-// the main kernel reads W as the high part.
-// 16-byte accesses, four in flight per thread (n4 = element count / 4).
-__device__ __forceinline__ float lo_part(float v) {
-    return __fsub_rn(v, __uint_as_float(__float_as_uint(v) & kTf32Mask));
-}
-
-__global__ void __launch_bounds__(256) split_tf32_kernel(const float4 *w, float4 *lo, int64_t n4) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += 4 * stride) {
-        float4 v[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (i + j * stride < n4)
-                v[j] = w[i + j * stride];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (i + j * stride < n4)
-                lo[i + j * stride] =
-                    make_float4(lo_part(v[j].x), lo_part(v[j].y), lo_part(v[j].z), lo_part(v[j].w));
-    }
-}
-
-// out[b, co, l] = bias[co] + sum over splits of the partial sums, in split order.
-__global__ void __launch_bounds__(256) reduce_splits_kernel(const float *partial, const float *bias,
-                                                            float *out, int splits, int C_out,
-                                                            int L_out, int64_t n) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        float acc = 0.0f;
-        for (int s = 0; s < splits; ++s)
-            acc = __fadd_rn(acc, partial[(int64_t)s * n + i]);
-        if (bias)
-            acc = __fadd_rn(acc, bias[(i / L_out) % C_out]);
-        out[i] = acc;
-    }
-}
-
-// The same sums four outputs at a time with 16-byte accesses (n % 4 == 0, out 16-byte
-// aligned, L_out >= 4 so that four consecutive outputs span at most two channels).
-__global__ void __launch_bounds__(256) reduce_splits_kernel4(const float4 *partial,
-                                                             const float *bias, float4 *out,
-                                                             int splits, int C_out, int L_out,
-                                                             int64_t n4) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 4
-        for (int s = 0; s < splits; ++s) {
-            const float4 p = partial[(int64_t)s * n4 + i];
-            acc.x = __fadd_rn(acc.x, p.x);
-            acc.y = __fadd_rn(acc.y, p.y);
-            acc.z = __fadd_rn(acc.z, p.z);
-            acc.w = __fadd_rn(acc.w, p.w);
-        }
-        if (bias) {
-            const int64_t row = (4 * i) / L_out;        // (b, co) row of the first output
-            const int l = (int)(4 * i - row * L_out);
-            const int co = (int)(row % C_out);
-            const int co_next = co + 1 == C_out ? 0 : co + 1;
-            const float b0 = bias[co], b1 = bias[co_next];
-            acc.x = __fadd_rn(acc.x, b0);
-            acc.y = __fadd_rn(acc.y, l + 1 < L_out ? b0 : b1);
-            acc.z = __fadd_rn(acc.z, l + 2 < L_out ? b0 : b1);
-            acc.w = __fadd_rn(acc.w, l + 3 < L_out ? b0 : b1);
-        }
-        out[i] = acc;
-    }
-}
-
 struct TfPlan {
     TfArgs A;
     size_t smem;
-    size_t ws_wlo, ws_partial, ws_total;   // workspace layout (bytes)
 };
-
-size_t align256(size_t x) { return (x + 255) / 256 * 256; }
-
-// Grid of a grid-stride elementwise kernel of 256-thread blocks over n elements.
-unsigned grid_for(int64_t n, int sms) {
-    const int64_t want = (n + 255) / 256, cap = 8LL * sms;
-    return (unsigned)(want < cap ? want : cap);
-}
 
 // Shared-memory layout of A for the given tile mode; false if it does not fit.
 bool layout_tf(const Problem &P, TfArgs &A, size_t *smem_out) {
@@ -660,14 +703,13 @@ bool layout_tf(const Problem &P, TfArgs &A, size_t *smem_out) {
     return true;
 }
 
-bool make_tf_plan(const Problem &P, TfPlan *out) {
+// The plan for blocks of N output channels; false if it does not fit.
+bool plan_for_n(const Problem &P, int N, TfPlan *out) {
     TfArgs A;
     memset(&A, 0, sizeof(A));
     A.P = P;
     const int Kg = P.cin_g * P.K;
-    if ((int64_t)P.B * P.L_out + kRows > INT32_MAX || (int64_t)P.B * P.C_in > INT32_MAX)
-        return false;   // flattened position and TMA row indices are 32-bit
-    A.N = P.cout_g < 256 ? P.cout_g : 256;
+    A.N = N;
     if (P.cout_g % A.N != 0)
         return false;
     A.n_cob = P.cout_g / A.N;
@@ -693,38 +735,44 @@ bool make_tf_plan(const Problem &P, TfPlan *out) {
     const int max_splits = A.num_kb / 8 > 0 ? A.num_kb / 8 : 1;   // at least 8 k-blocks a split
     if (splits > max_splits)
         splits = max_splits;
+    if (splits > kMaxSplits)
+        splits = kMaxSplits;
     if (splits < 1)
         splits = 1;
-    A.kb_per_split = (A.num_kb + splits - 1) / splits;
-    A.splits = (A.num_kb + A.kb_per_split - 1) / A.kb_per_split;
+    // The splits' partial sums meet in the owners' stage memory: S slots of the owned
+    // chunks' [128][16] fp32 blocks must fit below the bias.
+    const int nchunk = A.N / 16;
+    for (;; --splits) {
+        A.kb_per_split = (A.num_kb + splits - 1) / splits;
+        A.splits = (A.num_kb + A.kb_per_split - 1) / A.kb_per_split;
+        A.n_own = (nchunk + A.splits - 1) / A.splits;
+        if (A.splits == 1 || (size_t)A.splits * A.n_own * 16 * 128 * 4 <= A.off_bias)
+            break;
+    }
     A.num_units = A.splits * base_units;
-    TfPlan pl;
-    pl.A = A;
-    pl.smem = smem;
-    const size_t wbytes = (size_t)P.C_out * Kg * 4;
-    pl.ws_wlo = 0;
-    pl.ws_partial = align256(wbytes);
-    pl.ws_total = pl.ws_partial +
-                  (A.splits > 1 ? align256((size_t)A.splits * P.B * P.C_out * P.L_out * 4) : 0);
-    *out = pl;
+    out->A = A;
+    out->smem = smem;
     return true;
 }
 
+bool make_tf_plan(const Problem &P, TfPlan *out) {
+    if ((int64_t)P.B * P.L_out + kRows > INT32_MAX || (int64_t)P.B * P.C_in > INT32_MAX)
+        return false;   // flattened position and TMA row indices are 32-bit
+    // (128-channel blocks, halving the reduction's volume where the reduction splits,
+    // measured slower: the producers then pace the contraction)
+    return plan_for_n(P, P.cout_g < 256 ? P.cout_g : 256, out);
+}
+
 template <int K, bool MASK>
-cudaError_t launch_tf_km(const TfPlan &pl, void *ws, cudaStream_t stream) {
+cudaError_t launch_tf_km(const TfPlan &pl, cudaStream_t stream) {
     const Problem &P = pl.A.P;
     TfArgs A = pl.A;
     A.status = device_status_ptr();
     if (!A.status)
         return cudaErrorInvalidDevice;
-    unsigned char *wsb = static_cast<unsigned char *>(ws);
-    float *wlo = reinterpret_cast<float *>(wsb + pl.ws_wlo);
-    A.partial = A.splits > 1 ? reinterpret_cast<float *>(wsb + pl.ws_partial) : nullptr;
     const int Kg = P.cin_g * P.K;
-    alignas(64) CUtensorMap mhi, mlo, mx;
+    alignas(64) CUtensorMap mhi, mx;
     if (!encode_2d(&mhi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, P.w, (uint64_t)Kg, (uint64_t)P.C_out, 4,
-                   kBK, (uint32_t)A.N, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&mlo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, wlo, (uint64_t)Kg, (uint64_t)P.C_out, 4,
                    kBK, (uint32_t)A.N, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, P.x, (uint64_t)P.L_in,
                    (uint64_t)P.B * P.C_in, 4, kBox, (uint32_t)A.nch, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -732,39 +780,35 @@ cudaError_t launch_tf_km(const TfPlan &pl, void *ws, cudaStream_t stream) {
     const int sms = sm_count();
     if (sms <= 0)
         return cudaErrorNoDevice;
-    const int64_t nw4 = (int64_t)P.C_out * Kg / 4;   // Kg is a multiple of 32
-    split_tf32_kernel<<<(unsigned)grid_for((nw4 + 3) / 4, sms), 256, 0, stream>>>(
-        static_cast<const float4 *>(P.w), reinterpret_cast<float4 *>(wlo), nw4);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess)
-        return e;
     auto kern = tc_tf32_kernel<K, MASK>;
-    e = ensure_smem(reinterpret_cast<const void *>(kern), (int)pl.smem);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), (int)pl.smem);
     if (e != cudaSuccess)
         return e;
-    const int grid = A.num_units < sms ? A.num_units : sms;
+    // split-K: one unit per CTA, the splits of a tile a cluster (units <= SMs by the plan)
+    const int grid = A.splits > 1 ? A.num_units : (A.num_units < sms ? A.num_units : sms);
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)A.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     timing_begin(stream);
-    kern<<<grid, kThreads, pl.smem, stream>>>(A, mhi, mlo, mx);
+    e = cudaLaunchKernelEx(&cfg, kern, A, mhi, mx);
     timing_end(stream);
-    e = cudaGetLastError();
-    if (e != cudaSuccess || A.splits == 1)
+    if (e != cudaSuccess)
         return e;
-    const int64_t n = (int64_t)P.B * P.C_out * P.L_out;
-    if (n % 4 == 0 && P.L_out >= 4 && (reinterpret_cast<uintptr_t>(P.out) & 15) == 0)
-        reduce_splits_kernel4<<<(unsigned)grid_for(n / 4, sms), 256, 0, stream>>>(
-            reinterpret_cast<const float4 *>(A.partial), static_cast<const float *>(P.bias),
-            static_cast<float4 *>(P.out), A.splits, P.C_out, P.L_out, n / 4);
-    else
-        reduce_splits_kernel<<<(unsigned)grid_for(n, sms), 256, 0, stream>>>(
-            A.partial, static_cast<const float *>(P.bias), static_cast<float *>(P.out), A.splits,
-            P.C_out, P.L_out, n);
     return cudaGetLastError();
 }
 
 template <int K>
-cudaError_t launch_tf_k(const TfPlan &pl, void *ws, cudaStream_t stream) {
-    return pl.A.P.mask ? launch_tf_km<K, true>(pl, ws, stream)
-                       : launch_tf_km<K, false>(pl, ws, stream);
+cudaError_t launch_tf_k(const TfPlan &pl, cudaStream_t stream) {
+    return pl.A.P.mask ? launch_tf_km<K, true>(pl, stream) : launch_tf_km<K, false>(pl, stream);
 }
 
 }  // namespace
@@ -791,25 +835,18 @@ bool tc_tf32_supported(const Problem &P) {
     return make_tf_plan(P, &pl);
 }
 
-size_t tc_tf32_workspace(const Problem &P) {
+int tc_tf32_splits(const Problem &P) {
     TfPlan pl;
-    return make_tf_plan(P, &pl) ? pl.ws_total : 0;
+    return make_tf_plan(P, &pl) ? pl.A.splits : 0;
 }
 
-int tc_tf32_launches(const Problem &P) {
+cudaError_t launch_tc_tf32(const Problem &P, cudaStream_t stream) {
     TfPlan pl;
-    return make_tf_plan(P, &pl) ? (pl.A.splits > 1 ? 3 : 2) : 0;
-}
-
-cudaError_t launch_tc_tf32(const Problem &P, void *workspace, cudaStream_t stream) {
-    TfPlan pl;
-    if (!make_tf_plan(P, &pl) || !workspace)
-        return cudaErrorInvalidValue;
-    if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    if (!make_tf_plan(P, &pl))
         return cudaErrorInvalidValue;
     switch (P.K) {
 #define DCN1D_K(K_) \
-    case K_: return launch_tf_k<K_>(pl, workspace, stream);
+    case K_: return launch_tf_k<K_>(pl, stream);
         DCN1D_K(1) DCN1D_K(2) DCN1D_K(3) DCN1D_K(4) DCN1D_K(5) DCN1D_K(6) DCN1D_K(7) DCN1D_K(8)
         DCN1D_K(9) DCN1D_K(10) DCN1D_K(11) DCN1D_K(12) DCN1D_K(13) DCN1D_K(14) DCN1D_K(15)
         DCN1D_K(16)

@@ -134,15 +134,18 @@ int64_t dcn1d_forward_lr_workspace_size(const dcn1d_tensor *x, const dcn1d_tenso
  *   bias     [C_out] or NULL
  *   out      [B, C_out, L_out]                     required, written entirely
  *
- * All floating tensors share one dtype (F32 or BF16); the arithmetic is fp32
- * (bf16 operands of the tensor-core contraction, fp32 accumulation), and `out`
- * is written in that same dtype ("conv1d" page: the computation stays in the
- * input dtype).  groups must divide C_in and C_out; offset_groups must divide
+ * All floating tensors share one dtype (F32, BF16 or F16), and `out` is
+ * written in that same dtype ("conv1d" page: the computation stays in the
+ * input dtype).  Positions and fractions are fp32 throughout.  F32: fp32
+ * interpolation and an fp32-accurate contraction (three TF32 products).
+ * BF16/F16: fp32 accumulation; the tensor-core path interpolates in 16-bit
+ * pairs (the fraction and x1 - x0 rounded to the dtype, then one fused
+ * multiply-add), the depthwise and generic paths in fp32.  groups must divide C_in and C_out; offset_groups must divide
  * C_in; stride >= 1, padding >= 0, dilation >= 1 ("conv1d" page, "Arguments").
  * `unconstrained` != 0 lets taps sample anywhere (dc1d page, "Usage").
  *
- * Needs no scratch memory: where the fastest path would (see
- * dcn1d_forward_workspace_size), a path without scratch runs instead.
+ * Needs no scratch memory: every path, the fp32 tensor-core one included,
+ * runs as one kernel launch without it.
  *
  * Returns DCN1D_OK, or DCN1D_ERR_NULL / _DTYPE / _SHAPE / _ARG / _UNSUPPORTED on
  * invalid arguments (nothing launched), DCN1D_ERR_LAUNCH if a launch failed.
@@ -153,12 +156,12 @@ int dcn1d_forward(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1
                   int unconstrained, dcn1d_tensor *out, void *stream);
 
 /*
- * Scratch memory (bytes) the fastest path for these arguments needs, or 0 when
- * it needs none; a negative value is minus the status code of invalid
- * arguments.  Host only.  The fp32 tensor-core path needs scratch: the low
- * tf32 part of the weight (C_out * (C_in/groups) * K floats; the weight itself
- * serves as the high part) and, when the reduction is split across CTAs, the
- * fp32 partial sums (splits * B * C_out * L_out floats).
+ * Scratch memory (bytes) the fastest path for these arguments needs: 0 for
+ * every valid argument set (the fp32 tensor-core path forms the weight's low
+ * tf32 part in shared memory and adds its split-K partial sums on chip); a
+ * negative value is minus the status code of invalid arguments.  Host only.
+ * The workspace forms of the entry points keep their signatures, so callers
+ * that size a workspace by this query keep working.
  */
 int64_t dcn1d_forward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *offsets,
                                      const dcn1d_tensor *mask, const dcn1d_tensor *weight,
@@ -170,11 +173,10 @@ int64_t dcn1d_forward_workspace_size(const dcn1d_tensor *x, const dcn1d_tensor *
  * dcn1d_forward with caller-provided scratch: `workspace` is a device buffer
  * of `workspace_bytes` bytes, 256-byte aligned, owned by the caller and used
  * only during the work enqueued on `stream` (calls that overlap on the GPU
- * must use different workspaces).  With at least
- * dcn1d_forward_workspace_size() bytes the fastest path runs; with less (or
- * NULL and 0) the call behaves exactly like dcn1d_forward.  A non-zero size
- * with a NULL pointer is DCN1D_ERR_NULL.  Other arguments and errors as for
- * dcn1d_forward.
+ * must use different workspaces).  No present path reads it
+ * (dcn1d_forward_workspace_size is 0), so the call behaves exactly like
+ * dcn1d_forward.  A non-zero size with a NULL pointer is DCN1D_ERR_NULL.
+ * Other arguments and errors as for dcn1d_forward.
  */
 int dcn1d_forward_ws(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const dcn1d_tensor *mask,
                      const dcn1d_tensor *weight, const dcn1d_tensor *bias, int64_t stride,
@@ -203,7 +205,8 @@ int dcn1d_forward_ws(const dcn1d_tensor *x, const dcn1d_tensor *offsets, const d
  *
  * Scratch limit: arguments whose fastest path needs more than 48 MiB
  * (dcn1d_forward_workspace_size) are rejected with DCN1D_ERR_UNSUPPORTED and
- * nothing is launched.  Arguments that need no scratch run as dcn1d_forward.
+ * nothing is launched.  Arguments that need no scratch run as dcn1d_forward --
+ * at present every valid argument set, since no forward path needs scratch.
  *
  * Sharing: every call on a device uses the same array and it keeps the last
  * call's contents; each call writes every scratch byte it reads, so nothing
@@ -423,8 +426,7 @@ int dcn1d_sample_index(const dcn1d_tensor *offsets, int64_t L_in, int64_t stride
                        float *frac, void *stream);
 
 /*
- * Which kernel dcn1d_forward_ws launches for these arguments when given at
- * least dcn1d_forward_workspace_size() bytes of scratch, as a static string
+ * Which kernel dcn1d_forward launches for these arguments, as a static string
  * ("direct", "depthwise", "tcgen05_bf16", "tcgen05_3xtf32"), or NULL if the
  * arguments are invalid.  Host only; launches nothing.  For tests and
  * benchmarks.

@@ -84,8 +84,12 @@ TF32_CASES = [
     ("short_rows_span_8_batches", 9, 64, 64, 8, 28, 1, 0, 1, 1, 1, True, False, 2.0),
     # two x windows per batch row do not fit beside N = 256 twice: row tiles instead
     ("flat_falls_back_to_rows", 2, 32, 256, 16, 300, 2, 0, 1, 1, 1, False, False, 2.0),
-    # L_out = 1, 16 reduction splits: the split sums take the one-output-at-a-time path
+    # L_out = 1: one tile, its reduction split across a cluster of 8 CTAs
     ("lout_1_scalar_reduce", 2, 256, 64, 16, 16, 1, 0, 1, 1, 1, False, False, 2.0),
+    # 24 and 21 tiles: clusters of 6 and 7 splits, so the 16 column chunks of a tile are
+    # owned unevenly (3 or 2 per CTA)
+    ("split6_uneven_chunk_owners", 37, 96, 256, 16, 128, 1, 0, 3, 1, 1, False, False, 1.5),
+    ("split7_uneven_chunk_owners", 32, 112, 256, 16, 128, 1, 0, 3, 1, 1, True, False, 1.5),
 ]
 
 
@@ -105,18 +109,26 @@ def test_tc_tf32_parity(case):
     assert err <= TOL["f32"], (name, err)
 
 
-def test_tf32_without_workspace_takes_the_direct_path():
-    """dcn1d_forward without scratch runs a path that needs none, with the same result."""
+def test_tf32_is_one_launch_without_workspace():
+    """The fp32 tensor-core path (split-K included) needs no scratch: dcn1d_forward without
+    any workspace runs it as one launch, bit for bit like a call given a workspace."""
     w = W.USAGE_F32.with_batch(2)
     td = to_dev(W.make_inputs(w, seed=2))
-    a = gpu_forward(w, td)
+    assert dcn.dcn1d_forward_workspace_size(td["x"], td["offsets"], td["mask"], td["weight"],
+                                            td["bias"], w.stride, w.padding, w.dilation,
+                                            w.groups, w.offset_groups, w.unconstrained) == 0
+    assert kernel_name(w, td) == "tcgen05_3xtf32"
+    a = dcn.dcn1d_forward(td["x"], td["offsets"], td["mask"], td["weight"], td["bias"],
+                          w.stride, w.padding, w.dilation, w.groups, w.offset_groups,
+                          w.unconstrained, workspace=torch.empty(1 << 20, dtype=torch.uint8,
+                                                                 device="cuda"))
     b = dcn.dcn1d_forward(td["x"], td["offsets"], td["mask"], td["weight"], td["bias"],
                           w.stride, w.padding, w.dilation, w.groups, w.offset_groups,
                           w.unconstrained, workspace=False)
     torch.cuda.synchronize()
     assert dcn.dcn1d_last_launch_count() == 1
-    err = (a.double() - b.double()).abs().max().item() / b.double().abs().max().item()
-    assert err <= 2e-5
+    assert dcn.dcn1d_device_status() == 0
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
 
 
 def test_tf32_deterministic_across_calls():
@@ -126,7 +138,7 @@ def test_tf32_deterministic_across_calls():
     launches = dcn.dcn1d_last_launch_count()
     b = gpu_forward(w, td)
     torch.cuda.synchronize()
-    assert launches >= 2
+    assert launches == 1
     assert torch.equal(a.view(torch.int32), b.view(torch.int32))
 
 
