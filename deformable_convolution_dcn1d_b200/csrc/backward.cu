@@ -141,73 +141,116 @@ __global__ void __launch_bounds__(256) sum_splits_kernel(const float *part, T *o
 struct SampArgs {
     Problem P;
     int nchunk;                  // channel chunks per offset group
+    int nlb;                     // blocks of kSgRows positions per (b, chunk, offset group)
+    int win;                     // shared-memory grad_x window per channel (0: none)
+    int margin;                  // window positions before the first receptive field
     const float *dcols;          // [B][C_in*K][L_out] or NULL
     float *cols;                 // [B][C_in*K][L_out] or NULL
     void *cols16;                // the same columns in the input's 16-bit type, or NULL
     float *gx, *goff, *gmask;    // fp32 scratch, each may be NULL
 };
 
-// Thread = (b, chunk, offset group, k, l), l fastest.
+constexpr int kSgRows = 256;     // output positions per sampling-gradient block
+
+// Block = (kSgRows consecutive positions l, channel chunk, offset group, b); thread = one
+// position, looping over the taps k and the chunk's channels.  The grad_x scatter of all
+// taps of the block's positions goes to a shared-memory window over the chunk's rows
+// ([nc][win] fp32, positions w0 .. w0+win-1); taps outside it (unconstrained offsets past
+// the margin) add to global memory directly, and the window is added to global memory
+// once, element by element, at the end.
 template <class T, bool MASK>
-__global__ void __launch_bounds__(256) sample_grad_kernel(const SampArgs a) {
+__global__ void __launch_bounds__(kSgRows) sample_grad_kernel(const SampArgs a) {
+    extern __shared__ float gxs[];
     const Problem &P = a.P;
-    const int64_t n = (int64_t)P.B * a.nchunk * P.offset_groups * P.K * P.L_out;
-    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= n)
-        return;
-    const int l = (int)(t % P.L_out);
-    int64_t r = t / P.L_out;
-    const int k = (int)(r % P.K);
-    r /= P.K;
-    const int og = (int)(r % P.offset_groups);
-    r /= P.offset_groups;
+    int64_t r = blockIdx.x;
+    const int lb = (int)(r % a.nlb);
+    r /= a.nlb;
     const int chunk = (int)(r % a.nchunk);
-    const int b = (int)(r / a.nchunk);
-
-    const int start = l * P.stride - P.padding;
-    const int64_t oidx = (((int64_t)b * P.offset_groups + og) * P.L_out + l) * P.K + k;
-    const float off = ld_f32(static_cast<const T *>(P.off) + oidx);
-    const float m = MASK ? ld_f32(static_cast<const T *>(P.mask) + oidx) : 1.0f;
-    const int span = P.dilation * (P.K - 1);
-    const float raw = __fadd_rn(__int2float_rn(start + k * P.dilation), off);
-    // The clamp passes the gradient inside its closed range (NaN: no gradient).
-    const bool gate = P.unconstrained ||
-                      (raw >= __int2float_rn(start) && raw <= __int2float_rn(start + span));
-    const Tap tp = sample_tap(start, k, P.dilation, span, off, P.unconstrained);
-    const float mf = __fmul_rn(m, tp.f), m1f = __fmul_rn(m, __fsub_rn(1.0f, tp.f));
-    const bool in0 = tp.i0 >= 0 && tp.i0 < P.L_in;
-    const bool in1 = tp.i0 >= -1 && tp.i0 < P.L_in - 1;
-
+    r /= a.nchunk;
+    const int og = (int)(r % P.offset_groups);
+    const int b = (int)(r / P.offset_groups);
+    const int l0 = lb * kSgRows;
+    const int l = l0 + (int)threadIdx.x;
     const int c_begin = og * P.cin_per_og + chunk * kChunk;
     const int c_end = min(c_begin + kChunk, (og + 1) * P.cin_per_og);
-    float s_off = 0.0f, s_mask = 0.0f;
-    for (int ci = c_begin; ci < c_end; ++ci) {
-        const T *row = static_cast<const T *>(P.x) + ((int64_t)b * P.C_in + ci) * P.L_in;
-        const float x0 = in0 ? ld_f32(row + tp.i0) : 0.0f;
-        const float x1 = in1 ? ld_f32(row + tp.i0 + 1) : 0.0f;
-        const float v = __fadd_rn(__fmul_rn(__fsub_rn(1.0f, tp.f), x0), __fmul_rn(tp.f, x1));
-        const int64_t cidx = (((int64_t)b * P.C_in + ci) * P.K + k) * P.L_out + l;
-        if (a.cols)
-            a.cols[cidx] = __fmul_rn(m, v);
-        if (sizeof(T) == 2 && a.cols16)
-            static_cast<T *>(a.cols16)[cidx] = from_f32<T>(__fmul_rn(m, v));
-        if (a.dcols) {
-            const float dv = a.dcols[cidx];
-            if (a.gx) {
-                float *gxr = a.gx + ((int64_t)b * P.C_in + ci) * P.L_in;
-                if (in0)
-                    atomicAdd(gxr + tp.i0, __fmul_rn(m1f, dv));
-                if (in1)
-                    atomicAdd(gxr + tp.i0 + 1, __fmul_rn(mf, dv));
+    const int nc = c_end - c_begin;
+    const bool window = a.gx && a.dcols && a.win > 0;
+    const int W = a.win;
+    const int w0 = l0 * P.stride - P.padding - a.margin;
+    if (window) {
+        for (int i = threadIdx.x; i < nc * W; i += blockDim.x)
+            gxs[i] = 0.0f;
+        __syncthreads();
+    }
+    if (l < P.L_out) {
+        const int start = l * P.stride - P.padding;
+        const int span = P.dilation * (P.K - 1);
+        for (int k = 0; k < P.K; ++k) {
+            const int64_t oidx = (((int64_t)b * P.offset_groups + og) * P.L_out + l) * P.K + k;
+            const float off = ld_f32(static_cast<const T *>(P.off) + oidx);
+            const float m = MASK ? ld_f32(static_cast<const T *>(P.mask) + oidx) : 1.0f;
+            const float raw = __fadd_rn(__int2float_rn(start + k * P.dilation), off);
+            // The clamp passes the gradient inside its closed range (NaN: no gradient).
+            const bool gate = P.unconstrained ||
+                              (raw >= __int2float_rn(start) && raw <= __int2float_rn(start + span));
+            const Tap tp = sample_tap(start, k, P.dilation, span, off, P.unconstrained);
+            const float mf = __fmul_rn(m, tp.f), m1f = __fmul_rn(m, __fsub_rn(1.0f, tp.f));
+            const bool in0 = tp.i0 >= 0 && tp.i0 < P.L_in;
+            const bool in1 = tp.i0 >= -1 && tp.i0 < P.L_in - 1;
+            // window-relative neighbours (unsigned compares also reject NaN-free far taps)
+            const int r0 = tp.i0 - w0;
+            const bool win0 = window && r0 >= 0 && r0 < W;
+            const bool win1 = window && r0 + 1 >= 0 && r0 + 1 < W;
+            float s_off = 0.0f, s_mask = 0.0f;
+            for (int ci = c_begin; ci < c_end; ++ci) {
+                const T *row = static_cast<const T *>(P.x) + ((int64_t)b * P.C_in + ci) * P.L_in;
+                const float x0 = in0 ? ld_f32(row + tp.i0) : 0.0f;
+                const float x1 = in1 ? ld_f32(row + tp.i0 + 1) : 0.0f;
+                const float v = __fadd_rn(__fmul_rn(__fsub_rn(1.0f, tp.f), x0), __fmul_rn(tp.f, x1));
+                const int64_t cidx = (((int64_t)b * P.C_in + ci) * P.K + k) * P.L_out + l;
+                if (a.cols)
+                    a.cols[cidx] = __fmul_rn(m, v);
+                if (sizeof(T) == 2 && a.cols16)
+                    static_cast<T *>(a.cols16)[cidx] = from_f32<T>(__fmul_rn(m, v));
+                if (a.dcols) {
+                    const float dv = a.dcols[cidx];
+                    if (a.gx) {
+                        float *gxr = a.gx + ((int64_t)b * P.C_in + ci) * P.L_in;
+                        float *wr = gxs + (ci - c_begin) * W;
+                        if (in0) {
+                            if (win0)
+                                atomicAdd(wr + r0, __fmul_rn(m1f, dv));
+                            else
+                                atomicAdd(gxr + tp.i0, __fmul_rn(m1f, dv));
+                        }
+                        if (in1) {
+                            if (win1)
+                                atomicAdd(wr + r0 + 1, __fmul_rn(mf, dv));
+                            else
+                                atomicAdd(gxr + tp.i0 + 1, __fmul_rn(mf, dv));
+                        }
+                    }
+                    s_off = __fmaf_rn(__fmul_rn(m, __fsub_rn(x1, x0)), dv, s_off);
+                    s_mask = __fmaf_rn(v, dv, s_mask);
+                }
             }
-            s_off = __fmaf_rn(__fmul_rn(m, __fsub_rn(x1, x0)), dv, s_off);
-            s_mask = __fmaf_rn(v, dv, s_mask);
+            if (a.dcols && a.goff && gate)
+                atomicAdd(a.goff + oidx, s_off);
+            if (a.dcols && a.gmask)
+                atomicAdd(a.gmask + oidx, s_mask);
         }
     }
-    if (a.goff && gate)
-        atomicAdd(a.goff + oidx, s_off);
-    if (a.gmask)
-        atomicAdd(a.gmask + oidx, s_mask);
+    if (window) {
+        __syncthreads();
+        // untouched (zero) entries add nothing: skipped
+        for (int i = threadIdx.x; i < nc * W; i += blockDim.x) {
+            const int c = i / W, w = i - c * W;
+            const int pos = w0 + w;
+            const float v = gxs[i];
+            if (v != 0.0f && pos >= 0 && pos < P.L_in)
+                atomicAdd(a.gx + ((int64_t)b * P.C_in + c_begin + c) * P.L_in + pos, v);
+        }
+    }
 }
 
 // dst[z][c][r] = src[z][r][c] for z < nz, r < R, c < Cc (16-bit elements): 32 x 32 tiles
@@ -240,9 +283,38 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(const T *gout, T *gbias,
     __shared__ float part[256];
     const int co = blockIdx.x;
     float s = 0.0f;
-    for (int64_t i = threadIdx.x; i < (int64_t)B * L_out; i += blockDim.x) {
-        const int b = (int)(i / L_out), l = (int)(i - (int64_t)b * L_out);
-        s = __fadd_rn(s, ld_f32(gout + ((int64_t)b * C_out + co) * L_out + l));
+    // 16-byte loads where every row allows them (VE elements each), four in flight per
+    // thread; each thread adds its elements in a fixed order
+    constexpr int VE = 16 / (int)sizeof(T);
+    if (L_out % VE == 0 && (reinterpret_cast<uintptr_t>(gout) & 15) == 0) {
+        const int nv = L_out / VE;
+        const int64_t n = (int64_t)B * nv;
+        auto at = [&](int64_t i) {
+            const int b = (int)(i / nv), j = (int)(i - (int64_t)b * nv);
+            return reinterpret_cast<const uint4 *>(gout + ((int64_t)b * C_out + co) * L_out) + j;
+        };
+        auto add = [&](uint4 u) {
+            const T *e = reinterpret_cast<const T *>(&u);
+#pragma unroll
+            for (int q = 0; q < VE; ++q)
+                s = __fadd_rn(s, to_f32(e[q]));
+        };
+        int64_t i = threadIdx.x;
+        for (; i + 3 * (int64_t)blockDim.x < n; i += 4 * (int64_t)blockDim.x) {
+            const uint4 u0 = __ldg(at(i)), u1 = __ldg(at(i + blockDim.x)),
+                        u2 = __ldg(at(i + 2 * blockDim.x)), u3 = __ldg(at(i + 3 * blockDim.x));
+            add(u0);
+            add(u1);
+            add(u2);
+            add(u3);
+        }
+        for (; i < n; i += blockDim.x)
+            add(__ldg(at(i)));
+    } else {
+        for (int64_t i = threadIdx.x; i < (int64_t)B * L_out; i += blockDim.x) {
+            const int b = (int)(i / L_out), l = (int)(i - (int64_t)b * L_out);
+            s = __fadd_rn(s, ld_f32(gout + ((int64_t)b * C_out + co) * L_out + l));
+        }
     }
     part[threadIdx.x] = s;
     __syncthreads();
@@ -257,8 +329,25 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(const T *gout, T *gbias,
 
 template <class T>
 __global__ void __launch_bounds__(256) write_out_kernel(const float *src, T *dst, int64_t n) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x)
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // four elements at a time (a 16-byte load) where both buffers are aligned for it
+    if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
+        (reinterpret_cast<uintptr_t>(dst) & (4 * sizeof(T) - 1)) == 0) {
+        const int64_t n4 = n / 4;
+        for (int64_t i = i0; i < n4; i += stride) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(src) + i);
+            T o[4] = {from_f32<T>(v.x), from_f32<T>(v.y), from_f32<T>(v.z), from_f32<T>(v.w)};
+            if constexpr (sizeof(T) == 2)
+                *reinterpret_cast<uint2 *>(dst + 4 * i) = *reinterpret_cast<const uint2 *>(o);
+            else
+                *reinterpret_cast<float4 *>(dst + 4 * i) = *reinterpret_cast<const float4 *>(o);
+        }
+        for (int64_t i = 4 * n4 + i0; i < n; i += stride)   // the last n % 4 elements
+            dst[i] = from_f32<T>(src[i]);
+        return;
+    }
+    for (int64_t i = i0; i < n; i += stride)
         dst[i] = from_f32<T>(src[i]);
 }
 
@@ -436,20 +525,32 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
         memset(&a, 0, sizeof(a));
         a.P = P;
         a.nchunk = (P.cin_per_og + kChunk - 1) / kChunk;
+        a.nlb = (P.L_out + kSgRows - 1) / kSgRows;
+        // grad_x window: the receptive fields of a block's positions, plus a margin for
+        // unconstrained taps; past 48 KB of shared memory, global atomics only
+        a.margin = P.unconstrained ? 16 : 0;
+        {
+            const int64_t w = (int64_t)(kSgRows - 1) * P.stride +
+                              (int64_t)P.dilation * (P.K - 1) + 2 + 2 * a.margin;
+            a.win = (w * kChunk * 4 <= 48 * 1024) ? (int)w : 0;
+        }
         a.dcols = dcols;
         a.cols = cols;
         a.cols16 = cols16;
         a.gx = gx;
         a.goff = goff;
         a.gmask = gmask;
-        const int64_t nt = (int64_t)P.B * a.nchunk * P.offset_groups * P.K * P.L_out;
-        const unsigned blocks = (unsigned)((nt + 255) / 256);
+        const int64_t nt = (int64_t)P.B * a.nchunk * P.offset_groups * P.L_out;
+        const int64_t blocks = (int64_t)P.B * P.offset_groups * a.nchunk * a.nlb;
+        const size_t shm = (gx && dcols) ? (size_t)a.win * kChunk * 4 : 0;
         if (nt == 0) {
             // empty batch: no columns, no sampling gradient
+        } else if (blocks >= (1LL << 31)) {
+            return cudaErrorInvalidValue;
         } else if (P.mask)
-            sample_grad_kernel<T, true><<<blocks, 256, 0, s>>>(a);
+            sample_grad_kernel<T, true><<<(unsigned)blocks, kSgRows, shm, s>>>(a);
         else
-            sample_grad_kernel<T, false><<<blocks, 256, 0, s>>>(a);
+            sample_grad_kernel<T, false><<<(unsigned)blocks, kSgRows, shm, s>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess)
             return e;
         n += nt > 0;

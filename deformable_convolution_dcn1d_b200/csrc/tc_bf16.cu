@@ -584,6 +584,8 @@ __global__ void __maxnreg__(96)
             // accumulator rows (each depends on its own operand row only) are never stored.
             const int l = T.lbase + row;
             const float start = (float)(l * P.stride - P.padding);
+            const float hi_bound = __fadd_rn(start, spanf);   // the receptive field's end
+            const float dil_f = (float)P.dilation;
             const uint32_t win_bits = kFloorMagicBits + (uint32_t)T.wx0;
             const int pos_first = first_pos(tcount);
             const int pos_last =
@@ -616,11 +618,15 @@ __global__ void __maxnreg__(96)
                         prefetch(t, T, og);   // not predicted: load now
                     float f[K], m[K];
                     tp.slow = 0;
+                    // start + k*d by repeated adds of d: exact (integers below 2^24), the
+                    // same value as the product
+                    float tap_base = start;
 #pragma unroll
                     for (int k = 0; k < K; ++k) {
-                        float pos = __fadd_rn(__fadd_rn(start, (float)(k * P.dilation)), raw_off[k]);
+                        float pos = __fadd_rn(tap_base, raw_off[k]);
+                        tap_base = __fadd_rn(tap_base, dil_f);
                         if (!P.unconstrained)
-                            pos = fminf(fmaxf(pos, start), __fadd_rn(start, spanf));
+                            pos = fminf(fmaxf(pos, start), hi_bound);
                         const float tt = __fadd_rd(pos, M);
                         const uint32_t rel = __float_as_uint(tt) - win_bits;   // i0 - wx0
                         f[k] = __fsub_rn(pos, __fsub_rn(tt, M));
