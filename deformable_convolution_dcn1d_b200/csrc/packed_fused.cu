@@ -84,6 +84,11 @@ struct FElem<__nv_bfloat16> {
     static __device__ __forceinline__ float round(float v) {
         return __bfloat162float(__float2bfloat16_rn(v));
     }
+    // both rounded with one paired conversion (the same value per element)
+    static __device__ __forceinline__ float2 round2(float2 v) {
+        const uint32_t u = pack(v.x, v.y);
+        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+    }
 };
 
 template <>
@@ -101,6 +106,9 @@ struct FElem<__half> {
     }
     static __device__ __forceinline__ float round(float v) {
         return __half2float(__float2half_rn(v));
+    }
+    static __device__ __forceinline__ float2 round2(float2 v) {
+        return __half22float2(__floats2half2_rn(v.x, v.y));
     }
 };
 
@@ -135,9 +143,16 @@ __device__ __forceinline__ int floor8(int w) {
 
 // Shared-memory parameter block (fp32): dw_w [C*K], dw_b [C], w [C*K], bias [C],
 // off_b [J], mask_b [J].
+// The layer's small parameters in shared memory (fp32).  dww [C][K] and dwb, fb [C] in
+// channel order; fw, offb, maskb per channel PAIR and tap, [C/2][K][2], so the drain reads
+// the values of its two channels for one tap with one 8-byte load (pair_at).
 struct Par {
     const float *dww, *dwb, *fw, *fb, *offb, *maskb;
 };
+
+__host__ __device__ __forceinline__ int pair_at(int c, int k, int K) {
+    return ((c >> 1) * K + k) * 2 + (c & 1);
+}
 
 __device__ __forceinline__ Par par_of(const float *base, int C, int K) {
     Par p;
@@ -192,10 +207,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
         const E *mb = static_cast<const E *>(T.mask_b);
         float *w = par_s;   // the layout of par_of
         for (int i = threadIdx.x; i < C * K; i += kFThreads) {
-            w[i] = ld_f32(dww + i);                                   // dw_w
-            w[C * K + C + i] = ld_f32(fw + i);                        // w
-            w[2 * C * K + 2 * C + i] = ob ? ld_f32(ob + i) : 0.0f;    // off_b
-            w[3 * C * K + 2 * C + i] = mb ? ld_f32(mb + i) : 0.0f;    // mask_b
+            const int pi = pair_at(i / K, i % K, K);
+            w[i] = ld_f32(dww + i);                                    // dw_w
+            w[C * K + C + pi] = ld_f32(fw + i);                        // w
+            w[2 * C * K + 2 * C + pi] = ob ? ld_f32(ob + i) : 0.0f;    // off_b
+            w[3 * C * K + 2 * C + pi] = mb ? ld_f32(mb + i) : 0.0f;    // mask_b
         }
         for (int i = threadIdx.x; i < C; i += kFThreads) {
             w[C * K + i] = dwb ? ld_f32(dwb + i) : 0.0f;              // dw_b
@@ -419,22 +435,22 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 for (int ip = 0; ip < kFCw / 2; ++ip) {
                     const int cA = ch0 + 2 * ip, cB = cA + 1;
                     const uint32_t xrA = xbuf + (uint32_t)cA * rowb, xrB = xrA + rowb;
-                    float2 acc = make_float2(p.fb[cA], p.fb[cB]);
+                    float2 acc = *reinterpret_cast<const float2 *>(p.fb + cA);   // cA even
 #pragma unroll
                     for (int k = 0; k < K; ++k) {
                         const int eA = (2 * ip) * K + k, eB = eA + K;   // register indices
+                        const int pk = pair_at(cA, k, K);
                         const float2 z = __fadd2_rn(
                             make_float2(__uint_as_float(vo[eA]), __uint_as_float(vo[eB])),
-                            make_float2(p.offb[cA * K + k], p.offb[cB * K + k]));
-                        const float2 off = make_float2(FElem<E>::round(z.x), FElem<E>::round(z.y));
+                            *reinterpret_cast<const float2 *>(p.offb + pk));
+                        const float2 off = FElem<E>::round2(z);
                         float2 m = make_float2(1.0f, 1.0f);
                         if (MASKHEAD) {
                             const float2 zm = __fadd2_rn(
                                 make_float2(__uint_as_float(vm[MASKHEAD ? eA : 0]),
                                             __uint_as_float(vm[MASKHEAD ? eB : 0])),
-                                make_float2(p.maskb[cA * K + k], p.maskb[cB * K + k]));
-                            m = make_float2(FElem<E>::round(fsigmoid(zm.x)),
-                                            FElem<E>::round(fsigmoid(zm.y)));
+                                *reinterpret_cast<const float2 *>(p.maskb + pk));
+                            m = FElem<E>::round2(make_float2(fsigmoid(zm.x), fsigmoid(zm.y)));
                         }
                         const float bk = __fadd_rn(startf, (float)(k * T.dilation));
                         float2 pos = __fadd2_rn(make_float2(bk, bk), off);
@@ -478,7 +494,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
                                               x0);
                         if (MASKHEAD)
                             v = __fmul2_rn(v, m);
-                        acc = __ffma2_rn(make_float2(p.fw[cA * K + k], p.fw[cB * K + k]), v, acc);
+                        acc = __ffma2_rn(*reinterpret_cast<const float2 *>(p.fw + pk), v, acc);
                     }
                     if (valid) {
                         orow[(int64_t)cA * T.L_out] = from_f32<E>(acc.x);
