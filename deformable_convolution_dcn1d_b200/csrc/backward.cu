@@ -157,9 +157,10 @@ constexpr int kSgRows = 256;     // output positions per sampling-gradient block
 // taps of the block's positions goes to a shared-memory window over the chunk's rows
 // ([nc][win] fp32, positions w0 .. w0+win-1); taps outside it (unconstrained offsets past
 // the margin) add to global memory directly, and the window is added to global memory
-// once, element by element, at the end.
+// once, element by element, at the end.  Six blocks an SM (40 registers): the loads in
+// flight, not the instruction count, set this kernel's pace.
 template <class T, bool MASK>
-__global__ void __launch_bounds__(kSgRows) sample_grad_kernel(const SampArgs a) {
+__global__ void __launch_bounds__(kSgRows, 6) sample_grad_kernel(const SampArgs a) {
     extern __shared__ float gxs[];
     const Problem &P = a.P;
     int64_t r = blockIdx.x;
@@ -202,18 +203,27 @@ __global__ void __launch_bounds__(kSgRows) sample_grad_kernel(const SampArgs a) 
             const bool win0 = window && r0 >= 0 && r0 < W;
             const bool win1 = window && r0 + 1 >= 0 && r0 + 1 < W;
             float s_off = 0.0f, s_mask = 0.0f;
-            for (int ci = c_begin; ci < c_end; ++ci) {
-                const T *row = static_cast<const T *>(P.x) + ((int64_t)b * P.C_in + ci) * P.L_in;
-                const float x0 = in0 ? ld_f32(row + tp.i0) : 0.0f;
-                const float x1 = in1 ? ld_f32(row + tp.i0 + 1) : 0.0f;
+            // The next channel's neighbours and column gradient are loaded while this
+            // channel's are used, so two channels' global loads are in flight a thread.
+            const T *row = static_cast<const T *>(P.x) + ((int64_t)b * P.C_in + c_begin) * P.L_in;
+            const int64_t cstride = (int64_t)P.K * P.L_out;   // column rows between channels
+            int64_t cidx = (((int64_t)b * P.C_in + c_begin) * P.K + k) * P.L_out + l;
+            float nx0 = in0 ? ld_f32(row + tp.i0) : 0.0f;
+            float nx1 = in1 ? ld_f32(row + tp.i0 + 1) : 0.0f;
+            float ndv = a.dcols ? a.dcols[cidx] : 0.0f;
+            for (int ci = c_begin; ci < c_end; ++ci, row += P.L_in, cidx += cstride) {
+                const float x0 = nx0, x1 = nx1, dv = ndv;
+                if (ci + 1 < c_end) {
+                    nx0 = in0 ? ld_f32(row + P.L_in + tp.i0) : 0.0f;
+                    nx1 = in1 ? ld_f32(row + P.L_in + tp.i0 + 1) : 0.0f;
+                    ndv = a.dcols ? a.dcols[cidx + cstride] : 0.0f;
+                }
                 const float v = __fadd_rn(__fmul_rn(__fsub_rn(1.0f, tp.f), x0), __fmul_rn(tp.f, x1));
-                const int64_t cidx = (((int64_t)b * P.C_in + ci) * P.K + k) * P.L_out + l;
                 if (a.cols)
                     a.cols[cidx] = __fmul_rn(m, v);
                 if (sizeof(T) == 2 && a.cols16)
                     static_cast<T *>(a.cols16)[cidx] = from_f32<T>(__fmul_rn(m, v));
                 if (a.dcols) {
-                    const float dv = a.dcols[cidx];
                     if (a.gx) {
                         float *gxr = a.gx + ((int64_t)b * P.C_in + ci) * P.L_in;
                         float *wr = gxs + (ci - c_begin) * W;
