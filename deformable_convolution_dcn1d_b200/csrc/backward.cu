@@ -415,6 +415,7 @@ struct WsLayout {
     size_t goutT, wT;    // tensor-core path: grad_out and W transposed (16-bit)
     int wsplits;
     bool tc;
+    bool fused;          // tensor-core path whose column gradients stay on chip
 };
 
 WsLayout ws_layout(const Problem &P, const BackwardGrads &G) {
@@ -423,9 +424,10 @@ WsLayout ws_layout(const Problem &P, const BackwardGrads &G) {
     const size_t ncol = (size_t)P.B * P.C_in * P.K * P.L_out * 4;
     const size_t noff = (size_t)P.B * P.offset_groups * P.L_out * P.K * 4;
     const bool need_dcols = G.x || G.off || G.mask;
+    w.fused = w.tc && need_dcols && gemm_sample_supported(P);
     size_t at = 0;
-    w.dcols = need_dcols ? at : SIZE_MAX;
-    at += need_dcols ? align256(ncol) : 0;
+    w.dcols = (need_dcols && !w.fused) ? at : SIZE_MAX;
+    at += (need_dcols && !w.fused) ? align256(ncol) : 0;
     w.cols = G.w ? at : SIZE_MAX;   // the tensor-core path keeps them in 16 bits
     at += G.w ? align256(w.tc ? ncol / 2 : ncol) : 0;
     w.goutT = (w.tc && need_dcols) ? at : SIZE_MAX;
@@ -495,7 +497,17 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
         if ((e = cudaGetLastError()) != cudaSuccess)
             return e;
         n += 2;
-        for (int gi = 0; gi < P.groups; ++gi) {
+        for (int gi = 0; L.fused && gi < P.groups; ++gi) {
+            // the column gradient's GEMM with the sampling gradient as its drain (the
+            // sampled columns too, when the weight gradient is wanted)
+            if ((e = launch_gemm_sample(P, gi, goutT + (int64_t)gi * P.cout_g,
+                                        wT + (int64_t)gi * Kg * P.cout_g,
+                                        want_cols ? cols16 : nullptr, gx, goff, gmask, s)) !=
+                cudaSuccess)
+                return e;
+            ++n;
+        }
+        for (int gi = 0; !L.fused && gi < P.groups; ++gi) {
             if ((e = launch_gemm_tc(P.dtype, goutT + (int64_t)gi * P.cout_g,
                                     (int64_t)P.B * P.L_out, P.C_out, 0, P.L_out, 0,
                                     wT + (int64_t)gi * Kg * P.cout_g, Kg, P.cout_g, 0, 0, 0,
@@ -530,7 +542,8 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
             return e;
         ++n;
     }
-    if (want_dcols || want_cols) {   // 2. sampling gradient and sampled columns
+    if ((want_dcols && !L.fused) || (want_cols && !(L.fused && want_dcols))) {
+        // 2. sampling gradient and sampled columns (the fused path did both already)
         SampArgs a;
         memset(&a, 0, sizeof(a));
         a.P = P;

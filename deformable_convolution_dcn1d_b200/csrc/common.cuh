@@ -88,6 +88,14 @@ struct BackwardGrads {
 };
 size_t backward_workspace(const Problem &P, const BackwardGrads &G);
 bool backward_uses_tensor_cores(const Problem &P, const BackwardGrads &G);
+// The backward's column-gradient GEMM with the sampling gradient fused into its drain
+// (gemm_tc.cu; 16-bit, K in {3, 4, 5, 7, 9}): for conv group g, grad_x / grad_offsets /
+// grad_mask accumulate into the fp32 buffers given (each may be NULL) and the sampled
+// columns go to cols16 (or not, if NULL); goutT_g and wT_g as for the plain GEMM.
+bool gemm_sample_supported(const Problem &P);
+cudaError_t launch_gemm_sample(const Problem &P, int g, const void *goutT_g, const void *wT_g,
+                               void *cols16, float *gx, float *goff, float *gmask,
+                               cudaStream_t stream);
 cudaError_t launch_backward(const Problem &P, const BackwardGrads &G, void *workspace,
                             cudaStream_t stream, int *launches);
 // PackedDeformConv1d's offset (and mask) predictor (trunk.cu): a depthwise convolution
