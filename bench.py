@@ -496,7 +496,16 @@ def run_backward_pass(args, w: W.Workload, peaks: dict, want_cpu: bool):
     barrier(ws)
     ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), ws) / args.steps
     per_gpu = 2 * w.flops() / (ms / 1e3) / 1e12
-    if gemm_kernel == "tcgen05_gemm":   # 16-bit operands on the tensor cores
+    if gemm_kernel == "tcgen05_gemm" and w.dtype == "f32":   # three TF32 products
+        pk = peaks["bf16_tflops"] * TF32_OVER_BF16
+        roof = {"bound": "tensor", "achieved": per_gpu, "peak": pk,
+                "unit": "TFLOP/s", "frac": per_gpu / pk, "traffic": None,
+                "kernel": "backward: two tcgen05 3xTF32 GEMMs (fp32-accurate) + sampling "
+                          "gradient + transposes",
+                "peak_source": f"tf32 dense peak (bf16 burst {peaks['source']} x 1.1/2.25 "
+                               f"nominal), flops counted once",
+                "frac_of_3pass_ceiling": per_gpu / (pk / 3.0)}
+    elif gemm_kernel == "tcgen05_gemm":   # 16-bit operands on the tensor cores
         roof = {"bound": "tensor", "achieved": per_gpu, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": per_gpu / peaks["bf16_tflops"], "traffic": None,
                 "kernel": "backward: two tcgen05 GEMMs (16-bit operands, fp32 accumulation) "

@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(256) sum_splits_kernel(const float *part, T *o
 
 struct SampArgs {
     Problem P;
+    int cols_ld;                 // row stride of `cols` (L_out, or L_out padded to 4)
     int nchunk;                  // channel chunks per offset group
     int nlb;                     // blocks of kSgRows positions per (b, chunk, offset group)
     int win;                     // shared-memory grad_x window per channel (0: none)
@@ -219,8 +220,9 @@ __global__ void __launch_bounds__(kSgRows, 6) sample_grad_kernel(const SampArgs 
                     ndv = a.dcols ? a.dcols[cidx + cstride] : 0.0f;
                 }
                 const float v = __fadd_rn(__fmul_rn(__fsub_rn(1.0f, tp.f), x0), __fmul_rn(tp.f, x1));
-                if (a.cols)
-                    a.cols[cidx] = __fmul_rn(m, v);
+                if (a.cols)   // row (b, ci, k) of the columns, cols_ld elements apart
+                    a.cols[(((int64_t)b * P.C_in + ci) * P.K + k) * a.cols_ld + l] =
+                        __fmul_rn(m, v);
                 if (sizeof(T) == 2 && a.cols16)
                     static_cast<T *>(a.cols16)[cidx] = from_f32<T>(__fmul_rn(m, v));
                 if (a.dcols) {
@@ -361,6 +363,18 @@ __global__ void __launch_bounds__(256) write_out_kernel(const float *src, T *dst
         dst[i] = from_f32<T>(src[i]);
 }
 
+// dst[row][0 .. L) = src[row][0 .. L) for every row, dst rows ld elements apart (the rest
+// of a dst row is not written: readers stop at L).
+__global__ void __launch_bounds__(256) pad_rows_kernel(const float *src, float *dst, int64_t rows,
+                                                       int L, int ld) {
+    const int64_t n = rows * L;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / L;
+        dst[r * ld + (i - r * L)] = __ldg(src + i);
+    }
+}
+
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Splits of the weight gradient's batch sum: the largest divisor of B that brings the
@@ -393,6 +407,21 @@ bool tc_backward(const Problem &P, const BackwardGrads &G) {
     return (int64_t)P.B * P.L_out < (1LL << 31) && rows < (1LL << 31);
 }
 
+// fp32 problems on the tensor cores (three TF32 products): the transposed grad_out and W
+// rows (C_out, C_out / groups elements) must be multiples of 16 bytes; the columns and
+// grad_out of the weight gradient are kept with rows padded to a multiple of 4.
+bool tc32_backward(const Problem &P, const BackwardGrads &G) {
+    if (P.dtype != DCN1D_F32)
+        return false;
+    if (P.C_out % 4 || P.cout_g % 4)
+        return false;
+    if ((reinterpret_cast<uintptr_t>(G.gout) & 15) || (reinterpret_cast<uintptr_t>(P.w) & 15))
+        return false;
+    const int64_t lp = (P.L_out + 3) / 4 * 4;
+    const int64_t rows = (int64_t)P.B * (P.C_in * P.K > P.C_out ? P.C_in * P.K : P.C_out);
+    return (int64_t)P.B * lp < (1LL << 31) && rows < (1LL << 31);
+}
+
 // Splits of the tensor-core weight-gradient GEMM's batch sum: the largest divisor of B
 // that brings its 128 x N tiles to about one or two waves of the SMs.
 int wgrad_splits_tc(const Problem &P) {
@@ -416,6 +445,9 @@ struct WsLayout {
     int wsplits;
     bool tc;
     bool fused;          // tensor-core path whose column gradients stay on chip
+    bool tc32;           // fp32 on the tensor cores (three TF32 products)
+    int lp;              // row stride of the columns (and of goutP) in elements
+    size_t goutP;        // tc32: grad_out with rows padded to lp (fp32)
 };
 
 WsLayout ws_layout(const Problem &P, const BackwardGrads &G) {
@@ -425,24 +457,31 @@ WsLayout ws_layout(const Problem &P, const BackwardGrads &G) {
     const size_t noff = (size_t)P.B * P.offset_groups * P.L_out * P.K * 4;
     const bool need_dcols = G.x || G.off || G.mask;
     w.fused = w.tc && need_dcols && gemm_sample_supported(P);
+    w.tc32 = !w.tc && tc32_backward(P, G);
+    w.lp = w.tc32 ? (P.L_out + 3) / 4 * 4 : P.L_out;
+    const size_t ncolp = (size_t)P.B * P.C_in * P.K * w.lp * 4;
+    const size_t tsz = w.tc32 ? 4 : 2;   // element size of the transposed copies
     size_t at = 0;
     w.dcols = (need_dcols && !w.fused) ? at : SIZE_MAX;
     at += (need_dcols && !w.fused) ? align256(ncol) : 0;
-    w.cols = G.w ? at : SIZE_MAX;   // the tensor-core path keeps them in 16 bits
-    at += G.w ? align256(w.tc ? ncol / 2 : ncol) : 0;
-    w.goutT = (w.tc && need_dcols) ? at : SIZE_MAX;
-    at += (w.tc && need_dcols) ? align256((size_t)P.B * P.C_out * P.L_out * 2) : 0;
-    w.wT = (w.tc && need_dcols) ? at : SIZE_MAX;
-    at += (w.tc && need_dcols) ? align256((size_t)P.C_out * P.cin_g * P.K * 2) : 0;
+    w.cols = G.w ? at : SIZE_MAX;   // the 16-bit tensor-core path keeps them in 16 bits
+    at += G.w ? align256(w.tc ? ncol / 2 : ncolp) : 0;
+    const bool tr = (w.tc || w.tc32) && need_dcols;
+    w.goutT = tr ? at : SIZE_MAX;
+    at += tr ? align256((size_t)P.B * P.C_out * P.L_out * tsz) : 0;
+    w.wT = tr ? at : SIZE_MAX;
+    at += tr ? align256((size_t)P.C_out * P.cin_g * P.K * tsz) : 0;
+    w.goutP = (w.tc32 && G.w) ? at : SIZE_MAX;
+    at += (w.tc32 && G.w) ? align256((size_t)P.B * P.C_out * w.lp * 4) : 0;
     w.gx = G.x ? at : SIZE_MAX;
     at += G.x ? align256((size_t)P.B * P.C_in * P.L_in * 4) : 0;
     w.goff = G.off ? at : SIZE_MAX;
     at += G.off ? align256(noff) : 0;
     w.gmask = G.mask ? at : SIZE_MAX;
     at += G.mask ? align256(noff) : 0;
-    w.wsplits = G.w ? (w.tc ? wgrad_splits_tc(P) : wgrad_splits(P)) : 1;
-    // the tensor-core GEMM writes fp32 slices even unsplit (then converted)
-    const bool parts = G.w && (w.wsplits > 1 || w.tc);
+    w.wsplits = G.w ? ((w.tc || w.tc32) ? wgrad_splits_tc(P) : wgrad_splits(P)) : 1;
+    // the tensor-core GEMMs write fp32 slices even unsplit (then converted)
+    const bool parts = G.w && (w.wsplits > 1 || w.tc || w.tc32);
     w.wpart = parts ? at : SIZE_MAX;
     at += parts ? align256((size_t)w.wsplits * P.C_out * P.cin_g * P.K * 4) : 0;
     w.total = at;
@@ -465,6 +504,7 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
     T *cols16 = (L.cols != SIZE_MAX && L.tc) ? reinterpret_cast<T *>(wsb + L.cols) : nullptr;
     T *goutT = L.goutT != SIZE_MAX ? reinterpret_cast<T *>(wsb + L.goutT) : nullptr;
     T *wT = L.wT != SIZE_MAX ? reinterpret_cast<T *>(wsb + L.wT) : nullptr;
+    float *goutP = L.goutP != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.goutP) : nullptr;
     float *gx = L.gx != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.gx) : nullptr;
     float *goff = L.goff != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.goff) : nullptr;
     float *gmask = L.gmask != SIZE_MAX ? reinterpret_cast<float *>(wsb + L.gmask) : nullptr;
@@ -517,6 +557,30 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
                 return e;
             ++n;
         }
+    } else if (want_dcols && P.B > 0 && L.tc32) {
+        // 1. fp32 on the tensor cores, three TF32 products: D[n][m] = sum_co goutT[n][g*cout_g
+        // + co] * wT[g][m][co] over the flattened rows n = b * L_out + l, stored to
+        // dcols[b][g*Kg + m][l]
+        const dim3 tb(256);
+        transpose_kernel<T><<<dim3((P.L_out + 31) / 32, (P.C_out + 31) / 32, P.B), tb, 0, s>>>(
+            gout, goutT, P.C_out, P.L_out, P.L_out, P.C_out, (int64_t)P.C_out * P.L_out,
+            (int64_t)P.L_out * P.C_out);
+        transpose_kernel<T><<<dim3((Kg + 31) / 32, (P.cout_g + 31) / 32, P.groups), tb, 0, s>>>(
+            w, wT, P.cout_g, Kg, Kg, P.cout_g, (int64_t)P.cout_g * Kg, (int64_t)Kg * P.cout_g);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+        n += 2;
+        for (int gi = 0; gi < P.groups; ++gi) {
+            if ((e = launch_gemm_x3(reinterpret_cast<const float *>(goutT) + (int64_t)gi * P.cout_g,
+                                    (int64_t)P.B * P.L_out, P.C_out, 0, 0, 0,
+                                    reinterpret_cast<const float *>(wT) +
+                                        (int64_t)gi * Kg * P.cout_g,
+                                    Kg, P.cout_g, 0, 0, 0, P.L_out, Kg, P.cout_g, 1, P.B, P.L_out,
+                                    dcols + (int64_t)gi * Kg * P.L_out, 1, P.L_out,
+                                    (int64_t)P.C_in * P.K * P.L_out, s)) != cudaSuccess)
+                return e;
+            ++n;
+        }
     } else if (want_dcols && P.B > 0) {
         // 1. dcols[b][g*Kg + m][l] = sum_co W[g*cout_g + co][m] * gout[b][g*cout_g + co][l]
         GemmArgs g;
@@ -547,6 +611,7 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
         SampArgs a;
         memset(&a, 0, sizeof(a));
         a.P = P;
+        a.cols_ld = L.lp;
         a.nchunk = (P.cin_per_og + kChunk - 1) / kChunk;
         a.nlb = (P.L_out + kSgRows - 1) / kSgRows;
         // grad_x window: the receptive fields of a block's positions, plus a margin for
@@ -603,6 +668,35 @@ cudaError_t run_backward(const Problem &P, const BackwardGrads &G, void *ws, cud
         if ((e = cudaGetLastError()) != cudaSuccess)
             return e;
         n += P.B > 0;
+    } else if (want_cols && L.tc32) {
+        // 3. fp32 on the tensor cores, as the 16-bit form above, with grad_out and the
+        // columns in rows padded to lp elements (TMA rows are multiples of 16 bytes)
+        const int S = L.wsplits, rps = P.B / S;
+        const int64_t nw = (int64_t)P.C_out * Kg;
+        if (P.B > 0) {
+            pad_rows_kernel<<<grid_1d((int64_t)P.B * P.C_out * P.L_out), 256, 0, s>>>(
+                reinterpret_cast<const float *>(gout), goutP, (int64_t)P.B * P.C_out, P.L_out,
+                L.lp);
+            if ((e = cudaGetLastError()) != cudaSuccess)
+                return e;
+            ++n;
+            for (int gi = 0; gi < P.groups; ++gi) {
+                if ((e = launch_gemm_x3(cols, (int64_t)P.B * P.C_in * P.K, L.lp, gi * Kg,
+                                        rps * P.C_in * P.K, P.C_in * P.K, goutP,
+                                        (int64_t)P.B * P.C_out, L.lp, gi * P.cout_g,
+                                        rps * P.C_out, P.C_out, Kg, P.cout_g, P.L_out, rps, S, 0,
+                                        wpart + (int64_t)gi * P.cout_g * Kg, 1, Kg,
+                                        (int64_t)P.C_out * Kg, s)) != cudaSuccess)
+                    return e;
+                ++n;
+            }
+            sum_splits_kernel<T><<<grid_1d(nw), 256, 0, s>>>(wpart, static_cast<T *>(G.w), S, nw);
+            if ((e = cudaGetLastError()) != cudaSuccess)
+                return e;
+            ++n;
+        } else if ((e = cudaMemsetAsync(G.w, 0, nw * sizeof(T), s)) != cudaSuccess) {
+            return e;
+        }
     } else if (want_cols) {
         // 3. gW[g*cout_g + co][m] = sum_b sum_l gout[b][g*cout_g + co][l] * cols[b][g*Kg + m][l]
         // (zeros for an empty batch).  Split s of the batch sum covers batches
@@ -677,7 +771,7 @@ size_t backward_workspace(const Problem &P, const BackwardGrads &G) {
 }
 
 bool backward_uses_tensor_cores(const Problem &P, const BackwardGrads &G) {
-    return tc_backward(P, G);
+    return tc_backward(P, G) || tc32_backward(P, G);
 }
 
 cudaError_t launch_backward(const Problem &P, const BackwardGrads &G, void *workspace,

@@ -93,6 +93,16 @@ bool backward_uses_tensor_cores(const Problem &P, const BackwardGrads &G);
 // grad_mask accumulate into the fp32 buffers given (each may be NULL) and the sampled
 // columns go to cols16 (or not, if NULL); goutT_g and wT_g as for the plain GEMM.
 bool gemm_sample_supported(const Problem &P);
+// The same GEMM on fp32 operands by three TF32 products (gemm_tc.cu): row strides multiples
+// of 4 elements, 16-byte aligned bases.  flat_rpz > 0: the M rows of every z form one range
+// (row m is row m of A; its output goes to C[(m / flat_rpz) * c_sz + (m % flat_rpz) * c_sm
+// + n * c_sn]) and the per-z A offsets are not used.
+bool gemm_x3_supported(const void *A, int64_t a_ld, const void *B, int64_t b_ld);
+cudaError_t launch_gemm_x3(const float *A, int64_t a_rows, int64_t a_ld, int a_row0,
+                           int a_row_z, int a_row_r, const float *B, int64_t b_rows, int64_t b_ld,
+                           int b_row0, int b_row_z, int b_row_r, int M, int N, int K, int R,
+                           int nz, int flat_rpz, float *C, int64_t c_sm, int64_t c_sn,
+                           int64_t c_sz, cudaStream_t stream);
 cudaError_t launch_gemm_sample(const Problem &P, int g, const void *goutT_g, const void *wT_g,
                                void *cols16, float *gx, float *goff, float *gmask,
                                cudaStream_t stream);

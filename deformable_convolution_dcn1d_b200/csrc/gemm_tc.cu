@@ -405,6 +405,213 @@ __global__ void __launch_bounds__(kSThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------------
+// The same GEMM for fp32 operands, accurate to fp32 through three TF32 products: each
+// operand v is split exactly into hi (v with its low 13 mantissa bits cleared; the tf32
+// MMA reads an fp32 container that way) and lo = v - hi, and the MMA accumulates
+// hi*hi + hi*lo + lo*hi.  TMA loads the fp32 tiles (32 elements = 128 bytes a row); while
+// the MMA works, the four drain warps write each stage's lo tiles next to them.
+//
+// Rows: with `flat`, the M rows of A and C run over z as well (row m of the whole problem
+// is row m of A; its output lands at C[(m / rpz) * c_sz + (m % rpz) * c_sm + n * c_sn]),
+// so short per-z row counts still fill 128-row tiles.
+
+constexpr int kXBK = 32;                 // fp32 reduction elements per stage
+constexpr int kXStages = 2;
+constexpr int kXThreads = 6 * 32;        // TMA, MMA, 4 lo-formers / drain
+
+struct GemmX3Args {
+    int M, N, K, R, NT;
+    int tiles_m, tiles_n;
+    int a_row0, a_row_z, a_row_r;
+    int b_row0, b_row_z, b_row_r;
+    int flat, rpz;                       // flat rows: rpz rows per z
+    float *C;
+    int64_t c_sm, c_sn, c_sz;
+    uint32_t a_bytes, b_bytes;           // one stage's A and B tiles (each also has a lo tile)
+    unsigned int *status;
+};
+
+__device__ __forceinline__ uint4 lds_v4x(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts_v4x(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t tf32_lo(uint32_t v) {
+    return __float_as_uint(__fsub_rn(__uint_as_float(v), __uint_as_float(v & 0xFFFFE000u)));
+}
+
+__global__ void __launch_bounds__(kXThreads, 1)
+    gemm_x3_kernel(const __grid_constant__ GemmX3Args G, const __grid_constant__ CUtensorMap amap,
+                   const __grid_constant__ CUtensorMap bmap) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int tile = blockIdx.x;
+    const int tn = tile % G.tiles_n;
+    const int tm = (tile / G.tiles_n) % G.tiles_m;
+    const int z = tile / (G.tiles_n * G.tiles_m);
+    const int m0 = tm * kGM, n0 = tn * G.NT;
+
+    const uint32_t sraw = smem_u32(smem_raw);
+    const uint32_t sbase = (sraw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - sraw);
+    // stage s: A hi, A lo, B hi, B lo
+    const uint32_t stage_bytes = 2 * (G.a_bytes + G.b_bytes);
+    auto a_hi = [&](int s) { return sbase + (uint32_t)s * stage_bytes; };
+    auto a_lo = [&](int s) { return a_hi(s) + G.a_bytes; };
+    auto b_hi = [&](int s) { return a_hi(s) + 2 * G.a_bytes; };
+    auto b_lo = [&](int s) { return b_hi(s) + G.b_bytes; };
+    const uint32_t bar0 = sbase + kXStages * stage_bytes;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (kXStages + s); };
+    auto lo_ready = [&](int s) { return bar0 + 8u * (2 * kXStages + s); };
+    const uint32_t dfull = bar0 + 8u * (3 * kXStages);
+    uint32_t *tmem_holder =
+        reinterpret_cast<uint32_t *>(smem + (bar0 - sbase) + 8 * (3 * kXStages + 2));
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kXStages; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+            mbar_init(lo_ready(s), 4);
+        }
+        mbar_init(dfull, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kGMma) {
+        tmem_alloc(smem_u32(tmem_holder), 256);
+        tc_fence_before();
+    }
+    if (warp == kGTma && lane == 0) {
+        tma_prefetch_desc(&amap);
+        tma_prefetch_desc(&bmap);
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const BoundedWait wait{abort_flag, kGWaitNs, G.status};
+    const int nkb = (G.K + kXBK - 1) / kXBK;
+    const int total = nkb * G.R;
+    // A's first row: flat rows index the whole problem, else z's block
+    const int a_row_base = G.flat ? m0 : G.a_row0 + z * G.a_row_z + m0;
+
+    if (warp == kGTma) {
+        if (lane == 0) {
+            int it = 0;
+            for (; it < total; ++it) {
+                const int r = it / nkb, kb = it - r * nkb;
+                const int s = it % kXStages;
+                const uint32_t ph = (uint32_t)(it / kXStages) & 1u;
+                if (!wait(empty(s), ph ^ 1u))
+                    break;
+                mbar_arrive_expect_tx(full(s), G.a_bytes + G.b_bytes);
+                tma_load_2d(a_hi(s), &amap, kb * kXBK, a_row_base + r * G.a_row_r, full(s));
+                tma_load_2d(b_hi(s), &bmap, kb * kXBK,
+                            G.b_row0 + z * G.b_row_z + r * G.b_row_r + n0, full(s));
+            }
+            volatile int never = 0;
+            const BoundedWait drain{&never, kGWaitNs, G.status};
+            for (int j = (it > kXStages ? it - kXStages : 0); j < it; ++j)
+                drain(full(j % kXStages), (uint32_t)(j / kXStages) & 1u);
+        }
+    } else if (warp == kGMma) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_tf32_ss_f32(kGM, G.NT);
+            for (int it = 0; it < total; ++it) {
+                const int s = it % kXStages;
+                const uint32_t ph = (uint32_t)(it / kXStages) & 1u;
+                if (!wait(full(s), ph) || !wait(lo_ready(s), ph))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kXBK / 8; ++kk) {   // 8 tf32 = 32 bytes a step
+                    const uint32_t o = 32u * kk;
+                    const uint64_t ah = sw128_kmajor_desc(a_hi(s) + o);
+                    const uint64_t al = sw128_kmajor_desc(a_lo(s) + o);
+                    const uint64_t bh = sw128_kmajor_desc(b_hi(s) + o);
+                    const uint64_t bl = sw128_kmajor_desc(b_lo(s) + o);
+                    mma_tf32_ss(tmem, ah, bh, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+                    mma_tf32_ss(tmem, ah, bl, idesc, 1u);
+                    mma_tf32_ss(tmem, al, bh, idesc, 1u);
+                }
+                mma_commit(empty(s));
+            }
+            mma_commit(dfull);
+            volatile int never = 0;
+            const BoundedWait drain{&never, kGWaitNs, G.status};
+            drain(dfull, 0);
+        }
+    } else {
+        // ---- lo parts of every stage (elementwise, so the swizzle does not matter), then
+        // the drain: warp w reads TMEM lanes 32 (w % 4) ..
+        const int dt = threadIdx.x - 64;                  // 0 .. 127
+        bool ok = true;
+        for (int it = 0; it < total && ok; ++it) {
+            const int s = it % kXStages;
+            ok = __all_sync(0xffffffffu, wait(full(s), (uint32_t)(it / kXStages) & 1u));
+            if (ok) {
+                for (uint32_t o = 16u * dt; o < G.a_bytes; o += 16u * 128u) {
+                    uint4 v = lds_v4x(a_hi(s) + o);
+                    v = make_uint4(tf32_lo(v.x), tf32_lo(v.y), tf32_lo(v.z), tf32_lo(v.w));
+                    sts_v4x(a_lo(s) + o, v);
+                }
+                for (uint32_t o = 16u * dt; o < G.b_bytes; o += 16u * 128u) {
+                    uint4 v = lds_v4x(b_hi(s) + o);
+                    v = make_uint4(tf32_lo(v.x), tf32_lo(v.y), tf32_lo(v.z), tf32_lo(v.w));
+                    sts_v4x(b_lo(s) + o, v);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(lo_ready(s));
+            }
+        }
+        const int q = warp % 4;
+        const int m = m0 + 32 * q + lane;
+        if (ok && __all_sync(0xffffffffu, wait(dfull, 0))) {
+            tc_fence_after();
+            float *Crow = nullptr;
+            if (m < G.M) {
+                const int zz = G.flat ? m / G.rpz : z;
+                const int mm = G.flat ? m - zz * G.rpz : m;
+                Crow = G.C + (int64_t)zz * G.c_sz + (int64_t)mm * G.c_sm;
+            }
+            for (int c = 0; c < G.NT; c += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c, v);
+                tmem_wait_ld();
+                if (Crow) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int n = n0 + c + i;
+                        if (n < G.N)
+                            Crow[(int64_t)n * G.c_sn] = __uint_as_float(v[i]);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kGMma) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
 }  // namespace
 
 // The A and B operands as 16-bit row-major [rows][cols] arrays (row strides in
@@ -476,6 +683,66 @@ cudaError_t launch_gemm_tc(int dtype, const void *A, int64_t a_rows, int64_t a_l
     else
         gemm_tc_kernel<__nv_bfloat16><<<(unsigned)blocks, kGThreads, smem_launch, stream>>>(G, amap,
                                                                                             bmap);
+    return cudaGetLastError();
+}
+
+// fp32 operands: row strides (elements) multiples of 4, 16-byte aligned bases.
+bool gemm_x3_supported(const void *A, int64_t a_ld, const void *B, int64_t b_ld) {
+    return !(reinterpret_cast<uintptr_t>(A) & 15) && !(reinterpret_cast<uintptr_t>(B) & 15) &&
+           a_ld % 4 == 0 && b_ld % 4 == 0;
+}
+
+cudaError_t launch_gemm_x3(const float *A, int64_t a_rows, int64_t a_ld, int a_row0,
+                           int a_row_z, int a_row_r, const float *B, int64_t b_rows, int64_t b_ld,
+                           int b_row0, int b_row_z, int b_row_r, int M, int N, int K, int R,
+                           int nz, int flat_rpz, float *C, int64_t c_sm, int64_t c_sn,
+                           int64_t c_sz, cudaStream_t stream) {
+    if (!gemm_x3_supported(A, a_ld, B, b_ld) || a_rows < 1 || b_rows < 1 ||
+        a_rows >= (1LL << 31) || b_rows >= (1LL << 31))
+        return cudaErrorInvalidValue;
+    GemmX3Args G;
+    memset(&G, 0, sizeof(G));
+    G.flat = flat_rpz > 0 ? 1 : 0;
+    G.rpz = flat_rpz;
+    G.M = G.flat ? M * nz : M;   // flat: the rows of every z in one range
+    G.N = N;
+    G.K = K;
+    G.R = R;
+    G.NT = N <= 128 ? (N <= 64 ? 64 : 128) : 256;
+    G.tiles_m = (G.M + kGM - 1) / kGM;
+    G.tiles_n = (N + G.NT - 1) / G.NT;
+    G.a_row0 = a_row0;
+    G.a_row_z = a_row_z;
+    G.a_row_r = a_row_r;
+    G.b_row0 = b_row0;
+    G.b_row_z = b_row_z;
+    G.b_row_r = b_row_r;
+    G.C = C;
+    G.c_sm = c_sm;
+    G.c_sn = c_sn;
+    G.c_sz = c_sz;
+    G.a_bytes = kGM * kXBK * 4;
+    G.b_bytes = (uint32_t)G.NT * kXBK * 4;
+    G.status = device_status_ptr();
+    if (!G.status)
+        return cudaErrorInvalidDevice;
+    const int64_t blocks = (int64_t)G.tiles_m * G.tiles_n * (G.flat ? 1 : nz);
+    if (blocks < 1 || blocks >= (1LL << 31))
+        return cudaErrorInvalidValue;
+    alignas(64) CUtensorMap amap, bmap;
+    if (!encode_2d_ld(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, A, (uint64_t)K, (uint64_t)a_rows,
+                      (uint64_t)a_ld, 4, kXBK, kGM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d_ld(&bmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, B, (uint64_t)K, (uint64_t)b_rows,
+                      (uint64_t)b_ld, 4, kXBK, (uint32_t)G.NT, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const size_t smem = (size_t)kXStages * 2 * (G.a_bytes + G.b_bytes) +
+                        8 * (3 * kXStages + 2) + 16 + 1024;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(gemm_x3_kernel),
+                                (int)(smem < 116 * 1024 ? 116 * 1024 : smem));
+    if (e != cudaSuccess)
+        return e;
+    gemm_x3_kernel<<<(unsigned)blocks, kXThreads, smem < 116 * 1024 ? 116 * 1024 : smem,
+                     stream>>>(G, amap, bmap);
     return cudaGetLastError();
 }
 
