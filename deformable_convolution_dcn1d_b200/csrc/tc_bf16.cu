@@ -30,8 +30,14 @@
 //    quarter's columns): tcgen05.ld the accumulator, add the bias, round to
 //    bf16 and store; lanes are consecutive l, so each store is 64 contiguous
 //    bytes of out[b, co, :].  A tile's epilogue runs after the producers have
-//    staged the first kStages k-blocks of their next tile, so the MMA resumes
-//    on ready stages as soon as the accumulator is free.
+//    staged the first kStages k-blocks of their next tile;
+//  * the accumulator alternates between tensor-memory columns [0, N) and
+//    [128, 128 + N) from tile to tile, so consecutive tiles share only
+//    [128, 256).  The epilogue drains that shared slot first, parking its
+//    values in shared memory and releasing the slot before storing them; the
+//    next tile's MMAs start on their own slot at once and add the shared part of
+//    the staged k-blocks as soon as it is released.  Channel blocks of at most
+//    128 rotate over three slots and never wait for a drain.
 // Stages are chained by mbarriers; every wait is bounded (sm100.cuh).
 #include <string.h>
 
@@ -58,8 +64,11 @@ constexpr int kTmaWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 18 * 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColD = 0;      // D: columns [0, N)
-constexpr uint32_t kColA = 256;    // A stages: columns [256 + 32 s, +32)
+// Accumulator: columns [0, N) for even tiles of a CTA, [128, 128 + N) for odd ones, so
+// columns [128, 256) are the only ones two consecutive tiles share (N > 128); N <= 128
+// tiles rotate over [0, 128), [128, 256), [256, 384).  A stages: [384 + 32 s, +32).
+constexpr int kSlotCols = 128;
+constexpr uint32_t kColA = 384;
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s
 
 struct TcArgs {
@@ -78,7 +87,10 @@ struct TcArgs {
     int pair_store;    // 1: L_out even and out 4-byte aligned (32-bit epilogue stores)
     int xtma;          // 1: x windows by TMA; 0 (L_in not a multiple of 8, even): by the
                        // loader warp's 4-byte cp.async copies into the same layout
-    uint32_t off_w, off_x, off_bias, off_pos, off_bar;   // shared-memory layout
+    int park;          // 1: the drain parks the shared accumulator slot's values in shared
+                       // memory (N > 128 and room for 32 KB), so it releases the slot
+                       // before its stores
+    uint32_t off_w, off_x, off_bias, off_pos, off_park, off_bar;   // shared-memory layout
     unsigned int *status;                       // device status word
     uint64_t wait_ns;                           // limit of every mbarrier wait
 };
@@ -87,6 +99,28 @@ struct TcArgs {
 // producer groups (group = i % 2), so each group owns every other stage of the ring (the
 // ring depth is even).  With contiguous halves a group walks its channels in order and
 // meets each offset group once; the parity split is the fallback for odd counts.
+// The accumulator of a CTA's tile number tc: its first column, the slot only it uses
+// (N > 128: 0 for even tiles, 2 for odd ones; N <= 128: tc % 3) and how many earlier
+// tiles used that slot.
+struct Acc {
+    uint32_t col;
+    int own;
+    uint32_t own_uses;
+};
+__device__ __forceinline__ Acc acc_of(uint32_t tc, bool two) {
+    Acc a;
+    if (two) {
+        a.col = (tc & 1u) ? (uint32_t)kSlotCols : 0u;
+        a.own = (tc & 1u) ? 2 : 0;
+        a.own_uses = tc / 2u;
+    } else {
+        a.own = (int)(tc % 3u);
+        a.col = (uint32_t)kSlotCols * (uint32_t)a.own;
+        a.own_uses = tc / 3u;
+    }
+    return a;
+}
+
 __device__ __forceinline__ int kb_at(const TcArgs &A, int i) {
     return A.half_kb ? ((i & 1) ? A.half_kb + (i >> 1) : (i >> 1)) : i;
 }
@@ -344,9 +378,10 @@ __global__ void __maxnreg__(96)
     auto bar_empty = [&](int s) { return bar0 + 8u * (kStages + s); };
     auto bar_afull = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
     const uint32_t bar_dfull = bar0 + 8u * (3 * kStages);
-    const uint32_t bar_dempty = bar0 + 8u * (3 * kStages + 1);
-    const uint32_t bar_drain = bar0 + 8u * (3 * kStages + 2);
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + A.off_bar + 8 * (3 * kStages + 3));
+    const uint32_t bar_drain = bar0 + 8u * (3 * kStages + 1);
+    // one per 128-column accumulator slot: the drain of the slot's last tile is done
+    auto bar_dfree = [&](int slot) { return bar0 + 8u * (3 * kStages + 2 + slot); };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + A.off_bar + 8 * (3 * kStages + 5));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     if (threadIdx.x == 0) {
@@ -358,8 +393,9 @@ __global__ void __maxnreg__(96)
             mbar_init(bar_afull(s), kProdWarps / 2);
         }
         mbar_init(bar_dfull, 1);
-        mbar_init(bar_dempty, kProdWarps);
         mbar_init(bar_drain, 1);
+        for (int j = 0; j < 3; ++j)
+            mbar_init(bar_dfree(j), kProdWarps);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -468,26 +504,68 @@ __global__ void __maxnreg__(96)
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
+            const bool two = A.N > kSlotCols;
             const uint32_t idesc = Elem<E>::idesc(128, A.N);
+            const uint32_t idesc_lo = Elem<E>::idesc(128, kSlotCols);
+            const uint32_t idesc_hi = Elem<E>::idesc(128, two ? A.N - kSlotCols : 32);
             uint32_t it = 0, tc = 0;
             for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
-                if (!wait(bar_dempty, (tc & 1u) ^ 1u))
+                const Acc acc = acc_of(tc, two);
+                // the own slot's last tile (two or three back) has been drained
+                if (acc.own_uses > 0 && !wait(bar_dfree(acc.own), (acc.own_uses - 1u) & 1u))
                     goto mma_done;
                 tc_fence_after();
+                const uint32_t d = tmem + acc.col;
+                // N > 128: the shared slot [128, 256) is the previous tile's, drained first.
+                // Until it is free, the staged k-blocks contract into the own part only and
+                // their shared part follows (at most a ring's worth of k-blocks).
+                bool sh_free = !two || tc == 0;
+                int pend = 0;
+                // the own part: even tiles channels [0, 128) at column 0, odd tiles
+                // channels [128, N) at column 256; the shared part is the other one
+                auto part = [&](bool own, int p, uint32_t s) {
+                    const bool lo = own == ((tc & 1u) == 0u);   // channels [0, 128)?
+                    const uint32_t wst = w_st0 + s * A.w_stage_bytes + (lo ? 0u : kSlotCols * 128u);
+                    const uint32_t dp = d + (lo ? 0u : (uint32_t)kSlotCols);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_bf16_ts(dp, tmem + kColA + 32u * s + 8u * kk,
+                                    sw128_kmajor_desc(wst + 32u * kk), lo ? idesc_lo : idesc_hi,
+                                    (p > 0 || kk > 0) ? 1u : 0u);
+                };
                 for (int pos = 0; pos < A.num_kb; ++pos, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
                     if (!wait(bar_full(s), ph) || !wait(bar_afull(s), ph))
                         goto mma_done;
                     tc_fence_after();
-                    const uint32_t wst = w_st0 + s * A.w_stage_bytes;
+                    if (sh_free) {
+                        const uint32_t wst = w_st0 + s * A.w_stage_bytes;
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        mma_bf16_ts(tmem + kColD, tmem + kColA + 32u * s + 8u * kk,
-                                    sw128_kmajor_desc(wst + 32u * kk), idesc,
-                                    (pos > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            mma_bf16_ts(d, tmem + kColA + 32u * s + 8u * kk,
+                                        sw128_kmajor_desc(wst + 32u * kk), idesc,
+                                        (pos > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(bar_empty(s));
+                        continue;
                     }
-                    mma_commit(bar_empty(s));
+                    part(true, pos, s);
+                    ++pend;
+                    const bool must = pend == kStages || pos == A.num_kb - 1;
+                    const uint32_t sh_par = (tc - 1u) & 1u;   // the shared slot's last drain
+                    if (must ? wait(bar_dfree(1), sh_par) : mbar_try_wait(bar_dfree(1), sh_par)) {
+                        tc_fence_after();
+                        for (int p = pos + 1 - pend; p <= pos; ++p) {
+                            const uint32_t sp = (it - (uint32_t)(pos - p)) % kStages;
+                            part(false, p, sp);
+                            mma_commit(bar_empty(sp));
+                        }
+                        pend = 0;
+                        sh_free = true;
+                    } else if (must) {
+                        goto mma_done;
+                    }
                 }
                 mma_commit(bar_dfull);
             }
@@ -516,9 +594,74 @@ __global__ void __maxnreg__(96)
             tc_fence_after();
             E *outp = static_cast<E *>(P.out) +
                                   ((int64_t)T.b * P.C_out + (int64_t)T.co0) * P.L_out + l;
-            for (int cc = h; cc < A.N / 16; cc += 4) {
+            const bool two = A.N > kSlotCols;
+            const Acc acc = acc_of(tcnt, two);
+            // N > 128: the chunks in the shared slot [128, 256) first (even tiles: channels
+            // 128.., odd tiles: channels 0..127), then the own slot's
+            const int n16 = A.N / 16, s16 = kSlotCols / 16;
+            const int sh_lo = two ? ((tcnt & 1u) ? 0 : s16) : 0;
+            const int sh_hi = two ? ((tcnt & 1u) ? s16 : n16) : 0;
+            // The shared slot's chunks (at most two a warp) first.  Parked: bias added,
+            // rounded and written to shared memory as packed pairs ([channel pair][row]
+            // words, each thread reading back its own), the slot released, then stored, so
+            // the next tile's MMAs wait only for the tensor-memory loads.  Otherwise stored
+            // before the release.
+            uint32_t *park = reinterpret_cast<uint32_t *>(smem + A.off_park) + row;
+#pragma unroll 1
+            for (int j = 0; j < 2; ++j) {
+                const int cc = sh_lo + h + 4 * j;
+                if (cc < sh_hi) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + acc.col + 16u * cc, v);
+                    tmem_wait_ld();
+                    if (A.park) {
+                        uint32_t *pw = park + (8 * (cc - sh_lo)) * kRows;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            pw[i * kRows] =
+                                Elem<E>::pack(__uint_as_float(v[2 * i]) + biasg[16 * cc + 2 * i],
+                                              __uint_as_float(v[2 * i + 1]) +
+                                                  biasg[16 * cc + 2 * i + 1]);
+                    } else if (valid) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int co = 16 * cc + i;
+                            outp[(int64_t)co * P.L_out] =
+                                from_f32<E>(__uint_as_float(v[i]) + biasg[co]);
+                        }
+                    }
+                }
+            }
+            if (two) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar_dfree(1));
+            }
+            if (A.park && valid) {
+                unsigned short *outs = reinterpret_cast<unsigned short *>(outp);
+#pragma unroll 1
+                for (int j = 0; j < 2; ++j) {
+                    const int cc = sh_lo + h + 4 * j;
+                    if (cc < sh_hi) {
+                        const uint32_t *pr = park + (8 * (cc - sh_lo)) * kRows;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint32_t w = pr[i * kRows];
+                            outs[(int64_t)(16 * cc + 2 * i) * P.L_out] = (unsigned short)(w & 0xFFFFu);
+                            outs[(int64_t)(16 * cc + 2 * i + 1) * P.L_out] =
+                                (unsigned short)(w >> 16);
+                        }
+                    }
+                }
+            }
+            // the own slot's chunks
+            {
+            const int c_begin = sh_lo == 0 ? sh_hi : 0;
+            const int c_end = sh_lo == 0 ? n16 : sh_lo;
+            for (int cc = c_begin + h; cc < c_end; cc += 4) {
                 uint32_t v[16];
-                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + kColD + 16u * cc, v);
+                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + acc.col + 16u * cc, v);
                 tmem_wait_ld();
                 if (valid) {
 #pragma unroll
@@ -532,7 +675,8 @@ __global__ void __maxnreg__(96)
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(bar_dempty);
+                mbar_arrive(bar_dfree(acc.own));
+            }
             return true;
         };
         int pend_t = -1;        // tile whose epilogue is still to do
@@ -762,8 +906,14 @@ bool make_plan(const Problem &P, Plan *out) {
     A.off_bias = A.off_x + kStages * A.x_stage_bytes;
     A.off_pos = A.off_bias + (uint32_t)((P.C_out * 4 + 15) / 16 * 16);
     // wide K: the producers' tap positions, [K][512] floats
-    A.off_bar = A.off_pos + (P.K >= kPosSmemMinK ? (uint32_t)(P.K * kProdThreads * 4) : 0u);
-    size_t smem = A.off_bar + 8 * (3 * kStages + 3) + 16 + 1024;   // + alignment slack
+    A.off_park = A.off_pos + (P.K >= kPosSmemMinK ? (uint32_t)(P.K * kProdThreads * 4) : 0u);
+    const size_t tail = 8 * (3 * kStages + 5) + 16 + 1024;   // barriers + alignment slack
+    // the drain's parked shared-slot values, [64 channel pairs][128 rows] words, where
+    // they fit
+    const uint32_t park_bytes = (uint32_t)(kSlotCols / 2 * kRows * 4);
+    A.park = (A.N > kSlotCols && A.off_park + park_bytes + tail <= 227 * 1024) ? 1 : 0;
+    A.off_bar = A.off_park + (A.park ? park_bytes : 0u);
+    size_t smem = A.off_bar + tail;
     if (smem > 227 * 1024)
         return false;
     // At least half the SM's shared memory, so two CTAs (each allocating all 512

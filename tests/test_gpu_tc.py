@@ -1,13 +1,15 @@
 """GPU parity of the fused tensor-core (tcgen05) bf16 path: shapes chosen so that the
 library selects it, asserted, then compared with the oracle; plus the device status word
 (no bounded wait may have given up)."""
+import numpy as np
 import pytest
 import torch
 
 import deformable_convolution_dcn1d_b200 as dcn
 import oracle
 import workloads as W
-from gpu_util import TOL, gpu_forward, kernel_name, norm_err, oracle_full, to_dev
+from gpu_util import (TOL, gpu_forward, kernel_name, norm_err, oracle_full, oracle_points,
+                      sample_points, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +59,45 @@ def test_named_dense_workloads_take_the_tensor_core_path(w):
     t = W.make_inputs(w.with_batch(1), seed=0)
     td = to_dev(t)
     assert kernel_name(w.with_batch(1), td) == "tcgen05_bf16"
+
+
+# Several tiles a CTA (more than 3 x 148), so the accumulator's placement cycles: channel
+# blocks of 128 rotate over three 128-column slots; wider ones alternate between columns
+# [0, N) and [128, 128 + N), sharing [128, 256) with the next tile.  The last case leaves
+# no room for the drain's parked values (16 KB of bias), so the shared slot is stored
+# before its release.
+MANY_TILES = [
+    # name, B, C_in, C_out, K, L_in, s, p, d, groups, og, mask, unc, off_scale
+    ("n128_three_slots", 8, 32, 128, 4, 10240, 1, 1, 1, 1, 2, True, False, 2.0),
+    ("n256_alternating_parked", 8, 32, 256, 4, 10240, 1, 2, 1, 1, 1, False, True, 3.0),
+    ("n192_alternating_parked", 6, 64, 192, 4, 12288, 1, 1, 1, 1, 4, True, True, 2.0),
+    ("n256_alternating_no_room_to_park", 1, 1024, 4096, 9, 8192, 2, 4, 2, 16, 16, False,
+     True, 2.0),
+]
+
+
+@pytest.mark.parametrize("case", MANY_TILES, ids=[c[0] for c in MANY_TILES])
+def test_tc_bf16_many_tiles_per_cta(case):
+    name, B, Ci, Co, K, L, s, p, d, G, og, mask, unc, sc = case
+    L_out = oracle.out_length(L, K, s, p, d)
+    w, t = W.small_case(23, B=B, C_in=Ci, C_out=Co, K=K, stride=s, padding=p, dilation=d,
+                        groups=G, offset_groups=og, L_in=L, L_out=L_out, dtype="bf16",
+                        mask=mask, unconstrained=unc, off_scale=sc)
+    td = to_dev(t)
+    assert kernel_name(w, td) == "tcgen05_bf16", kernel_name(w, td)
+    y = gpu_forward(w, td)
+    assert dcn.dcn1d_device_status() == 0
+    # every channel of two positions in each of several tiles, both halves of the
+    # channel block, plus whole rows and random points
+    ls = sorted({0, 127, 128, 255, 256 + 77, 3 * 128 + 5, L_out // 2, L_out - 1})
+    bs = sorted({0, B - 1})
+    grid = np.array([(b, co, l) for b in bs for l in ls for co in range(Co)], dtype=np.int64)
+    rows = [(0, 0), (B - 1, Co - 1), (0, 128 % Co), (B - 1, Co // 2 - 1)]
+    pts = np.concatenate([grid, sample_points(w, 4096, seed=11, rows=rows)])
+    r = oracle_points(w, t, pts)
+    yc = y.double().cpu().numpy()[pts[:, 0], pts[:, 1], pts[:, 2]]
+    err = norm_err(yc, r)
+    assert err <= TOL["bf16"], (name, err)
 
 
 def test_device_status_clean_after_many_launches():
