@@ -37,11 +37,18 @@
 //    values in shared memory and releasing the slot before storing them; the
 //    next tile's MMAs start on their own slot at once and add the shared part of
 //    the staged k-blocks as soon as it is released.  Channel blocks of at most
-//    128 rotate over three slots and never wait for a drain.
+//    128 rotate over three slots and never wait for a drain;
+//  * the last, partial round of tiles: when it holds at most half a grid, the
+//    kernel is launched as clusters of two CTAs and the two CTAs of a cluster
+//    each take half of one such tile's k-blocks; the second sends its fp32
+//    partial sum through distributed shared memory into the first one's freed
+//    weight stages, and the first adds it in its drain.
 // Stages are chained by mbarriers; every wait is bounded (sm100.cuh).
 #include <string.h>
 
+#include <mutex>
 #include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "sampler.cuh"
@@ -87,6 +94,9 @@ struct TcArgs {
     int pair_store;    // 1: L_out even and out 4-byte aligned (32-bit epilogue stores)
     int xtma;          // 1: x windows by TMA; 0 (L_in not a multiple of 8, even): by the
                        // loader warp's 4-byte cp.async copies into the same layout
+    int pair_tail;     // 1: launched as clusters of two CTAs; when the last round holds at
+                       // most half a grid of tiles, the two CTAs of a cluster each take half
+                       // of one such tile's reduction (positions [0, n/2) and [n/2, n))
     int park;          // 1: the drain parks the shared accumulator slot's values in shared
                        // memory (N > 128 and room for 32 KB), so it releases the slot
                        // before its stores
@@ -123,6 +133,41 @@ __device__ __forceinline__ Acc acc_of(uint32_t tc, bool two) {
 
 __device__ __forceinline__ int kb_at(const TcArgs &A, int i) {
     return A.half_kb ? ((i & 1) ? A.half_kb + (i >> 1) : (i >> 1)) : i;
+}
+
+// The i-th unit of work of this CTA: tile t, pipeline positions [p0, p1), and whether it
+// is a whole tile (part 0), the first half of a split tile whose result this CTA stores
+// (part 1, cluster rank 0) or the second half, sent to the first as a partial sum (part 2).
+// Tiles go round-robin over the grid; the last, partial round is split in halves between
+// the CTAs of a cluster when it fits in half the grid.  t < 0: no more work.
+struct Work {
+    int t, p0, p1, part;
+};
+__device__ __forceinline__ Work work_at(const TcArgs &A, int i) {
+    const int grid = (int)gridDim.x, c = (int)blockIdx.x;
+    const int full = A.num_tiles / grid;
+    const int tail = A.num_tiles - full * grid;
+    Work w{-1, 0, A.num_kb, 0};
+    if (i < full) {
+        w.t = i * grid + c;
+    } else if (i == full && tail > 0) {
+        if (A.pair_tail && 2 * tail <= grid) {
+            if ((c >> 1) < tail) {
+                w.t = full * grid + (c >> 1);
+                const int h = A.num_kb / 2;
+                if (c & 1) {
+                    w.p0 = h;
+                    w.part = 2;
+                } else {
+                    w.p1 = h;
+                    w.part = 1;
+                }
+            }
+        } else if (c < tail) {
+            w.t = full * grid + c;
+        }
+    }
+    return w;
 }
 
 struct Tile {
@@ -425,10 +470,13 @@ __global__ void __maxnreg__(96)
         const E *xbase = static_cast<const E *>(P.x);
         const int words = A.nbox * (kBox / 2);   // 4-byte words per staged row
         if (!STALL) {
-            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
-                const Tile T = decode_tile(A, t);
+            for (int wi = 0;; ++wi) {
+                const Work Wk = work_at(A, wi);
+                if (Wk.t < 0)
+                    break;
+                const Tile T = decode_tile(A, Wk.t);
                 const int xrow0 = T.b * P.C_in + T.g * P.cin_g;
-                for (int pos = 0; pos < A.num_kb; ++pos, ++it) {
+                for (int pos = Wk.p0; pos < Wk.p1; ++pos, ++it) {
                     const int kb = kb_at(A, pos);
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
@@ -473,10 +521,13 @@ __global__ void __maxnreg__(96)
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && !STALL) {
             uint32_t it = 0;
-            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
-                const Tile T = decode_tile(A, t);
+            for (int wi = 0;; ++wi) {
+                const Work Wk = work_at(A, wi);
+                if (Wk.t < 0)
+                    break;
+                const Tile T = decode_tile(A, Wk.t);
                 const int xrow0 = T.b * P.C_in + T.g * P.cin_g;
-                for (int pos = 0; pos < A.num_kb; ++pos, ++it) {
+                for (int pos = Wk.p0; pos < Wk.p1; ++pos, ++it) {
                     const int kb = kb_at(A, pos);
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
@@ -509,7 +560,10 @@ __global__ void __maxnreg__(96)
             const uint32_t idesc_lo = Elem<E>::idesc(128, kSlotCols);
             const uint32_t idesc_hi = Elem<E>::idesc(128, two ? A.N - kSlotCols : 32);
             uint32_t it = 0, tc = 0;
-            for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x, ++tc) {
+            for (int wi = 0;; ++wi, ++tc) {
+                const Work Wk = work_at(A, wi);
+                if (Wk.t < 0)
+                    break;
                 const Acc acc = acc_of(tc, two);
                 // the own slot's last tile (two or three back) has been drained
                 if (acc.own_uses > 0 && !wait(bar_dfree(acc.own), (acc.own_uses - 1u) & 1u))
@@ -531,9 +585,9 @@ __global__ void __maxnreg__(96)
                     for (int kk = 0; kk < kBK / 16; ++kk)
                         mma_bf16_ts(dp, tmem + kColA + 32u * s + 8u * kk,
                                     sw128_kmajor_desc(wst + 32u * kk), lo ? idesc_lo : idesc_hi,
-                                    (p > 0 || kk > 0) ? 1u : 0u);
+                                    (p > Wk.p0 || kk > 0) ? 1u : 0u);
                 };
-                for (int pos = 0; pos < A.num_kb; ++pos, ++it) {
+                for (int pos = Wk.p0; pos < Wk.p1; ++pos, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
                     if (!wait(bar_full(s), ph) || !wait(bar_afull(s), ph))
@@ -545,14 +599,14 @@ __global__ void __maxnreg__(96)
                         for (int kk = 0; kk < kBK / 16; ++kk) {
                             mma_bf16_ts(d, tmem + kColA + 32u * s + 8u * kk,
                                         sw128_kmajor_desc(wst + 32u * kk), idesc,
-                                        (pos > 0 || kk > 0) ? 1u : 0u);
+                                        (pos > Wk.p0 || kk > 0) ? 1u : 0u);
                         }
                         mma_commit(bar_empty(s));
                         continue;
                     }
                     part(true, pos, s);
                     ++pend;
-                    const bool must = pend == kStages || pos == A.num_kb - 1;
+                    const bool must = pend == kStages || pos == Wk.p1 - 1;
                     const uint32_t sh_par = (tc - 1u) & 1u;   // the shared slot's last drain
                     if (must ? wait(bar_dfree(1), sh_par) : mbar_try_wait(bar_dfree(1), sh_par)) {
                         tc_fence_after();
@@ -713,16 +767,25 @@ __global__ void __maxnreg__(96)
         // This warp's group takes the positions whose ring index tcount*num_kb + pos has
         // its parity, so each ring stage always has the same consumer group, even when a
         // tile has an odd number of k-blocks (a parity wait is never a phase ahead).
-        auto first_pos = [&](uint32_t tcnt) {
-            return (int)(((uint32_t)par ^ (tcnt * (uint32_t)A.num_kb)) & 1u);
+        // positions [p0, p1) of a work unit whose first one has ring index base
+        auto first_pos = [&](uint32_t base, int p0) {
+            return p0 + (int)(((uint32_t)par ^ base) & 1u);
         };
-        if (kAhead && (int)blockIdx.x < A.num_tiles && first_pos(0) < A.num_kb) {
-            const Tile T0 = decode_tile(A, blockIdx.x);
-            prefetch(blockIdx.x, T0, seg_og(T0, first_pos(0)));
+        {
+            const Work W0 = work_at(A, 0);
+            if (kAhead && W0.t >= 0 && first_pos(0, W0.p0) < W0.p1) {
+                const Tile T0 = decode_tile(A, W0.t);
+                prefetch(W0.t, T0, seg_og(T0, first_pos(0, W0.p0)));
+            }
         }
-        for (int t = blockIdx.x; t < A.num_tiles; t += gridDim.x) {
+        uint32_t itbase = 0;    // ring index of the current unit's first position
+        for (int wi = 0;; ++wi) {
+            const Work Wk = work_at(A, wi);
+            if (Wk.t < 0)
+                break;
+            const int t = Wk.t;
             const Tile T = decode_tile(A, t);
-            const int t_next = t + (int)gridDim.x;
+            const uint32_t itnext = itbase + (uint32_t)(Wk.p1 - Wk.p0);
             // Rows past L_out (the last tile's) sample with row 0's offsets: their taps are
             // finite and read the window or the bounds-checked slow path, and their
             // accumulator rows (each depends on its own operand row only) are never stored.
@@ -731,10 +794,10 @@ __global__ void __maxnreg__(96)
             const float hi_bound = __fadd_rn(start, spanf);   // the receptive field's end
             const float dil_f = (float)P.dilation;
             const uint32_t win_bits = kFloorMagicBits + (uint32_t)T.wx0;
-            const int pos_first = first_pos(tcount);
+            const int pos_first = first_pos(itbase, Wk.p0);
             const int pos_last =
-                pos_first < A.num_kb ? pos_first + ((A.num_kb - 1 - pos_first) / 2) * 2 : 0;
-            const int og_last = pos_first < A.num_kb ? seg_og(T, pos_last) : 0;   // this warp's last
+                pos_first < Wk.p1 ? pos_first + ((Wk.p1 - 1 - pos_first) / 2) * 2 : 0;
+            const int og_last = pos_first < Wk.p1 ? seg_og(T, pos_last) : 0;   // this warp's last
             const E *xb = static_cast<const E *>(P.x) + (int64_t)T.b * P.C_in * P.L_in;
             Taps<K> tp;
             // Offset group of the first channel of this warp's first segment; it only
@@ -742,10 +805,11 @@ __global__ void __maxnreg__(96)
             int og_cur = -1;
             int og = (T.g * P.cin_g) / P.cin_per_og;
             int og_next_c = (og + 1) * P.cin_per_og - T.g * P.cin_g;   // group-relative
-            const int kb_first_stage = (A.num_kb < kStages ? A.num_kb : kStages);
-            for (int pos = pos_first; pos < A.num_kb; pos += 2) {
+            const int npos = Wk.p1 - Wk.p0;
+            const int kb_first_stage = (npos < kStages ? npos : kStages);
+            for (int pos = pos_first; pos < Wk.p1; pos += 2) {
                 const int kb = kb_at(A, pos);
-                const uint32_t it = tcount * (uint32_t)A.num_kb + (uint32_t)pos;
+                const uint32_t it = itbase + (uint32_t)(pos - Wk.p0);
                 const int s = it % kStages;
                 const uint32_t ph = (it / kStages) & 1u;
                 const int kk0 = kb * kBK + kSeg * half;
@@ -798,10 +862,12 @@ __global__ void __maxnreg__(96)
                     if constexpr (kAhead) {
                         if (og < og_last)
                             prefetch(t, T, og + 1);
-                        else if (t_next < A.num_tiles) {
-                            const Tile Tn = decode_tile(A, t_next);   // once per tile
-                            if (first_pos(tcount + 1) < A.num_kb)
-                                prefetch(t_next, Tn, seg_og(Tn, first_pos(tcount + 1)));
+                        else {
+                            const Work Wn = work_at(A, wi + 1);   // once per tile
+                            if (Wn.t >= 0 && first_pos(itnext, Wn.p0) < Wn.p1) {
+                                const Tile Tn = decode_tile(A, Wn.t);
+                                prefetch(Wn.t, Tn, seg_og(Tn, first_pos(itnext, Wn.p0)));
+                            }
                         }
                     }
                 }
@@ -829,7 +895,7 @@ __global__ void __maxnreg__(96)
                     if (lane == 0)
                         mbar_arrive(bar_afull(s));
                 }
-                if (pend_t >= 0 && pos + 2 >= kb_first_stage) {
+                if (pend_t >= 0 && (pos - Wk.p0) + 2 >= kb_first_stage) {
                     if (!epilogue(pend_t, pend_cnt))
                         goto prod_done;
                     pend_t = -1;
@@ -840,8 +906,12 @@ __global__ void __maxnreg__(96)
                     goto prod_done;
                 pend_t = -1;
             }
-            pend_t = t;
-            pend_cnt = tcount++;
+            if (Wk.part == 0) {   // a split unit is finished at the teardown
+                pend_t = t;
+                pend_cnt = tcount;
+            }
+            ++tcount;
+            itbase = itnext;
         }
         if (pend_t >= 0)
             epilogue(pend_t, pend_cnt);
@@ -850,6 +920,62 @@ __global__ void __maxnreg__(96)
 
     // ---------------------------------------------------------------- teardown
     tc_fence_before();
+    {
+        // A split last unit.  Every thread of both CTAs of the cluster reaches this point
+        // on every path, aborts included, so both cluster barriers always complete.
+        const int full = A.num_tiles / (int)gridDim.x;
+        const Work Wl = work_at(A, full);
+        if (Wl.t >= 0 && Wl.part != 0) {
+            // 1: every MMA of both CTAs has completed (each issuer waited for its drain
+            // commit; each loader for its copies), so the first CTA's weight stages are
+            // free to take the second CTA's partial sum, [N/4][128 rows][4] fp32
+            cluster_barrier();
+            tc_fence_after();
+            const int q = warp % 4, h = warp / 4, row = 32 * q + lane;
+            const Acc acc = acc_of((uint32_t)full, A.N > kSlotCols);
+            if (Wl.part == 2 && warp < kProdWarps) {
+                const uint32_t dst = cluster_map(w_st0, 0);
+                for (int cc = h; cc < A.N / 16; cc += 4) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + acc.col + 16u * cc, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        st_cluster_v4(dst + 16u * ((uint32_t)(4 * cc + g) * kRows + (uint32_t)row),
+                                      v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+                }
+            }
+            // 2: the partial sum is in place
+            cluster_barrier();
+            if (Wl.part == 1 && warp < kProdWarps) {
+                const Tile T = decode_tile(A, Wl.t);
+                const int l = T.lbase + row;
+                const float *biasg = bias_s + T.co0;
+                const float4 *part = reinterpret_cast<const float4 *>(smem + A.off_w) + row;
+                E *outp = static_cast<E *>(P.out) +
+                          ((int64_t)T.b * P.C_out + (int64_t)T.co0) * P.L_out + l;
+                for (int cc = h; cc < A.N / 16; cc += 4) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + acc.col + 16u * cc, v);
+                    tmem_wait_ld();
+                    if (l < P.L_out) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const float4 pv = part[(4 * cc + g) * kRows];
+                            const float pg[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int co = 16 * cc + 4 * g + i;
+                                outp[(int64_t)co * P.L_out] = from_f32<E>(
+                                    (__uint_as_float(v[4 * g + i]) + pg[i]) + biasg[co]);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+        }
+    }
     __syncthreads();
     if (warp == kMmaWarp) {
         __syncwarp();
@@ -925,6 +1051,33 @@ bool make_plan(const Problem &P, Plan *out) {
     return true;
 }
 
+// Whether clusters of two CTAs of this kernel and shared-memory size can cover all `sms`
+// SMs at once (asked once per kernel and size).
+bool pair_clusters_fit(const void *kern, int smem, int sms) {
+    static std::mutex mu;
+    static std::vector<std::pair<std::pair<const void *, int>, bool>> memo;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const auto &m : memo)
+        if (m.first.first == kern && m.first.second == smem)
+            return m.second;
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)sms);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const bool ok = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && 2 * n >= sms;
+    cudaGetLastError();   // a refused query leaves no error behind
+    memo.push_back({{kern, smem}, ok});
+    return ok;
+}
+
 template <class E, int K, bool MASK, bool STALL = false>
 cudaError_t launch_km(const Plan &pl, cudaStream_t stream) {
     const Problem &P = pl.A.P;
@@ -945,10 +1098,31 @@ cudaError_t launch_km(const Plan &pl, cudaStream_t stream) {
     const int sms = sm_count();
     if (sms <= 0)
         return cudaErrorNoDevice;
-    const int grid = pl.A.num_tiles < sms ? pl.A.num_tiles : sms;
+    TcArgs A = pl.A;
+    // The last round's tiles split in halves between the CTAs of 2-CTA clusters, when that
+    // round holds at most half a grid of tiles and the whole grid fits as clusters.
+    const int tail = A.num_tiles % sms;
+    const bool pair = !STALL && sms % 2 == 0 && A.num_kb >= 2 && tail > 0 && 2 * tail <= sms &&
+                      pair_clusters_fit(reinterpret_cast<const void *>(kern), (int)pl.smem, sms);
+    A.pair_tail = pair ? 1 : 0;
+    const int grid = pair ? sms : (A.num_tiles < sms ? A.num_tiles : sms);
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pair ? 2u : 1u;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pair ? 1 : 0;
     timing_begin(stream);
-    kern<<<grid, kThreads, pl.smem, stream>>>(pl.A, wmap, xmap);
+    e = cudaLaunchKernelEx(&cfg, kern, A, wmap, xmap);
     timing_end(stream);
+    if (e != cudaSuccess)
+        return e;
     return cudaGetLastError();
 }
 
