@@ -105,10 +105,6 @@ struct TcArgs {
     uint64_t wait_ns;                           // limit of every mbarrier wait
 };
 
-// The k-block at pipeline position i of a tile.  Positions alternate between the two
-// producer groups (group = i % 2), so each group owns every other stage of the ring (the
-// ring depth is even).  With contiguous halves a group walks its channels in order and
-// meets each offset group once; the parity split is the fallback for odd counts.
 // The accumulator of a CTA's tile number tc: its first column, the slot only it uses
 // (N > 128: 0 for even tiles, 2 for odd ones; N <= 128: tc % 3) and how many earlier
 // tiles used that slot.
@@ -131,6 +127,12 @@ __device__ __forceinline__ Acc acc_of(uint32_t tc, bool two) {
     return a;
 }
 
+// The k-block at pipeline position i of a tile.  The two producer groups take the
+// positions by the parity of their ring index, so each group owns every other stage of
+// the ring (the ring depth is even), and the ring index parity alternates with the
+// position.  With contiguous halves (positions 0, 1, 2, 3, ... -> k-blocks 0, n/2, 1,
+// n/2 + 1, ...) a group walks its channels in order and meets each offset group once;
+// otherwise the positions are the k-blocks themselves.
 __device__ __forceinline__ int kb_at(const TcArgs &A, int i) {
     return A.half_kb ? ((i & 1) ? A.half_kb + (i >> 1) : (i >> 1)) : i;
 }
