@@ -1054,14 +1054,24 @@ bool make_plan(const Problem &P, Plan *out) {
 }
 
 // Whether clusters of two CTAs of this kernel and shared-memory size can cover all `sms`
-// SMs at once (asked once per kernel and size).
+// SMs of the current device at once (asked once per device, kernel and size; the record
+// keeps the last 64 answers).
 bool pair_clusters_fit(const void *kern, int smem, int sms) {
+    struct Seen {
+        int dev;
+        const void *kern;
+        int smem, sms;
+        bool ok;
+    };
     static std::mutex mu;
-    static std::vector<std::pair<std::pair<const void *, int>, bool>> memo;
+    static std::vector<Seen> memo;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return false;
     std::lock_guard<std::mutex> lock(mu);
     for (const auto &m : memo)
-        if (m.first.first == kern && m.first.second == smem)
-            return m.second;
+        if (m.dev == dev && m.kern == kern && m.smem == smem && m.sms == sms)
+            return m.ok;
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
     cfg.gridDim = dim3((unsigned)sms);
@@ -1076,7 +1086,9 @@ bool pair_clusters_fit(const void *kern, int smem, int sms) {
     int n = 0;
     const bool ok = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && 2 * n >= sms;
     cudaGetLastError();   // a refused query leaves no error behind
-    memo.push_back({{kern, smem}, ok});
+    if (memo.size() >= 64)
+        memo.erase(memo.begin());
+    memo.push_back({dev, kern, smem, sms, ok});
     return ok;
 }
 
