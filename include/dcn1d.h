@@ -440,9 +440,9 @@ const char *dcn1d_forward_kernel_name(const dcn1d_tensor *x, const dcn1d_tensor 
 /*
  * For benchmarks: the next dcn1d_forward / dcn1d_forward_ws call on this host
  * thread records `begin` (a cudaEvent_t) on its stream right before launching
- * its main kernel and `end` right after it, then forgets both.  A forward that
- * launches helper kernels (weight split, split-K reduction) keeps them outside
- * the pair.  NULL events record nothing.
+ * its kernel and `end` right after it, then forgets both.  Every forward is one
+ * kernel launch, so the pair brackets all of its device work.  NULL events record
+ * nothing.
  */
 void dcn1d_set_timing_events(void *begin, void *end);
 
