@@ -73,6 +73,10 @@ MANY_TILES = [
     ("n192_alternating_parked", 6, 64, 192, 4, 12288, 1, 1, 1, 1, 4, True, True, 2.0),
     ("n256_alternating_no_room_to_park", 1, 1024, 4096, 9, 8192, 2, 4, 2, 16, 16, False,
      True, 2.0),
+    # last rounds of 50 and 60 tiles, split between the CTAs of 2-CTA clusters: three
+    # k-blocks (halves of one and two), and K = 16 in two 256-channel blocks
+    ("k3_mask_odd_kblocks_split_tail", 6, 64, 256, 3, 13696, 1, 1, 1, 1, 2, True, False, 2.0),
+    ("k16_two_blocks_split_tail", 2, 128, 512, 16, 16048, 1, 0, 3, 1, 1, False, False, 1.5),
 ]
 
 
